@@ -1,0 +1,115 @@
+"""Seeded synthetic inputs shared by the tests, the benchmark and the oracle leg.
+
+This module draws random numbers and lays them out; it holds none of the
+attention arithmetic.  Recipe (the same for every workload):
+
+* q, K, V: i.i.d. N(0, 1) in bf16 (torch normal in fp32, rounded to bf16),
+  drawn from ``torch.Generator(device).manual_seed(seed)`` with seeds
+  ``base+0`` (q), ``base+1`` (K), ``base+2`` (V);
+* seqlens: integers uniform on the closed interval [lo, hi] from seed
+  ``base+3`` on a CPU generator (so every device sees the same lengths);
+* cache rows at or past ``seqlens[b]`` hold random values too, or NaN when
+  ``poison=True`` (a read past the end then shows up as NaN in the output);
+* ``q_gain`` multiplies q before rounding (a "peaky" softmax when > 1).
+
+Layouts are the ones of the C ABI: decode q [B,Hq,d], caches [B,Tmax,Hkv,d];
+prefill q [B,S,Hq,d], k/v [B,S,Hkv,d].
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+
+def _normal(shape, seed: int, device, gain: float = 1.0) -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    x = torch.empty(shape, dtype=torch.float32, device=device)
+    # fill in slices so a 34 GB cache never needs a 68 GB fp32 temporary
+    flat = x.view(-1)
+    step = 1 << 28
+    for s in range(0, flat.numel(), step):
+        flat[s:s + step].normal_(generator=g)
+    if gain != 1.0:
+        x.mul_(gain)
+    return x.to(torch.bfloat16)
+
+
+def _normal_bf16(shape, seed: int, device) -> torch.Tensor:
+    """N(0,1) bf16 drawn in slices straight into a bf16 buffer (large caches)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    flat = out.view(-1)
+    step = 1 << 27
+    tmp = torch.empty(min(step, max(flat.numel(), 1)), dtype=torch.float32, device=device)
+    for s in range(0, flat.numel(), step):
+        n = min(step, flat.numel() - s)
+        t = tmp[:n]
+        t.normal_(generator=g)
+        flat[s:s + n].copy_(t)
+    return out
+
+
+def seqlens_uniform(B: int, lo: int, hi: int, seed: int) -> torch.Tensor:
+    """B integers uniform on [lo, hi] (inclusive), CPU int32."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return torch.randint(lo, hi + 1, (B,), generator=g, dtype=torch.int64).to(torch.int32)
+
+
+@dataclass
+class DecodeInputs:
+    q: torch.Tensor          # [B,Hq,d] bf16
+    k_cache: torch.Tensor    # [B,Tmax,Hkv,d] bf16
+    v_cache: torch.Tensor    # [B,Tmax,Hkv,d] bf16
+    seqlens: torch.Tensor    # [B] int32, same device as q
+    scale: float
+
+
+def make_decode(B: int, Hq: int, Hkv: int, d: int, Tmax: int, seqlens=None, *, device="cpu",
+                seed: int = 0, scale: float | None = None, poison: bool = False,
+                q_gain: float = 1.0, seqlen_range=None) -> DecodeInputs:
+    """Decode inputs.  ``seqlens``: None -> every sequence holds Tmax tokens;
+    an int -> all equal; a list/tensor -> as given; or ``seqlen_range=(lo,hi)``
+    draws them uniformly with seed ``seed+3``."""
+    if seqlen_range is not None:
+        sl = seqlens_uniform(B, seqlen_range[0], seqlen_range[1], seed + 3)
+    elif seqlens is None:
+        sl = torch.full((B,), Tmax, dtype=torch.int32)
+    elif isinstance(seqlens, int):
+        sl = torch.full((B,), seqlens, dtype=torch.int32)
+    else:
+        sl = torch.as_tensor(seqlens, dtype=torch.int32).cpu()
+    q = _normal((B, Hq, d), seed + 0, device, q_gain)
+    big = B * Tmax * Hkv * d > (1 << 26)
+    mk = _normal_bf16 if big else _normal
+    k = mk((B, Tmax, Hkv, d), seed + 1, device)
+    v = mk((B, Tmax, Hkv, d), seed + 2, device)
+    if poison:
+        nan = torch.tensor(float("nan"), dtype=torch.bfloat16, device=device)
+        for b in range(B):
+            t = int(sl[b])
+            if t < Tmax:
+                k[b, t:].fill_(nan)
+                v[b, t:].fill_(nan)
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    return DecodeInputs(q, k, v, sl.to(device), scale)
+
+
+@dataclass
+class PrefillInputs:
+    q: torch.Tensor   # [B,S,Hq,d] bf16
+    k: torch.Tensor   # [B,S,Hkv,d] bf16
+    v: torch.Tensor   # [B,S,Hkv,d] bf16
+    scale: float
+
+
+def make_prefill(B: int, S: int, Hq: int, Hkv: int, d: int, *, device="cpu", seed: int = 0,
+                 q_gain: float = 1.0) -> PrefillInputs:
+    q = _normal((B, S, Hq, d), seed + 0, device, q_gain)
+    k = _normal((B, S, Hkv, d), seed + 1, device)
+    v = _normal((B, S, Hkv, d), seed + 2, device)
+    return PrefillInputs(q, k, v, 1.0 / float(d) ** 0.5)

@@ -1,0 +1,49 @@
+"""The five synthetic workloads, by what they are and their sizes.
+
+Shapes follow the pages: the 32/8/128 head geometry read off a config file in
+deepconcepts.dev "Checking it on a real system", the 32-query / 2-KV-head
+geometry of inferencex.semianalysis.com "Engineering details" (KV head
+replication), and the causal prefill of anrans.github.io attention-variants.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    d: int
+    Tmax: int
+    seqlen_range: tuple | None = None   # None: every sequence holds Tmax tokens
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+
+@dataclass(frozen=True)
+class PrefillWorkload:
+    name: str
+    B: int
+    S: int
+    Hq: int
+    Hkv: int
+    d: int
+
+
+TINY_DECODE = DecodeWorkload("tiny decode B1 Hq8 Hkv2 d128 T256", 1, 8, 2, 128, 256)
+QWEN3_8B_DECODE = DecodeWorkload("Qwen3-8B-shaped decode B49 Hq32 Hkv8 d128 T8192", 49, 32, 8, 128, 8192)
+VARLEN_DECODE = tuple(
+    DecodeWorkload(f"variable-length decode B64 Hq32 Hkv{h} d128 T~U[512,32768]", 64, 32, h, 128, 32768,
+                   (512, 32768))
+    for h in (32, 8, 4, 1)
+)
+EXTREME_GROUP_DECODE = DecodeWorkload(
+    "extreme grouping decode (Qwen3.5-style, 32 q heads / 2 KV heads) B16 d128 T131072", 16, 32, 2, 128, 131072)
+CAUSAL_PREFILL = PrefillWorkload("causal GQA prefill B4 S8192 Hq32 Hkv8 d128", 4, 8192, 32, 8, 128)
+
+DECODE_WORKLOADS = (TINY_DECODE, QWEN3_8B_DECODE) + VARLEN_DECODE + (EXTREME_GROUP_DECODE,)

@@ -1,0 +1,313 @@
+/*
+ * gqa_oracle.c -- plain, slow, fp64 CPU oracle for grouped-query attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path (the
+ * CUDA library and its Python binding) never calls it and shares no code,
+ * header, table or helper with it.
+ *
+ * What it computes, and where the pages define it:
+ *
+ *  - Consecutive group mapping, kv_head = q_head / (Hq / Hkv), Hq divisible
+ *    by Hkv: "Share keys and values without confusing query-head identity"
+ *    (study.greatitself.com, grouped-query and multi-query attention), and the
+ *    eight-to-two mapping check in "Shared KV can still produce different
+ *    outputs" (lihaoran.work/?p=2890).
+ *  - Raw KV-cache bytes = 2 x layers x tokens x kv_heads x head_dim x bytes:
+ *    "KV-head count determines the raw cache ratio" (lihaoran.work/?p=2890),
+ *    "Three numbers that people expect to move together"
+ *    (deepconcepts.dev, Grouped-Query Attention).
+ *  - Per query head, softmax(q K^T * scale) V with the head's own
+ *    distribution: "Shared KV can still produce different outputs"
+ *    (lihaoran.work/?p=2890).
+ *  - The expanded formulation: each query head gets its own explicit copy of
+ *    the K and V rows of its KV head (the repeat_interleave form), then plain
+ *    per-head attention: "Kernels do not need to copy the KV heads"
+ *    (anrans.github.io attention-variants, version 1 of its example).
+ *  - Causal prefill: row r attends to tokens t <= r (lower triangle including
+ *    the diagonal), masked scores excluded from the softmax: same section,
+ *    the tril mask of its example.
+ *
+ * Everything is done in double precision.  Inputs are the bf16 bit patterns
+ * the GPU sees; bf16 is the upper 16 bits of an IEEE-754 binary32, so the
+ * conversion below is exact.  The softmax is the two-pass form: maximum, then
+ * exp(s - max) weights, then the weighted sum divided by the sum of weights.
+ *
+ * Readings taken where the pages are silent (each is listed in the design
+ * notes of the repository):
+ *  - decode: the query sees every cached token t < seqlens[b] (no other mask);
+ *  - an empty history (seqlens[b] == 0) gives an all-zero output row;
+ *  - outputs are fp64; callers compare rounded GPU outputs against them.
+ *
+ * Threads (pthreads) split the work over (batch, query head) pairs; each
+ * pair is computed by exactly the same sequential code.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_NO_MEMORY 2
+
+/* ---- definitions the pages fix ------------------------------------------ */
+
+/* kv head used by query head h under the consecutive grouping; -1 when the
+ * grouping is not regular (Hq not divisible by Hkv) or h is out of range. */
+int gqa_oracle_kv_head(int h, int Hq, int Hkv)
+{
+    if (Hq <= 0 || Hkv <= 0 || h < 0 || h >= Hq) return -1;
+    if (Hq % Hkv != 0) return -1;
+    int group = Hq / Hkv;
+    return h / group;
+}
+
+/* raw KV-cache payload in bytes: K and V, for every layer, token, kv head and
+ * head coordinate. */
+long long gqa_oracle_kv_bytes(long long layers, long long tokens, long long kv_heads,
+                              long long head_dim, long long bytes_per_elem)
+{
+    return 2LL * layers * tokens * kv_heads * head_dim * bytes_per_elem;
+}
+
+/* bf16 bit pattern -> double: the pattern is the top half of a binary32. */
+static double bf16_to_double(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+void gqa_oracle_bf16_to_f64(const uint16_t *x, double *y, long long n)
+{
+    for (long long i = 0; i < n; ++i) y[i] = bf16_to_double(x[i]);
+}
+
+/* ---- one query row against an explicit per-head copy of K and V --------- */
+
+/* out[0:d] = sum_t softmax_t(scale * q.K[t]) V[t] over t < n, two-pass.
+ * K, V are the head's own (already repeated) rows, row-major [n][d]. */
+static void attend_row(const double *q, const double *K, const double *V, long long n, int d,
+                       double scale, double *scores, double *out)
+{
+    for (int j = 0; j < d; ++j) out[j] = 0.0;
+    if (n <= 0) return;
+    double m = -INFINITY;
+    for (long long t = 0; t < n; ++t) {
+        double s = 0.0;
+        for (int j = 0; j < d; ++j) s += q[j] * K[t * d + j];
+        s *= scale;
+        scores[t] = s;
+        if (s > m) m = s;
+    }
+    double denom = 0.0;
+    for (long long t = 0; t < n; ++t) {
+        double w = exp(scores[t] - m);
+        scores[t] = w;
+        denom += w;
+    }
+    for (long long t = 0; t < n; ++t) {
+        double w = scores[t];
+        for (int j = 0; j < d; ++j) out[j] += w * V[t * d + j];
+    }
+    for (int j = 0; j < d; ++j) out[j] /= denom;
+}
+
+/* ---- decode -------------------------------------------------------------- */
+
+typedef struct {
+    const uint16_t *q, *k, *v;
+    const int32_t *seqlens;
+    int B, Hq, Hkv, d, Tmax;
+    double scale;
+    double *out;
+    int tid, nthreads;
+    int status;
+} decode_job;
+
+static void *decode_worker(void *arg)
+{
+    decode_job *J = (decode_job *)arg;
+    const int d = J->d;
+    double *qrow = (double *)malloc(sizeof(double) * (size_t)d);
+    double *Kh = (double *)malloc(sizeof(double) * (size_t)J->Tmax * (size_t)d);
+    double *Vh = (double *)malloc(sizeof(double) * (size_t)J->Tmax * (size_t)d);
+    double *sc = (double *)malloc(sizeof(double) * (size_t)(J->Tmax > 0 ? J->Tmax : 1));
+    if (!qrow || !Kh || !Vh || !sc) {
+        J->status = ORACLE_NO_MEMORY;
+        free(qrow); free(Kh); free(Vh); free(sc);
+        return NULL;
+    }
+    long long pairs = (long long)J->B * J->Hq;
+    for (long long p = J->tid; p < pairs; p += J->nthreads) {
+        int b = (int)(p / J->Hq), h = (int)(p % J->Hq);
+        int kvh = gqa_oracle_kv_head(h, J->Hq, J->Hkv);
+        long long T = J->seqlens[b];
+        /* explicit repeat: this query head's own copy of its KV head's rows */
+        for (long long t = 0; t < T; ++t) {
+            size_t src = (((size_t)b * J->Tmax + (size_t)t) * J->Hkv + (size_t)kvh) * (size_t)d;
+            for (int j = 0; j < d; ++j) {
+                Kh[t * d + j] = bf16_to_double(J->k[src + j]);
+                Vh[t * d + j] = bf16_to_double(J->v[src + j]);
+            }
+        }
+        size_t qo = ((size_t)b * J->Hq + (size_t)h) * (size_t)d;
+        for (int j = 0; j < d; ++j) qrow[j] = bf16_to_double(J->q[qo + j]);
+        attend_row(qrow, Kh, Vh, T, d, J->scale, sc, J->out + qo);
+    }
+    free(qrow); free(Kh); free(Vh); free(sc);
+    return NULL;
+}
+
+/* q [B,Hq,d], k/v [B,Tmax,Hkv,d] bf16 bits, seqlens [B] (0 <= seqlens <= Tmax),
+ * out [B,Hq,d] fp64.  Returns 0 on success. */
+int gqa_oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                      const int32_t *seqlens, int B, int Hq, int Hkv, int d, int Tmax,
+                      double scale, double *out, int nthreads)
+{
+    if (!q || !k || !v || !seqlens || !out) return ORACLE_BAD_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Tmax < 0) return ORACLE_BAD_ARG;
+    if (Hq % Hkv != 0) return ORACLE_BAD_ARG;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > Tmax) return ORACLE_BAD_ARG;
+    if (nthreads < 1) nthreads = 1;
+    if ((long long)nthreads > (long long)B * Hq) nthreads = B * Hq;
+    decode_job *jobs = (decode_job *)calloc((size_t)nthreads, sizeof(decode_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) { free(jobs); free(th); return ORACLE_NO_MEMORY; }
+    for (int i = 0; i < nthreads; ++i) {
+        decode_job J = {q, k, v, seqlens, B, Hq, Hkv, d, Tmax, scale, out, i, nthreads, ORACLE_OK};
+        jobs[i] = J;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, decode_worker, &jobs[i]);
+    decode_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    int st = ORACLE_OK;
+    for (int i = 0; i < nthreads; ++i) if (jobs[i].status != ORACLE_OK) st = jobs[i].status;
+    free(jobs); free(th);
+    return st;
+}
+
+/* ---- causal prefill ------------------------------------------------------ */
+
+typedef struct {
+    const uint16_t *q, *k, *v;
+    int B, S, Hq, Hkv, d;
+    double scale;
+    const int32_t *rows; /* NULL: every row; else nrows (b, h, r) triples */
+    long long nrows;
+    double *out;
+    int tid, nthreads;
+    int status;
+} prefill_job;
+
+/* every row of one (b, h): row r sees tokens 0..r inclusive */
+static void prefill_head(const prefill_job *J, int b, int h, double *Kh, double *Vh,
+                         double *qrow, double *sc)
+{
+    const int d = J->d, S = J->S;
+    int kvh = gqa_oracle_kv_head(h, J->Hq, J->Hkv);
+    /* explicit repeat of the whole KV head for this query head */
+    for (long long t = 0; t < S; ++t) {
+        size_t src = (((size_t)b * S + (size_t)t) * J->Hkv + (size_t)kvh) * (size_t)d;
+        for (int j = 0; j < d; ++j) {
+            Kh[t * d + j] = bf16_to_double(J->k[src + j]);
+            Vh[t * d + j] = bf16_to_double(J->v[src + j]);
+        }
+    }
+    for (long long r = 0; r < S; ++r) {
+        size_t qo = (((size_t)b * S + (size_t)r) * J->Hq + (size_t)h) * (size_t)d;
+        for (int j = 0; j < d; ++j) qrow[j] = bf16_to_double(J->q[qo + j]);
+        attend_row(qrow, Kh, Vh, r + 1, d, J->scale, sc, J->out + qo);
+    }
+}
+
+static void *prefill_worker(void *arg)
+{
+    prefill_job *J = (prefill_job *)arg;
+    const int d = J->d, S = J->S;
+    double *Kh = (double *)malloc(sizeof(double) * (size_t)S * (size_t)d);
+    double *Vh = (double *)malloc(sizeof(double) * (size_t)S * (size_t)d);
+    double *qrow = (double *)malloc(sizeof(double) * (size_t)d);
+    double *sc = (double *)malloc(sizeof(double) * (size_t)S);
+    if (!Kh || !Vh || !qrow || !sc) {
+        J->status = ORACLE_NO_MEMORY;
+        free(Kh); free(Vh); free(qrow); free(sc);
+        return NULL;
+    }
+    long long pairs = (long long)J->B * J->Hq;
+    for (long long p = J->tid; p < pairs; p += J->nthreads) {
+        int b = (int)(p / J->Hq), h = (int)(p % J->Hq);
+        if (!J->rows) {
+            prefill_head(J, b, h, Kh, Vh, qrow, sc);
+            continue;
+        }
+        /* subset mode: compute every listed row that belongs to (b, h) */
+        int have_kv = 0;
+        for (long long i = 0; i < J->nrows; ++i) {
+            const int32_t *e = J->rows + 3 * i;
+            if (e[0] != b || e[1] != h) continue;
+            int kvh = gqa_oracle_kv_head(h, J->Hq, J->Hkv);
+            if (!have_kv) {
+                long long rmax = 0;
+                for (long long u = i; u < J->nrows; ++u) {
+                    const int32_t *f = J->rows + 3 * u;
+                    if (f[0] == b && f[1] == h && f[2] > rmax) rmax = f[2];
+                }
+                for (long long t = 0; t <= rmax; ++t) {
+                    size_t src = (((size_t)b * S + (size_t)t) * J->Hkv + (size_t)kvh) * (size_t)d;
+                    for (int j = 0; j < d; ++j) {
+                        Kh[t * d + j] = bf16_to_double(J->k[src + j]);
+                        Vh[t * d + j] = bf16_to_double(J->v[src + j]);
+                    }
+                }
+                have_kv = 1;
+            }
+            long long r = e[2];
+            size_t qo = (((size_t)b * S + (size_t)r) * J->Hq + (size_t)h) * (size_t)d;
+            for (int j = 0; j < d; ++j) qrow[j] = bf16_to_double(J->q[qo + j]);
+            attend_row(qrow, Kh, Vh, r + 1, d, J->scale, sc, J->out + (size_t)i * (size_t)d);
+        }
+    }
+    free(Kh); free(Vh); free(qrow); free(sc);
+    return NULL;
+}
+
+/* q [B,S,Hq,d], k/v [B,S,Hkv,d] bf16 bits.  rows == NULL: out [B,S,Hq,d] fp64
+ * for every row.  rows != NULL: nrows (b, h, r) int32 triples; out [nrows,d]
+ * holds those rows in the order given.  Returns 0 on success. */
+int gqa_oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, int B, int S,
+                       int Hq, int Hkv, int d, double scale, const int32_t *rows,
+                       long long nrows, double *out, int nthreads)
+{
+    if (!q || !k || !v || !out) return ORACLE_BAD_ARG;
+    if (B <= 0 || S <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return ORACLE_BAD_ARG;
+    if (Hq % Hkv != 0) return ORACLE_BAD_ARG;
+    if (rows) {
+        if (nrows < 0) return ORACLE_BAD_ARG;
+        for (long long i = 0; i < nrows; ++i) {
+            const int32_t *e = rows + 3 * i;
+            if (e[0] < 0 || e[0] >= B || e[1] < 0 || e[1] >= Hq || e[2] < 0 || e[2] >= S)
+                return ORACLE_BAD_ARG;
+        }
+    }
+    if (nthreads < 1) nthreads = 1;
+    if ((long long)nthreads > (long long)B * Hq) nthreads = B * Hq;
+    prefill_job *jobs = (prefill_job *)calloc((size_t)nthreads, sizeof(prefill_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) { free(jobs); free(th); return ORACLE_NO_MEMORY; }
+    for (int i = 0; i < nthreads; ++i) {
+        prefill_job J = {q, k, v, B, S, Hq, Hkv, d, scale, rows, nrows, out, i, nthreads, ORACLE_OK};
+        jobs[i] = J;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, prefill_worker, &jobs[i]);
+    prefill_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    int st = ORACLE_OK;
+    for (int i = 0; i < nthreads; ++i) if (jobs[i].status != ORACLE_OK) st = jobs[i].status;
+    free(jobs); free(th);
+    return st;
+}

@@ -1,0 +1,314 @@
+"""Pins for the fp64 oracle: each check ties it to something other than itself.
+
+* golden values printed on the pages (tests/golden/, each line cited);
+* closed forms (the two-query example, one cached token, a zero query);
+* library routines for special cases (torch scaled_dot_product_attention in
+  fp64 for the MHA endpoint and for causal prefill, torch's own bf16 -> fp64
+  conversion, torch.repeat_interleave for the expanded form);
+* a grouped, copy-free restatement (queries of a group as extra rows against
+  one shared KV head) that must agree with the oracle's explicit repeat;
+* brute force in plain Python on tiny shapes with distinct per-head inputs;
+* invariants (swapping two KV heads together with their query groups swaps
+  the outputs group by group).
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from grouped_query_attention_02_b200 import inputs
+from tests._tolerance import compare
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for ln in f:
+            ln = ln.strip()
+            if ln and not ln.startswith("#"):
+                yield ln
+
+
+# ---------------------------------------------------------------- mapping
+
+
+def test_mapping_matches_pages(oracle_mod):
+    n = 0
+    for ln in _lines("mapping.txt"):
+        head, rest = ln.split(":")
+        Hq, Hkv = map(int, head.split())
+        expect = [int(x) for x in rest.split()[:Hq]]
+        assert [oracle_mod.kv_head(h, Hq, Hkv) for h in range(Hq)] == expect
+        n += 1
+    assert n == 2
+
+
+def test_mapping_endpoints_and_irregular(oracle_mod):
+    assert [oracle_mod.kv_head(h, 12, 12) for h in range(12)] == list(range(12))  # MHA
+    assert [oracle_mod.kv_head(h, 71, 1) for h in range(71)] == [0] * 71          # MQA, 71 heads
+    assert oracle_mod.kv_head(0, 6, 4) == -1      # 6 query heads cannot split into 4 groups
+    assert oracle_mod.kv_head(8, 8, 2) == -1      # out of range
+    assert oracle_mod.kv_head(-1, 8, 2) == -1
+
+
+# ---------------------------------------------------------------- byte model
+
+
+def test_kv_bytes_match_pages(oracle_mod):
+    n = 0
+    for ln in _lines("kv_bytes.txt"):
+        f = ln.split()
+        L, T, H, d, b, expect = (int(x) for x in f[:6])
+        assert oracle_mod.kv_bytes(L, T, H, d, b) == expect, ln
+        n += 1
+    assert n == 9
+
+
+def test_kv_bytes_ratios(oracle_mod):
+    # two-head GQA stores a quarter of eight-head MHA's raw cache; query heads never enter
+    assert 4 * oracle_mod.kv_bytes(32, 4096, 2, 128, 2) == oracle_mod.kv_bytes(32, 4096, 8, 128, 2)
+    # an 8k-token request of the 36-layer, 8-KV-head config: 1.125 GiB (the page rounds to 1.13)
+    assert oracle_mod.kv_bytes(36, 8192, 8, 128, 2) == 1.125 * 2 ** 30
+    assert oracle_mod.kv_bytes(32, 1, 32, 128, 2) == 4 * oracle_mod.kv_bytes(32, 1, 8, 128, 2) == 512 * 1024
+
+
+def test_capacity_exercise(oracle_mod):
+    for ln in _lines("capacity.txt"):
+        L, H, d, w, expect = ln.split()
+        free = (80 - float(w) - 4) * 2 ** 30
+        per_request = oracle_mod.kv_bytes(int(L), 4096, int(H), int(d), 2)
+        assert int(free // per_request) == int(expect)
+
+
+# ---------------------------------------------------------------- bf16
+
+
+def test_bf16_conversion_exhaustive(oracle_mod):
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ours = oracle_mod.bf16_bits_to_f64(bits)
+    ref = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], ref[~nan])
+
+
+# ---------------------------------------------------------------- closed forms
+
+
+def _bf(x):
+    return torch.tensor(x, dtype=torch.float64).to(torch.bfloat16)
+
+
+def test_two_query_example(oracle_mod):
+    keys, values, queries = [], [], []
+    for ln in _lines("two_query.txt"):
+        f = ln.split()
+        {"key": keys, "value": values, "query": queries}[f[0]].append([float(x) for x in f[1:]])
+    d = 2
+    q = _bf([queries])                       # [1, 2 heads, 2]
+    k = _bf([[[kk] for kk in keys]])         # [1, T=2, 1 kv head, 2]
+    v = _bf([[[vv] for vv in values]])
+    out = oracle_mod.decode(q, k, v, [2], 1.0 / math.sqrt(d))
+    a, b = out[0, 0, 0], out[0, 1, 0]
+    c = math.exp(-1.0 / math.sqrt(2.0))
+    assert a == pytest.approx((10 + 20 * c) / (1 + c), rel=1e-14)
+    assert b == pytest.approx((10 * c + 20) / (1 + c), rel=1e-14)
+    assert (round(a, 6), round(b, 6)) == (13.302385, 16.697615)
+    assert not math.isclose(a, b)            # shared K/V, distinct queries, distinct outputs
+    assert a + b == pytest.approx(30.0, rel=1e-14)   # mirror symmetry of the example
+    assert out[0, 0, 1] == 0.0 and out[0, 1, 1] == 0.0
+
+
+def test_single_cached_token_returns_its_value_row(oracle_mod):
+    x = inputs.make_decode(2, 8, 2, 16, 5, seqlens=[1, 1], seed=11)
+    out = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    v = x.v_cache.double().numpy()
+    for h in range(8):
+        for b in range(2):
+            assert np.array_equal(out[b, h], v[b, 0, h // 4])
+
+
+def test_zero_query_averages_values(oracle_mod):
+    x = inputs.make_decode(2, 6, 2, 16, 7, seqlens=[7, 3], seed=5)
+    q0 = torch.zeros_like(x.q)
+    out = oracle_mod.decode(q0, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    v = x.v_cache.double().numpy()
+    for b, T in enumerate([7, 3]):
+        for h in range(6):
+            np.testing.assert_allclose(out[b, h], v[b, :T, h // 3].mean(axis=0), rtol=0, atol=1e-14)
+
+
+def test_empty_history_gives_zero(oracle_mod):
+    x = inputs.make_decode(2, 4, 2, 16, 4, seqlens=[0, 4], seed=2)
+    out = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    assert np.all(out[0] == 0.0)
+    assert np.any(out[1] != 0.0)
+
+
+def test_rejects_irregular_or_bad_lengths(oracle_mod):
+    x = inputs.make_decode(1, 6, 2, 16, 4, seed=1)
+    with pytest.raises(ValueError):
+        oracle_mod.decode(x.q, x.k_cache[:, :, :1].expand(1, 4, 4, 16).contiguous(), x.v_cache[:, :, :1]
+                          .expand(1, 4, 4, 16).contiguous(), x.seqlens, x.scale)
+    with pytest.raises(ValueError):
+        oracle_mod.decode(x.q, x.k_cache, x.v_cache, [5], x.scale)
+
+
+# ---------------------------------------------------------------- library routines
+
+
+def _sdpa(q, k, v, scale, causal=False):
+    return torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=scale, is_causal=causal)
+
+
+def test_mha_endpoint_equals_library_sdpa(oracle_mod):
+    x = inputs.make_decode(2, 4, 4, 16, 9, seqlens=[9, 5], seed=21)
+    out = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    for b, T in enumerate([9, 5]):
+        q = x.q[b].double()[:, None, :]                     # [H,1,d]
+        k = x.k_cache[b, :T].double().transpose(0, 1)       # [H,T,d]
+        v = x.v_cache[b, :T].double().transpose(0, 1)
+        ref = _sdpa(q, k, v, x.scale)[:, 0, :].numpy()
+        np.testing.assert_allclose(out[b], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_mqa_endpoint_equals_library_sdpa(oracle_mod):
+    x = inputs.make_decode(2, 6, 1, 16, 8, seqlens=[8, 2], seed=22)
+    out = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    for b, T in enumerate([8, 2]):
+        q = x.q[b].double()[:, None, :]
+        k = x.k_cache[b, :T, 0].double()[None].expand(6, T, 16)
+        v = x.v_cache[b, :T, 0].double()[None].expand(6, T, 16)
+        np.testing.assert_allclose(out[b], _sdpa(q, k, v, x.scale)[:, 0, :].numpy(), rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_mha_equals_library_causal_sdpa(oracle_mod):
+    x = inputs.make_prefill(2, 9, 4, 4, 16, seed=23)
+    out = oracle_mod.prefill_causal(x.q, x.k, x.v, x.scale)
+    ref = _sdpa(x.q.double().transpose(1, 2), x.k.double().transpose(1, 2), x.v.double().transpose(1, 2),
+                x.scale, causal=True).transpose(1, 2).numpy()
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_grouped_equals_expanded_tiny(oracle_mod):
+    """The page's equivalence case: B=2, T=9, 12 query heads, 3 KV heads, d=16, causal."""
+    B, T, Hq, Hkv, d = 2, 9, 12, 3, 16
+    rep = Hq // Hkv
+    x = inputs.make_prefill(B, T, Hq, Hkv, d, seed=24)
+    gqa = oracle_mod.prefill_causal(x.q, x.k, x.v, x.scale)
+    # expanded: physically repeat K/V along the head axis with the library routine, then MHA
+    k_rep = x.k.repeat_interleave(rep, dim=2).contiguous()
+    v_rep = x.v.repeat_interleave(rep, dim=2).contiguous()
+    mha = oracle_mod.prefill_causal(x.q, k_rep, v_rep, x.scale)
+    np.testing.assert_array_equal(gqa, mha)
+    # grouped without copies: a group's rep query heads become rep*T extra rows against one KV head
+    q = x.q.double()                     # [B,T,Hq,d]
+    k = x.k.double()
+    v = x.v.double()
+    causal = torch.ones(T, T, dtype=torch.bool).tril()
+    for j in range(Hkv):
+        qg = q[:, :, j * rep:(j + 1) * rep, :].permute(0, 2, 1, 3).reshape(B, rep * T, d)
+        s = (qg @ k[:, :, j, :].transpose(1, 2)) * x.scale             # [B, rep*T, T]
+        s = s.view(B, rep, T, T).masked_fill(~causal, float("-inf"))
+        o = torch.softmax(s, dim=-1).reshape(B, rep * T, T) @ v[:, :, j, :]
+        o = o.view(B, rep, T, d).permute(0, 2, 1, 3).numpy()
+        np.testing.assert_allclose(gqa[:, :, j * rep:(j + 1) * rep, :], o, rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_row_subset_matches_full(oracle_mod):
+    x = inputs.make_prefill(2, 11, 6, 2, 16, seed=25)
+    full = oracle_mod.prefill_causal(x.q, x.k, x.v, x.scale)
+    rows = [(1, 5, 10), (0, 0, 0), (1, 2, 3), (0, 5, 7), (1, 5, 0)]
+    sub = oracle_mod.prefill_causal(x.q, x.k, x.v, x.scale, rows=rows)
+    for i, (b, h, r) in enumerate(rows):
+        np.testing.assert_array_equal(sub[i], full[b, r, h])
+
+
+# ---------------------------------------------------------------- brute force
+
+
+def _brute_decode(q, k, v, seqlens, scale):
+    """Plain-Python loops over flat lists; mapping written as integer division."""
+    B, Hq, d = len(q), len(q[0]), len(q[0][0])
+    Hkv = len(k[0][0])
+    out = [[[0.0] * d for _ in range(Hq)] for _ in range(B)]
+    for b in range(B):
+        for h in range(Hq):
+            kv = h * Hkv // Hq
+            T = seqlens[b]
+            if T == 0:
+                continue
+            s = [scale * sum(q[b][h][j] * k[b][t][kv][j] for j in range(d)) for t in range(T)]
+            w = [math.exp(x) for x in s]        # inputs are small: no max shift needed
+            z = math.fsum(w)
+            for j in range(d):
+                out[b][h][j] = math.fsum(w[t] * v[b][t][kv][j] for t in range(T)) / z
+    return out
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(1, 1), (4, 1), (6, 2), (8, 2), (12, 3), (71, 1)])
+@pytest.mark.parametrize("d", [2, 16])
+def test_brute_force_decode(oracle_mod, Hq, Hkv, d):
+    seqlens = [9, 1, 3, 2, 0]
+    x = inputs.make_decode(5, Hq, Hkv, d, 9, seqlens=seqlens, seed=100 + Hq + d)
+    got = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    ref = _brute_decode(x.q.double().tolist(), x.k_cache.double().tolist(), x.v_cache.double().tolist(),
+                        seqlens, x.scale)
+    np.testing.assert_allclose(got, np.array(ref), rtol=1e-12, atol=1e-13)
+
+
+def test_brute_force_prefill(oracle_mod):
+    B, S, Hq, Hkv, d = 2, 5, 6, 2, 4
+    x = inputs.make_prefill(B, S, Hq, Hkv, d, seed=31)
+    got = oracle_mod.prefill_causal(x.q, x.k, x.v, x.scale)
+    q, k, v = x.q.double().tolist(), x.k.double().tolist(), x.v.double().tolist()
+    for b in range(B):
+        for r in range(S):
+            for h in range(Hq):
+                kv = h // (Hq // Hkv)
+                w = [math.exp(x.scale * sum(q[b][r][h][j] * k[b][t][kv][j] for j in range(d)))
+                     for t in range(r + 1)]
+                z = math.fsum(w)
+                for j in range(d):
+                    ref = math.fsum(w[t] * v[b][t][kv][j] for t in range(r + 1)) / z
+                    assert got[b, r, h, j] == pytest.approx(ref, rel=1e-12, abs=1e-13)
+
+
+# ---------------------------------------------------------------- invariants
+
+
+def test_swapping_kv_heads_with_their_groups_swaps_outputs(oracle_mod):
+    B, Hq, Hkv, d, T = 2, 8, 2, 16, 6
+    x = inputs.make_decode(B, Hq, Hkv, d, T, seed=41)
+    base = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    g = Hq // Hkv
+    perm_kv = [1, 0]
+    perm_q = [perm_kv[h // g] * g + h % g for h in range(Hq)]
+    out = oracle_mod.decode(x.q[:, perm_q].contiguous(), x.k_cache[:, :, perm_kv].contiguous(),
+                            x.v_cache[:, :, perm_kv].contiguous(), x.seqlens, x.scale)
+    np.testing.assert_array_equal(out, base[:, perm_q])
+    # swapping only the KV heads must change the outputs (the mapping is not symmetric)
+    out2 = oracle_mod.decode(x.q, x.k_cache[:, :, perm_kv].contiguous(), x.v_cache[:, :, perm_kv].contiguous(),
+                             x.seqlens, x.scale)
+    assert not np.allclose(out2, base)
+
+
+def test_distinct_queries_in_a_group_give_distinct_outputs(oracle_mod):
+    x = inputs.make_decode(1, 8, 2, 16, 32, seed=42)
+    out = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    for h in range(1, 4):
+        assert not np.allclose(out[0, 0], out[0, h])
+
+
+def test_tight_tolerance_sees_one_dropped_token(oracle_mod):
+    """At the tiny decode shape, an off-by-one in the cached length breaks the tight gate."""
+    x = inputs.make_decode(1, 8, 2, 128, 256, seed=0)
+    full = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    short = oracle_mod.decode(x.q, x.k_cache, x.v_cache, [255], x.scale)
+    assert compare(short, full)["tight_violations"] > 0
+    assert compare(full, full)["tight_violations"] == 0
