@@ -1,0 +1,469 @@
+"""Benchmark: GQA decode on one B200 (or N independent GPUs), through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--rows all|none]
+
+One step is one decode step (split-KV kernel + combine) over the Qwen3-8B-shaped
+workload: 49 sequences, 32 query heads / 8 KV heads, d=128, 8192 cached tokens
+each, bf16 N(0,1) synthetic inputs already resident in HBM.  The cache
+(1.64 GB) is larger than the 126 MB L2, so no flush is needed between steps.
+The headline value is unique-KV bytes (2 * sum(T) * Hkv * d * 2) per second;
+tokens/s (sequences decoded per second, one layer) rides along.
+
+The JSON line also carries the other hot-path rows measured the same way
+(tiny decode, variable-length sweep, extreme grouping, the expanded repeat-KV
+baseline, causal prefill), the roofline of the dominant kernel, the clocks
+seen during the timed region, an end-to-end figure with host buffers, and the
+fp64 CPU oracle timed on a bounded sample of the same workload.
+
+With N > 1 (torchrun), every rank decodes its own 49 sequences (its shard of
+a 49*N batch; weak scaling, no collective on the data path); the step time is
+the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+PROFILES = os.path.join(ROOT, "profiles")
+METRIC = "GQA decode unique-KV HBM GB/s (% of B200 peak) and decode tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- host helpers (no GPU needed)
+
+def unique_kv_bytes(seqlens, Hkv: int, d: int) -> int:
+    """K and V rows actually cached: 2 * sum(T) * Hkv * d * 2 bytes (bf16)."""
+    return 2 * int(sum(int(t) for t in seqlens)) * Hkv * d * 2
+
+
+def decode_flops(seqlens, Hq: int, d: int) -> int:
+    """4 * Hq * d per cached token: q.k and p.v, independent of Hkv."""
+    return 4 * int(sum(int(t) for t in seqlens)) * Hq * d
+
+
+def prefill_causal_flops(B: int, S: int, Hq: int, d: int) -> int:
+    """4 * d per unmasked (query, key) pair per head; row r sees r + 1 keys."""
+    return 4 * d * B * Hq * S * (S + 1) // 2
+
+
+def rank_seed(rank: int, base: int = 0) -> int:
+    return base + 1000 * rank
+
+
+def shard_of(rank: int, world: int, per_rank: int):
+    """Global sequence indices owned by `rank` when each rank decodes per_rank sequences."""
+    return list(range(rank * per_rank, (rank + 1) * per_rank))
+
+
+def aggregate(values_per_rank, times_per_rank):
+    """Whole-job throughput: all units over the slowest rank's time."""
+    t = max(times_per_rank)
+    return sum(values_per_rank) / t, t
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    for f in ("decode.cu", "prefill.cu", "ptx.cuh", "internal.h", "api.cu"):
+        p = os.path.join(ROOT, "grouped_query_attention_02_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(name: str):
+    """dram read+write bytes per launch from a committed ncu summary, if it matches the current kernels."""
+    p = os.path.join(PROFILES, name)
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("kernel_source_digest") != kernel_source_digest():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU measurement
+
+def _events(torch):
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def time_decode(gqa, torch, x, steps: int, warmup: int, expanded=None):
+    """Mean step time and mean split-kernel time (ms) over `steps` timed decode steps."""
+    out = torch.empty_like(x.q)
+    call = (lambda: gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out)) if expanded is None else \
+        (lambda: gqa.gqa_decode_expanded(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out,
+                                         k_rep=expanded[0], v_rep=expanded[1]))
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    kev = [_events(torch) for _ in range(steps)]
+    s0, s1 = _events(torch)
+    launches = 0
+    s0.record()
+    for i in range(steps):
+        gqa.gqa_set_profile_events(*kev[i])
+        call()
+        launches += gqa.gqa_last_launch_count()
+    s1.record()
+    gqa.gqa_set_profile_events(None, None)
+    torch.cuda.synchronize()
+    step_ms = s0.elapsed_time(s1) / steps
+    kern_ms = sum(a.elapsed_time(b) for a, b in kev) / steps
+    return step_ms, kern_ms, launches, out
+
+
+def time_prefill(gqa, torch, p, steps: int, warmup: int):
+    out = torch.empty_like(p.q)
+    for _ in range(warmup):
+        gqa.gqa_prefill_causal(p.q, p.k, p.v, out=out)
+    torch.cuda.synchronize()
+    kev = [_events(torch) for _ in range(steps)]
+    s0, s1 = _events(torch)
+    launches = 0
+    s0.record()
+    for i in range(steps):
+        gqa.gqa_set_profile_events(*kev[i])
+        gqa.gqa_prefill_causal(p.q, p.k, p.v, out=out)
+        launches += gqa.gqa_last_launch_count()
+    s1.record()
+    gqa.gqa_set_profile_events(None, None)
+    torch.cuda.synchronize()
+    return s0.elapsed_time(s1) / steps, sum(a.elapsed_time(b) for a, b in kev) / steps, launches
+
+
+def time_e2e(gqa, torch, x, steps: int):
+    """Host buffers in, host result out: pinned H2D of q, K, V, seqlens + decode + D2H of out, per step."""
+    hq = x.q.cpu().pin_memory()
+    hk = x.k_cache.cpu().pin_memory()
+    hv = x.v_cache.cpu().pin_memory()
+    hs = x.seqlens.cpu().pin_memory()
+    hout = torch.empty(x.q.shape, dtype=torch.bfloat16).pin_memory()
+    dq, dk, dv, ds = (torch.empty_like(t, device="cuda") for t in (hq, hk, hv, hs))
+    dout = torch.empty_like(dq)
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        ds.copy_(hs, non_blocking=True)
+        gqa.gqa_decode(dq, dk, dv, ds, x.scale, out=dout)
+        hout.copy_(dout, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    s0, s1 = _events(torch)
+    s0.record()
+    for _ in range(steps):
+        step()
+    s1.record()
+    torch.cuda.synchronize()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs))
+    d2h = hout.numel() * hout.element_size()
+    ok = torch.equal(hout, dout.cpu())
+    del dq, dk, dv, ds, dout
+    return s0.elapsed_time(s1) / steps, h2d, d2h, ok
+
+
+def cpu_oracle_sample(x, target_s: float = 12.0, max_seqs: int | None = None):
+    """Time the fp64 oracle on the first n sequences of the workload (all heads), n sized to ~target_s."""
+    import oracle
+
+    sl = x.seqlens.cpu().tolist()
+    Hkv, d = x.k_cache.shape[2], x.k_cache.shape[3]
+    B = len(sl)
+    cores = oracle.default_threads()
+
+    def run(n):
+        T = max(1, max(sl[:n]))
+        kk = x.k_cache[:n, :T].cpu()
+        vv = x.v_cache[:n, :T].cpu()
+        t0 = time.perf_counter()
+        oracle.decode(x.q[:n].cpu(), kk, vv, sl[:n], x.scale, nthreads=cores)
+        return time.perf_counter() - t0
+
+    t1 = run(1)
+    n = max(1, min(B if max_seqs is None else max_seqs, int(target_s / max(t1, 1e-3))))
+    tn = run(n) if n > 1 else t1
+    ub = unique_kv_bytes(sl[:n], Hkv, d)
+    return {"value": ub / tn / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n} of {B} sequences, every query head, {sum(sl[:n])} cached tokens; "
+                      f"{tn:.2f} s wall on {cores} threads",
+            "seconds": tn, "tokens_per_s": n / tn}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--rows", choices=["all", "none"], default="all")
+    ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the host-buffer measurement")
+    ap.add_argument("--cpu-baseline", choices=["on", "off"], default="on")
+    args = ap.parse_args()
+
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        print(f"--gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+
+    from grouped_query_attention_02_b200 import inputs, workloads
+
+    w = workloads.QWEN3_8B_DECODE
+    base_cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.Tmax,
+                "global_batch": w.B * max(world, 1), "parallelism": f"dp{max(world, 1)} (batch-sharded, no collective)",
+                "l2": "inputs larger than L2 (1.64 GB cache vs 126 MB); no flush"}
+
+    if args.impl == "reference":
+        # the reference arm is the fp64 CPU oracle, on rank 0 only
+        if rank != 0:
+            return
+        import oracle
+
+        # inputs on the host: one sequence per step keeps a step to a few seconds
+        xs = inputs.make_decode(2, w.Hq, w.Hkv, w.d, w.Tmax, device="cpu", seed=0)
+        cores = oracle.default_threads()
+        times = []
+        for i in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            oracle.decode(xs.q[:1], xs.k_cache[:1], xs.v_cache[:1], xs.seqlens[:1], xs.scale, nthreads=cores)
+            dt = time.perf_counter() - t0
+            if i >= args.warmup:
+                times.append(dt)
+        t = sum(times) / len(times)
+        ub = unique_kv_bytes([w.Tmax], w.Hkv, w.d)
+        val = ub / t / 1e9
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": base_cfg,
+                "cpu_baseline": {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                                 "sample": f"one of {w.B} sequences per step (all {w.Hq} query heads, "
+                                           f"{w.Tmax} cached tokens)"},
+                "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import grouped_query_attention_02_b200 as gqa
+
+    gqa.load()
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+
+    peaks = load_peaks()
+    x = inputs.make_decode(w.B, w.Hq, w.Hkv, w.d, w.Tmax, device="cuda", seed=rank_seed(rank))
+    sl = x.seqlens.cpu().tolist()
+    U = unique_kv_bytes(sl, w.Hkv, w.d)
+    alg_bytes = U + 2 * x.q.numel() * 2   # cache + q in + out
+
+    # warm-up + barrier, then the timed steps bracketed by barrier + synchronize
+    out = torch.empty_like(x.q)
+    for _ in range(args.warmup):
+        gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    kev = [_events(torch) for _ in range(args.steps)]
+    s0, s1 = _events(torch)
+    launches = 0
+    with ClockSampler(local_rank) as clk:
+        time.sleep(0.25)
+        s0.record()
+        for i in range(args.steps):
+            gqa.gqa_set_profile_events(*kev[i])
+            gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out)
+            launches += gqa.gqa_last_launch_count()
+        s1.record()
+        torch.cuda.synchronize()
+    gqa.gqa_set_profile_events(None, None)
+    if dist:
+        dist.barrier()
+    step_ms = s0.elapsed_time(s1) / args.steps
+    kern_ms = sum(a.elapsed_time(b) for a, b in kev) / args.steps
+    if dist:
+        t = torch.tensor([step_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms_max = float(t.item())
+    else:
+        step_ms_max = step_ms
+    status = gqa.gqa_get_last_device_status()
+    value = U * max(world, 1) / (step_ms_max * 1e-3) / 1e9
+    tokens_per_s = w.B * max(world, 1) / (step_ms_max * 1e-3)
+
+    # ---- end to end through the public API with host buffers (every rank; slowest rank counts)
+    e2e_err = None
+    if args.e2e_steps > 0:
+        try:
+            e2e_ms, h2d, d2h, ok = time_e2e(gqa, torch, x, args.e2e_steps)
+        except RuntimeError as e:  # pinned memory exhausted, etc.
+            e2e_ms, h2d, d2h, ok, e2e_err = float("nan"), 0, 0, False, str(e)[:200]
+    else:
+        e2e_ms, h2d, d2h, ok, e2e_err = float("nan"), 0, 0, False, "skipped (--e2e-steps 0)"
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank != 0:
+        if dist:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    achieved = alg_bytes / (kern_ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": max(world, 1), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "accumulate": "fp32", "data": "synthetic", "config": base_cfg,
+        "tokens_per_s": tokens_per_s, "frac_of_hbm_peak_step": value / max(world, 1) / peaks["hbm_gbs"],
+        "gpu_launches": launches, "device_status": status,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": profile_traffic("decode_split_qwen3_8b.json"),
+                     "kernel": "decode_split_kernel<4>", "kernel_ms": kern_ms, "algorithmic_bytes": alg_bytes,
+                     "peak_source": f"{peaks.get('source')} hbm_gbs (copy bandwidth)"},
+        "clocks": clk.summary(),
+    }
+
+    line["e2e"] = {"value": (U * max(world, 1) / (e2e_ms * 1e-3) / 1e9) if e2e_err is None else None,
+                   "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                   "result_matches_device": ok}
+    if e2e_err:
+        line["e2e"]["error"] = e2e_err
+
+    # ---- the other rows of the hot path
+    if args.rows == "all" and max(world, 1) == 1:
+        rows = {}
+        del out
+        for ww in (workloads.TINY_DECODE,) + workloads.VARLEN_DECODE + (workloads.EXTREME_GROUP_DECODE,):
+            xx = inputs.make_decode(ww.B, ww.Hq, ww.Hkv, ww.d, ww.Tmax, device="cuda", seed=0,
+                                    seqlen_range=ww.seqlen_range)
+            sll = xx.seqlens.cpu().tolist()
+            uu = unique_kv_bytes(sll, ww.Hkv, ww.d)
+            st_ms, k_ms, n, _ = time_decode(gqa, torch, xx, 10 if ww.B * ww.Tmax > 1e5 else 50, 3)
+            rows[ww.name] = {"ms_per_step": st_ms, "kernel_ms": k_ms, "unique_kv_GBps": uu / (st_ms * 1e-3) / 1e9,
+                             "frac_hbm": uu / (st_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                             "tokens_per_s": ww.B / (st_ms * 1e-3), "launches_per_step": n / (10 if ww.B * ww.Tmax > 1e5 else 50)}
+            del xx
+            torch.cuda.empty_cache()
+        # expanded repeat-KV baseline on the headline workload
+        k_rep = torch.empty((w.B, w.Tmax, w.Hq, w.d), dtype=torch.bfloat16, device="cuda")
+        v_rep = torch.empty_like(k_rep)
+        st_ms, k_ms, n, _ = time_decode(gqa, torch, x, 5, 2, expanded=(k_rep, v_rep))
+        rows["expanded repeat-KV baseline, " + w.name] = {
+            "ms_per_step": st_ms, "unique_kv_GBps": U / (st_ms * 1e-3) / 1e9,
+            "bytes_moved_per_step": U + 2 * U * w.group + U * w.group,
+            "slowdown_vs_grouped": st_ms / step_ms}
+        del k_rep, v_rep
+        torch.cuda.empty_cache()
+        # causal prefill
+        pw = workloads.CAUSAL_PREFILL
+        try:
+            p = inputs.make_prefill(pw.B, pw.S, pw.Hq, pw.Hkv, pw.d, device="cuda", seed=0)
+            st_ms, k_ms, n = time_prefill(gqa, torch, p, 10, 3)
+            fl = prefill_causal_flops(pw.B, pw.S, pw.Hq, pw.d)
+            rows[pw.name] = {"ms_per_step": st_ms, "kernel_ms": k_ms, "TFLOPs": fl / (st_ms * 1e-3) / 1e12,
+                             "frac_bf16_peak": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                             "peak_tflops": peaks["bf16_tflops"]}
+        except gqa.GQAError as e:
+            rows[pw.name] = {"error": str(e)}
+        line["rows"] = rows
+
+    # ---- the fp64 oracle on a bounded sample, host cores of this machine
+    if max(world, 1) == 1 and args.cpu_baseline == "on":
+        line["cpu_baseline"] = cpu_oracle_sample(x)
+
+    print(json.dumps(line))
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,1 +1,231 @@
-"""B200-native grouped-query attention: decode and causal prefill behind a C ABI."""
+"""B200-native grouped-query attention: decode and causal prefill behind a C ABI.
+
+This module is the thin Python binding of ``libgqa.so`` (``include/gqa.h``):
+it checks tensor dtypes/shapes/devices, passes raw pointers, sizes and the
+current CUDA stream through ctypes, and turns status codes into exceptions.
+Every step of the computation runs in the library's CUDA kernels; there is no
+fallback.  If the library is missing the first call raises ``RuntimeError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "GQAError", "gqa_decode", "gqa_prefill_causal", "gqa_decode_expanded", "gqa_decode_expanded_bytes",
+    "gqa_decode_plan", "gqa_get_last_device_status", "gqa_selftest_wait_timeout", "gqa_set_profile_events",
+    "gqa_last_launch_count", "gqa_release", "gqa_status_string", "gqa_version", "library_path", "load",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libgqa.so")
+_lib = None
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+
+EXPORTS = {
+    # name: (restype, argtypes)
+    "gqa_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp]),
+    "gqa_prefill_causal": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
+    "gqa_decode_expanded": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp]),
+    "gqa_decode_expanded_bytes": (ctypes.c_size_t, [_i, _i, _i, _i]),
+    "gqa_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
+                             ctypes.POINTER(ctypes.c_size_t)]),
+    "gqa_get_last_device_status": (_i, [_vp]),
+    "gqa_selftest_wait_timeout": (_i, [_i, _vp]),
+    "gqa_set_profile_events": (_i, [_vp, _vp]),
+    "gqa_last_launch_count": (_i, []),
+    "gqa_release": (None, []),
+    "gqa_status_string": (ctypes.c_char_p, [_i]),
+    "gqa_version": (ctypes.c_char_p, []),
+}
+
+
+class GQAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_text(status)} (status {status})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """Load libgqa.so (built in-tree by ``python -m grouped_query_attention_02_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libgqa.so is not built ({_LIB_PATH}); run "
+                               "`python -m grouped_query_attention_02_b200.build` -- there is no fallback path")
+        lib = ctypes.CDLL(_LIB_PATH)
+        for name, (res, args) in EXPORTS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_text(status: int) -> str:
+    return load().gqa_status_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise GQAError(status, where)
+
+
+def _stream_ptr(stream):
+    import torch
+
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype, ndim, device=None):
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def gqa_decode(q, k_cache, v_cache, seqlens, scale=None, out=None, stream=None):
+    """q [B,Hq,d], k_cache/v_cache [B,Tmax,Hkv,d] bf16, seqlens [B] int32 (device) -> out [B,Hq,d] bf16."""
+    import torch
+
+    _need(q, "q", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    _need(k_cache, "k_cache", torch.bfloat16, 4, q.device)
+    _need(v_cache, "v_cache", torch.bfloat16, 4, q.device)
+    _need(seqlens, "seqlens", torch.int32, 1, q.device)
+    Bk, Tmax, Hkv, dk = k_cache.shape
+    if (Bk, dk) != (B, d) or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, k_cache, v_cache and seqlens")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out", torch.bfloat16, 3, q.device)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    if scale is None:
+        scale = 1.0 / d ** 0.5
+    st = load().gqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(), B, Hq, Hkv, d,
+                           Tmax, float(scale), out.data_ptr(), _stream_ptr(stream))
+    _check(st, "gqa_decode")
+    return out
+
+
+def gqa_decode_expanded(q, k_cache, v_cache, seqlens, scale=None, out=None, k_rep=None, v_rep=None, stream=None):
+    """The repeat-KV baseline: same result as gqa_decode, K/V copied g times first."""
+    import torch
+
+    _need(q, "q", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    _need(k_cache, "k_cache", torch.bfloat16, 4, q.device)
+    _need(v_cache, "v_cache", torch.bfloat16, 4, q.device)
+    _need(seqlens, "seqlens", torch.int32, 1, q.device)
+    Bk, Tmax, Hkv, dk = k_cache.shape
+    if (Bk, dk) != (B, d) or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, k_cache, v_cache and seqlens")
+    if out is None:
+        out = torch.empty_like(q)
+    rep_shape = (B, Tmax, Hq, d)
+    if k_rep is None:
+        k_rep = torch.empty(rep_shape, dtype=torch.bfloat16, device=q.device)
+    if v_rep is None:
+        v_rep = torch.empty(rep_shape, dtype=torch.bfloat16, device=q.device)
+    for t, n in ((out, "out"), (k_rep, "k_rep"), (v_rep, "v_rep")):
+        _need(t, n, torch.bfloat16, t.dim(), q.device)
+    if tuple(k_rep.shape) != rep_shape or tuple(v_rep.shape) != rep_shape:
+        raise ValueError(f"k_rep/v_rep must have shape {rep_shape}")
+    if scale is None:
+        scale = 1.0 / d ** 0.5
+    st = load().gqa_decode_expanded(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(), B, Hq,
+                                    Hkv, d, Tmax, float(scale), out.data_ptr(), k_rep.data_ptr(), v_rep.data_ptr(),
+                                    _stream_ptr(stream))
+    _check(st, "gqa_decode_expanded")
+    return out
+
+
+def gqa_prefill_causal(q, k, v, out=None, stream=None):
+    """q [B,S,Hq,d], k/v [B,S,Hkv,d] bf16 -> out [B,S,Hq,d] bf16 (causal, scale 1/sqrt(d))."""
+    import torch
+
+    _need(q, "q", torch.bfloat16, 4)
+    B, S, Hq, d = q.shape
+    _need(k, "k", torch.bfloat16, 4, q.device)
+    _need(v, "v", torch.bfloat16, 4, q.device)
+    Bk, Sk, Hkv, dk = k.shape
+    if (Bk, Sk, dk) != (B, S, d) or v.shape != k.shape:
+        raise ValueError("shape mismatch between q, k and v")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out", torch.bfloat16, 4, q.device)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    st = load().gqa_prefill_causal(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, S, Hq, Hkv, d, out.data_ptr(),
+                                   _stream_ptr(stream))
+    _check(st, "gqa_prefill_causal")
+    return out
+
+
+def gqa_decode_expanded_bytes(B, Tmax, Hq, d):
+    return int(load().gqa_decode_expanded_bytes(B, Tmax, Hq, d))
+
+
+def gqa_decode_plan(B, Hq, Hkv, d, Tmax, num_sms):
+    """(chunk, nsplit, workspace_bytes) gqa_decode uses on a device with num_sms SMs."""
+    c, n, w = _i(), _i(), ctypes.c_size_t()
+    _check(load().gqa_decode_plan(B, Hq, Hkv, d, Tmax, num_sms, ctypes.byref(c), ctypes.byref(n), ctypes.byref(w)),
+           "gqa_decode_plan")
+    return c.value, n.value, w.value
+
+
+def gqa_get_last_device_status(stream=None) -> int:
+    return int(load().gqa_get_last_device_status(_stream_ptr(stream)))
+
+
+def gqa_selftest_wait_timeout(timeout_us: int, stream=None):
+    _check(load().gqa_selftest_wait_timeout(int(timeout_us), _stream_ptr(stream)), "gqa_selftest_wait_timeout")
+
+
+def gqa_set_profile_events(before=None, after=None):
+    """before/after: torch.cuda.Event(enable_timing=True) or None (turns the hook off)."""
+    for ev in (before, after):
+        if ev is not None and not ev.cuda_event:
+            ev.record()          # torch creates the underlying cudaEvent_t lazily, on first record
+    b = None if before is None else ctypes.c_void_p(before.cuda_event)
+    a = None if after is None else ctypes.c_void_p(after.cuda_event)
+    _check(load().gqa_set_profile_events(b, a), "gqa_set_profile_events")
+
+
+def gqa_last_launch_count() -> int:
+    return int(load().gqa_last_launch_count())
+
+
+def gqa_release():
+    load().gqa_release()
+
+
+def gqa_status_string(status: int) -> str:
+    return status_text(status)
+
+
+def gqa_version() -> str:
+    return load().gqa_version().decode()

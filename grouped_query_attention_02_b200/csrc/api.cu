@@ -1,0 +1,325 @@
+// api.cu -- the C ABI of libgqa.so (declared in include/gqa.h): argument
+// checks, split planning, TMA tensor maps, the per-device workspace and the
+// launches.  Everything here is host code except the device status word.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <mutex>
+#include <unordered_map>
+
+#include "../../include/gqa.h"
+#include "internal.h"
+
+namespace {
+
+using namespace gqa;
+
+__device__ int g_status_word;  // first error a kernel recorded (0 = none)
+static_assert(kStatusTimeout == GQA_ERR_DEVICE_TIMEOUT, "device and host timeout codes differ");
+
+constexpr unsigned long long kWaitBudgetNs = 1000000000ull;  // a bounded wait gives up after ~1 s
+
+struct DeviceState {
+    void *ws = nullptr;
+    size_t ws_bytes = 0;
+    int num_sms = 0;
+    int *status = nullptr;
+};
+
+std::mutex g_mu;
+std::unordered_map<int, DeviceState> g_devices;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+cudaEvent_t g_ev_before = nullptr, g_ev_after = nullptr;
+thread_local int g_last_launches = 0;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gqa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA; }
+
+// Per-device state (SM count, status-word address); caller holds g_mu.
+gqa_status device_state(DeviceState **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+    DeviceState &st = g_devices[dev];
+    if (st.num_sms == 0) {
+        if (cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return GQA_ERR_CUDA;
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return GQA_ERR_CUDA;
+        st.status = static_cast<int *>(p);
+    }
+    *out = &st;
+    return GQA_OK;
+}
+
+gqa_status ensure_workspace(DeviceState *st, size_t bytes)
+{
+    if (bytes <= st->ws_bytes) return GQA_OK;
+    if (st->ws) cudaFree(st->ws);
+    st->ws = nullptr;
+    st->ws_bytes = 0;
+    if (cudaMalloc(&st->ws, bytes) != cudaSuccess) {
+        cudaGetLastError();
+        return GQA_ERR_OUT_OF_MEMORY;
+    }
+    st->ws_bytes = bytes;
+    return GQA_OK;
+}
+
+gqa_status get_encoder()
+{
+    if (g_encode) return GQA_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return GQA_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return GQA_OK;
+}
+
+// 4-D bf16 map over a [n3][n2][n1][n0] row-major tensor, box {64, 1, rows, 1},
+// 128-byte swizzle: one box is `rows` rows of one 64-column half of a head.
+gqa_status encode_4d(CUtensorMap *tm, const void *base, uint64_t n0, uint64_t n1, uint64_t n2, uint64_t n3,
+                     uint32_t box_rows)
+{
+    cuuint64_t dims[4] = {n0, n1, n2, n3};
+    cuuint64_t strides[3] = {n0 * 2, n0 * n1 * 2, n0 * n1 * n2 * 2};
+    cuuint32_t box[4] = {64, 1, box_rows, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_CUDA;
+}
+
+gqa_status check_decode_args(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq,
+                             int Hkv, int d, int Tmax, const void *out)
+{
+    if (!q || !k || !v || !seqlens || !out) return GQA_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Tmax <= 0) return GQA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
+    if (d != kHeadDim) return GQA_ERR_UNSUPPORTED;
+    if (B > 65535 || Hq > 65535) return GQA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GQA_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return GQA_ERR_MISALIGNED;
+    return GQA_OK;
+}
+
+struct Plan {
+    int chunk, nsplit, hb, nhb;
+    size_t ws_bytes;
+};
+
+Plan make_plan(int B, int Hq, int Hkv, int Tmax, int num_sms)
+{
+    const int g = Hq / Hkv;
+    Plan p;
+    p.hb = decode_heads_per_cta(g);
+    p.nhb = (g + p.hb - 1) / p.hb;
+    const long long tiles = (Tmax + kDecodeTile - 1) / kDecodeTile;
+    const long long base = (long long)B * Hkv * p.nhb;
+    const long long slots = (long long)num_sms * kDecodeCtasPerSm;
+    // cost in units of "one stage per resident CTA": waves x tiles per split, plus the
+    // partials' round trip and one extra launch when the history is split
+    double best = 1e300;
+    int best_s = 1;
+    const long long smax = tiles < 4096 ? tiles : 4096;
+    for (long long s = 1; s <= smax; ++s) {
+        const long long ct = (tiles + s - 1) / s;
+        const long long se = (tiles + ct - 1) / ct;
+        if (se != s) continue;
+        const long long waves = (base * se + slots - 1) / slots;
+        double cost = (double)waves * (double)ct;
+        if (se > 1) {
+            const double part_bytes = 2.0 * B * Hq * se * (kHeadDim + 2) * 4.0;
+            cost += part_bytes / (double)(kDecodeTile * 512) / (double)slots + 2.0;
+        }
+        if (cost < best - 1e-9) {
+            best = cost;
+            best_s = (int)se;
+        }
+    }
+    p.chunk = (int)(((tiles + best_s - 1) / best_s) * kDecodeTile);
+    p.nsplit = (Tmax + p.chunk - 1) / p.chunk;
+    p.ws_bytes = p.nsplit > 1 ? (size_t)B * Hq * p.nsplit * (kHeadDim + 2) * sizeof(float) : 0;
+    return p;
+}
+
+gqa_status run_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq, int Hkv,
+                      int Tmax, float scale, void *out, cudaStream_t stream, int *launches)
+{
+    DeviceState *st = nullptr;
+    gqa_status s = device_state(&st);
+    if (s != GQA_OK) return s;
+    if ((s = get_encoder()) != GQA_OK) return s;
+    const Plan p = make_plan(B, Hq, Hkv, Tmax, st->num_sms);
+    if (p.nsplit > 1 && (s = ensure_workspace(st, p.ws_bytes)) != GQA_OK) return s;
+    if (Hkv * p.nhb > 65535) return GQA_ERR_UNSUPPORTED;
+
+    CUtensorMap tmK, tmV;
+    if ((s = encode_4d(&tmK, k, kHeadDim, Hkv, Tmax, B, kDecodeTile)) != GQA_OK) return s;
+    if ((s = encode_4d(&tmV, v, kHeadDim, Hkv, Tmax, B, kDecodeTile)) != GQA_OK) return s;
+
+    DecodeArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.seqlens = seqlens;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.part_o = static_cast<float *>(st->ws);
+    a.part_ml = a.part_o ? a.part_o + (size_t)B * Hq * p.nsplit * kHeadDim : nullptr;
+    a.status = st->status;
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.Tmax = Tmax;
+    a.group = Hq / Hkv;
+    a.chunk = p.chunk;
+    a.nsplit = p.nsplit;
+    a.nhb = p.nhb;
+    a.qscale = scale * 1.4426950408889634f;  // log2(e): the softmax runs in base 2
+    a.wait_budget_ns = kWaitBudgetNs;
+
+    if (g_ev_before) cudaEventRecord(g_ev_before, stream);
+    if ((s = cuda_status(launch_decode_split(tmK, tmV, a, stream))) != GQA_OK) return s;
+    if (g_ev_after) cudaEventRecord(g_ev_after, stream);
+    int n = 1;
+    if (p.nsplit > 1) {
+        if ((s = cuda_status(launch_decode_combine(a, stream))) != GQA_OK) return s;
+        ++n;
+    }
+    *launches += n;
+    return GQA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens, int B, int Hq,
+                      int Hkv, int d, int Tmax, float scale, void *out, void *stream)
+{
+    g_last_launches = 0;
+    gqa_status s = check_decode_args(q, k_cache, v_cache, seqlens, B, Hq, Hkv, d, Tmax, out);
+    if (s != GQA_OK) return s;
+    std::lock_guard<std::mutex> lk(g_mu);
+    return run_decode(q, k_cache, v_cache, seqlens, B, Hq, Hkv, Tmax, scale, out,
+                      static_cast<cudaStream_t>(stream), &g_last_launches);
+}
+
+size_t gqa_decode_expanded_bytes(int B, int Tmax, int Hq, int d)
+{
+    if (B <= 0 || Tmax <= 0 || Hq <= 0 || d <= 0) return 0;
+    return (size_t)B * (size_t)Tmax * (size_t)Hq * (size_t)d * 2u;
+}
+
+gqa_status gqa_decode_expanded(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                               int B, int Hq, int Hkv, int d, int Tmax, float scale, void *out, void *k_rep,
+                               void *v_rep, void *stream)
+{
+    g_last_launches = 0;
+    gqa_status s = check_decode_args(q, k_cache, v_cache, seqlens, B, Hq, Hkv, d, Tmax, out);
+    if (s != GQA_OK) return s;
+    if (!k_rep || !v_rep) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(k_rep) || !aligned16(v_rep)) return GQA_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if ((s = cuda_status(launch_repeat_kv(k_cache, v_cache, seqlens, k_rep, v_rep, B, Tmax, Hq, Hkv, st))) != GQA_OK)
+        return s;
+    g_last_launches = 1;
+    return run_decode(q, k_rep, v_rep, seqlens, B, Hq, Hq, Tmax, scale, out, st, &g_last_launches);
+}
+
+gqa_status gqa_decode_plan(int B, int Hq, int Hkv, int d, int Tmax, int num_sms, int *chunk, int *nsplit,
+                           size_t *workspace_bytes)
+{
+    if (!chunk || !nsplit || !workspace_bytes) return GQA_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Tmax <= 0 || num_sms <= 0) return GQA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
+    if (d != kHeadDim) return GQA_ERR_UNSUPPORTED;
+    const Plan p = make_plan(B, Hq, Hkv, Tmax, num_sms);
+    *chunk = p.chunk;
+    *nsplit = p.nsplit;
+    *workspace_bytes = p.ws_bytes;
+    return GQA_OK;
+}
+
+gqa_status gqa_prefill_causal(const void *q, const void *k, const void *v, int B, int S, int Hq, int Hkv, int d,
+                              void *out, void *stream)
+{
+    g_last_launches = 0;
+    if (!q || !k || !v || !out) return GQA_ERR_INVALID_ARG;
+    if (B <= 0 || S <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return GQA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
+    if (d != kHeadDim) return GQA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GQA_ERR_MISALIGNED;
+    (void)stream;
+    return GQA_ERR_UNSUPPORTED;
+}
+
+gqa_status gqa_get_last_device_status(void *stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GQA_ERR_CUDA;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status_word, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(int)) != cudaSuccess) return GQA_ERR_CUDA;
+    return static_cast<gqa_status>(v);
+}
+
+gqa_status gqa_selftest_wait_timeout(int timeout_us, void *stream)
+{
+    g_last_launches = 0;
+    if (timeout_us <= 0 || timeout_us > 10000000) return GQA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState *st = nullptr;
+    gqa_status s = device_state(&st);
+    if (s != GQA_OK) return s;
+    s = cuda_status(launch_wait_timeout_selftest(st->status, (unsigned long long)timeout_us * 1000ull,
+                                                 static_cast<cudaStream_t>(stream)));
+    if (s == GQA_OK) g_last_launches = 1;
+    return s;
+}
+
+gqa_status gqa_set_profile_events(void *before, void *after)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    if ((before == nullptr) != (after == nullptr)) return GQA_ERR_INVALID_ARG;
+    g_ev_before = static_cast<cudaEvent_t>(before);
+    g_ev_after = static_cast<cudaEvent_t>(after);
+    return GQA_OK;
+}
+
+int gqa_last_launch_count(void) { return g_last_launches; }
+
+void gqa_release(void)
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    int cur = 0;
+    cudaGetDevice(&cur);
+    for (auto &kv : g_devices) {
+        if (kv.second.ws) {
+            cudaSetDevice(kv.first);
+            cudaFree(kv.second.ws);
+        }
+    }
+    g_devices.clear();
+    cudaSetDevice(cur);
+}
+
+const char *gqa_status_string(gqa_status s)
+{
+    switch (s) {
+    case GQA_OK: return "ok";
+    case GQA_ERR_INVALID_ARG: return "invalid argument";
+    case GQA_ERR_UNSUPPORTED: return "unsupported shape";
+    case GQA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case GQA_ERR_OUT_OF_MEMORY: return "workspace allocation failed";
+    case GQA_ERR_CUDA: return "CUDA error";
+    case GQA_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    }
+    return "unknown status";
+}
+
+const char *gqa_version(void) { return "gqa-b200 0.1"; }
+
+}  // extern "C"

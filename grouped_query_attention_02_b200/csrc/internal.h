@@ -1,0 +1,51 @@
+// internal.h -- host-side interface between the C ABI (api.cu) and the kernel
+// translation units (decode.cu, prefill.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gqa {
+
+constexpr int kHeadDim = 128;       // the one head size this build implements
+constexpr int kDecodeTile = 64;     // tokens per TMA stage of the decode kernel
+constexpr int kDecodeCtasPerSm = 2; // resident decode CTAs per SM (shared-memory bound)
+constexpr int kStatusTimeout = 6;   // device status word: a bounded wait gave up
+
+struct DecodeArgs {
+    const __nv_bfloat16 *q;   // [B,Hq,d]
+    const int32_t *seqlens;   // [B], device
+    __nv_bfloat16 *out;       // [B,Hq,d]
+    float *part_o;            // [B,Hq,nsplit,d]   (nsplit > 1)
+    float *part_ml;           // [B,Hq,nsplit,2]   (nsplit > 1)
+    int *status;              // device status word
+    int B, Hq, Hkv, Tmax, group, chunk, nsplit, nhb;
+    float qscale;             // scale * log2(e)
+    unsigned long long wait_budget_ns;
+};
+
+// Heads of one group handled by one decode CTA for group size g.
+int decode_heads_per_cta(int g);
+size_t decode_smem_bytes(int heads_per_cta);
+
+cudaError_t launch_decode_split(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeArgs &a,
+                                cudaStream_t stream);
+cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t stream);
+cudaError_t launch_repeat_kv(const void *k, const void *v, const int32_t *seqlens, void *k_rep, void *v_rep,
+                             int B, int Tmax, int Hq, int Hkv, cudaStream_t stream);
+cudaError_t launch_wait_timeout_selftest(int *status, unsigned long long budget_ns, cudaStream_t stream);
+
+struct PrefillArgs {
+    __nv_bfloat16 *out;       // [B,S,Hq,d]
+    int *status;
+    int B, S, Hq, Hkv, group;
+    float qscale;             // log2(e) / sqrt(d)
+    unsigned long long wait_budget_ns;
+};
+
+cudaError_t launch_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                           const PrefillArgs &a, cudaStream_t stream);
+
+}  // namespace gqa

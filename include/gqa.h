@@ -1,0 +1,156 @@
+/*
+ * gqa.h -- C ABI of libgqa.so: grouped-query attention (GQA) on one B200.
+ *
+ * The operator.  Hq query heads are split into Hkv consecutive groups of
+ * g = Hq / Hkv heads; query head h reads KV head h / g.  Hq must be a
+ * multiple of Hkv.  MHA (Hkv == Hq) and MQA (Hkv == 1) are the two ends of
+ * the same operator.  Definitions: study.greatitself.com "grouped-query and
+ * multi-query attention" (mapping paragraph); lihaoran.work/?p=2890 "Shared KV
+ * can still produce different outputs" (each query head keeps its own
+ * softmax(q K^T / sqrt(d)) V); anrans.github.io attention-variants "Kernels do
+ * not need to copy the KV heads" (a group's query heads read one shared KV
+ * head, read once, never copied; causal mask as a lower triangle).
+ *
+ * Conventions shared by every entry point.
+ *  - Tensors are bf16 (IEEE binary32 with the low 16 bits dropped), dense and
+ *    row-major in the layouts named below; all device pointers must be
+ *    16-byte aligned.  Accumulation is fp32; outputs are rounded to bf16.
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy
+ *    default stream.  Every call only enqueues work on `stream` and returns;
+ *    no call synchronises the host, and the caller owns every tensor and the
+ *    stream.  Results are ready when the stream has reached them.
+ *  - Host-side argument checks run before anything is enqueued; a failed
+ *    check returns its status and enqueues nothing.  A CUDA launch error is
+ *    returned as GQA_ERR_CUDA.
+ *  - The library keeps, per device, a grow-only workspace for split-KV
+ *    partial results (allocated with cudaMalloc on first need) and a cache of
+ *    TMA tensor maps keyed by pointer and shape.  gqa_release() frees both.
+ *    Calls that share the workspace on one device must be ordered on one
+ *    stream (or otherwise serialised by the caller).
+ *  - Only head_dim d == 128 is implemented (GQA_ERR_UNSUPPORTED otherwise).
+ */
+#ifndef GQA_H_
+#define GQA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gqa_status {
+    GQA_OK = 0,
+    GQA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, Hq % Hkv != 0 */
+    GQA_ERR_UNSUPPORTED = 2,    /* a valid shape this build does not implement (d != 128) */
+    GQA_ERR_MISALIGNED = 3,     /* a pointer not 16-byte aligned */
+    GQA_ERR_OUT_OF_MEMORY = 4,  /* the workspace could not be allocated */
+    GQA_ERR_CUDA = 5,           /* a CUDA runtime/driver call or launch failed */
+    GQA_ERR_DEVICE_TIMEOUT = 6  /* a kernel gave up a bounded wait (read by gqa_get_last_device_status) */
+} gqa_status;
+
+/*
+ * gqa_decode -- one decode step over a bf16 KV cache.
+ *
+ *   q        [B, Hq, d]        the step's query, one row per (sequence, query head)
+ *   k_cache  [B, Tmax, Hkv, d] keys of every cached token (the step's own token included)
+ *   v_cache  [B, Tmax, Hkv, d] values, same layout
+ *   seqlens  [B] int32, DEVICE memory: cached tokens of each sequence
+ *   scale    multiplier of q.k (normally 1/sqrt(d))
+ *   out      [B, Hq, d]        out[b,h] = sum_{t < seqlens[b]} softmax_t(scale q[b,h].k[b,t,h/g]) v[b,t,h/g]
+ *
+ * Sequence b attends to every cached token t < seqlens[b]; rows at or past
+ * seqlens[b] are never used (they may hold anything, NaN included).
+ * Preconditions not checked on the host (checking needs a device read):
+ * 0 <= seqlens[b] <= Tmax; values outside are clamped to [0, Tmax].  A
+ * sequence with seqlens[b] == 0 gets an all-zero output row.
+ *
+ * Each K/V tile is fetched once by TMA and shared by the g query heads of its
+ * group.  Long or uneven histories are split across CTAs (split-KV) and the
+ * partial results merged by a second kernel, through the library workspace.
+ */
+gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                      int B, int Hq, int Hkv, int d, int Tmax, float scale, void *out, void *stream);
+
+/*
+ * gqa_prefill_causal -- causal self-attention over whole prompts.
+ *
+ *   q    [B, S, Hq, d]
+ *   k, v [B, S, Hkv, d]
+ *   out  [B, S, Hq, d]   out[b,r,h] = sum_{t <= r} softmax_t(q[b,r,h].k[b,t,h/g] / sqrt(d)) v[b,t,h/g]
+ *
+ * Row r sees tokens 0..r (lower triangle including the diagonal); the scale
+ * is 1/sqrt(d).  QK^T and PV run on the tcgen05 tensor cores with fp32
+ * accumulators in tensor memory; the softmax weights are rounded to bf16
+ * before the PV product.  No workspace.
+ */
+gqa_status gqa_prefill_causal(const void *q, const void *k, const void *v, int B, int S, int Hq, int Hkv,
+                              int d, void *out, void *stream);
+
+/*
+ * gqa_decode_expanded -- the same decode computed the wasteful way, kept as a
+ * baseline: every KV head is first physically repeated g times into the
+ * caller's buffers k_rep/v_rep [B, Tmax, Hq, d] (rows t < seqlens[b] are
+ * written, the rest untouched), then the decode kernel runs with one query
+ * head per KV head.  Same arguments and result as gqa_decode; the buffers
+ * must each hold gqa_decode_expanded_bytes(B, Tmax, Hq, d) bytes.
+ */
+gqa_status gqa_decode_expanded(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                               int B, int Hq, int Hkv, int d, int Tmax, float scale, void *out,
+                               void *k_rep, void *v_rep, void *stream);
+
+/* Bytes of ONE repeated cache (k_rep or v_rep) for gqa_decode_expanded; 0 on bad sizes. */
+size_t gqa_decode_expanded_bytes(int B, int Tmax, int Hq, int d);
+
+/*
+ * gqa_decode_plan -- the split-KV plan gqa_decode uses, for a device with
+ * num_sms SMs: tokens per split (*chunk, a multiple of the 64-token tile),
+ * number of splits (*nsplit) and workspace bytes it needs (*workspace_bytes,
+ * 0 when nsplit == 1).  Pure host arithmetic; touches no device.
+ */
+gqa_status gqa_decode_plan(int B, int Hq, int Hkv, int d, int Tmax, int num_sms, int *chunk, int *nsplit,
+                           size_t *workspace_bytes);
+
+/*
+ * gqa_get_last_device_status -- synchronises `stream`, then reads and clears
+ * the device's status word.  Kernels never trap: a kernel that gives up a
+ * bounded wait (about a second) records GQA_ERR_DEVICE_TIMEOUT there and
+ * returns.  Returns GQA_OK when nothing was recorded, GQA_ERR_CUDA when the
+ * synchronisation itself failed.
+ */
+gqa_status gqa_get_last_device_status(void *stream);
+
+/*
+ * gqa_selftest_wait_timeout -- enqueues one tiny kernel that waits on a
+ * shared-memory barrier nothing will ever complete, bounded to about
+ * timeout_us microseconds, and records GQA_ERR_DEVICE_TIMEOUT.  Used by the
+ * tests to show that a stuck wait returns instead of hanging the GPU.
+ */
+gqa_status gqa_selftest_wait_timeout(int timeout_us, void *stream);
+
+/*
+ * gqa_set_profile_events -- measurement hook.  When both are non-NULL
+ * (cudaEvent_t passed as void*), every later gqa_decode / gqa_prefill_causal /
+ * gqa_decode_expanded records `before` on its stream immediately before its
+ * dominant kernel (the split-KV decode kernel; the prefill kernel) and
+ * `after` immediately after it.  NULL, NULL turns the hook off.
+ */
+gqa_status gqa_set_profile_events(void *before, void *after);
+
+/* Number of kernels the most recent call on this host thread enqueued. */
+int gqa_last_launch_count(void);
+
+/* Frees the workspace and tensor-map cache of every device the library used. */
+void gqa_release(void);
+
+/* Text for a status code (static storage). */
+const char *gqa_status_string(gqa_status status);
+
+/* Library version, e.g. "gqa-b200 0.1". */
+const char *gqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_H_ */

@@ -1,0 +1,186 @@
+"""GPU parity of the decode path against the fp64 oracle, through the C ABI.
+
+Small cases are compared element by element over every output; the full-size
+workloads are compared on sampled sequences (every query head of each sampled
+sequence), the oracle reading only those sequences' cached rows.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import grouped_query_attention_02_b200 as gqa
+from grouped_query_attention_02_b200 import inputs, workloads
+from tests._tolerance import assert_close
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _oracle_rows(oracle_mod, x, bs):
+    """Oracle outputs for sequences bs, one sequence at a time (copies only [0:T_b] rows)."""
+    sl = x.seqlens.cpu().tolist()
+    res = []
+    for b in bs:
+        T = max(1, sl[b])
+        o = oracle_mod.decode(x.q[b:b + 1].cpu(), x.k_cache[b:b + 1, :T].cpu(), x.v_cache[b:b + 1, :T].cpu(),
+                              [sl[b]], x.scale)
+        res.append(o[0])
+    return np.stack(res)
+
+
+def _run(x, **kw):
+    out = gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, **kw)
+    torch.cuda.synchronize()
+    assert gqa.gqa_get_last_device_status() == 0
+    return out
+
+
+def _check_all(oracle_mod, x, out):
+    ref = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens.cpu(), x.scale)
+    return assert_close(out.double().cpu().numpy(), ref)
+
+
+# ---------------------------------------------------------------- the workloads
+
+
+def test_tiny_decode_full(oracle_mod):
+    w = workloads.TINY_DECODE
+    x = inputs.make_decode(w.B, w.Hq, w.Hkv, w.d, w.Tmax, device=DEV, seed=0)
+    _check_all(oracle_mod, x, _run(x))
+
+
+def test_qwen3_8b_shaped_decode_full(oracle_mod):
+    w = workloads.QWEN3_8B_DECODE
+    x = inputs.make_decode(w.B, w.Hq, w.Hkv, w.d, w.Tmax, device=DEV, seed=0)
+    _check_all(oracle_mod, x, _run(x))
+
+
+@pytest.mark.parametrize("w", workloads.VARLEN_DECODE, ids=lambda w: f"Hkv{w.Hkv}")
+def test_variable_length_decode_sampled(oracle_mod, w):
+    x = inputs.make_decode(w.B, w.Hq, w.Hkv, w.d, w.Tmax, device=DEV, seed=0, seqlen_range=w.seqlen_range)
+    out = _run(x)
+    sl = x.seqlens.cpu()
+    bs = sorted({int(sl.argmin()), int(sl.argmax()), 0, 1, w.B // 2, w.B - 1})
+    assert_close(out[bs].double().cpu().numpy(), _oracle_rows(oracle_mod, x, bs))
+
+
+def test_extreme_grouping_decode_sampled(oracle_mod):
+    w = workloads.EXTREME_GROUP_DECODE
+    x = inputs.make_decode(w.B, w.Hq, w.Hkv, w.d, w.Tmax, device=DEV, seed=0)
+    out = _run(x)
+    bs = [0, 7, 15]
+    assert_close(out[bs].double().cpu().numpy(), _oracle_rows(oracle_mod, x, bs))
+
+
+# ---------------------------------------------------------------- edges
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 4), (6, 2), (8, 2), (32, 4), (32, 2), (32, 1), (71, 1)])
+def test_group_sizes(oracle_mod, Hq, Hkv):
+    x = inputs.make_decode(3, Hq, Hkv, 128, 300, seqlens=[300, 129, 17], device=DEV, seed=Hq * 10 + Hkv)
+    _check_all(oracle_mod, x, _run(x))
+
+
+def test_tile_edges_and_empty(oracle_mod):
+    lens = [0, 1, 2, 63, 64, 65, 127, 128, 129, 1000, 1024, 1025]
+    x = inputs.make_decode(len(lens), 8, 2, 128, 1025, seqlens=lens, device=DEV, seed=3)
+    out = _run(x)
+    assert torch.all(out[0] == 0)
+    _check_all(oracle_mod, x, out)
+
+
+def test_split_boundaries(oracle_mod):
+    # a long single sequence is split; lengths straddling the split chunk must merge exactly
+    B, Hq, Hkv, Tmax = 2, 8, 2, 20000
+    chunk, nsplit, _ = gqa.gqa_decode_plan(B, Hq, Hkv, 128, Tmax, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert nsplit > 1
+    lens = [chunk + 1, min(Tmax, 2 * chunk - 1)]
+    x = inputs.make_decode(B, Hq, Hkv, 128, Tmax, seqlens=lens, device=DEV, seed=4)
+    _check_all(oracle_mod, x, _run(x))
+
+
+def test_nan_poisoned_padding_is_never_read(oracle_mod):
+    lens = [5, 64, 100, 777]
+    x = inputs.make_decode(4, 16, 4, 128, 800, seqlens=lens, device=DEV, seed=5, poison=True)
+    out = _run(x)
+    assert not torch.isnan(out).any()
+    _check_all(oracle_mod, x, out)
+
+
+def test_peaky_softmax(oracle_mod):
+    x = inputs.make_decode(4, 32, 8, 128, 2048, seqlens=[2048, 1500, 33, 700], device=DEV, seed=6, q_gain=8.0)
+    _check_all(oracle_mod, x, _run(x))
+
+
+def test_lengths_outside_the_cache_are_clamped(oracle_mod):
+    x = inputs.make_decode(2, 8, 2, 128, 128, seqlens=[128, 0], device=DEV, seed=7)
+    out_ref = _run(x)
+    x.seqlens = torch.tensor([128 + 50, -3], dtype=torch.int32, device=DEV)
+    out = _run(x)
+    assert torch.equal(out, out_ref)
+    assert torch.all(out[1] == 0)
+
+
+def test_non_default_stream_and_out_buffer(oracle_mod):
+    x = inputs.make_decode(2, 8, 2, 128, 512, seqlens=[512, 300], device=DEV, seed=8)
+    s = torch.cuda.Stream()
+    out = torch.full_like(x.q, float("nan"))
+    with torch.cuda.stream(s):
+        gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out, stream=s)
+    s.synchronize()
+    _check_all(oracle_mod, x, out)
+
+
+def test_repeated_calls_are_deterministic():
+    x = inputs.make_decode(8, 32, 8, 128, 4096, device=DEV, seed=9)
+    a = _run(x).clone()
+    b = _run(x)
+    assert torch.equal(a, b)
+
+
+# ---------------------------------------------------------------- expanded baseline
+
+
+def test_expanded_baseline_matches_oracle(oracle_mod):
+    x = inputs.make_decode(3, 32, 8, 128, 1500, seqlens=[1500, 999, 64], device=DEV, seed=10)
+    out = gqa.gqa_decode_expanded(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    torch.cuda.synchronize()
+    assert gqa.gqa_last_launch_count() >= 2
+    _check_all(oracle_mod, x, out)
+
+
+def test_expanded_copy_is_a_real_repeat():
+    x = inputs.make_decode(2, 8, 2, 128, 100, seqlens=[100, 40], device=DEV, seed=11)
+    k_rep = torch.zeros((2, 100, 8, 128), dtype=torch.bfloat16, device=DEV)
+    v_rep = torch.zeros_like(k_rep)
+    gqa.gqa_decode_expanded(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, k_rep=k_rep, v_rep=v_rep)
+    torch.cuda.synchronize()
+    for b, T in enumerate([100, 40]):
+        assert torch.equal(k_rep[b, :T], x.k_cache[b, :T].repeat_interleave(4, dim=1))
+        assert torch.equal(v_rep[b, :T], x.v_cache[b, :T].repeat_interleave(4, dim=1))
+        assert torch.all(k_rep[b, T:] == 0)
+
+
+# ---------------------------------------------------------------- failure detection
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(oracle_mod):
+    gqa.gqa_selftest_wait_timeout(2000)
+    assert gqa.gqa_get_last_device_status() == 6
+    assert gqa.gqa_get_last_device_status() == 0          # read-and-clear
+    x = inputs.make_decode(1, 8, 2, 128, 256, device=DEV, seed=12)
+    _check_all(oracle_mod, x, _run(x))
+
+
+def test_profile_events_bracket_the_decode_kernel():
+    x = inputs.make_decode(16, 32, 8, 128, 4096, device=DEV, seed=13)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gqa.gqa_set_profile_events(e0, e1)
+    try:
+        _run(x)
+    finally:
+        gqa.gqa_set_profile_events(None, None)
+    assert e0.elapsed_time(e1) > 0
