@@ -12,7 +12,7 @@ import ctypes
 import os
 
 __all__ = [
-    "GQAError", "gqa_decode", "gqa_prefill_causal", "gqa_decode_expanded", "gqa_decode_expanded_bytes",
+    "GQAError", "gqa_decode", "gqa_decode_noalloc", "gqa_prefill_causal", "gqa_decode_expanded", "gqa_decode_expanded_bytes",
     "gqa_decode_plan", "gqa_get_last_device_status", "gqa_selftest_wait_timeout", "gqa_set_profile_events",
     "gqa_last_launch_count", "gqa_release", "gqa_status_string", "gqa_version", "library_path", "load",
 ]
@@ -27,6 +27,7 @@ _i = ctypes.c_int
 EXPORTS = {
     # name: (restype, argtypes)
     "gqa_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp]),
+    "gqa_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp]),
     "gqa_prefill_causal": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "gqa_decode_expanded": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp]),
     "gqa_decode_expanded_bytes": (ctypes.c_size_t, [_i, _i, _i, _i]),
@@ -127,6 +128,35 @@ def gqa_decode(q, k_cache, v_cache, seqlens, scale=None, out=None, stream=None):
     st = load().gqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(), B, Hq, Hkv, d,
                            Tmax, float(scale), out.data_ptr(), _stream_ptr(stream))
     _check(st, "gqa_decode")
+    return out
+
+
+def gqa_decode_noalloc(q, k_cache, v_cache, seqlens, scale=None, out=None, stream=None):
+    """gqa_decode without any device allocation by the library (its split partials live in a fixed
+    32 MiB array inside libgqa.so).  For callers whose device memory is fully reserved by their own
+    pool, or whose decode loop cannot absorb cudaMalloc.  `out` should be preallocated by such a
+    caller; calls that overlap on the GPU race on the shared array."""
+    import torch
+
+    _need(q, "q", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    _need(k_cache, "k_cache", torch.bfloat16, 4, q.device)
+    _need(v_cache, "v_cache", torch.bfloat16, 4, q.device)
+    _need(seqlens, "seqlens", torch.int32, 1, q.device)
+    Bk, Tmax, Hkv, dk = k_cache.shape
+    if (Bk, dk) != (B, d) or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, k_cache, v_cache and seqlens")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out", torch.bfloat16, 3, q.device)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    if scale is None:
+        scale = 1.0 / d ** 0.5
+    st = load().gqa_decode_noalloc(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(), B, Hq,
+                                   Hkv, d, Tmax, float(scale), out.data_ptr(), _stream_ptr(stream))
+    _check(st, "gqa_decode_noalloc")
     return out
 
 

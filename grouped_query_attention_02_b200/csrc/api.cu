@@ -194,6 +194,19 @@ gqa_status run_decode(const void *q, const void *k, const void *v, const int32_t
 
 }  // namespace
 
+namespace gqa {
+
+int *device_status_word()
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState *st = nullptr;
+    return device_state(&st) == GQA_OK ? st->status : nullptr;
+}
+
+void set_last_launch_count(int n) { g_last_launches = n; }
+
+}  // namespace gqa
+
 extern "C" {
 
 gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens, int B, int Hq,

@@ -45,6 +45,11 @@ struct PrefillArgs {
     unsigned long long wait_budget_ns;
 };
 
+// The current device's status word (address of the library's device variable), or null.
+int *device_status_word();
+// Sets what gqa_last_launch_count() reports on this host thread.
+void set_last_launch_count(int n);
+
 cudaError_t launch_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV,
                            const PrefillArgs &a, cudaStream_t stream);
 

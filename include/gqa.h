@@ -73,6 +73,36 @@ gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache, c
                       int B, int Hq, int Hkv, int d, int Tmax, float scale, void *out, void *stream);
 
 /*
+ * gqa_decode_noalloc -- gqa_decode for callers that cannot let a library
+ * allocate device memory.  (This entry point is an engineering addition; the
+ * pages describe no counterpart.)
+ *
+ * Who needs it: a serving engine that reserves nearly all of the GPU for its
+ * own memory pool (typically to size its KV cache) has nothing left for a
+ * library's cudaMalloc, and a latency-critical decode loop cannot absorb
+ * cudaMalloc's implicit synchronisation and unpredictable cost.  This call
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *
+ * Arguments, layouts, result and the other error codes are those of
+ * gqa_decode; the caller still owns and passes every input and output.  The
+ * split-KV partials go to a fixed 32 MiB array compiled into the library,
+ * which every GPU that loads the library holds until the process exits.
+ *  - Returns GQA_ERR_UNSUPPORTED when the partials of this shape
+ *    (workspace_bytes of gqa_decode_plan: B*Hq*nsplit*(d+2)*4 bytes) exceed
+ *    32 MiB; gqa_decode handles such shapes.
+ *  - The first call on a device looks up the array's device address once,
+ *    with that device current; make that first call before any stream
+ *    capture.
+ *  - Every call on a device shares the one array and it keeps the last
+ *    call's contents; nothing in it needs to start at zero because each call
+ *    writes every partial it later reads.  Calls whose kernels overlap on the
+ *    GPU (different streams, no ordering between them) race on the array and
+ *    give wrong results: order them, e.g. on one stream.
+ */
+gqa_status gqa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
+                              int B, int Hq, int Hkv, int d, int Tmax, float scale, void *out, void *stream);
+
+/*
  * gqa_prefill_causal -- causal self-attention over whole prompts.
  *
  *   q    [B, S, Hq, d]

@@ -1,0 +1,73 @@
+"""gqa_decode_noalloc through the C ABI: same results as gqa_decode, no device allocation.
+
+The entry point exists for callers that cannot let a library allocate device
+memory (a serving engine whose pool already holds the GPU, a decode loop that
+cannot absorb cudaMalloc).  Its split partials live in a fixed 32 MiB array
+inside libgqa.so.  This file is collected last so that a run stopping at the
+first failure has already run every other test; it also passes on its own in
+a fresh process.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import pytest
+import torch
+
+import grouped_query_attention_02_b200 as gqa
+from grouped_query_attention_02_b200 import inputs
+from tests._tolerance import assert_close
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _call_noalloc(lib, x, out):
+    B, Hq, d = x.q.shape
+    _, Tmax, Hkv, _ = x.k_cache.shape
+    return lib.gqa_decode_noalloc(x.q.data_ptr(), x.k_cache.data_ptr(), x.v_cache.data_ptr(), x.seqlens.data_ptr(),
+                                  B, Hq, Hkv, d, Tmax, ctypes.c_float(x.scale), out.data_ptr(),
+                                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+@pytest.mark.parametrize("shape", [
+    # (B, Hq, Hkv, Tmax, seqlens): the second splits the history, so the scratch really holds partials
+    (1, 8, 2, 256, None),
+    (8, 32, 8, 8192, [8192, 8000, 4097, 64, 1, 0, 3000, 8191]),
+    (3, 32, 2, 20000, [20000, 12345, 777]),
+], ids=["tiny", "split-8x8192", "group16-split"])
+def test_matches_gqa_decode_on_two_calls_in_a_row(shape):
+    B, Hq, Hkv, Tmax, lens = shape
+    lib = gqa.load()
+    x = inputs.make_decode(B, Hq, Hkv, 128, Tmax, seqlens=lens, device=DEV, seed=77)
+    ref = gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+    torch.cuda.synchronize()
+    ref64 = ref.double().cpu().numpy()
+    for call in range(2):
+        out = torch.full_like(x.q, float("nan"))
+        assert _call_noalloc(lib, x, out) == 0
+        torch.cuda.synchronize()
+        assert gqa.gqa_get_last_device_status() == 0
+        assert_close(out.double().cpu().numpy(), ref64)
+    if B == 8:
+        assert gqa.gqa_decode_plan(B, Hq, Hkv, 128, Tmax, torch.cuda.get_device_properties(0).multi_processor_count)[1] > 1
+
+
+def test_rejects_partials_larger_than_the_fixed_scratch():
+    # 128 sequences x 32 query heads, 32768-token caches: the plan's partials need 65 MiB > 32 MiB
+    B, Hq, Hkv, Tmax = 128, 32, 8, 32768
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    _, nsplit, ws = gqa.gqa_decode_plan(B, Hq, Hkv, 128, Tmax, sms)
+    if ws <= 32 << 20:
+        pytest.skip("this GPU's plan fits the scratch")
+    q = torch.zeros((B, Hq, 128), dtype=torch.bfloat16, device=DEV)
+    k = torch.empty((B, Tmax, Hkv, 128), dtype=torch.bfloat16, device=DEV)
+    v = torch.empty_like(k)
+    sl = torch.full((B,), Tmax, dtype=torch.int32, device=DEV)
+    out = torch.empty_like(q)
+    lib = gqa.load()
+    st = lib.gqa_decode_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), sl.data_ptr(), B, Hq, Hkv, 128, Tmax,
+                                ctypes.c_float(0.088), out.data_ptr(), None)
+    assert st == 2, gqa.gqa_status_string(st)
+    assert gqa.gqa_last_launch_count() == 0
