@@ -266,8 +266,32 @@ gqa_status gqa_prefill_causal(const void *q, const void *k, const void *v, int B
     if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
     if (d != kHeadDim) return GQA_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GQA_ERR_MISALIGNED;
-    (void)stream;
-    return GQA_ERR_UNSUPPORTED;
+    if (B > 65535 || S > (1 << 30)) return GQA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState *st = nullptr;
+    gqa_status s = device_state(&st);
+    if (s != GQA_OK) return s;
+    if ((s = get_encoder()) != GQA_OK) return s;
+    CUtensorMap tmQ, tmK, tmV;
+    if ((s = encode_4d(&tmQ, q, kHeadDim, Hq, S, B, 128)) != GQA_OK) return s;
+    if ((s = encode_4d(&tmK, k, kHeadDim, Hkv, S, B, 128)) != GQA_OK) return s;
+    if ((s = encode_4d(&tmV, v, kHeadDim, Hkv, S, B, 128)) != GQA_OK) return s;
+    PrefillArgs a;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.status = st->status;
+    a.B = B;
+    a.S = S;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.group = Hq / Hkv;
+    a.qscale = 1.4426950408889634f / std::sqrt((float)d);   // log2(e) / sqrt(d): base-2 softmax
+    a.wait_budget_ns = kWaitBudgetNs;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (g_ev_before) cudaEventRecord(g_ev_before, cs);
+    if ((s = cuda_status(launch_prefill(tmQ, tmK, tmV, a, cs))) != GQA_OK) return s;
+    if (g_ev_after) cudaEventRecord(g_ev_after, cs);
+    g_last_launches = 1;
+    return GQA_OK;
 }
 
 gqa_status gqa_get_last_device_status(void *stream)
