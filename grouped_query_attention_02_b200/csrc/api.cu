@@ -108,21 +108,23 @@ gqa_status check_decode_args(const void *q, const void *k, const void *v, const 
 }
 
 struct Plan {
-    int chunk, nsplit, hb, nhb;
+    int tile, chunk, nsplit, hb, nhb;
     size_t ws_bytes;
 };
 
 Plan make_plan(int B, int Hq, int Hkv, int Tmax, int num_sms)
 {
     const int g = Hq / Hkv;
+    const DecodeShape sh = decode_shape(g);
     Plan p;
-    p.hb = decode_heads_per_cta(g);
-    p.nhb = (g + p.hb - 1) / p.hb;
-    const long long tiles = (Tmax + kDecodeTile - 1) / kDecodeTile;
+    p.tile = sh.tile;
+    p.hb = sh.heads_per_cta;
+    p.nhb = sh.nhb;
+    const long long tiles = (Tmax + sh.tile - 1) / sh.tile;
     const long long base = (long long)B * Hkv * p.nhb;
-    const long long slots = (long long)num_sms * kDecodeCtasPerSm;
-    // cost in units of "one stage per resident CTA": waves x tiles per split, plus the
-    // partials' round trip and one extra launch when the history is split
+    const long long slots = (long long)num_sms * sh.ctas_per_sm;
+    // cost in units of "one stage per resident CTA": waves x (tiles per split + start-up),
+    // plus the partials' round trip and one extra launch when the history is split
     double best = 1e300;
     int best_s = 1;
     const long long smax = tiles < 4096 ? tiles : 4096;
@@ -131,17 +133,18 @@ Plan make_plan(int B, int Hq, int Hkv, int Tmax, int num_sms)
         const long long se = (tiles + ct - 1) / ct;
         if (se != s) continue;
         const long long waves = (base * se + slots - 1) / slots;
-        double cost = (double)waves * (double)ct;
+        // each CTA also pays a fixed start-up (barriers, query rows, pipeline fill): about one tile
+        double cost = (double)waves * ((double)ct + 1.0);
         if (se > 1) {
             const double part_bytes = 2.0 * B * Hq * se * (kHeadDim + 2) * 4.0;
-            cost += part_bytes / (double)(kDecodeTile * 512) / (double)slots + 2.0;
+            cost += part_bytes / (double)(sh.tile * 512) / (double)slots + 2.0 * kDecodeTile / sh.tile;
         }
         if (cost < best - 1e-9) {
             best = cost;
             best_s = (int)se;
         }
     }
-    p.chunk = (int)(((tiles + best_s - 1) / best_s) * kDecodeTile);
+    p.chunk = (int)(((tiles + best_s - 1) / best_s) * sh.tile);
     p.nsplit = (Tmax + p.chunk - 1) / p.chunk;
     p.ws_bytes = p.nsplit > 1 ? (size_t)B * Hq * p.nsplit * (kHeadDim + 2) * sizeof(float) : 0;
     return p;
@@ -159,8 +162,8 @@ gqa_status run_decode(const void *q, const void *k, const void *v, const int32_t
     if (Hkv * p.nhb > 65535) return GQA_ERR_UNSUPPORTED;
 
     CUtensorMap tmK, tmV;
-    if ((s = encode_4d(&tmK, k, kHeadDim, Hkv, Tmax, B, kDecodeTile)) != GQA_OK) return s;
-    if ((s = encode_4d(&tmV, v, kHeadDim, Hkv, Tmax, B, kDecodeTile)) != GQA_OK) return s;
+    if ((s = encode_4d(&tmK, k, kHeadDim, Hkv, Tmax, B, p.tile)) != GQA_OK) return s;
+    if ((s = encode_4d(&tmV, v, kHeadDim, Hkv, Tmax, B, p.tile)) != GQA_OK) return s;
 
     DecodeArgs a;
     a.q = static_cast<const __nv_bfloat16 *>(q);

@@ -398,19 +398,28 @@ int decode_heads_per_cta(int g)
     return 8;
 }
 
-size_t decode_smem_bytes(int hb)
+DecodeShape decode_shape(int g)
 {
-    switch (hb) {
-    case 1: return SmemLayout<1>::bytes + 1024;
-    case 2: return SmemLayout<2>::bytes + 1024;
-    case 4: return SmemLayout<4>::bytes + 1024;
-    default: return SmemLayout<8>::bytes + 1024;
+    DecodeShape s;
+    s.tensor_cores = (g >= 3 && g <= 32);
+    if (s.tensor_cores) {
+        s.tile = 128;
+        s.heads_per_cta = g;
+        s.nhb = 1;
+        s.ctas_per_sm = 1;
+    } else {
+        s.tile = kDecodeTile;
+        s.heads_per_cta = decode_heads_per_cta(g);
+        s.nhb = (g + s.heads_per_cta - 1) / s.heads_per_cta;
+        s.ctas_per_sm = kDecodeCtasPerSm;
     }
+    return s;
 }
 
 cudaError_t launch_decode_split(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeArgs &a,
                                 cudaStream_t stream)
 {
+    if (decode_shape(a.group).tensor_cores) return launch_decode_tc(tmK, tmV, a, stream);
     switch (decode_heads_per_cta(a.group)) {
     case 1: return launch_split_hb<1>(tmK, tmV, a, stream);
     case 2: return launch_split_hb<2>(tmK, tmV, a, stream);

@@ -10,8 +10,8 @@
 namespace gqa {
 
 constexpr int kHeadDim = 128;       // the one head size this build implements
-constexpr int kDecodeTile = 64;     // tokens per TMA stage of the decode kernel
-constexpr int kDecodeCtasPerSm = 2; // resident decode CTAs per SM (shared-memory bound)
+constexpr int kDecodeTile = 64;     // tokens per TMA stage of the CUDA-core decode kernel
+constexpr int kDecodeCtasPerSm = 2; // resident CUDA-core decode CTAs per SM (shared-memory bound)
 constexpr int kStatusTimeout = 6;   // device status word: a bounded wait gave up
 
 struct DecodeArgs {
@@ -26,12 +26,24 @@ struct DecodeArgs {
     unsigned long long wait_budget_ns;
 };
 
-// Heads of one group handled by one decode CTA for group size g.
-int decode_heads_per_cta(int g);
-size_t decode_smem_bytes(int heads_per_cta);
+// How the decode of group size g is laid out: the kernel family (tensor cores for
+// 3 <= g <= 32, CUDA cores otherwise), its token tile (TMA box rows and split
+// granularity), query heads per CTA, CTAs per SM for the split planner.
+struct DecodeShape {
+    bool tensor_cores;
+    int tile;          // tokens per pipeline stage
+    int heads_per_cta; // query heads one CTA serves
+    int nhb;           // CTAs per (sequence, KV head, split)
+    int ctas_per_sm;
+};
+DecodeShape decode_shape(int g);
+int decode_heads_per_cta(int g);   // CUDA-core kernel only
 
+// Launches the decode kernel decode_shape(a.group) names; the tensor maps' box must be decode_shape().tile rows.
 cudaError_t launch_decode_split(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeArgs &a,
                                 cudaStream_t stream);
+cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeArgs &a,
+                             cudaStream_t stream);
 cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t stream);
 cudaError_t launch_repeat_kv(const void *k, const void *v, const int32_t *seqlens, void *k_rep, void *v_rep,
                              int B, int Tmax, int Hq, int Hkv, cudaStream_t stream);

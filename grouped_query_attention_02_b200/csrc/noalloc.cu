@@ -60,13 +60,13 @@ gqa_status scratch_for_current_device(float **scratch, int *num_sms)
     return GQA_OK;
 }
 
-// [B][Tmax][Hkv][d] bf16 cache, boxes of kDecodeTile rows of one 64-column half, 128-byte swizzle.
-gqa_status encode_cache_map(CUtensorMap *tm, const void *base, int B, int Tmax, int Hkv)
+// [B][Tmax][Hkv][d] bf16 cache, boxes of `rows` rows of one 64-column half, 128-byte swizzle.
+gqa_status encode_cache_map(CUtensorMap *tm, const void *base, int B, int Tmax, int Hkv, int rows)
 {
     const uint64_t d = kHeadDim;
     cuuint64_t dims[4] = {d, (cuuint64_t)Hkv, (cuuint64_t)Tmax, (cuuint64_t)B};
     cuuint64_t strides[3] = {d * 2, d * Hkv * 2, d * Hkv * (uint64_t)Tmax * 2};
-    cuuint32_t box[4] = {64, 1, (cuuint32_t)kDecodeTile, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = g_na_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -100,13 +100,13 @@ extern "C" gqa_status gqa_decode_noalloc(const void *q, const void *k_cache, con
     if ((s = gqa_decode_plan(B, Hq, Hkv, d, Tmax, num_sms, &chunk, &nsplit, &need)) != GQA_OK) return s;
     if (need > kScratchBytes) return GQA_ERR_UNSUPPORTED;   // partials would not fit the fixed scratch
     const int g = Hq / Hkv;
-    const int hb = decode_heads_per_cta(g);
-    const int nhb = (g + hb - 1) / hb;
+    const DecodeShape sh = decode_shape(g);
+    const int nhb = sh.nhb;
     if ((long long)Hkv * nhb > 65535) return GQA_ERR_UNSUPPORTED;
 
     CUtensorMap tmK, tmV;
-    if ((s = encode_cache_map(&tmK, k_cache, B, Tmax, Hkv)) != GQA_OK) return s;
-    if ((s = encode_cache_map(&tmV, v_cache, B, Tmax, Hkv)) != GQA_OK) return s;
+    if ((s = encode_cache_map(&tmK, k_cache, B, Tmax, Hkv, sh.tile)) != GQA_OK) return s;
+    if ((s = encode_cache_map(&tmV, v_cache, B, Tmax, Hkv, sh.tile)) != GQA_OK) return s;
 
     DecodeArgs a;
     a.q = static_cast<const __nv_bfloat16 *>(q);
