@@ -55,8 +55,9 @@ def test_matches_gqa_decode_on_two_calls_in_a_row(shape):
 
 
 def test_rejects_partials_larger_than_the_fixed_scratch():
-    # 128 sequences x 32 query heads, 32768-token caches: the plan's partials need 65 MiB > 32 MiB
-    B, Hq, Hkv, Tmax = 128, 32, 8, 32768
+    # 1100 sequences x 32 query heads over one KV head, 4096-token caches: on 148 SMs the plan
+    # splits each history in two and the partials need 34.9 MiB > 32 MiB
+    B, Hq, Hkv, Tmax = 1100, 32, 1, 4096
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     _, nsplit, ws = gqa.gqa_decode_plan(B, Hq, Hkv, 128, Tmax, sms)
     if ws <= 32 << 20:
