@@ -80,7 +80,7 @@ def load_peaks():
         return dict(FALLBACK_PEAKS)
 
 
-DECODE_SOURCES = ("decode.cu", "ptx.cuh", "internal.h")
+DECODE_SOURCES = ("decode.cu", "decode_tc.cu", "ptx.cuh", "internal.h")
 PREFILL_SOURCES = ("prefill.cu", "ptx.cuh", "internal.h")
 
 
@@ -281,6 +281,30 @@ def cpu_oracle_sample(x, target_s: float = 12.0):
             "seconds": spent, "tokens_per_s": n * reps / spent}
 
 
+def decode_kernel_name(g: int) -> str:
+    """Which decode kernel the library launches for group size g (label only)."""
+    if 3 <= g <= 32:
+        return f"decode_tc_kernel<{16 if g <= 16 else 32}>"
+    return f"decode_split_kernel<{1 if g <= 1 else 2 if g <= 2 else 4 if g <= 4 else 8}>"
+
+
+def prefill_only(gqa, torch, inputs, workloads, args):
+    """Time the causal prefill workload alone (B sequences of 8192 tokens, 32/8 heads, d=128)."""
+    pw = workloads.CAUSAL_PREFILL
+    peaks = load_peaks()
+    p = inputs.make_prefill(args.prefill_batch, pw.S, pw.Hq, pw.Hkv, pw.d, device="cuda", seed=0)
+    st_ms, k_ms, n = time_prefill(gqa, torch, p, args.steps, args.warmup)
+    fl = prefill_causal_flops(args.prefill_batch, pw.S, pw.Hq, pw.d)
+    print(json.dumps({"metric": "causal GQA prefill TFLOP/s", "value": fl / (st_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": st_ms,
+                      "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": pw.name, "B": args.prefill_batch},
+                      "roofline": {"bound": "tensor", "achieved": fl / (k_ms * 1e-3) / 1e12,
+                                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                   "frac": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+                      "gpu_launches": n, "device_status": gqa.gqa_get_last_device_status()}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -290,6 +314,9 @@ def main():
     ap.add_argument("--rows", choices=["all", "none"], default="all")
     ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the host-buffer measurement")
     ap.add_argument("--cpu-baseline", choices=["on", "off"], default="on")
+    ap.add_argument("--mode", choices=["decode", "prefill"], default="decode",
+                    help="prefill: time only the causal prefill workload (used for its ncu captures)")
+    ap.add_argument("--prefill-batch", type=int, default=4, help="sequences in --mode prefill")
     args = ap.parse_args()
 
     import torch
@@ -341,6 +368,9 @@ def main():
 
     gqa.load()
     torch.cuda.set_device(local_rank)
+    if args.mode == "prefill":
+        prefill_only(gqa, torch, inputs, workloads, args)
+        return
     dist = None
     if world > 1:
         import datetime
@@ -418,8 +448,8 @@ def main():
         "tokens_per_s": tokens_per_s, "frac_of_hbm_peak_step": value / max(world, 1) / peaks["hbm_gbs"],
         "gpu_launches": launches, "device_status": status,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": profile_traffic("decode_split_qwen3_8b.md"),
-                     "kernel": "decode_split_kernel<4>", "kernel_ms": kern_ms, "algorithmic_bytes": alg_bytes,
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": profile_traffic("decode_tc_qwen3_8b.md"),
+                     "kernel": decode_kernel_name(w.group), "kernel_ms": kern_ms, "algorithmic_bytes": alg_bytes,
                      "peak_source": f"{peaks.get('source')} hbm_gbs (copy bandwidth)"},
         "clocks": clk.summary(),
     }
@@ -461,9 +491,14 @@ def main():
             p = inputs.make_prefill(pw.B, pw.S, pw.Hq, pw.Hkv, pw.d, device="cuda", seed=0)
             st_ms, k_ms, n = time_prefill(gqa, torch, p, 10, 3)
             fl = prefill_causal_flops(pw.B, pw.S, pw.Hq, pw.d)
+            t1 = profile_traffic("prefill_causal_b1_s8192.md", PREFILL_SOURCES)
             rows[pw.name] = {"ms_per_step": st_ms, "kernel_ms": k_ms, "TFLOPs": fl / (st_ms * 1e-3) / 1e12,
-                             "frac_bf16_peak": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
-                             "peak_tflops": peaks["bf16_tflops"]}
+                             "roofline": {"bound": "tensor", "achieved": fl / (k_ms * 1e-3) / 1e12,
+                                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                          "frac": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                                          "traffic": None if t1 is None else t1 * pw.B,
+                                          "traffic_note": "ncu capture at B=1 scaled by B (traffic is per sequence)",
+                                          "peak_source": f"{peaks.get('source')} bf16_tflops (cuBLAS burst)"}}
         except gqa.GQAError as e:
             rows[pw.name] = {"error": str(e)}
         line["rows"] = rows
