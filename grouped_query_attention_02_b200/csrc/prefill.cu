@@ -117,6 +117,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r)
         : "memory");
 }
 
+// max of three floats in one instruction (PTX max.f32 with three sources, sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -570,23 +578,29 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (!wait_or_fail(&bar[PS_FULL + w], j & 1, a, err)) { ok = false; break; }
             tc_fence_after();
             const bool diag = (j == qt);
-            // pass 1: the row maximum of the raw scores (keys after the row hidden on the diagonal)
-            float pm[8];
+            // pass 1: the row maximum of the raw scores (keys after the row hidden on the diagonal);
+            // two 32-column loads per wait, three-input max, four independent partial maxima
+            float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sr[32];
-                tmem_ld32(tS + c * 32, sr);
+            for (int c2 = 0; c2 < 4; c2 += 2) {
+                uint32_t sr[64];
+                tmem_ld32(tS + c2 * 32, sr);
+                tmem_ld32(tS + c2 * 32 + 32, sr + 32);
                 tmem_wait_ld();
+                if (diag) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float v = (diag && c * 32 + i > r) ? -INFINITY : __uint_as_float(sr[i]);
-                    pm[i & 7] = fmaxf(pm[i & 7], v);
+                    for (int i = 0; i < 64; ++i)
+                        if (c2 * 32 + i > r) sr[i] = __float_as_uint(-INFINITY);
+                }
+#pragma unroll
+                for (int i = 0; i < 64; i += 8) {
+                    pm[0] = fmax3(pm[0], __uint_as_float(sr[i + 0]), __uint_as_float(sr[i + 1]));
+                    pm[1] = fmax3(pm[1], __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
+                    pm[2] = fmax3(pm[2], __uint_as_float(sr[i + 4]), __uint_as_float(sr[i + 5]));
+                    pm[3] = fmax3(pm[3], __uint_as_float(sr[i + 6]), __uint_as_float(sr[i + 7]));
                 }
             }
-            const float mraw = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+            const float mraw = fmaxf(fmax3(pm[0], pm[1], pm[2]), pm[3]);
             const float m_new = fmaxf(m_run, mraw * a.qscale);
             const bool move = (m_new > m_run + kRescaleThreshold);
             const float m_use = move ? m_new : m_run;
@@ -609,23 +623,29 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                             make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t sr[32];
-                tmem_ld32(tS + c * 32, sr);
+            for (int c2 = 0; c2 < 4; c2 += 2) {
+                uint32_t sr[64];
+                tmem_ld32(tS + c2 * 32, sr);
+                tmem_ld32(tS + c2 * 32 + 32, sr + 32);
                 tmem_wait_ld();
-                uint32_t pk[16];
+                if (diag) {
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    float2 e = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), sc2, nm2);
-                    if (diag) {
-                        if (c * 32 + i > r) e.x = -INFINITY;
-                        if (c * 32 + i + 1 > r) e.y = -INFINITY;
-                    }
-                    const float2 pe = make_float2(ex2(e.x), ex2(e.y));
-                    ps[(i >> 1) & 3] = __fadd2_rn(ps[(i >> 1) & 3], pe);
-                    pk[i >> 1] = pack_bf16x2(pe.x, pe.y);
+                    for (int i = 0; i < 64; ++i)
+                        if (c2 * 32 + i > r) sr[i] = __float_as_uint(-INFINITY);
                 }
-                tmem_st16(tS + c * 16, pk);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const float2 e = __ffma2_rn(
+                            make_float2(__uint_as_float(sr[h * 32 + i]), __uint_as_float(sr[h * 32 + i + 1])), sc2, nm2);
+                        const float2 pe = make_float2(ex2(e.x), ex2(e.y));
+                        ps[(i >> 1) & 3] = __fadd2_rn(ps[(i >> 1) & 3], pe);
+                        pk[i >> 1] = pack_bf16x2(pe.x, pe.y);
+                    }
+                    tmem_st16(tS + (c2 + h) * 16, pk);
+                }
             }
             tmem_wait_st();
             const float rs = (ps[0].x + ps[0].y) + (ps[1].x + ps[1].y) + (ps[2].x + ps[2].y) + (ps[3].x + ps[3].y);
