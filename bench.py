@@ -284,7 +284,7 @@ def cpu_oracle_sample(x, target_s: float = 12.0):
 def decode_kernel_name(g: int) -> str:
     """Which decode kernel the library launches for group size g (label only)."""
     if 3 <= g <= 32:
-        return f"decode_tc_kernel<{16 if g <= 16 else 32}>"
+        return f"decode_persistent_kernel<{16 if g <= 16 else 32}>"
     return f"decode_split_kernel<{1 if g <= 1 else 2 if g <= 2 else 4 if g <= 4 else 8}>"
 
 
@@ -317,6 +317,8 @@ def main():
     ap.add_argument("--mode", choices=["decode", "prefill"], default="decode",
                     help="prefill: time only the causal prefill workload (used for its ncu captures)")
     ap.add_argument("--prefill-batch", type=int, default=4, help="sequences in --mode prefill")
+    ap.add_argument("--decode-workload", default="Qwen3-8B",
+                    help="name prefix of the decode workload timed as the headline (profiling other rows)")
     args = ap.parse_args()
 
     import torch
@@ -329,7 +331,7 @@ def main():
 
     from grouped_query_attention_02_b200 import inputs, workloads
 
-    w = workloads.QWEN3_8B_DECODE
+    w = next(x for x in workloads.DECODE_WORKLOADS if x.name.startswith(args.decode_workload))
     base_cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.Tmax,
                 "global_batch": w.B * max(world, 1), "parallelism": f"dp{max(world, 1)} (batch-sharded, no collective)",
                 "l2": "inputs larger than L2 (1.64 GB cache vs 126 MB); no flush"}
@@ -381,7 +383,8 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
 
     peaks = load_peaks()
-    x = inputs.make_decode(w.B, w.Hq, w.Hkv, w.d, w.Tmax, device="cuda", seed=rank_seed(rank))
+    x = inputs.make_decode(w.B, w.Hq, w.Hkv, w.d, w.Tmax, device="cuda", seed=rank_seed(rank),
+                           seqlen_range=w.seqlen_range)
     sl = x.seqlens.cpu().tolist()
     U = unique_kv_bytes(sl, w.Hkv, w.d)
     alg_bytes = U + 2 * x.q.numel() * 2   # cache + q in + out

@@ -16,8 +16,10 @@ using namespace gqa;
 
 __device__ int g_status_word;  // first error a kernel recorded (0 = none)
 static_assert(kStatusTimeout == GQA_ERR_DEVICE_TIMEOUT, "device and host timeout codes differ");
+static_assert(kStatusMisaligned == GQA_ERR_MISALIGNED, "device and host alignment codes differ");
 
 constexpr unsigned long long kWaitBudgetNs = 1000000000ull;  // a bounded wait gives up after ~1 s
+constexpr size_t kWorkspaceBudget = size_t(256) << 20;        // split partials of one call, at most
 
 struct DeviceState {
     void *ws = nullptr;
@@ -107,20 +109,60 @@ gqa_status check_decode_args(const void *q, const void *k, const void *v, const 
     return GQA_OK;
 }
 
-struct Plan {
-    int tile, chunk, nsplit, hb, nhb;
-    size_t ws_bytes;
-};
+gqa_status run_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq, int Hkv,
+                      int Tmax, float scale, void *out, cudaStream_t stream, int *launches);
 
-Plan make_plan(int B, int Hq, int Hkv, int Tmax, int num_sms)
+}  // namespace
+
+namespace gqa {
+
+int *device_status_word()
+{
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState *st = nullptr;
+    return device_state(&st) == GQA_OK ? st->status : nullptr;
+}
+
+void set_last_launch_count(int n) { g_last_launches = n; }
+
+static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_t ws_budget)
 {
     const int g = Hq / Hkv;
     const DecodeShape sh = decode_shape(g);
-    Plan p;
+    DecodePlan p{};
     p.tile = sh.tile;
     p.hb = sh.heads_per_cta;
     p.nhb = sh.nhb;
+    p.tensor_cores = sh.tensor_cores;
     const long long tiles = (Tmax + sh.tile - 1) / sh.tile;
+    if (sh.tensor_cores) {
+        // the device cuts histories from the real lengths (decode_plan_kernel); the host only bounds
+        // the pieces per sequence (at most 64, fewer when their partials would not fit the budget)
+        // and sizes the workspace for that bound
+        const size_t per_piece = (size_t)B * Hq * (kHeadDim + 2) * 4 + (size_t)B * 16;
+        long long cap = 64;
+        if (cap > tiles) cap = tiles;
+        const long long fit = per_piece ? (long long)(ws_budget / per_piece) : cap;
+        if (fit < cap) cap = fit < 1 ? 1 : fit;
+        const long long cmin = (tiles + cap - 1) / cap;
+        p.nsplit = (int)((tiles + cmin - 1) / cmin);
+        p.chunk = (int)(cmin * sh.tile);
+        size_t off = 0;
+        p.off_hdr = off;
+        off += 256;
+        p.off_nsb = off;
+        off += round256((size_t)B * 4) * 2;   // pieces per sequence, then the planner's scratch
+        p.off_items = off;
+        off += round256((size_t)B * p.nsplit * 16);
+        p.off_po = off;
+        off += round256((size_t)B * Hq * p.nsplit * kHeadDim * 4);
+        p.off_pml = off;
+        off += round256((size_t)B * Hq * p.nsplit * 2 * 4);
+        p.ws_bytes = off;
+        return p;
+    }
     const long long base = (long long)B * Hkv * p.nhb;
     const long long slots = (long long)num_sms * sh.ctas_per_sm;
     // cost in units of "one stage per resident CTA": waves x (tiles per split + start-up),
@@ -146,32 +188,32 @@ Plan make_plan(int B, int Hq, int Hkv, int Tmax, int num_sms)
     }
     p.chunk = (int)(((tiles + best_s - 1) / best_s) * sh.tile);
     p.nsplit = (Tmax + p.chunk - 1) / p.chunk;
+    p.off_po = 0;
+    p.off_pml = (size_t)B * Hq * p.nsplit * kHeadDim * 4;
     p.ws_bytes = p.nsplit > 1 ? (size_t)B * Hq * p.nsplit * (kHeadDim + 2) * sizeof(float) : 0;
     return p;
 }
 
-gqa_status run_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq, int Hkv,
-                      int Tmax, float scale, void *out, cudaStream_t stream, int *launches)
+int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq, int Hkv,
+                   int Tmax, float scale, void *out, void *ws, const DecodePlan &p, int num_sms, int *status,
+                   cudaStream_t stream, int *launches, cudaEvent_t ev_before, cudaEvent_t ev_after)
 {
-    DeviceState *st = nullptr;
-    gqa_status s = device_state(&st);
-    if (s != GQA_OK) return s;
+    gqa_status s;
     if ((s = get_encoder()) != GQA_OK) return s;
-    const Plan p = make_plan(B, Hq, Hkv, Tmax, st->num_sms);
-    if (p.nsplit > 1 && (s = ensure_workspace(st, p.ws_bytes)) != GQA_OK) return s;
-    if (Hkv * p.nhb > 65535) return GQA_ERR_UNSUPPORTED;
-
-    CUtensorMap tmK, tmV;
+    if ((long long)Hkv * p.nhb > 65535) return GQA_ERR_UNSUPPORTED;
+    if (p.ws_bytes > 0 && !ws) return GQA_ERR_INVALID_ARG;
+    CUtensorMap tmK, tmV, tmQ;
     if ((s = encode_4d(&tmK, k, kHeadDim, Hkv, Tmax, B, p.tile)) != GQA_OK) return s;
     if ((s = encode_4d(&tmV, v, kHeadDim, Hkv, Tmax, B, p.tile)) != GQA_OK) return s;
 
-    DecodeArgs a;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    DecodeArgs a{};
     a.q = static_cast<const __nv_bfloat16 *>(q);
     a.seqlens = seqlens;
     a.out = static_cast<__nv_bfloat16 *>(out);
-    a.part_o = static_cast<float *>(st->ws);
-    a.part_ml = a.part_o ? a.part_o + (size_t)B * Hq * p.nsplit * kHeadDim : nullptr;
-    a.status = st->status;
+    a.part_o = w ? reinterpret_cast<float *>(w + p.off_po) : nullptr;
+    a.part_ml = w ? reinterpret_cast<float *>(w + p.off_pml) : nullptr;
+    a.status = status;
     a.B = B;
     a.Hq = Hq;
     a.Hkv = Hkv;
@@ -182,33 +224,63 @@ gqa_status run_decode(const void *q, const void *k, const void *v, const int32_t
     a.nhb = p.nhb;
     a.qscale = scale * 1.4426950408889634f;  // log2(e): the softmax runs in base 2
     a.wait_budget_ns = kWaitBudgetNs;
-
-    if (g_ev_before) cudaEventRecord(g_ev_before, stream);
-    if ((s = cuda_status(launch_decode_split(tmK, tmV, a, stream))) != GQA_OK) return s;
-    if (g_ev_after) cudaEventRecord(g_ev_after, stream);
-    int n = 1;
-    if (p.nsplit > 1) {
+    a.num_ctas = num_sms;
+    int n = 0;
+    if (p.tensor_cores) {
+        a.plan_hdr = reinterpret_cast<int *>(w + p.off_hdr);
+        a.nsplit_b = reinterpret_cast<int *>(w + p.off_nsb);
+        a.plan_scratch = reinterpret_cast<int *>(w + p.off_nsb + round256((size_t)B * 4));
+        a.items = reinterpret_cast<int4 *>(w + p.off_items);
+        // the group's query rows as a 3-D map (d, heads, batch): one box = N rows of one 64-column half
+        const int N = a.group <= 16 ? 16 : 32;
+        cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)Hq, (cuuint64_t)B};
+        cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)kHeadDim * Hq * 2};
+        cuuint32_t box[3] = {64, (cuuint32_t)N, 1};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return GQA_ERR_CUDA;
+        if ((s = cuda_status(launch_decode_plan(a, stream))) != GQA_OK) return s;
+        ++n;
+        if (ev_before) cudaEventRecord(ev_before, stream);
+        if ((s = cuda_status(launch_decode_tc(tmK, tmV, tmQ, a, stream))) != GQA_OK) return s;
+        if (ev_after) cudaEventRecord(ev_after, stream);
+        ++n;
         if ((s = cuda_status(launch_decode_combine(a, stream))) != GQA_OK) return s;
         ++n;
+    } else {
+        if (ev_before) cudaEventRecord(ev_before, stream);
+        if ((s = cuda_status(launch_decode_split(tmK, tmV, a, stream))) != GQA_OK) return s;
+        if (ev_after) cudaEventRecord(ev_after, stream);
+        ++n;
+        if (p.nsplit > 1) {
+            if ((s = cuda_status(launch_decode_combine(a, stream))) != GQA_OK) return s;
+            ++n;
+        }
     }
     *launches += n;
     return GQA_OK;
 }
 
-}  // namespace
+}  // namespace gqa
 
-namespace gqa {
+namespace {
 
-int *device_status_word()
+gqa_status run_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq, int Hkv,
+                      int Tmax, float scale, void *out, cudaStream_t stream, int *launches)
 {
-    std::lock_guard<std::mutex> lk(g_mu);
     DeviceState *st = nullptr;
-    return device_state(&st) == GQA_OK ? st->status : nullptr;
+    gqa_status s = device_state(&st);
+    if (s != GQA_OK) return s;
+    const DecodePlan p = decode_plan_host(B, Hq, Hkv, Tmax, st->num_sms, kWorkspaceBudget);
+    if (p.ws_bytes > 0 && (s = ensure_workspace(st, p.ws_bytes)) != GQA_OK) return s;
+    return static_cast<gqa_status>(decode_enqueue(q, k, v, seqlens, B, Hq, Hkv, Tmax, scale, out, st->ws, p,
+                                                  st->num_sms, st->status, stream, launches, g_ev_before,
+                                                  g_ev_after));
 }
 
-void set_last_launch_count(int n) { g_last_launches = n; }
-
-}  // namespace gqa
+}  // namespace
 
 extern "C" {
 
@@ -253,7 +325,7 @@ gqa_status gqa_decode_plan(int B, int Hq, int Hkv, int d, int Tmax, int num_sms,
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Tmax <= 0 || num_sms <= 0) return GQA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
     if (d != kHeadDim) return GQA_ERR_UNSUPPORTED;
-    const Plan p = make_plan(B, Hq, Hkv, Tmax, num_sms);
+    const DecodePlan p = decode_plan_host(B, Hq, Hkv, Tmax, num_sms, kWorkspaceBudget);
     *chunk = p.chunk;
     *nsplit = p.nsplit;
     *workspace_bytes = p.ws_bytes;

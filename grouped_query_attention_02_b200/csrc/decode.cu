@@ -314,7 +314,7 @@ __global__ void __launch_bounds__(kD) decode_combine_kernel(const DecodeArgs a)
     const int h = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
     int T = a.seqlens[b];
     T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
-    int nv = (T + a.chunk - 1) / a.chunk;
+    int nv = a.nsplit_b ? a.nsplit_b[b] : (T + a.chunk - 1) / a.chunk;
     nv = nv > a.nsplit ? a.nsplit : nv;
     const size_t row = (size_t)b * a.Hq + h;
     const float *ml = a.part_ml + row * a.nsplit * 2;
@@ -419,7 +419,6 @@ DecodeShape decode_shape(int g)
 cudaError_t launch_decode_split(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeArgs &a,
                                 cudaStream_t stream)
 {
-    if (decode_shape(a.group).tensor_cores) return launch_decode_tc(tmK, tmV, a, stream);
     switch (decode_heads_per_cta(a.group)) {
     case 1: return launch_split_hb<1>(tmK, tmV, a, stream);
     case 2: return launch_split_hb<2>(tmK, tmV, a, stream);

@@ -1,28 +1,36 @@
-// decode_tc.cu -- GQA decode with the dot products on the tcgen05 tensor cores.
+// decode_tc.cu -- GQA decode with the dot products on the tcgen05 tensor cores,
+// scheduled from the actual sequence lengths.
 //
-// Same contract as decode_split_kernel (one CTA per (sequence b, KV head,
-// split), split partials merged by decode_combine_kernel), but the group's g
-// query heads are the N dimension of two small matrix products per 128-token
-// tile, with the tokens as the 128-row M dimension:
+// Per (sequence b, KV head) the group's g query heads are the N dimension of
+// two small matrix products per 128-token tile, with the tokens as the
+// 128-row M dimension:
 //
-//   S^T [128 tokens x N] = K_tile [128 x d] . Q_g^T        (A = K, K-major; B = Q, K-major)
+//   S^T [128 tokens x N] = K_tile [128 x d] . Q_g^T           (A = K, K-major; B = Q, K-major)
 //   O^T [d x N]         += V_tile^T [d x 128] . P^T [128 x N]  (A = V, MN-major; B = P^T, MN-major)
 //
-// N is g rounded up to 16 or 32 (extra query rows are zero).  The softmax
-// weights enter the second product as two bf16 terms (hi + lo), so the
-// result carries them to about 2^-17 relative, like an fp32 weight.  Each K/V tile is
-// fetched from HBM once by TMA and serves every head of the group ("Kernels do
-// not need to copy the KV heads", anrans.github.io attention-variants: the
-// group's query heads become extra rows against one shared KV head).
+// N is g rounded up to 16 or 32.  Each K/V tile is fetched from HBM once by TMA
+// and serves every head of the group ("Kernels do not need to copy the KV
+// heads", anrans.github.io attention-variants: the group's query heads become
+// extra rows against one shared KV head).  The softmax weights enter the
+// second product as two bf16 terms (hi + lo), so the result carries them to
+// about 2^-17 relative, like an fp32 weight.
 //
-// The softmax runs on 128 threads, one token per thread (TMEM lane = token
-// for S^T, lane = d for O^T).  The running maximum of each head is CTA-wide
-// and only moves when some score exceeds it by more than 8 (log2 units); in
-// the common case a tile costs one warp vote and one group barrier, no
-// reduction.  When it moves, the tile maximum is reduced across the CTA, the
-// per-thread partial sums and the O^T accumulator in TMEM are rescaled.
+// Scheduling.  The host cannot see the lengths (they live on the device), so
+// decode_plan_kernel reads them and cuts every history into pieces of C tiles,
+// C chosen from the total work so that there are about eight rounds of pieces,
+// and lists the pieces longest first.  decode_persistent_kernel then runs one
+// CTA per SM; each CTA claims (piece, KV head) units from an atomic counter
+// and keeps its TMA / MMA / softmax pipeline running across units, writing
+// one partial result (o, m, l) per unit; decode_combine_kernel merges them.
 //
-// Warps: 0..3 softmax + epilogue, 4 TMA producer, 5 TMEM allocator + MMA issuer.
+// The softmax runs on one 128-thread warpgroup per 16 heads, one token per
+// thread (TMEM lane = token for S^T, lane = d for O^T).  The running maximum
+// of each head only moves when some score exceeds it by more than 8 (log2
+// units); in the common case a tile costs one warp vote and one group barrier.
+//
+// Warps: 0..4*nwg-1 softmax + epilogue (nwg = N/16), then the TMA producer
+// (it also claims units and loads the group's query rows), then the TMEM
+// allocator + MMA issuer.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -34,33 +42,40 @@ constexpr int kD = kHeadDim;
 constexpr int kTok = 128;                 // tokens per tile (the M of S^T)
 constexpr int kTile = kTok * kD * 2;      // 32 KB: one K or V tile
 constexpr int kHalf = kTile / 2;          // one 64-column half
-constexpr int kThreads = 192;
-constexpr int kSoftmax = 128;
+constexpr int kWG = 128;                  // threads of one softmax warpgroup (one token each)
+constexpr int kHPW = 16;                  // heads per softmax warpgroup
+constexpr int kQD = 4;                    // depth of the unit queue in shared memory
 constexpr float kMoveThreshold = 8.0f;
+constexpr int kPlanThreads = 1024;
+constexpr int kPlanMaxC = 4096;           // remainder sizes sorted by a shared-memory histogram up to this
 
 template <int N>
 struct TcCfg {
+    static constexpr int nwg = N / kHPW;                      // softmax warpgroups, 16 heads each
+    static constexpr int threads = kWG * nwg + 64;            // + TMA warp + MMA warp
     static constexpr int stages = 3;
     static constexpr int stage_bytes = 2 * kTile;             // K then V
-    static constexpr int q_off = stages * stage_bytes;        // Q: [2 halves][N rows][128 B], swizzled
+    static constexpr int q_off = stages * stage_bytes;        // Q[2 buffers]: [2 halves][N rows][128 B], swizzled
     static constexpr int q_half = N * 128;
-    static constexpr int p_off = q_off + 2 * q_half;          // P^T hi, then lo: [N/8][16 token groups][8][8] bf16
+    static constexpr int q_bytes = 2 * q_half;
+    static constexpr int p_off = q_off + 2 * q_bytes;         // P^T hi, then lo: [N/8][16 token groups][8][8] bf16
     static constexpr int p_bytes = N * kTok * 2;
     static constexpr int red_off = p_off + 2 * p_bytes;       // [2][4][N] floats: tile maxima per warp
-    static constexpr int lsum_off = red_off + 2 * 4 * N * 4;  // [4][N] floats: l partials per warp
-    static constexpr int vote_off = lsum_off + 4 * N * 4;     // [2][4] ints
-    static constexpr int bar_off = vote_off + 32;
-    // barriers: k_full[3], v_full[3], kv_empty[3], s_full[2], s_free[2], p_full, p_free, o_full, drain, grp
-    static constexpr int nbars = 18;
+    static constexpr int lsum_off = red_off + 2 * 4 * N * 4;  // [2 O buffers][4][N] floats: l partials per warp
+    static constexpr int vote_off = lsum_off + 2 * 4 * N * 4; // [nwg][2][4] ints
+    static constexpr int queue_off = vote_off + nwg * 32;     // kQD units of 8 ints
+    static constexpr int bar_off = queue_off + kQD * 32;
+    static constexpr int nbars = 32 + nwg;
     static constexpr int tmem_off = bar_off + nbars * 8;
     static constexpr int err_off = tmem_off + 8;
     static constexpr int bytes = err_off + 8;
-    static constexpr uint32_t tmem_cols = (3 * N <= 32) ? 32 : (3 * N <= 64 ? 64 : 128);
-    static_assert(bytes + 1024 <= 227 * 1024, "shared memory budget");
+    static constexpr uint32_t tmem_cols = (4 * N <= 64) ? 64 : 128;   // S[2] and O[2], N columns each
+    static_assert(bytes <= 227 * 1024, "shared memory budget");
 };
 
+// barrier slots
 enum : int { K_FULL = 0, V_FULL = 3, KV_EMPTY = 6, S_FULL = 9, S_FREE = 11, P_FULL = 13, P_FREE = 14, O_FULL = 15,
-             DRAIN = 16, GRP = 17 };
+             O_FREE = 17, Q_FULL = 19, Q_EMPTY = 21, I_FULL = 23, I_EMPTY = 27, DRAIN = 31, GRP = 32 };
 
 __device__ __forceinline__ void record_status(int *status, int code)
 {
@@ -82,8 +97,8 @@ __device__ __forceinline__ bool wait_or_fail(uint64_t *bar, uint32_t parity, con
     return true;
 }
 
-// Barrier among the 128 softmax threads on an mbarrier, so that it gives up (bounded) like every other wait
-// instead of blocking forever when another role has failed.  `uses` counts this thread's earlier syncs.
+// Barrier among one warpgroup's 128 threads on an mbarrier, so that it gives up (bounded) like every
+// other wait instead of blocking forever when another role has failed.  `uses` counts earlier syncs.
 __device__ __forceinline__ bool group_sync(uint64_t *grp, int &uses, const DecodeArgs &a, volatile int *err)
 {
     mbar_arrive(grp);
@@ -92,68 +107,187 @@ __device__ __forceinline__ bool group_sync(uint64_t *grp, int &uses, const Decod
     return r;
 }
 
-template <int N>
-__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&r)[N])
-{
-    if constexpr (N == 16) {
-        tmem_ld16(taddr, r);
-    } else {
-        uint32_t (&lo)[16] = *reinterpret_cast<uint32_t (*)[16]>(&r[0]);
-        uint32_t (&hi)[16] = *reinterpret_cast<uint32_t (*)[16]>(&r[16]);
-        tmem_ld16(taddr, lo);
-        tmem_ld16(taddr + 16, hi);
-    }
-}
-
-template <int N>
-__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const uint32_t (&r)[N])
-{
-    if constexpr (N == 16) {
-        tmem_st16(taddr, r);
-    } else {
-        const uint32_t (&lo)[16] = *reinterpret_cast<const uint32_t (*)[16]>(&r[0]);
-        const uint32_t (&hi)[16] = *reinterpret_cast<const uint32_t (*)[16]>(&r[16]);
-        tmem_st16(taddr, lo);
-        tmem_st16(taddr + 16, hi);
-    }
-}
-
 __device__ __forceinline__ uint32_t pack2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// 3-D tiled load (d, heads, batch) of the group's query rows.
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *tm, uint64_t *bar, int c0, int c1, int c2)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------------------------
+// Exclusive scan of n ints in shared memory by the whole block.
+__device__ void block_exclusive_scan(int *v, int n, int *warp_tot)
+{
+    const int tid = threadIdx.x, nt = blockDim.x;
+    const int per = (n + nt - 1) / nt;
+    const int lo = min(n, tid * per), hi = min(n, lo + per);
+    int run = 0;
+    for (int i = lo; i < hi; ++i) run += v[i];
+    int x = run;   // inclusive scan of the per-thread runs
+    const int lane = tid & 31, w = tid >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tot[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        int t = lane < (nt >> 5) ? warp_tot[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, t, o);
+            if (lane >= o) t += y;
+        }
+        if (lane < (nt >> 5)) warp_tot[lane] = t;
+    }
+    __syncthreads();
+    int base = x - run + (w > 0 ? warp_tot[w - 1] : 0);
+    for (int i = lo; i < hi; ++i) {
+        const int c = v[i];
+        v[i] = base;
+        base += c;
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ int block_sum(int part, int *red_i, int *out)
+{
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) red_i[w] = part;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int s = 0;
+        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += red_i[i];
+        *out = s;
+    }
+    __syncthreads();
+    return *out;
+}
+
+// Cuts every history into pieces of C tiles and lists them longest first:
+// plan_hdr = {claim counter (reset to 0), pieces, C}; nsplit_b[b] = pieces of sequence b;
+// items[i] = {b, piece index, first token, end token}.  Full pieces come first, then the
+// shorter last pieces in decreasing length (a counting sort).
+__global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeArgs a, int slots)
+{
+    __shared__ long long red_ll[32];
+    __shared__ int red_i[32];
+    __shared__ int warp_tot[32];
+    __shared__ int hist[kPlanMaxC];
+    __shared__ int cursor[kPlanMaxC];
+    __shared__ int s_C, s_sum;
+    int *full_off = a.plan_scratch;     // per-sequence offsets of the full pieces (B ints, global)
+
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    long long tot = 0;
+    int mx = 0;
+    for (int b = tid; b < a.B; b += blockDim.x) {
+        int T = a.seqlens[b];
+        T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
+        const int tl = (T + kTok - 1) / kTok;
+        tot += tl;
+        mx = max(mx, tl);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if (lane == 0) {
+        red_ll[w] = tot;
+        red_i[w] = mx;
+    }
+    for (int i = tid; i < kPlanMaxC; i += blockDim.x) {
+        hist[i] = 0;
+        cursor[i] = 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        long long T = 0;
+        int M = 0;
+        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+            T += red_ll[i];
+            M = max(M, red_i[i]);
+        }
+        // about eight rounds of (piece, KV head) units per persistent CTA, never more than nsplit pieces
+        long long C = (T * a.Hkv + 8LL * slots - 1) / (8LL * slots);
+        const long long cmin = (M + a.nsplit - 1) / a.nsplit;
+        if (C < cmin) C = cmin;
+        if (C > M) C = M;
+        if (C < 1) C = 1;
+        s_C = (int)C;
+    }
+    __syncthreads();
+    const int C = s_C;
+    const bool sort_rem = C <= kPlanMaxC;
+    int npieces = 0;
+    for (int b = tid; b < a.B; b += blockDim.x) {
+        int T = a.seqlens[b];
+        T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
+        const int tl = (T + kTok - 1) / kTok;
+        const int rem = tl % C;
+        full_off[b] = tl / C;
+        a.nsplit_b[b] = tl / C + (rem > 0 ? 1 : 0);
+        npieces += tl / C + (rem > 0 ? 1 : 0);
+        if (rem > 0 && sort_rem) atomicAdd(&hist[C - 1 - rem], 1);   // reversed: longest remainder first
+    }
+    __syncthreads();
+    const int P = block_sum(npieces, red_i, &s_sum);
+    int nfull = 0;
+    for (int b = tid; b < a.B; b += blockDim.x) nfull += full_off[b];
+    const int F = block_sum(nfull, red_i, &s_sum);
+    block_exclusive_scan(full_off, a.B, warp_tot);
+    if (sort_rem) block_exclusive_scan(hist, C, warp_tot);   // hist[C-1-r]: remainders longer than r
+    for (int b = tid; b < a.B; b += blockDim.x) {
+        int T = a.seqlens[b];
+        T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
+        const int tl = (T + kTok - 1) / kTok;
+        const int full = tl / C, rem = tl % C;
+        for (int s = 0; s < full; ++s)
+            a.items[full_off[b] + s] = make_int4(b, s, s * C * kTok, min((s + 1) * C * kTok, T));
+        if (rem > 0) {
+            const int k = C - 1 - rem;
+            const int pos = sort_rem ? F + hist[k] + atomicAdd(&cursor[k], 1) : F + atomicAdd(&cursor[0], 1);
+            a.items[pos] = make_int4(b, full, full * C * kTok, T);
+        }
+    }
+    if (tid == 0) {
+        a.plan_hdr[0] = 0;   // claim counter
+        a.plan_hdr[1] = P;
+        a.plan_hdr[2] = C;
+    }
+}
+
+// ---------------------------------------------------------------------------------------------
 template <int N>
-__global__ void __launch_bounds__(kThreads, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const DecodeArgs a)
+__global__ void __launch_bounds__(TcCfg<N>::threads, 1)
+decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                         const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a)
 {
     using C = TcCfg<N>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-
-    const int split = blockIdx.x;
-    const int kvh = blockIdx.y;
-    const int b = blockIdx.z;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-
-    int T = a.seqlens[b];
-    T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
-    const int t_begin = split * a.chunk;
-    const int t_end = min(t_begin + a.chunk, T);
-    const int h0 = kvh * a.group;
-    const int g = a.group;
-
-    if (t_end <= t_begin) {
-        if (a.nsplit == 1) {
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            for (int i = threadIdx.x; i < g * (kD / 8); i += kThreads)
-                reinterpret_cast<uint4 *>(a.out + ((size_t)b * a.Hq + h0) * kD)[i] = z;
-        }
+    // the 128-byte swizzle needs 1024-byte aligned tiles; the whole budget is used, so there is no room
+    // to realign: a misaligned window is reported and the CTA does nothing
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) record_status(a.status, kStatusMisaligned);
         return;
     }
-    const int ntiles = (t_end - t_begin + kTok - 1) / kTok;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = a.group;
 
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + C::bar_off);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::tmem_off);
@@ -161,9 +295,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     float *red = reinterpret_cast<float *>(smem + C::red_off);
     float *lsum = reinterpret_cast<float *>(smem + C::lsum_off);
     volatile int *vote = reinterpret_cast<volatile int *>(smem + C::vote_off);
-    uint8_t *qs = smem + C::q_off;
+    volatile int *queue = reinterpret_cast<volatile int *>(smem + C::queue_off);
     uint8_t *ps = smem + C::p_off;
 
+    const int producer_warp = 4 * C::nwg, mma_warp = 4 * C::nwg + 1;
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::stages; ++s) {
             mbar_init(&bar[K_FULL + s], 1);
@@ -172,26 +307,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar[S_FULL + s], 1);
-            mbar_init(&bar[S_FREE + s], kSoftmax);
+            mbar_init(&bar[S_FREE + s], kWG * C::nwg);
+            mbar_init(&bar[O_FULL + s], 1);
+            mbar_init(&bar[O_FREE + s], kWG * C::nwg);
+            mbar_init(&bar[Q_FULL + s], 1);
+            mbar_init(&bar[Q_EMPTY + s], 1);
         }
-        mbar_init(&bar[P_FULL], kSoftmax);
+        mbar_init(&bar[P_FULL], kWG * C::nwg);
         mbar_init(&bar[P_FREE], 1);
-        mbar_init(&bar[O_FULL], 1);
+        for (int s = 0; s < kQD; ++s) {
+            mbar_init(&bar[I_FULL + s], 1);
+            mbar_init(&bar[I_EMPTY + s], 1 + kWG * C::nwg);
+        }
         mbar_init(&bar[DRAIN], 1);
-        mbar_init(&bar[GRP], kSoftmax);
+        for (int w = 0; w < C::nwg; ++w) mbar_init(&bar[GRP + w], kWG);
         *err = 0;
         fence_barrier_init();
     }
-    // the group's query rows, bf16, K-major with the 128-byte swizzle; rows g..N-1 are zero
-    for (int i = threadIdx.x; i < N * (kD / 8); i += kThreads) {
-        const int n = i / (kD / 8), c16 = i % (kD / 8);        // row, 16-byte chunk of the 256-byte row
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (n < g) v = reinterpret_cast<const uint4 *>(a.q + ((size_t)b * a.Hq + h0 + n) * kD)[c16];
-        const int half = c16 >> 3, c = c16 & 7;
-        *reinterpret_cast<uint4 *>(qs + half * C::q_half + n * 128 + ((c ^ (n & 7)) << 4)) = v;
-    }
-    fence_proxy_async_smem();
-    if (warp == 5) {
+    if (warp == mma_warp) {
         tmem_alloc(tmem_slot, C::tmem_cols);
         tmem_relinquish();
     }
@@ -200,179 +333,283 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS[2] = {tmem, tmem + N};
-    const uint32_t tO = tmem + 2 * N;
+    const uint32_t tO[2] = {tmem + 2 * N, tmem + 3 * N};
 
-    if (warp == 4) {
-        // ---------------- TMA producer
+    if (warp == producer_warp) {
+        // ---------------- claims units, loads the group's query rows and streams the K/V tiles
         if (lane == 0) {
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            int issued = 0;
-            for (int j = 0; j < ntiles; ++j) {
-                const int s = j % C::stages;
-                if (j >= C::stages && !wait_or_fail(&bar[KV_EMPTY + s], ((j / C::stages) - 1) & 1, a, err)) break;
-                uint8_t *ks = smem + s * C::stage_bytes;
-                const int t0 = t_begin + j * kTok;
-                mbar_arrive_expect_tx(&bar[K_FULL + s], kTile);
-                tma_load_4d(ks, &tmK, &bar[K_FULL + s], 0, kvh, t0, b);
-                tma_load_4d(ks + kHalf, &tmK, &bar[K_FULL + s], 64, kvh, t0, b);
-                mbar_arrive_expect_tx(&bar[V_FULL + s], kTile);
-                tma_load_4d(ks + kTile, &tmV, &bar[V_FULL + s], 0, kvh, t0, b);
-                tma_load_4d(ks + kTile + kHalf, &tmV, &bar[V_FULL + s], 64, kvh, t0, b);
-                ++issued;
+            tma_prefetch_desc(&tmQ);
+            const int units = a.plan_hdr[1] * a.Hkv;
+            int tcount = 0, icount = 0, issued_tiles = 0;
+            while (true) {
+                const int u = atomicAdd(&a.plan_hdr[0], 1);
+                const int slot = icount % kQD;
+                if (icount >= kQD && !wait_or_fail(&bar[I_EMPTY + slot], ((icount / kQD) - 1) & 1, a, err)) break;
+                volatile int *q = queue + slot * 8;
+                if (u >= units) {
+                    q[4] = -1;                         // no more work
+                    mbar_arrive(&bar[I_FULL + slot]);
+                    break;
+                }
+                const int4 it = a.items[u / a.Hkv];
+                const int kvh = u % a.Hkv;
+                q[0] = it.x;
+                q[1] = kvh;
+                q[2] = it.y;
+                q[3] = it.z;
+                q[4] = it.w;
+                mbar_arrive(&bar[I_FULL + slot]);
+                const int qb = icount & 1;
+                if (icount >= 2 && !wait_or_fail(&bar[Q_EMPTY + qb], ((icount >> 1) - 1) & 1, a, err)) break;
+                uint8_t *qs = smem + C::q_off + qb * C::q_bytes;
+                mbar_arrive_expect_tx(&bar[Q_FULL + qb], C::q_bytes);
+                tma_load_3d(qs, &tmQ, &bar[Q_FULL + qb], 0, kvh * g, it.x);
+                tma_load_3d(qs + C::q_half, &tmQ, &bar[Q_FULL + qb], 64, kvh * g, it.x);
+                const int ntl = (it.w - it.z + kTok - 1) / kTok;
+                bool ok = true;
+                for (int jj = 0; jj < ntl; ++jj, ++tcount) {
+                    const int s = tcount % C::stages;
+                    if (tcount >= C::stages &&
+                        !wait_or_fail(&bar[KV_EMPTY + s], ((tcount / C::stages) - 1) & 1, a, err)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *ks = smem + s * C::stage_bytes;
+                    const int t0 = it.z + jj * kTok;
+                    mbar_arrive_expect_tx(&bar[K_FULL + s], kTile);
+                    tma_load_4d(ks, &tmK, &bar[K_FULL + s], 0, kvh, t0, it.x);
+                    tma_load_4d(ks + kHalf, &tmK, &bar[K_FULL + s], 64, kvh, t0, it.x);
+                    mbar_arrive_expect_tx(&bar[V_FULL + s], kTile);
+                    tma_load_4d(ks + kTile, &tmV, &bar[V_FULL + s], 0, kvh, t0, it.x);
+                    tma_load_4d(ks + kTile + kHalf, &tmV, &bar[V_FULL + s], 64, kvh, t0, it.x);
+                    issued_tiles = tcount + 1;
+                }
+                ++icount;
+                if (!ok) break;
             }
-            for (int j = issued - 1; j >= 0 && j >= issued - C::stages; --j) {
-                const uint32_t ph = (j / C::stages) & 1;
-                mbar_wait(&bar[K_FULL + j % C::stages], ph, a.wait_budget_ns);
-                mbar_wait(&bar[V_FULL + j % C::stages], ph, a.wait_budget_ns);
+            // leave no copy in flight
+            for (int t = issued_tiles - 1; t >= 0 && t >= issued_tiles - C::stages; --t) {
+                const uint32_t ph = (t / C::stages) & 1;
+                mbar_wait(&bar[K_FULL + t % C::stages], ph, a.wait_budget_ns);
+                mbar_wait(&bar[V_FULL + t % C::stages], ph, a.wait_budget_ns);
             }
+            for (int i = icount - 1; i >= 0 && i >= icount - 2; --i)
+                mbar_wait(&bar[Q_FULL + (i & 1)], (i >> 1) & 1, a.wait_budget_ns);
         }
-    } else if (warp == 5) {
+    } else if (warp == mma_warp) {
         // ---------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc_s = umma_idesc_bf16(kTok, N, 0, 0);   // K (K-major) . Q^T (K-major)
             const uint32_t idesc_o = umma_idesc_bf16(kD, N, 1, 1);     // V^T (MN-major) . P^T (MN-major)
-            const uint32_t q_addr = smem_u32(qs);
             const uint32_t p_addr = smem_u32(ps);
+            int tcount = 0, icount = 0;
             bool ok = true;
-            int pv_done = 0;
-            for (int j = 0; ok && j <= ntiles; ++j) {
-                if (j < ntiles) {
-                    const int s = j % C::stages;
-                    if (!wait_or_fail(&bar[K_FULL + s], (j / C::stages) & 1, a, err)) { ok = false; break; }
-                    if (j >= 2 && !wait_or_fail(&bar[S_FREE + (j & 1)], ((j >> 1) - 1) & 1, a, err)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t k_addr = smem_u32(smem + s * C::stage_bytes);
-#pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint32_t ka = k_addr + (ks >> 2) * kHalf + (ks & 3) * 32;
-                        const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
-                        umma_bf16_ss(tS[j & 1], umma_smem_desc(ka, 16, 1024, 2), umma_smem_desc(qa, 16, 1024, 2),
-                                     idesc_s, ks > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&bar[S_FULL + (j & 1)]);
-                }
-                if (j >= 1) {
-                    const int jp = j - 1;
-                    const int s = jp % C::stages;
-                    if (!wait_or_fail(&bar[P_FULL], jp & 1, a, err)) { ok = false; break; }
-                    if (!wait_or_fail(&bar[V_FULL + s], (jp / C::stages) & 1, a, err)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t v_addr = smem_u32(smem + s * C::stage_bytes + kTile);
-                    // O^T += V^T P_hi^T + V^T P_lo^T: the weights carried as a sum of two bf16 terms
-#pragma unroll
-                    for (int part = 0; part < 2; ++part) {
-#pragma unroll
-                        for (int ks = 0; ks < kTok / 16; ++ks) {
-                            // A = V^T: 16 tokens (two 8-row groups, 1024 B apart), 64-column blocks kHalf apart
-                            // B = P^T: 16 tokens (two 128-byte core-matrix groups), 8-head blocks 2048 B apart
-                            umma_bf16_ss(tO, umma_smem_desc(v_addr + ks * 2048, kHalf, 1024, 2),
-                                         umma_smem_desc(p_addr + part * C::p_bytes + ks * 256, 128, 2048, 0),
-                                         idesc_o, (jp > 0 || part > 0 || ks > 0) ? 1u : 0u);
+            while (ok) {
+                const int slot = icount % kQD;
+                if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
+                volatile int *q = queue + slot * 8;
+                const int t_begin = q[3], t_end = q[4];
+                mbar_arrive(&bar[I_EMPTY + slot]);
+                if (t_end < 0) break;
+                const int ntl = (t_end - t_begin + kTok - 1) / kTok;
+                const int qb = icount & 1, ob = icount & 1;
+                if (!wait_or_fail(&bar[Q_FULL + qb], (icount >> 1) & 1, a, err)) break;
+                if (icount >= 2 && !wait_or_fail(&bar[O_FREE + ob], ((icount >> 1) - 1) & 1, a, err)) break;
+                const uint32_t q_addr = smem_u32(smem + C::q_off + qb * C::q_bytes);
+                for (int jj = 0; jj <= ntl; ++jj) {
+                    if (jj < ntl) {
+                        const int T = tcount + jj;
+                        const int s = T % C::stages;
+                        if (!wait_or_fail(&bar[K_FULL + s], (T / C::stages) & 1, a, err)) { ok = false; break; }
+                        if (T >= 2 && !wait_or_fail(&bar[S_FREE + (T & 1)], ((T >> 1) - 1) & 1, a, err)) {
+                            ok = false;
+                            break;
                         }
+                        tc_fence_after();
+                        const uint32_t k_addr = smem_u32(smem + s * C::stage_bytes);
+#pragma unroll
+                        for (int ks = 0; ks < kD / 16; ++ks) {
+                            const uint32_t ka = k_addr + (ks >> 2) * kHalf + (ks & 3) * 32;
+                            const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
+                            umma_bf16_ss(tS[T & 1], umma_smem_desc(ka, 16, 1024, 2), umma_smem_desc(qa, 16, 1024, 2),
+                                         idesc_s, ks > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&bar[S_FULL + (T & 1)]);
                     }
-                    umma_commit(&bar[P_FREE]);
-                    umma_commit(&bar[KV_EMPTY + s]);
-                    ++pv_done;
+                    if (jj >= 1) {
+                        const int T = tcount + jj - 1;
+                        const int s = T % C::stages;
+                        if (!wait_or_fail(&bar[P_FULL], T & 1, a, err)) { ok = false; break; }
+                        if (!wait_or_fail(&bar[V_FULL + s], (T / C::stages) & 1, a, err)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t v_addr = smem_u32(smem + s * C::stage_bytes + kTile);
+                        // O^T += V^T P_hi^T + V^T P_lo^T: the weights carried as a sum of two bf16 terms
+#pragma unroll
+                        for (int part = 0; part < 2; ++part) {
+#pragma unroll
+                            for (int ks = 0; ks < kTok / 16; ++ks) {
+                                // A = V^T: 16 tokens (two 8-row groups, 1024 B apart), 64-column blocks kHalf apart
+                                // B = P^T: 16 tokens (two 128-byte core-matrix groups), 8-head blocks 2048 B apart
+                                umma_bf16_ss(tO[ob], umma_smem_desc(v_addr + ks * 2048, kHalf, 1024, 2),
+                                             umma_smem_desc(p_addr + part * C::p_bytes + ks * 256, 128, 2048, 0),
+                                             idesc_o, (jj > 1 || part > 0 || ks > 0) ? 1u : 0u);
+                            }
+                        }
+                        umma_commit(&bar[P_FREE]);
+                        umma_commit(&bar[KV_EMPTY + s]);
+                    }
                 }
+                if (!ok) break;
+                umma_commit(&bar[O_FULL + ob]);
+                umma_commit(&bar[Q_EMPTY + qb]);
+                tcount += ntl;
+                ++icount;
             }
-            if (ok && pv_done == ntiles) umma_commit(&bar[O_FULL]);
             umma_commit(&bar[DRAIN]);
             mbar_wait(&bar[DRAIN], 0, a.wait_budget_ns);
         }
     } else {
-        // ---------------- softmax: thread t owns token t of each tile (and d = t of O^T)
-        const int t = threadIdx.x;                 // warps 0..3: TMEM lane quarter = warp
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        float m_use[N], l_part[N];
-#pragma unroll
-        for (int h = 0; h < N; ++h) {
-            m_use[h] = -INFINITY;
-            l_part[h] = 0.f;
-        }
+        // ---------------- softmax warpgroup wg: heads 16*wg .. 16*wg+15; thread t owns token t of
+        // each tile (TMEM lane t of S^T) and column d = t of O^T
+        const int wg = warp >> 2;
+        const int quarter = warp & 3;              // TMEM lane quarter this warp may access
+        const int t = quarter * 32 + lane;
+        const int hs = wg * kHPW;                  // first head (column) of this warpgroup
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        volatile int *myvote = vote + wg * 8;
+        int tcount = 0, icount = 0, uses = 0;
         bool ok = true;
-        int uses = 0;
-        for (int j = 0; j < ntiles; ++j) {
-            const int sb = j & 1;
-            if (!wait_or_fail(&bar[S_FULL + sb], (j >> 1) & 1, a, err)) { ok = false; break; }
+        // The epilogue of a unit (its O^T from TMEM to the partials) runs after the next unit's first
+        // tile, so that waiting for the unit's last PV product overlaps useful work.
+        bool pend = false;
+        int pb = 0, pkvh = 0, psplit = 0, pob = 0;
+        float pm[kHPW];
+        auto epilogue = [&]() -> bool {
+            if (!group_sync(&bar[GRP + wg], uses, a, err)) return false;      // lsum[pob] complete
+            if (!wait_or_fail(&bar[O_FULL + pob], (((icount - 1) >> 1)) & 1, a, err)) return false;
             tc_fence_after();
-            uint32_t raw[N];
-            tmem_ld_row<N>(tS[sb] + lane_off, raw);
+            uint32_t o[kHPW];
+            tmem_ld16(tO[pob] + lane_off + hs, o);
             tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&bar[S_FREE + sb]);
-
-            const bool valid = (t_begin + j * kTok + t) < t_end;
-            float x[N];
-            bool over = false;
+            const float *ls = lsum + pob * 4 * N;
+            const int d = t;
 #pragma unroll
-            for (int h = 0; h < N; ++h) {
-                x[h] = valid ? __uint_as_float(raw[h]) * a.qscale : -INFINITY;
-                over |= x[h] > m_use[h] + kMoveThreshold;
-            }
-            const int wflag = __any_sync(0xffffffffu, over) ? 1 : 0;
-            if (lane == 0) vote[sb * 4 + warp] = wflag;
-            if (!group_sync(&bar[GRP], uses, a, err)) { ok = false; break; }
-            const bool any_move = (vote[sb * 4 + 0] | vote[sb * 4 + 1] | vote[sb * 4 + 2] | vote[sb * 4 + 3]) != 0;
-            float alpha[N];
-            bool rescale_o = false;
-#pragma unroll
-            for (int h = 0; h < N; ++h) alpha[h] = 1.f;
-            if (any_move) {
-                // CTA-wide maximum of this tile, per head
-#pragma unroll
-                for (int h = 0; h < N; ++h) {
-                    float mx = x[h];
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-                    if (lane == 0) red[(sb * 4 + warp) * N + h] = mx;
+            for (int h = 0; h < kHPW; ++h) {
+                const int hg = hs + h;
+                if (hg >= g) break;
+                const float L = ls[hg] + ls[N + hg] + ls[2 * N + hg] + ls[3 * N + hg];
+                const size_t prow = ((size_t)pb * a.Hq + pkvh * g + hg) * a.nsplit + psplit;
+                a.part_o[prow * kD + d] = __uint_as_float(o[h]);
+                if (d == 0) {
+                    a.part_ml[prow * 2 + 0] = pm[h];
+                    a.part_ml[prow * 2 + 1] = L;
                 }
-                if (!group_sync(&bar[GRP], uses, a, err)) { ok = false; break; }
+            }
+            tc_fence_before();
+            mbar_arrive(&bar[O_FREE + pob]);
+            pend = false;
+            return true;
+        };
+        while (ok) {
+            const int slot = icount % kQD;
+            if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
+            volatile int *qq = queue + slot * 8;
+            const int b = qq[0], kvh = qq[1], split = qq[2], t_begin = qq[3], t_end = qq[4];
+            mbar_arrive(&bar[I_EMPTY + slot]);
+            if (t_end < 0) {
+                if (pend) epilogue();   // the pending unit is icount - 1, as in the loop
+                break;
+            }
+            const int ntl = (t_end - t_begin + kTok - 1) / kTok;
+            const int ob = icount & 1;
+            float m_use[kHPW], l_part[kHPW];
 #pragma unroll
-                for (int h = 0; h < N; ++h) {
-                    const float* rr = red + sb * 4 * N + h;
-                    const float tm = fmaxf(fmaxf(rr[0], rr[N]), fmaxf(rr[2 * N], rr[3 * N]));
-                    const float m_new = fmaxf(m_use[h], tm);
-                    if (m_new > m_use[h] + kMoveThreshold) {
-                        alpha[h] = ex2(m_use[h] - m_new);     // 0 on the first tile
-                        m_use[h] = m_new;
-                        l_part[h] *= alpha[h];
-                        rescale_o = true;
+            for (int h = 0; h < kHPW; ++h) {
+                m_use[h] = -INFINITY;
+                l_part[h] = 0.f;
+            }
+            for (int jj = 0; jj < ntl; ++jj) {
+                const int T = tcount + jj;
+                const int sb = T & 1;
+                if (!wait_or_fail(&bar[S_FULL + sb], (T >> 1) & 1, a, err)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t raw[kHPW];
+                tmem_ld16(tS[sb] + lane_off + hs, raw);
+                tmem_wait_ld();
+                tc_fence_before();
+                mbar_arrive(&bar[S_FREE + sb]);
+
+                const bool valid = (t_begin + jj * kTok + t) < t_end;
+                float x[kHPW];
+                bool over = false;
+#pragma unroll
+                for (int h = 0; h < kHPW; ++h) {
+                    x[h] = valid ? __uint_as_float(raw[h]) * a.qscale : -INFINITY;
+                    over |= x[h] > m_use[h] + kMoveThreshold;
+                }
+                const int wflag = __any_sync(0xffffffffu, over) ? 1 : 0;
+                if (lane == 0) myvote[sb * 4 + quarter] = wflag;
+                if (!group_sync(&bar[GRP + wg], uses, a, err)) { ok = false; break; }
+                const bool any_move = (myvote[sb * 4 + 0] | myvote[sb * 4 + 1] | myvote[sb * 4 + 2] |
+                                       myvote[sb * 4 + 3]) != 0;
+                float alpha[kHPW];
+                bool rescale_o = false;
+#pragma unroll
+                for (int h = 0; h < kHPW; ++h) alpha[h] = 1.f;
+                if (any_move) {
+                    // this tile's maximum over all 128 tokens, per head
+#pragma unroll
+                    for (int h = 0; h < kHPW; ++h) {
+                        float mx = x[h];
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                        if (lane == 0) red[(sb * 4 + quarter) * N + hs + h] = mx;
+                    }
+                    if (!group_sync(&bar[GRP + wg], uses, a, err)) { ok = false; break; }
+#pragma unroll
+                    for (int h = 0; h < kHPW; ++h) {
+                        const float *rr = red + sb * 4 * N + hs + h;
+                        const float tm = fmaxf(fmaxf(rr[0], rr[N]), fmaxf(rr[2 * N], rr[3 * N]));
+                        const float m_new = fmaxf(m_use[h], tm);
+                        if (m_new > m_use[h] + kMoveThreshold) {
+                            alpha[h] = ex2(m_use[h] - m_new);     // 0 on the unit's first tile
+                            m_use[h] = m_new;
+                            l_part[h] *= alpha[h];
+                            rescale_o = true;
+                        }
+                    }
+                    rescale_o = rescale_o && (jj > 0);          // uniform: the warpgroup saw the same maxima
+                }
+                float p[kHPW];
+#pragma unroll
+                for (int h = 0; h < kHPW; ++h) {
+                    p[h] = ex2(x[h] - m_use[h]);
+                    l_part[h] += p[h];
+                }
+                if (T >= 1) {
+                    // previous PV done: P buffer free and this unit's O stable
+                    if (!wait_or_fail(&bar[P_FREE], (T - 1) & 1, a, err)) { ok = false; break; }
+                    tc_fence_after();
+                    if (rescale_o) {
+                        uint32_t o[kHPW];
+                        tmem_ld16(tO[ob] + lane_off + hs, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int h = 0; h < kHPW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+                        tmem_st16(tO[ob] + lane_off + hs, o);
+                        tmem_wait_st();
                     }
                 }
-                rescale_o = rescale_o && (j > 0);             // uniform: every thread saw the same maxima
-            }
-            float p[N];
-#pragma unroll
-            for (int h = 0; h < N; ++h) {
-                p[h] = ex2(x[h] - m_use[h]);
-                l_part[h] += p[h];
-            }
-            if (j >= 1) {
-                if (!wait_or_fail(&bar[P_FREE], (j - 1) & 1, a, err)) { ok = false; break; }
-                tc_fence_after();
-                if (rescale_o) {
-                    uint32_t o[N];
-                    tmem_ld_row<N>(tO + lane_off, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int h = 0; h < N; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-                    tmem_st_row<N>(tO + lane_off, o);
-                    tmem_wait_st();
-                }
-            }
-            // Rows past the history may hold anything (NaN included) and the tensor cores would form
-            // 0 * NaN: in a partial tile the masked tokens zero their own V row once it has landed.
-            if (t_end - (t_begin + j * kTok) < kTok) {
-                const int st = j % C::stages;
-                if (!valid) {
-                    if (!wait_or_fail(&bar[V_FULL + st], (j / C::stages) & 1, a, err)) { ok = false; break; }
+                // Rows past the history may hold anything (NaN included) and the tensor cores would form
+                // 0 * NaN: in a partial tile the masked tokens zero their own V row once it has landed.
+                if (wg == 0 && t_end - (t_begin + jj * kTok) < kTok && !valid) {
+                    const int st = T % C::stages;
+                    if (!wait_or_fail(&bar[V_FULL + st], (T / C::stages) & 1, a, err)) { ok = false; break; }
                     uint8_t *vrow = smem + st * C::stage_bytes + kTile + t * 128;
                     const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
@@ -381,98 +618,91 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant_
                         *reinterpret_cast<uint4 *>(vrow + kHalf + c * 16) = z;
                     }
                 }
-            }
-            // P^T, MN-major without swizzle: core matrices of 8 tokens x 8 heads (128 B).  Each weight is
-            // stored as hi = bf16(p) plus lo = bf16(p - hi), so the PV product sees p to about 2^-17.
+                // P^T, MN-major without swizzle: core matrices of 8 tokens x 8 heads (128 B), each weight
+                // as hi = bf16(p) plus lo = bf16(p - hi)
 #pragma unroll
-            for (int hb = 0; hb < N / 8; ++hb) {
-                uint32_t hi[4], lo[4];
+                for (int hb = 0; hb < kHPW / 8; ++hb) {
+                    uint32_t hi[4], lo[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float a0 = p[hb * 8 + 2 * e], a1 = p[hb * 8 + 2 * e + 1];
-                    hi[e] = pack2(a0, a1);
-                    lo[e] = pack2(a0 - bf16_lo(hi[e]), a1 - bf16_hi(hi[e]));
+                    for (int e = 0; e < 4; ++e) {
+                        const float a0 = p[hb * 8 + 2 * e], a1 = p[hb * 8 + 2 * e + 1];
+                        hi[e] = pack2(a0, a1);
+                        lo[e] = pack2(a0 - bf16_lo(hi[e]), a1 - bf16_hi(hi[e]));
+                    }
+                    uint8_t *dst = ps + (hs / 8 + hb) * 2048 + (t >> 3) * 128 + (t & 7) * 16;
+                    *reinterpret_cast<uint4 *>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(dst + C::p_bytes) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                 }
-                uint8_t *dst = ps + hb * 2048 + (t >> 3) * 128 + (t & 7) * 16;
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(dst + C::p_bytes) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bar[P_FULL]);
+                // the previous unit's epilogue, now that its last PV has long been issued
+                if (jj == 0 && pend && !epilogue()) { ok = false; break; }
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bar[P_FULL]);
-        }
-        // sums of the weights per head over the CTA's tokens
-        if (ok) {
+            if (!ok) break;
+            // this unit's weight sums per head, reduced over each warp's 32 tokens; the CTA-wide sum is
+            // finished in the (deferred) epilogue
 #pragma unroll
-            for (int h = 0; h < N; ++h) {
+            for (int h = 0; h < kHPW; ++h) {
                 float v = l_part[h];
                 v += __shfl_xor_sync(0xffffffffu, v, 16);
                 v += __shfl_xor_sync(0xffffffffu, v, 8);
                 v += __shfl_xor_sync(0xffffffffu, v, 4);
                 v += __shfl_xor_sync(0xffffffffu, v, 2);
                 v += __shfl_xor_sync(0xffffffffu, v, 1);
-                if (lane == 0) lsum[warp * N + h] = v;
+                if (lane == 0) lsum[ob * 4 * N + quarter * N + hs + h] = v;
             }
-            ok = group_sync(&bar[GRP], uses, a, err);
-        }
-        if (ok && wait_or_fail(&bar[O_FULL], 0, a, err)) {
-            tc_fence_after();
-            uint32_t o[N];
-            tmem_ld_row<N>(tO + lane_off, o);
-            tmem_wait_ld();
-            const int d = t;
+            pend = true;
+            pb = b;
+            pkvh = kvh;
+            psplit = split;
+            pob = ob;
 #pragma unroll
-            for (int h = 0; h < N; ++h) {
-                if (h >= g) break;
-                const float L = lsum[h] + lsum[N + h] + lsum[2 * N + h] + lsum[3 * N + h];
-                const float O = __uint_as_float(o[h]);
-                const size_t row = (size_t)b * a.Hq + h0 + h;
-                if (a.nsplit == 1) {
-                    a.out[row * kD + d] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
-                } else {
-                    const size_t prow = row * a.nsplit + split;
-                    a.part_o[prow * kD + d] = O;
-                    if (d == 0) {
-                        a.part_ml[prow * 2 + 0] = m_use[h];
-                        a.part_ml[prow * 2 + 1] = L;
-                    }
-                }
-            }
+            for (int h = 0; h < kHPW; ++h) pm[h] = m_use[h];
+            tcount += ntl;
+            ++icount;
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == mma_warp) {
         tc_fence_after();
         tmem_dealloc(tmem, C::tmem_cols);
     }
 }
 
 template <int N>
-cudaError_t launch_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeArgs &a, cudaStream_t stream)
+cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, const CUtensorMap &tmQ,
+                              const DecodeArgs &a, cudaStream_t stream)
 {
-    const int smem = TcCfg<N>::bytes + 1024;
+    const int smem = TcCfg<N>::bytes;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e =
+            cudaFuncSetAttribute(decode_persistent_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    dim3 grid(a.nsplit, a.Hkv, a.B);
-    decode_tc_kernel<N><<<grid, kThreads, smem, stream>>>(tmK, tmV, a);
+    decode_persistent_kernel<N><<<a.num_ctas, TcCfg<N>::threads, smem, stream>>>(tmK, tmV, tmQ, a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeArgs &a,
-                             cudaStream_t stream)
+cudaError_t launch_decode_plan(const DecodeArgs &a, cudaStream_t stream)
 {
-    if (a.group <= 16) return launch_tc<16>(tmK, tmV, a, stream);
-    if (a.group <= 32) return launch_tc<32>(tmK, tmV, a, stream);
+    decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(a, a.num_ctas);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, const CUtensorMap &tmQ,
+                             const DecodeArgs &a, cudaStream_t stream)
+{
+    if (a.group <= 16) return launch_persistent<16>(tmK, tmV, tmQ, a, stream);
+    if (a.group <= 32) return launch_persistent<32>(tmK, tmV, tmQ, a, stream);
     return cudaErrorInvalidValue;
 }
 

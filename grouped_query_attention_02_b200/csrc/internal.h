@@ -13,6 +13,7 @@ constexpr int kHeadDim = 128;       // the one head size this build implements
 constexpr int kDecodeTile = 64;     // tokens per TMA stage of the CUDA-core decode kernel
 constexpr int kDecodeCtasPerSm = 2; // resident CUDA-core decode CTAs per SM (shared-memory bound)
 constexpr int kStatusTimeout = 6;   // device status word: a bounded wait gave up
+constexpr int kStatusMisaligned = 3; // device status word: a kernel found its shared memory misaligned
 
 struct DecodeArgs {
     const __nv_bfloat16 *q;   // [B,Hq,d]
@@ -24,7 +25,28 @@ struct DecodeArgs {
     int B, Hq, Hkv, Tmax, group, chunk, nsplit, nhb;
     float qscale;             // scale * log2(e)
     unsigned long long wait_budget_ns;
+    // device-planned schedule (tensor-core path): see decode_tc.cu
+    int *plan_hdr;            // {claim counter, pieces, C}
+    int *nsplit_b;            // [B] pieces per sequence (the combine reads it when non-null)
+    int *plan_scratch;        // [B] planner scratch
+    int4 *items;              // [B * nsplit] pieces, longest first
+    int num_ctas;             // persistent CTAs (one per SM)
 };
+
+// Host plan of a decode call and the layout of its workspace.
+struct DecodePlan {
+    int tile, chunk, nsplit, hb, nhb;
+    bool tensor_cores;
+    size_t off_hdr, off_nsb, off_items, off_po, off_pml, ws_bytes;
+};
+// ws_budget bounds the split partials of the tensor-core path (more pieces per sequence when it allows).
+DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_t ws_budget);
+
+// Enqueues one decode (all kernels) on `stream` with the workspace `ws` laid out by `p`.
+// Returns 0 or a gqa_status code; adds the kernels launched to *launches.
+int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq, int Hkv,
+                   int Tmax, float scale, void *out, void *ws, const DecodePlan &p, int num_sms, int *status,
+                   cudaStream_t stream, int *launches, cudaEvent_t ev_before, cudaEvent_t ev_after);
 
 // How the decode of group size g is laid out: the kernel family (tensor cores for
 // 3 <= g <= 32, CUDA cores otherwise), its token tile (TMA box rows and split
@@ -39,11 +61,12 @@ struct DecodeShape {
 DecodeShape decode_shape(int g);
 int decode_heads_per_cta(int g);   // CUDA-core kernel only
 
-// Launches the decode kernel decode_shape(a.group) names; the tensor maps' box must be decode_shape().tile rows.
+// Launches the CUDA-core decode kernel (group sizes outside the tensor-core range).
 cudaError_t launch_decode_split(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeArgs &a,
                                 cudaStream_t stream);
-cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeArgs &a,
-                             cudaStream_t stream);
+cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, const CUtensorMap &tmQ,
+                             const DecodeArgs &a, cudaStream_t stream);
+cudaError_t launch_decode_plan(const DecodeArgs &a, cudaStream_t stream);
 cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t stream);
 cudaError_t launch_repeat_kv(const void *k, const void *v, const int32_t *seqlens, void *k_rep, void *v_rep,
                              int B, int Tmax, int Hq, int Hkv, cudaStream_t stream);

@@ -87,9 +87,11 @@ gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache, c
  * gqa_decode; the caller still owns and passes every input and output.  The
  * split-KV partials go to a fixed 32 MiB array compiled into the library,
  * which every GPU that loads the library holds until the process exits.
- *  - Returns GQA_ERR_UNSUPPORTED when the partials of this shape
- *    (workspace_bytes of gqa_decode_plan: B*Hq*nsplit*(d+2)*4 bytes) exceed
- *    32 MiB; gqa_decode handles such shapes.
+ *  - The split plan is gqa_decode's with the pieces per sequence reduced
+ *    until the workspace (split partials of about B*Hq*nsplit*(d+2)*4 bytes
+ *    plus the piece list) fits; returns GQA_ERR_UNSUPPORTED when even one
+ *    piece per sequence does not fit 32 MiB (B*Hq*(d+2)*4 bytes > 32 MiB);
+ *    gqa_decode handles such shapes.
  *  - The first call on a device looks up the array's device address once,
  *    with that device current; make that first call before any stream
  *    capture.
@@ -134,9 +136,12 @@ size_t gqa_decode_expanded_bytes(int B, int Tmax, int Hq, int d);
 
 /*
  * gqa_decode_plan -- the split-KV plan gqa_decode uses, for a device with
- * num_sms SMs: tokens per split (*chunk, a multiple of the 64-token tile),
- * number of splits (*nsplit) and workspace bytes it needs (*workspace_bytes,
- * 0 when nsplit == 1).  Pure host arithmetic; touches no device.
+ * num_sms SMs: tokens per split (*chunk, a multiple of the kernel's token
+ * tile), number of splits (*nsplit) and workspace bytes it needs
+ * (*workspace_bytes).  For group sizes 3..32 (the tensor-core kernel) the
+ * histories are cut on the device from the actual lengths: *chunk is then the
+ * smallest piece and *nsplit the most pieces one sequence can get, and the
+ * workspace also holds the piece list.  Pure host arithmetic; touches no device.
  */
 gqa_status gqa_decode_plan(int B, int Hq, int Hkv, int d, int Tmax, int num_sms, int *chunk, int *nsplit,
                            size_t *workspace_bytes);

@@ -101,7 +101,13 @@ def test_split_plan_covers_the_history(lib, w):
     chunk, nsplit, ws = gqa.gqa_decode_plan(w.B, w.Hq, w.Hkv, w.d, w.Tmax, 148)
     assert chunk % 64 == 0 and chunk > 0
     assert nsplit * chunk >= w.Tmax and (nsplit - 1) * chunk < w.Tmax
-    assert ws == (w.B * w.Hq * nsplit * (128 + 2) * 4 if nsplit > 1 else 0)
+    partials = w.B * w.Hq * nsplit * (128 + 2) * 4
+    if 3 <= w.group <= 32:
+        # tensor-core path: pieces are cut on the device from the real lengths (at most nsplit per
+        # sequence); the workspace also holds the piece list
+        assert ws >= partials
+    else:
+        assert ws == (partials if nsplit > 1 else 0)
 
 
 def test_split_plan_fills_the_machine(lib):

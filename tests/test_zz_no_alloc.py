@@ -55,13 +55,10 @@ def test_matches_gqa_decode_on_two_calls_in_a_row(shape):
 
 
 def test_rejects_partials_larger_than_the_fixed_scratch():
-    # 1100 sequences x 32 query heads over one KV head, 4096-token caches: on 148 SMs the plan
-    # splits each history in two and the partials need 34.9 MiB > 32 MiB
-    B, Hq, Hkv, Tmax = 1100, 32, 1, 4096
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
-    _, nsplit, ws = gqa.gqa_decode_plan(B, Hq, Hkv, 128, Tmax, sms)
-    if ws <= 32 << 20:
-        pytest.skip("this GPU's plan fits the scratch")
+    # 2048 sequences x 32 query heads: even one piece per sequence needs 2048*32*130*4 B = 34 MB of
+    # partials, more than the 32 MiB array
+    B, Hq, Hkv, Tmax = 2048, 32, 8, 256
+    assert B * Hq * (128 + 2) * 4 > 32 << 20
     q = torch.zeros((B, Hq, 128), dtype=torch.bfloat16, device=DEV)
     k = torch.empty((B, Tmax, Hkv, 128), dtype=torch.bfloat16, device=DEV)
     v = torch.empty_like(k)
