@@ -247,7 +247,7 @@ int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *s
         if ((s = cuda_status(launch_decode_tc(tmK, tmV, tmQ, a, stream))) != GQA_OK) return s;
         if (ev_after) cudaEventRecord(ev_after, stream);
         ++n;
-        if ((s = cuda_status(launch_decode_combine(a, stream))) != GQA_OK) return s;
+        if ((s = cuda_status(launch_decode_combine(a, stream, true))) != GQA_OK) return s;
         ++n;
     } else {
         if (ev_before) cudaEventRecord(ev_before, stream);

@@ -308,24 +308,53 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
 }
 
-// Merge the split partials of one (b, query head): out = sum_s o_s 2^(m_s-M) / sum_s l_s 2^(m_s-M).
+// Merge the split partials of one (b, query head):
+// out = sum_s o_s 2^(m_s-M) / sum_s l_s 2^(m_s-M), M = max_s m_s.  The (m, l) pairs are read by all
+// threads at once (one split per thread), the maximum and the weights go through shared memory, and
+// the weighted sum over o_s is unrolled so that its loads are in flight together.
 __global__ void __launch_bounds__(kD) decode_combine_kernel(const DecodeArgs a)
 {
+    // launched as a programmatic dependent of the split kernel: wait for its results
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ float wgt[kD];
+    __shared__ float red[kD / 32];
     const int h = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
     int T = a.seqlens[b];
     T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
     int nv = a.nsplit_b ? a.nsplit_b[b] : (T + a.chunk - 1) / a.chunk;
+    // with the device plan, a history of one piece (or none) was written out by the split kernel
+    if (a.nsplit_b && nv <= 1) return;
     nv = nv > a.nsplit ? a.nsplit : nv;
     const size_t row = (size_t)b * a.Hq + h;
     const float *ml = a.part_ml + row * a.nsplit * 2;
     const float *po = a.part_o + row * a.nsplit * kD;
+    // M = max over the splits
     float M = -INFINITY;
-    for (int s = 0; s < nv; ++s) M = fmaxf(M, ml[2 * s]);
+    for (int s = j; s < nv; s += kD) M = fmaxf(M, ml[2 * s]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if ((j & 31) == 0) red[j >> 5] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
     float Lsum = 0.f, O = 0.f;
-    for (int s = 0; s < nv; ++s) {
-        const float f = ex2(ml[2 * s] - M);
-        Lsum += ml[2 * s + 1] * f;
-        O += po[(size_t)s * kD + j] * f;
+    for (int c = 0; c < nv; c += kD) {
+        const int n = min(kD, nv - c);
+        __syncthreads();
+        if (j < n) wgt[j] = ex2(ml[2 * (c + j)] - M);
+        __syncthreads();
+        int s = 0;
+        for (; s + 4 <= n; s += 4) {
+            const float o0 = po[(size_t)(c + s + 0) * kD + j], o1 = po[(size_t)(c + s + 1) * kD + j];
+            const float o2 = po[(size_t)(c + s + 2) * kD + j], o3 = po[(size_t)(c + s + 3) * kD + j];
+            const float l0 = ml[2 * (c + s + 0) + 1], l1 = ml[2 * (c + s + 1) + 1];
+            const float l2 = ml[2 * (c + s + 2) + 1], l3 = ml[2 * (c + s + 3) + 1];
+            O += o0 * wgt[s] + o1 * wgt[s + 1] + o2 * wgt[s + 2] + o3 * wgt[s + 3];
+            Lsum += l0 * wgt[s] + l1 * wgt[s + 1] + l2 * wgt[s + 2] + l3 * wgt[s + 3];
+        }
+        for (; s < n; ++s) {
+            O += po[(size_t)(c + s) * kD + j] * wgt[s];
+            Lsum += ml[2 * (c + s) + 1] * wgt[s];
+        }
     }
     a.out[row * kD + j] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
 }
@@ -427,11 +456,18 @@ cudaError_t launch_decode_split(const CUtensorMap &tmK, const CUtensorMap &tmV, 
     }
 }
 
-cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t stream)
+cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t stream, bool pdl)
 {
-    dim3 grid(a.Hq, a.B);
-    decode_combine_kernel<<<grid, kD, 0, stream>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.Hq, a.B);
+    cfg.blockDim = dim3(kD);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_combine_kernel, a);
 }
 
 cudaError_t launch_repeat_kv(const void *k, const void *v, const int32_t *seqlens, void *k_rep, void *v_rep,

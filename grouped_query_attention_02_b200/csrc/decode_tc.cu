@@ -20,8 +20,11 @@
 // C chosen from the total work so that there are about eight rounds of pieces,
 // and lists the pieces longest first.  decode_persistent_kernel then runs one
 // CTA per SM; each CTA claims (piece, KV head) units from an atomic counter
-// and keeps its TMA / MMA / softmax pipeline running across units, writing
-// one partial result (o, m, l) per unit; decode_combine_kernel merges them.
+// and keeps its TMA / MMA / softmax pipeline running across units.  A unit
+// that covers its whole history writes the output; otherwise it writes a
+// partial result (o, m, l) that decode_combine_kernel merges.  The three
+// kernels are chained with programmatic dependent launch, so each one's
+// launch and prologue overlap the previous one.
 //
 // The softmax runs on one 128-thread warpgroup per 16 heads, one token per
 // thread (TMEM lane = token for S^T, lane = d for O^T).  The running maximum
@@ -190,6 +193,8 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     __shared__ int s_C, s_sum;
     int *full_off = a.plan_scratch;     // per-sequence offsets of the full pieces (B ints, global)
 
+    // the persistent kernel may start its prologue now; it reads this plan only after griddepcontrol.wait
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     long long tot = 0;
     int mx = 0;
@@ -255,6 +260,11 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
         const int tl = (T + kTok - 1) / kTok;
         const int full = tl / C, rem = tl % C;
+        if (tl == 0) {
+            // no cached token: no unit will touch this sequence, its output rows are zero
+            uint4 *o = reinterpret_cast<uint4 *>(a.out + (size_t)b * a.Hq * kD);
+            for (int i = 0; i < a.Hq * kD / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
+        }
         for (int s = 0; s < full; ++s)
             a.items[full_off[b] + s] = make_int4(b, s, s * C * kTok, min((s + 1) * C * kTok, T));
         if (rem > 0) {
@@ -331,6 +341,10 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // everything below may read what decode_plan_kernel wrote; the combine kernel may be scheduled
+    // now (it waits for this grid to finish before it reads anything)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS[2] = {tmem, tmem + N};
     const uint32_t tO[2] = {tmem + 2 * N, tmem + 3 * N};
@@ -495,16 +509,30 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             tmem_wait_ld();
             const float *ls = lsum + pob * 4 * N;
             const int d = t;
+            const int npieces = a.nsplit_b[pb];
+            if (npieces == 1) {
+                // the whole history in one unit: normalise and write the output
 #pragma unroll
-            for (int h = 0; h < kHPW; ++h) {
-                const int hg = hs + h;
-                if (hg >= g) break;
-                const float L = ls[hg] + ls[N + hg] + ls[2 * N + hg] + ls[3 * N + hg];
-                const size_t prow = ((size_t)pb * a.Hq + pkvh * g + hg) * a.nsplit + psplit;
-                a.part_o[prow * kD + d] = __uint_as_float(o[h]);
-                if (d == 0) {
-                    a.part_ml[prow * 2 + 0] = pm[h];
-                    a.part_ml[prow * 2 + 1] = L;
+                for (int h = 0; h < kHPW; ++h) {
+                    const int hg = hs + h;
+                    if (hg >= g) break;
+                    const float L = ls[hg] + ls[N + hg] + ls[2 * N + hg] + ls[3 * N + hg];
+                    const float O = __uint_as_float(o[h]);
+                    a.out[((size_t)pb * a.Hq + pkvh * g + hg) * kD + d] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+                }
+            } else {
+                // one piece of several: a partial (o, m, l) for decode_combine_kernel
+#pragma unroll
+                for (int h = 0; h < kHPW; ++h) {
+                    const int hg = hs + h;
+                    if (hg >= g) break;
+                    const float L = ls[hg] + ls[N + hg] + ls[2 * N + hg] + ls[3 * N + hg];
+                    const size_t prow = ((size_t)pb * a.Hq + pkvh * g + hg) * a.nsplit + psplit;
+                    a.part_o[prow * kD + d] = __uint_as_float(o[h]);
+                    if (d == 0) {
+                        a.part_ml[prow * 2 + 0] = pm[h];
+                        a.part_ml[prow * 2 + 1] = L;
+                    }
                 }
             }
             tc_fence_before();
@@ -686,8 +714,19 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
-    decode_persistent_kernel<N><<<a.num_ctas, TcCfg<N>::threads, smem, stream>>>(tmK, tmV, tmQ, a);
-    return cudaGetLastError();
+    // programmatic dependent launch: the prologue overlaps decode_plan_kernel, which the kernel
+    // waits for (griddepcontrol.wait) before reading the plan
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.num_ctas);
+    cfg.blockDim = dim3(TcCfg<N>::threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_persistent_kernel<N>, tmK, tmV, tmQ, a);
 }
 
 }  // namespace

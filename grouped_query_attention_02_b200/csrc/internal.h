@@ -67,7 +67,8 @@ cudaError_t launch_decode_split(const CUtensorMap &tmK, const CUtensorMap &tmV, 
 cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, const CUtensorMap &tmQ,
                              const DecodeArgs &a, cudaStream_t stream);
 cudaError_t launch_decode_plan(const DecodeArgs &a, cudaStream_t stream);
-cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t stream);
+// pdl: launched as a programmatic dependent of the previous kernel on the stream
+cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t stream, bool pdl = false);
 cudaError_t launch_repeat_kv(const void *k, const void *v, const int32_t *seqlens, void *k_rep, void *v_rep,
                              int B, int Tmax, int Hq, int Hkv, cudaStream_t stream);
 cudaError_t launch_wait_timeout_selftest(int *status, unsigned long long budget_ns, cudaStream_t stream);
