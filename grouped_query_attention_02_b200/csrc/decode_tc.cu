@@ -72,7 +72,8 @@ struct TcCfg {
     static constexpr int tmem_off = bar_off + nbars * 8;
     static constexpr int err_off = tmem_off + 8;
     static constexpr int bytes = err_off + 8;
-    static constexpr uint32_t tmem_cols = (4 * N <= 64) ? 64 : 128;   // S[2] and O[2], N columns each
+    // S[2] (N columns each) and O[2] (2N columns each: the hi and lo products side by side)
+    static constexpr uint32_t tmem_cols = (6 * N <= 128) ? 128 : 256;
     static_assert(bytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -347,7 +348,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS[2] = {tmem, tmem + N};
-    const uint32_t tO[2] = {tmem + 2 * N, tmem + 3 * N};
+    const uint32_t tO[2] = {tmem + 2 * N, tmem + 4 * N};   // columns [0,N): V^T P_hi^T, [N,2N): V^T P_lo^T
 
     if (warp == producer_warp) {
         // ---------------- claims units, loads the group's query rows and streams the K/V tiles
@@ -416,7 +417,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         // ---------------- MMA issuer
         if (lane == 0) {
             const uint32_t idesc_s = umma_idesc_bf16(kTok, N, 0, 0);   // K (K-major) . Q^T (K-major)
-            const uint32_t idesc_o = umma_idesc_bf16(kD, N, 1, 1);     // V^T (MN-major) . P^T (MN-major)
+            const uint32_t idesc_o = umma_idesc_bf16(kD, 2 * N, 1, 1); // V^T (MN-major) . [P_hi | P_lo]^T (MN-major)
             const uint32_t p_addr = smem_u32(ps);
             int tcount = 0, icount = 0;
             bool ok = true;
@@ -459,17 +460,15 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                         if (!wait_or_fail(&bar[V_FULL + s], (T / C::stages) & 1, a, err)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t v_addr = smem_u32(smem + s * C::stage_bytes + kTile);
-                        // O^T += V^T P_hi^T + V^T P_lo^T: the weights carried as a sum of two bf16 terms
+                        // [O_hi | O_lo] += V^T [P_hi | P_lo]^T in one product of width 2N: the lo blocks
+                        // follow the hi blocks at the same 2048-byte stride, so they are simply more columns
 #pragma unroll
-                        for (int part = 0; part < 2; ++part) {
-#pragma unroll
-                            for (int ks = 0; ks < kTok / 16; ++ks) {
-                                // A = V^T: 16 tokens (two 8-row groups, 1024 B apart), 64-column blocks kHalf apart
-                                // B = P^T: 16 tokens (two 128-byte core-matrix groups), 8-head blocks 2048 B apart
-                                umma_bf16_ss(tO[ob], umma_smem_desc(v_addr + ks * 2048, kHalf, 1024, 2),
-                                             umma_smem_desc(p_addr + part * C::p_bytes + ks * 256, 128, 2048, 0),
-                                             idesc_o, (jj > 1 || part > 0 || ks > 0) ? 1u : 0u);
-                            }
+                        for (int ks = 0; ks < kTok / 16; ++ks) {
+                            // A = V^T: 16 tokens (two 8-row groups, 1024 B apart), 64-column blocks kHalf apart
+                            // B = P^T: 16 tokens (two 128-byte core-matrix groups), 8-head blocks 2048 B apart
+                            umma_bf16_ss(tO[ob], umma_smem_desc(v_addr + ks * 2048, kHalf, 1024, 2),
+                                         umma_smem_desc(p_addr + ks * 256, 128, 2048, 0), idesc_o,
+                                         (jj > 1 || ks > 0) ? 1u : 0u);
                         }
                         umma_commit(&bar[P_FREE]);
                         umma_commit(&bar[KV_EMPTY + s]);
@@ -504,9 +503,12 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             if (!group_sync(&bar[GRP + wg], uses, a, err)) return false;      // lsum[pob] complete
             if (!wait_or_fail(&bar[O_FULL + pob], (((icount - 1) >> 1)) & 1, a, err)) return false;
             tc_fence_after();
-            uint32_t o[kHPW];
+            uint32_t o[kHPW], olo[kHPW];
             tmem_ld16(tO[pob] + lane_off + hs, o);
+            tmem_ld16(tO[pob] + lane_off + N + hs, olo);
             tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < kHPW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) + __uint_as_float(olo[h]));
             const float *ls = lsum + pob * 4 * N;
             const int d = t;
             const int npieces = a.nsplit_b[pb];
@@ -624,12 +626,15 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     if (!wait_or_fail(&bar[P_FREE], (T - 1) & 1, a, err)) { ok = false; break; }
                     tc_fence_after();
                     if (rescale_o) {
-                        uint32_t o[kHPW];
-                        tmem_ld16(tO[ob] + lane_off + hs, o);
-                        tmem_wait_ld();
 #pragma unroll
-                        for (int h = 0; h < kHPW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-                        tmem_st16(tO[ob] + lane_off + hs, o);
+                        for (int part = 0; part < 2; ++part) {   // the hi and the lo columns
+                            uint32_t o[kHPW];
+                            tmem_ld16(tO[ob] + lane_off + part * N + hs, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int h = 0; h < kHPW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+                            tmem_st16(tO[ob] + lane_off + part * N + hs, o);
+                        }
                         tmem_wait_st();
                     }
                 }
