@@ -459,7 +459,7 @@ def main():
         "tokens_per_s": tokens_per_s, "frac_of_hbm_peak_step": value / max(world, 1) / peaks["hbm_gbs"],
         "gpu_launches": launches, "device_status": status,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": profile_traffic("decode_tc_qwen3_8b.md"),
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": profile_traffic("decode_persistent_qwen3_8b.md"),
                      "kernel": decode_kernel_name(w.group), "kernel_ms": kern_ms, "algorithmic_bytes": alg_bytes,
                      "peak_source": f"{peaks.get('source')} hbm_gbs (copy bandwidth)"},
         "clocks": clk.summary(),

@@ -22,11 +22,12 @@
  *  - Host-side argument checks run before anything is enqueued; a failed
  *    check returns its status and enqueues nothing.  A CUDA launch error is
  *    returned as GQA_ERR_CUDA.
- *  - The library keeps, per device, a grow-only workspace for split-KV
- *    partial results (allocated with cudaMalloc on first need) and a cache of
- *    TMA tensor maps keyed by pointer and shape.  gqa_release() frees both.
- *    Calls that share the workspace on one device must be ordered on one
- *    stream (or otherwise serialised by the caller).
+ *  - The library keeps, per device, a grow-only workspace for the split-KV
+ *    plan and partial results (allocated with cudaMalloc on first need);
+ *    gqa_release() frees it.  TMA tensor maps are encoded on the host for
+ *    every call (kernel parameters, nothing is cached).  Calls that share the
+ *    workspace on one device must be ordered on one stream (or otherwise
+ *    serialised by the caller).
  *  - Only head_dim d == 128 is implemented (GQA_ERR_UNSUPPORTED otherwise).
  */
 #ifndef GQA_H_
@@ -66,8 +67,12 @@ typedef enum gqa_status {
  * sequence with seqlens[b] == 0 gets an all-zero output row.
  *
  * Each K/V tile is fetched once by TMA and shared by the g query heads of its
- * group.  Long or uneven histories are split across CTAs (split-KV) and the
- * partial results merged by a second kernel, through the library workspace.
+ * group.  For 3 <= g <= 32 the products run on the tcgen05 tensor cores and
+ * the histories are cut into pieces on the device from the actual lengths
+ * (longest first), processed by one persistent CTA per SM; pieces of one
+ * history are merged by a log-sum-exp combine kernel.  Other group sizes use
+ * a CUDA-core kernel with a host-side split.  Either way the work goes
+ * through the library workspace.
  */
 gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens,
                       int B, int Hq, int Hkv, int d, int Tmax, float scale, void *out, void *stream);
@@ -150,7 +155,9 @@ gqa_status gqa_decode_plan(int B, int Hq, int Hkv, int d, int Tmax, int num_sms,
  * gqa_get_last_device_status -- synchronises `stream`, then reads and clears
  * the device's status word.  Kernels never trap: a kernel that gives up a
  * bounded wait (about a second) records GQA_ERR_DEVICE_TIMEOUT there and
- * returns.  Returns GQA_OK when nothing was recorded, GQA_ERR_CUDA when the
+ * returns; one that finds its shared-memory window not 1024-byte aligned
+ * (which the 128-byte swizzle needs) records GQA_ERR_MISALIGNED and does
+ * nothing.  Returns GQA_OK when nothing was recorded, GQA_ERR_CUDA when the
  * synchronisation itself failed.
  */
 gqa_status gqa_get_last_device_status(void *stream);
