@@ -12,6 +12,11 @@ attention arithmetic.  Recipe (the same for every workload):
   ``poison=True`` (a read past the end then shows up as NaN in the output);
 * ``q_gain`` multiplies q before rounding (a "peaky" softmax when > 1).
 
+FP8 caches (``make_decode_fp8``): the same N(0, 1) draws divided by a
+per-tensor scale, clamped to the largest finite E4M3 value (448) and stored as
+E4M3 codes (torch's float8_e4m3fn cast, round to nearest even); rows past the
+history hold the NaN code 0x7F when ``poison=True``.
+
 Layouts are the ones of the C ABI: decode q [B,Hq,d], caches [B,Tmax,Hkv,d];
 prefill q [B,S,Hq,d], k/v [B,S,Hkv,d].
 """
@@ -97,6 +102,61 @@ def make_decode(B: int, Hq: int, Hkv: int, d: int, Tmax: int, seqlens=None, *, d
     if scale is None:
         scale = 1.0 / float(d) ** 0.5
     return DecodeInputs(q, k, v, sl.to(device), scale)
+
+
+@dataclass
+class DecodeFp8Inputs:
+    q: torch.Tensor          # [B,Hq,d] bf16
+    k_cache: torch.Tensor    # [B,Tmax,Hkv,d] uint8, E4M3 codes
+    v_cache: torch.Tensor    # [B,Tmax,Hkv,d] uint8, E4M3 codes
+    k_scale: float           # a key is e4m3(code) * k_scale
+    v_scale: float           # a value is e4m3(code) * v_scale
+    seqlens: torch.Tensor    # [B] int32, same device as q
+    scale: float
+
+
+def _normal_e4m3(shape, seed: int, device, inv_scale: float) -> torch.Tensor:
+    """N(0,1) / scale, clamped to +-448 and cast to E4M3 codes, drawn in slices."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    out = torch.empty(shape, dtype=torch.uint8, device=device)
+    flat = out.view(-1)
+    step = 1 << 27
+    tmp = torch.empty(min(step, max(flat.numel(), 1)), dtype=torch.float32, device=device)
+    for s in range(0, flat.numel(), step):
+        n = min(step, flat.numel() - s)
+        t = tmp[:n]
+        t.normal_(generator=g)
+        t.mul_(inv_scale).clamp_(-448.0, 448.0)
+        flat[s:s + n].copy_(t.to(torch.float8_e4m3fn).view(torch.uint8))
+    return out
+
+
+def make_decode_fp8(B: int, Hq: int, Hkv: int, d: int, Tmax: int, seqlens=None, *, device="cpu",
+                    seed: int = 0, scale: float | None = None, poison: bool = False, q_gain: float = 1.0,
+                    seqlen_range=None, k_scale: float = 0.0135, v_scale: float = 0.0142) -> DecodeFp8Inputs:
+    """Decode inputs over an FP8 (E4M3) cache with per-tensor scales; ``seqlens`` as in make_decode.
+    The default scales map about six standard deviations onto the largest E4M3 value."""
+    if seqlen_range is not None:
+        sl = seqlens_uniform(B, seqlen_range[0], seqlen_range[1], seed + 3)
+    elif seqlens is None:
+        sl = torch.full((B,), Tmax, dtype=torch.int32)
+    elif isinstance(seqlens, int):
+        sl = torch.full((B,), seqlens, dtype=torch.int32)
+    else:
+        sl = torch.as_tensor(seqlens, dtype=torch.int32).cpu()
+    q = _normal((B, Hq, d), seed + 0, device, q_gain)
+    k = _normal_e4m3((B, Tmax, Hkv, d), seed + 1, device, 1.0 / k_scale)
+    v = _normal_e4m3((B, Tmax, Hkv, d), seed + 2, device, 1.0 / v_scale)
+    if poison:
+        for b in range(B):
+            t = int(sl[b])
+            if t < Tmax:
+                k[b, t:].fill_(0x7F)
+                v[b, t:].fill_(0x7F)
+    if scale is None:
+        scale = 1.0 / float(d) ** 0.5
+    return DecodeFp8Inputs(q, k, v, float(k_scale), float(v_scale), sl.to(device), scale)
 
 
 @dataclass

@@ -63,6 +63,19 @@ def _bits(x) -> np.ndarray:
     return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
 
 
+def _bytes(x) -> np.ndarray:
+    """FP8 tensor (torch float8_e4m3fn or uint8, any device) or uint8 array -> contiguous uint8 numpy."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint8
+        return np.ascontiguousarray(x)
+    import torch
+
+    t = x.detach().cpu().contiguous()
+    if t.dtype != torch.uint8:
+        t = t.view(torch.uint8)
+    return np.ascontiguousarray(t.numpy())
+
+
 class Oracle:
     """ctypes view of one compiled copy of gqa_oracle.c."""
 
@@ -77,6 +90,11 @@ class Oracle:
         lib.gqa_oracle_decode.restype = ctypes.c_int
         lib.gqa_oracle_decode.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 5 + [
             ctypes.c_double, ctypes.c_void_p, ctypes.c_int]
+        lib.gqa_oracle_e4m3_to_f64.restype = None
+        lib.gqa_oracle_e4m3_to_f64.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong]
+        lib.gqa_oracle_decode_fp8.restype = ctypes.c_int
+        lib.gqa_oracle_decode_fp8.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_double] * 2 + [ctypes.c_void_p] + [
+            ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_void_p, ctypes.c_int]
         lib.gqa_oracle_prefill.restype = ctypes.c_int
         lib.gqa_oracle_prefill.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 5 + [
             ctypes.c_double, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p, ctypes.c_int]
@@ -92,6 +110,29 @@ class Oracle:
         b = np.ascontiguousarray(bits, dtype=np.uint16)
         out = np.empty(b.shape, dtype=np.float64)
         self.lib.gqa_oracle_bf16_to_f64(b.ctypes.data, out.ctypes.data, b.size)
+        return out
+
+    def e4m3_to_f64(self, bytes_: np.ndarray) -> np.ndarray:
+        b = np.ascontiguousarray(bytes_, dtype=np.uint8)
+        out = np.empty(b.shape, dtype=np.float64)
+        self.lib.gqa_oracle_e4m3_to_f64(b.ctypes.data, out.ctypes.data, b.size)
+        return out
+
+    def decode_fp8(self, q, k8, v8, k_scale: float, v_scale: float, seqlens, scale: float,
+                   nthreads: int | None = None) -> np.ndarray:
+        """q [B,Hq,d] bf16; k8/v8 [B,Tmax,Hkv,d] E4M3 bytes (uint8 or float8_e4m3fn) -> out fp64."""
+        qb, kb, vb = _bits(q), _bytes(k8), _bytes(v8)
+        B, Hq, d = qb.shape
+        B2, Tmax, Hkv, d2 = kb.shape
+        assert B2 == B and d2 == d and vb.shape == kb.shape
+        sl = np.ascontiguousarray(np.asarray(
+            seqlens.cpu().numpy() if hasattr(seqlens, "cpu") else seqlens, dtype=np.int32))
+        out = np.zeros((B, Hq, d), dtype=np.float64)
+        st = self.lib.gqa_oracle_decode_fp8(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, float(k_scale),
+                                            float(v_scale), sl.ctypes.data, B, Hq, Hkv, d, Tmax, float(scale),
+                                            out.ctypes.data, nthreads or default_threads())
+        if st != 0:
+            raise ValueError(f"oracle fp8 decode rejected its arguments (status {st})")
         return out
 
     def decode(self, q, k_cache, v_cache, seqlens, scale: float, nthreads: int | None = None) -> np.ndarray:
@@ -159,6 +200,14 @@ def bf16_bits_to_f64(bits):
 
 def decode(q, k_cache, v_cache, seqlens, scale, nthreads=None):
     return _get().decode(q, k_cache, v_cache, seqlens, scale, nthreads)
+
+
+def e4m3_to_f64(bytes_):
+    return _get().e4m3_to_f64(bytes_)
+
+
+def decode_fp8(q, k8, v8, k_scale, v_scale, seqlens, scale, nthreads=None):
+    return _get().decode_fp8(q, k8, v8, k_scale, v_scale, seqlens, scale, nthreads)
 
 
 def prefill_causal(q, k, v, scale, rows=None, nthreads=None):

@@ -27,6 +27,10 @@
  *  - Causal prefill: row r attends to tokens t <= r (lower triangle including
  *    the diagonal), masked scores excluded from the softmax: same section,
  *    the tril mask of its example.
+ *  - FP8 KV cache: the cache stored in FP8 instead of bf16 ("Other ways to
+ *    shrink the KV cache", anrans.github.io attention-variants: K and V in
+ *    FP8, as serving engines support); every element is the E4M3 value of its
+ *    byte times a per-tensor scale, and the attention is the same as above.
  *
  * Everything is done in double precision.  Inputs are the bf16 bit patterns
  * the GPU sees; bf16 is the upper 16 bits of an IEEE-754 binary32, so the
@@ -86,6 +90,24 @@ void gqa_oracle_bf16_to_f64(const uint16_t *x, double *y, long long n)
     for (long long i = 0; i < n; ++i) y[i] = bf16_to_double(x[i]);
 }
 
+/* FP8 E4M3 (the "fn" variant: no infinities) byte -> double, from the format's
+ * definition: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits;
+ * exponent 0 encodes subnormals m * 2^-9; exponent 15 with mantissa 7 is NaN. */
+static double e4m3_to_double(uint8_t x)
+{
+    const int sign = (x >> 7) & 1, e = (x >> 3) & 0xF, m = x & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+void gqa_oracle_e4m3_to_f64(const uint8_t *x, double *y, long long n)
+{
+    for (long long i = 0; i < n; ++i) y[i] = e4m3_to_double(x[i]);
+}
+
 /* ---- one query row against an explicit per-head copy of K and V --------- */
 
 /* out[0:d] = sum_t softmax_t(scale * q.K[t]) V[t] over t < n, two-pass.
@@ -126,6 +148,9 @@ typedef struct {
     double *out;
     int tid, nthreads;
     int status;
+    /* FP8 caches (k8, v8 non-NULL): element value = e4m3(byte) * k_scale (or v_scale) */
+    const uint8_t *k8, *v8;
+    double k_scale, v_scale;
 } decode_job;
 
 static void *decode_worker(void *arg)
@@ -150,8 +175,13 @@ static void *decode_worker(void *arg)
         for (long long t = 0; t < T; ++t) {
             size_t src = (((size_t)b * J->Tmax + (size_t)t) * J->Hkv + (size_t)kvh) * (size_t)d;
             for (int j = 0; j < d; ++j) {
-                Kh[t * d + j] = bf16_to_double(J->k[src + j]);
-                Vh[t * d + j] = bf16_to_double(J->v[src + j]);
+                if (J->k8) {
+                    Kh[t * d + j] = e4m3_to_double(J->k8[src + j]) * J->k_scale;
+                    Vh[t * d + j] = e4m3_to_double(J->v8[src + j]) * J->v_scale;
+                } else {
+                    Kh[t * d + j] = bf16_to_double(J->k[src + j]);
+                    Vh[t * d + j] = bf16_to_double(J->v[src + j]);
+                }
             }
         }
         size_t qo = ((size_t)b * J->Hq + (size_t)h) * (size_t)d;
@@ -162,13 +192,36 @@ static void *decode_worker(void *arg)
     return NULL;
 }
 
+static int run_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint8_t *k8,
+                      const uint8_t *v8, double k_scale, double v_scale, const int32_t *seqlens, int B,
+                      int Hq, int Hkv, int d, int Tmax, double scale, double *out, int nthreads);
+
 /* q [B,Hq,d], k/v [B,Tmax,Hkv,d] bf16 bits, seqlens [B] (0 <= seqlens <= Tmax),
  * out [B,Hq,d] fp64.  Returns 0 on success. */
 int gqa_oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                       const int32_t *seqlens, int B, int Hq, int Hkv, int d, int Tmax,
                       double scale, double *out, int nthreads)
 {
-    if (!q || !k || !v || !seqlens || !out) return ORACLE_BAD_ARG;
+    if (!k || !v) return ORACLE_BAD_ARG;
+    return run_decode(q, k, v, NULL, NULL, 1.0, 1.0, seqlens, B, Hq, Hkv, d, Tmax, scale, out, nthreads);
+}
+
+/* The same decode over an FP8 (E4M3) cache with per-tensor scales: every cached
+ * element is e4m3(byte) * k_scale (keys) or e4m3(byte) * v_scale (values). */
+int gqa_oracle_decode_fp8(const uint16_t *q, const uint8_t *k8, const uint8_t *v8, double k_scale,
+                          double v_scale, const int32_t *seqlens, int B, int Hq, int Hkv, int d, int Tmax,
+                          double scale, double *out, int nthreads)
+{
+    if (!k8 || !v8) return ORACLE_BAD_ARG;
+    return run_decode(q, NULL, NULL, k8, v8, k_scale, v_scale, seqlens, B, Hq, Hkv, d, Tmax, scale, out,
+                      nthreads);
+}
+
+static int run_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint8_t *k8,
+                      const uint8_t *v8, double k_scale, double v_scale, const int32_t *seqlens, int B,
+                      int Hq, int Hkv, int d, int Tmax, double scale, double *out, int nthreads)
+{
+    if (!q || !seqlens || !out) return ORACLE_BAD_ARG;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0 || Tmax < 0) return ORACLE_BAD_ARG;
     if (Hq % Hkv != 0) return ORACLE_BAD_ARG;
     for (int b = 0; b < B; ++b)
@@ -179,7 +232,8 @@ int gqa_oracle_decode(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
     if (!jobs || !th) { free(jobs); free(th); return ORACLE_NO_MEMORY; }
     for (int i = 0; i < nthreads; ++i) {
-        decode_job J = {q, k, v, seqlens, B, Hq, Hkv, d, Tmax, scale, out, i, nthreads, ORACLE_OK};
+        decode_job J = {q, k, v, seqlens, B, Hq, Hkv, d, Tmax, scale, out, i, nthreads, ORACLE_OK,
+                        k8, v8, k_scale, v_scale};
         jobs[i] = J;
     }
     for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, decode_worker, &jobs[i]);

@@ -37,6 +37,14 @@ MUTANTS = {
     "prefill key cache indexed with S and Hq": (
         "size_t src = (((size_t)b * S + (size_t)t) * J->Hkv + (size_t)kvh) * (size_t)d;",
         "size_t src = (((size_t)b * S + (size_t)t) * J->Hq + (size_t)kvh) * (size_t)d;"),
+    "e4m3 exponent bias 8": ("else v = ldexp(1.0 + m / 8.0, e - 7);", "else v = ldexp(1.0 + m / 8.0, e - 8);"),
+    "e4m3 subnormals one binade low": ("if (e == 0) v = ldexp((double)m, -9);",
+                                       "if (e == 0) v = ldexp((double)m, -10);"),
+    "e4m3 NaN code read as a number": ("if (e == 15 && m == 7) return NAN;", "if (e == 16) return NAN;"),
+    "fp8 key scale dropped": ("Kh[t * d + j] = e4m3_to_double(J->k8[src + j]) * J->k_scale;",
+                              "Kh[t * d + j] = e4m3_to_double(J->k8[src + j]);"),
+    "fp8 values scaled by the key scale": ("Vh[t * d + j] = e4m3_to_double(J->v8[src + j]) * J->v_scale;",
+                                           "Vh[t * d + j] = e4m3_to_double(J->v8[src + j]) * J->k_scale;"),
 }
 
 

@@ -312,3 +312,73 @@ def test_tight_tolerance_sees_one_dropped_token(oracle_mod):
     short = oracle_mod.decode(x.q, x.k_cache, x.v_cache, [255], x.scale)
     assert compare(short, full)["tight_violations"] > 0
     assert compare(full, full)["tight_violations"] == 0
+
+
+# ---------------------------------------------------------------- FP8 (E4M3) KV cache
+
+
+def _e4m3_f64(codes):
+    """torch's own E4M3 -> float64 conversion (a library routine, independent of the oracle)."""
+    t = torch.as_tensor(np.asarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def test_e4m3_conversion_exhaustive(oracle_mod):
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle_mod.e4m3_to_f64(codes)
+    ref = _e4m3_f64(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
+    assert np.array_equal(np.signbit(got[ok]), np.signbit(ref[ok]))   # 0x80 is -0
+
+
+def test_e4m3_format_constants(oracle_mod):
+    """Fixed points of the E4M3 format (1 sign, 4 exponent bits biased by 7, 3 mantissa bits,
+    no infinities): zero, the smallest subnormal 2^-9, the largest subnormal 7 * 2^-9, the smallest
+    normal 2^-6, one, the largest finite value 448, and the two NaN codes."""
+    codes = [0x00, 0x01, 0x07, 0x08, 0x38, 0x7E, 0xFE, 0xB8, 0x7F, 0xFF]
+    got = oracle_mod.e4m3_to_f64(np.array(codes, dtype=np.uint8))
+    want = [0.0, 2.0 ** -9, 7 * 2.0 ** -9, 2.0 ** -6, 1.0, 448.0, -448.0, -1.0]
+    assert list(got[:8]) == want
+    assert np.isnan(got[8]) and np.isnan(got[9])
+
+
+def test_fp8_decode_at_unit_scales_equals_the_bf16_decode(oracle_mod):
+    """Every finite E4M3 value is exact in bf16, so at unit scales the FP8 decode is the bf16 decode
+    of the widened cache, bit for bit."""
+    x = inputs.make_decode_fp8(3, 8, 2, 16, 11, seqlens=[11, 4, 0], seed=51, k_scale=1.0, v_scale=1.0)
+    got = oracle_mod.decode_fp8(x.q, x.k_cache, x.v_cache, 1.0, 1.0, x.seqlens, x.scale)
+    kb = x.k_cache.view(torch.float8_e4m3fn).to(torch.bfloat16)
+    vb = x.v_cache.view(torch.float8_e4m3fn).to(torch.bfloat16)
+    ref = oracle_mod.decode(x.q, kb, vb, x.seqlens, x.scale)
+    np.testing.assert_array_equal(got, ref)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (6, 1)])
+def test_fp8_decode_with_scales_equals_library_sdpa(oracle_mod, Hq, Hkv):
+    """Keys scale the scores and values scale the output: torch SDPA in fp64 on the dequantised
+    cache (torch's E4M3 conversion times the per-tensor scales)."""
+    d, T = 16, 10
+    lens = [10, 3]
+    ks, vs = 0.0213, 0.37
+    x = inputs.make_decode_fp8(2, Hq, Hkv, d, T, seqlens=lens, seed=52 + Hq, k_scale=ks, v_scale=vs)
+    got = oracle_mod.decode_fp8(x.q, x.k_cache, x.v_cache, ks, vs, x.seqlens, x.scale)
+    g = Hq // Hkv
+    k = torch.from_numpy(_e4m3_f64(x.k_cache.numpy())) * ks
+    v = torch.from_numpy(_e4m3_f64(x.v_cache.numpy())) * vs
+    for b, n in enumerate(lens):
+        q = x.q[b].double()[:, None, :]
+        kk = k[b, :n].transpose(0, 1).repeat_interleave(g, dim=0)
+        vv = v[b, :n].transpose(0, 1).repeat_interleave(g, dim=0)
+        ref = _sdpa(q, kk, vv, x.scale)[:, 0, :].numpy()
+        np.testing.assert_allclose(got[b], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_fp8_rows_past_the_history_are_never_read(oracle_mod):
+    x = inputs.make_decode_fp8(2, 8, 2, 16, 12, seqlens=[5, 12], seed=53, poison=True)
+    y = inputs.make_decode_fp8(2, 8, 2, 16, 12, seqlens=[5, 12], seed=53, poison=False)
+    a = oracle_mod.decode_fp8(x.q, x.k_cache, x.v_cache, x.k_scale, x.v_scale, x.seqlens, x.scale)
+    b = oracle_mod.decode_fp8(y.q, y.k_cache, y.v_cache, y.k_scale, y.v_scale, y.seqlens, y.scale)
+    assert np.isfinite(a).all()
+    np.testing.assert_array_equal(a, b)
