@@ -12,7 +12,7 @@ import ctypes
 import os
 
 __all__ = [
-    "GQAError", "gqa_decode", "gqa_decode_noalloc", "gqa_prefill_causal", "gqa_decode_expanded", "gqa_decode_expanded_bytes",
+    "GQAError", "gqa_decode", "gqa_decode_fp8", "gqa_decode_noalloc", "gqa_prefill_causal", "gqa_decode_expanded", "gqa_decode_expanded_bytes",
     "gqa_decode_plan", "gqa_get_last_device_status", "gqa_selftest_wait_timeout", "gqa_set_profile_events",
     "gqa_last_launch_count", "gqa_release", "gqa_status_string", "gqa_version", "library_path", "load",
 ]
@@ -27,6 +27,8 @@ _i = ctypes.c_int
 EXPORTS = {
     # name: (restype, argtypes)
     "gqa_decode": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp]),
+    "gqa_decode_fp8": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                            _vp, _vp]),
     "gqa_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp]),
     "gqa_prefill_causal": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "gqa_decode_expanded": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp]),
@@ -128,6 +130,39 @@ def gqa_decode(q, k_cache, v_cache, seqlens, scale=None, out=None, stream=None):
     st = load().gqa_decode(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(), B, Hq, Hkv, d,
                            Tmax, float(scale), out.data_ptr(), _stream_ptr(stream))
     _check(st, "gqa_decode")
+    return out
+
+
+def gqa_decode_fp8(q, k_cache, v_cache, seqlens, k_scale, v_scale, scale=None, out=None, stream=None):
+    """q [B,Hq,d] bf16; k_cache/v_cache [B,Tmax,Hkv,d] E4M3 codes (torch.uint8 or torch.float8_e4m3fn);
+    a key is e4m3(code) * k_scale, a value e4m3(code) * v_scale; seqlens [B] int32 (device)
+    -> out [B,Hq,d] bf16."""
+    import torch
+
+    _need(q, "q", torch.bfloat16, 3)
+    B, Hq, d = q.shape
+    if k_cache.dtype == torch.float8_e4m3fn:
+        k_cache = k_cache.view(torch.uint8)
+    if v_cache.dtype == torch.float8_e4m3fn:
+        v_cache = v_cache.view(torch.uint8)
+    _need(k_cache, "k_cache", torch.uint8, 4, q.device)
+    _need(v_cache, "v_cache", torch.uint8, 4, q.device)
+    _need(seqlens, "seqlens", torch.int32, 1, q.device)
+    Bk, Tmax, Hkv, dk = k_cache.shape
+    if (Bk, dk) != (B, d) or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, k_cache, v_cache and seqlens")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out", torch.bfloat16, 3, q.device)
+        if out.shape != q.shape:
+            raise ValueError("out must have q's shape")
+    if scale is None:
+        scale = 1.0 / d ** 0.5
+    st = load().gqa_decode_fp8(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), seqlens.data_ptr(), B, Hq, Hkv,
+                               d, Tmax, float(scale), float(k_scale), float(v_scale), out.data_ptr(),
+                               _stream_ptr(stream))
+    _check(st, "gqa_decode_fp8")
     return out
 
 

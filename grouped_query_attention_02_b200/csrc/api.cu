@@ -96,6 +96,22 @@ gqa_status encode_4d(CUtensorMap *tm, const void *base, uint64_t n0, uint64_t n1
     return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_CUDA;
 }
 
+// 4-D map over E4M3 codes [n3][n2][n1][128] (one byte each), box {128, 1, rows, 1}, 128-byte swizzle:
+// one box is `rows` whole rows of one head.
+gqa_status encode_4d_codes(CUtensorMap *tm, const void *base, uint64_t n1, uint64_t n2, uint64_t n3,
+                           uint32_t box_rows)
+{
+    const uint64_t n0 = kHeadDim;
+    cuuint64_t dims[4] = {n0, n1, n2, n3};
+    cuuint64_t strides[3] = {n0, n0 * n1, n0 * n1 * n2};
+    cuuint32_t box[4] = {(cuuint32_t)n0, 1, box_rows, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_CUDA;
+}
+
 gqa_status check_decode_args(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq,
                              int Hkv, int d, int Tmax, const void *out)
 {
@@ -110,7 +126,8 @@ gqa_status check_decode_args(const void *q, const void *k, const void *v, const 
 }
 
 gqa_status run_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq, int Hkv,
-                      int Tmax, float scale, void *out, cudaStream_t stream, int *launches);
+                      int Tmax, float scale, void *out, cudaStream_t stream, int *launches,
+                      const Fp8Scales *fp8 = nullptr);
 
 }  // namespace
 
@@ -127,10 +144,18 @@ void set_last_launch_count(int n) { g_last_launches = n; }
 
 static size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
-DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_t ws_budget)
+DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_t ws_budget, bool fp8)
 {
     const int g = Hq / Hkv;
-    const DecodeShape sh = decode_shape(g);
+    DecodeShape sh = decode_shape(g);
+    if (fp8) {
+        // the FP8 kernel is the tensor-core one for every group size it takes (g <= 32)
+        sh.tensor_cores = true;
+        sh.tile = 128;
+        sh.heads_per_cta = g;
+        sh.nhb = 1;
+        sh.ctas_per_sm = 1;
+    }
     DecodePlan p{};
     p.tile = sh.tile;
     p.hb = sh.heads_per_cta;
@@ -196,15 +221,22 @@ DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_
 
 int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq, int Hkv,
                    int Tmax, float scale, void *out, void *ws, const DecodePlan &p, int num_sms, int *status,
-                   cudaStream_t stream, int *launches, cudaEvent_t ev_before, cudaEvent_t ev_after)
+                   cudaStream_t stream, int *launches, cudaEvent_t ev_before, cudaEvent_t ev_after,
+                   const Fp8Scales *fp8)
 {
     gqa_status s;
     if ((s = get_encoder()) != GQA_OK) return s;
     if ((long long)Hkv * p.nhb > 65535) return GQA_ERR_UNSUPPORTED;
     if (p.ws_bytes > 0 && !ws) return GQA_ERR_INVALID_ARG;
+    if (fp8 && (!p.tensor_cores || p.tile != 128 || Hq / Hkv > 32)) return GQA_ERR_UNSUPPORTED;
     CUtensorMap tmK, tmV, tmQ;
-    if ((s = encode_4d(&tmK, k, kHeadDim, Hkv, Tmax, B, p.tile)) != GQA_OK) return s;
-    if ((s = encode_4d(&tmV, v, kHeadDim, Hkv, Tmax, B, p.tile)) != GQA_OK) return s;
+    if (fp8) {
+        if ((s = encode_4d_codes(&tmK, k, Hkv, Tmax, B, 128)) != GQA_OK) return s;
+        if ((s = encode_4d_codes(&tmV, v, Hkv, Tmax, B, 128)) != GQA_OK) return s;
+    } else {
+        if ((s = encode_4d(&tmK, k, kHeadDim, Hkv, Tmax, B, p.tile)) != GQA_OK) return s;
+        if ((s = encode_4d(&tmV, v, kHeadDim, Hkv, Tmax, B, p.tile)) != GQA_OK) return s;
+    }
 
     uint8_t *w = static_cast<uint8_t *>(ws);
     DecodeArgs a{};
@@ -223,6 +255,10 @@ int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *s
     a.nsplit = p.nsplit;
     a.nhb = p.nhb;
     a.qscale = scale * 1.4426950408889634f;  // log2(e): the softmax runs in base 2
+    if (fp8) {
+        a.qk_factor = a.qscale * fp8->k_scale;
+        a.o_factor = fp8->v_scale * (1.0f / 128.0f);
+    }
     a.wait_budget_ns = kWaitBudgetNs;
     a.num_ctas = num_sms;
     int n = 0;
@@ -244,7 +280,7 @@ int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *s
         if ((s = cuda_status(launch_decode_plan(a, stream))) != GQA_OK) return s;
         ++n;
         if (ev_before) cudaEventRecord(ev_before, stream);
-        if ((s = cuda_status(launch_decode_tc(tmK, tmV, tmQ, a, stream))) != GQA_OK) return s;
+        if ((s = cuda_status(launch_decode_tc(tmK, tmV, tmQ, a, stream, fp8 != nullptr))) != GQA_OK) return s;
         if (ev_after) cudaEventRecord(ev_after, stream);
         ++n;
         if ((s = cuda_status(launch_decode_combine(a, stream, true))) != GQA_OK) return s;
@@ -268,16 +304,17 @@ int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *s
 namespace {
 
 gqa_status run_decode(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq, int Hkv,
-                      int Tmax, float scale, void *out, cudaStream_t stream, int *launches)
+                      int Tmax, float scale, void *out, cudaStream_t stream, int *launches,
+                      const Fp8Scales *fp8)
 {
     DeviceState *st = nullptr;
     gqa_status s = device_state(&st);
     if (s != GQA_OK) return s;
-    const DecodePlan p = decode_plan_host(B, Hq, Hkv, Tmax, st->num_sms, kWorkspaceBudget);
+    const DecodePlan p = decode_plan_host(B, Hq, Hkv, Tmax, st->num_sms, kWorkspaceBudget, fp8 != nullptr);
     if (p.ws_bytes > 0 && (s = ensure_workspace(st, p.ws_bytes)) != GQA_OK) return s;
     return static_cast<gqa_status>(decode_enqueue(q, k, v, seqlens, B, Hq, Hkv, Tmax, scale, out, st->ws, p,
                                                   st->num_sms, st->status, stream, launches, g_ev_before,
-                                                  g_ev_after));
+                                                  g_ev_after, fp8));
 }
 
 }  // namespace
@@ -293,6 +330,21 @@ gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache, c
     std::lock_guard<std::mutex> lk(g_mu);
     return run_decode(q, k_cache, v_cache, seqlens, B, Hq, Hkv, Tmax, scale, out,
                       static_cast<cudaStream_t>(stream), &g_last_launches);
+}
+
+gqa_status gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens, int B,
+                          int Hq, int Hkv, int d, int Tmax, float scale, float k_scale, float v_scale, void *out,
+                          void *stream)
+{
+    g_last_launches = 0;
+    gqa_status s = check_decode_args(q, k_cache, v_cache, seqlens, B, Hq, Hkv, d, Tmax, out);
+    if (s != GQA_OK) return s;
+    if (!std::isfinite(scale) || !std::isfinite(k_scale) || !std::isfinite(v_scale)) return GQA_ERR_INVALID_ARG;
+    if (Hq / Hkv > 32) return GQA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    const Fp8Scales sc{k_scale, v_scale};
+    return run_decode(q, k_cache, v_cache, seqlens, B, Hq, Hkv, Tmax, scale, out,
+                      static_cast<cudaStream_t>(stream), &g_last_launches, &sc);
 }
 
 size_t gqa_decode_expanded_bytes(int B, int Tmax, int Hq, int d)

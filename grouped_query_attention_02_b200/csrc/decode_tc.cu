@@ -34,6 +34,8 @@
 // Warps: 0..4*nwg-1 softmax + epilogue (nwg = N/16), then the TMA producer
 // (it also claims units and loads the group's query rows), then the TMEM
 // allocator + MMA issuer.
+#include <cuda_fp16.h>
+
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -52,34 +54,49 @@ constexpr float kMoveThreshold = 8.0f;
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanMaxC = 4096;           // remainder sizes sorted by a shared-memory histogram up to this
 
-template <int N>
+// F8 = false: bf16 cache; the K and V tiles go from TMA straight to the tensor cores.
+// F8 = true: FP8 (E4M3) cache.  TMA brings the raw code tiles (16 KB each) into a ring; one converter
+// warpgroup widens them exactly to f16 (every E4M3 value is an f16 value): the keys into tensor
+// memory, where they are the A operand of S^T, the values into a 128-byte-swizzled f16 tile in shared
+// memory.  Q is converted in place to f16 with a power-of-two scale per head, and P enters the second
+// product as f16 hi + lo terms (of 128 p, so that small weights stay normal), with f16 MMAs throughout.
+template <int N, bool F8>
 struct TcCfg {
     static constexpr int nwg = N / kHPW;                      // softmax warpgroups, 16 heads each
-    static constexpr int threads = kWG * nwg + 64;            // + TMA warp + MMA warp
-    static constexpr int stages = 3;
-    static constexpr int stage_bytes = 2 * kTile;             // K then V
-    static constexpr int q_off = stages * stage_bytes;        // Q[2 buffers]: [2 halves][N rows][128 B], swizzled
+    static constexpr int conv_warps = F8 ? 4 : 0;             // FP8: the converter warpgroup
+    static constexpr int threads = kWG * nwg + 32 * conv_warps + 64;   // + TMA warp + MMA warp
+    static constexpr int stages = F8 ? 4 : 3;
+    static constexpr int stage_bytes = F8 ? kTile : 2 * kTile;   // K then V (FP8: two 16 KB code tiles)
+    static constexpr int vc_off = stages * stage_bytes;       // FP8: two converted f16 V tiles
+    static constexpr int vc_bytes = F8 ? 2 * kTile : 0;
+    static constexpr int q_off = vc_off + vc_bytes;           // Q[2 buffers]: [2 halves][N rows][128 B], swizzled
     static constexpr int q_half = N * 128;
     static constexpr int q_bytes = 2 * q_half;
-    static constexpr int p_off = q_off + 2 * q_bytes;         // P^T hi, then lo: [N/8][16 token groups][8][8] bf16
+    static constexpr int p_off = q_off + 2 * q_bytes;         // P^T hi, then lo: [N/8][16 token groups][8][8] 16-bit
     static constexpr int p_bytes = N * kTok * 2;
     static constexpr int red_off = p_off + 2 * p_bytes;       // [2][4][N] floats: tile maxima per warp
     static constexpr int lsum_off = red_off + 2 * 4 * N * 4;  // [2 O buffers][4][N] floats: l partials per warp
-    static constexpr int vote_off = lsum_off + 2 * 4 * N * 4; // [nwg][2][4] ints
+    static constexpr int qfac_off = lsum_off + 2 * 4 * N * 4; // FP8: [2 Q buffers][N] score factors per head
+    static constexpr int vote_off = qfac_off + (F8 ? 2 * N * 4 : 0);   // [nwg][2][4] ints
     static constexpr int queue_off = vote_off + nwg * 32;     // kQD units of 8 ints
     static constexpr int bar_off = queue_off + kQD * 32;
-    static constexpr int nbars = 32 + nwg;
+    static constexpr int nbars = F8 ? 52 : 32 + nwg;
     static constexpr int tmem_off = bar_off + nbars * 8;
     static constexpr int err_off = tmem_off + 8;
     static constexpr int bytes = err_off + 8;
+    // FP8: K[2] (64 columns each: 128 f16 keys per token, packed in pairs) first, then as below.
     // S[2] (N columns each) and O[2] (2N columns each: the hi and lo products side by side)
-    static constexpr uint32_t tmem_cols = (6 * N <= 128) ? 128 : 256;
+    static constexpr uint32_t s_base = F8 ? 128 : 0;
+    static constexpr uint32_t tmem_used = s_base + 6 * N;
+    static constexpr uint32_t tmem_cols = tmem_used <= 128 ? 128 : (tmem_used <= 256 ? 256 : 512);
     static_assert(bytes <= 227 * 1024, "shared memory budget");
 };
 
 // barrier slots
 enum : int { K_FULL = 0, V_FULL = 3, KV_EMPTY = 6, S_FULL = 9, S_FREE = 11, P_FULL = 13, P_FREE = 14, O_FULL = 15,
-             O_FREE = 17, Q_FULL = 19, Q_EMPTY = 21, I_FULL = 23, I_EMPTY = 27, DRAIN = 31, GRP = 32 };
+             O_FREE = 17, Q_FULL = 19, Q_EMPTY = 21, I_FULL = 23, I_EMPTY = 27, DRAIN = 31, GRP = 32,
+             // FP8 only: raw code ring, converted K (tensor memory), converted V (shared memory), converted Q
+             R_FULL = 34, R_EMPTY = 38, KT_FULL = 42, KT_FREE = 44, VC_FULL = 46, VC_FREE = 48, QC_FULL = 50 };
 
 __device__ __forceinline__ void record_status(int *status, int code)
 {
@@ -281,13 +298,30 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     }
 }
 
+// Two E4M3 codes (low byte first) -> f16x2, exact.
+__device__ __forceinline__ void e4m3x4_to_f16x4(uint32_t w, uint32_t &lo, uint32_t &hi)
+{
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
+{
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float f16_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
+__device__ __forceinline__ float f16_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
+
 // ---------------------------------------------------------------------------------------------
-template <int N>
-__global__ void __launch_bounds__(TcCfg<N>::threads, 1)
+template <int N, bool F8>
+__global__ void __launch_bounds__(TcCfg<N, F8>::threads, 1)
 decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a)
 {
-    using C = TcCfg<N>;
+    using C = TcCfg<N, F8>;
     // the 128-byte swizzle needs 1024-byte aligned tiles; the whole budget is used, so there is no room
     // to realign: a misaligned window is reported and the CTA does nothing
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -305,16 +339,33 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     volatile int *err = reinterpret_cast<volatile int *>(smem + C::err_off);
     float *red = reinterpret_cast<float *>(smem + C::red_off);
     float *lsum = reinterpret_cast<float *>(smem + C::lsum_off);
+    float *qfac = reinterpret_cast<float *>(smem + C::qfac_off);
     volatile int *vote = reinterpret_cast<volatile int *>(smem + C::vote_off);
     volatile int *queue = reinterpret_cast<volatile int *>(smem + C::queue_off);
     uint8_t *ps = smem + C::p_off;
 
-    const int producer_warp = 4 * C::nwg, mma_warp = 4 * C::nwg + 1;
+    const int conv_warp0 = 4 * C::nwg;
+    const int producer_warp = conv_warp0 + C::conv_warps, mma_warp = producer_warp + 1;
+    constexpr int unit_readers = 1 + kWG * C::nwg + 32 * C::conv_warps;   // MMA + softmax + converter
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::stages; ++s) {
-            mbar_init(&bar[K_FULL + s], 1);
-            mbar_init(&bar[V_FULL + s], 1);
-            mbar_init(&bar[KV_EMPTY + s], 1);
+        if constexpr (F8) {
+            for (int s = 0; s < C::stages; ++s) {
+                mbar_init(&bar[R_FULL + s], 1);
+                mbar_init(&bar[R_EMPTY + s], kWG);
+            }
+            for (int s = 0; s < 2; ++s) {
+                mbar_init(&bar[KT_FULL + s], kWG);
+                mbar_init(&bar[KT_FREE + s], 1);
+                mbar_init(&bar[VC_FULL + s], kWG);
+                mbar_init(&bar[VC_FREE + s], 1);
+                mbar_init(&bar[QC_FULL + s], kWG);
+            }
+        } else {
+            for (int s = 0; s < C::stages; ++s) {
+                mbar_init(&bar[K_FULL + s], 1);
+                mbar_init(&bar[V_FULL + s], 1);
+                mbar_init(&bar[KV_EMPTY + s], 1);
+            }
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar[S_FULL + s], 1);
@@ -328,7 +379,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         mbar_init(&bar[P_FREE], 1);
         for (int s = 0; s < kQD; ++s) {
             mbar_init(&bar[I_FULL + s], 1);
-            mbar_init(&bar[I_EMPTY + s], 1 + kWG * C::nwg);
+            mbar_init(&bar[I_EMPTY + s], unit_readers);
         }
         mbar_init(&bar[DRAIN], 1);
         for (int w = 0; w < C::nwg; ++w) mbar_init(&bar[GRP + w], kWG);
@@ -347,8 +398,9 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS[2] = {tmem, tmem + N};
-    const uint32_t tO[2] = {tmem + 2 * N, tmem + 4 * N};   // columns [0,N): V^T P_hi^T, [N,2N): V^T P_lo^T
+    const uint32_t tS[2] = {tmem + C::s_base, tmem + C::s_base + N};
+    // columns [0,N): V^T P_hi^T, [N,2N): V^T P_lo^T
+    const uint32_t tO[2] = {tmem + C::s_base + 2 * N, tmem + C::s_base + 4 * N};
 
     if (warp == producer_warp) {
         // ---------------- claims units, loads the group's query rows and streams the K/V tiles
@@ -386,19 +438,31 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 bool ok = true;
                 for (int jj = 0; jj < ntl; ++jj, ++tcount) {
                     const int s = tcount % C::stages;
-                    if (tcount >= C::stages &&
-                        !wait_or_fail(&bar[KV_EMPTY + s], ((tcount / C::stages) - 1) & 1, a, err)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *ks = smem + s * C::stage_bytes;
                     const int t0 = it.z + jj * kTok;
-                    mbar_arrive_expect_tx(&bar[K_FULL + s], kTile);
-                    tma_load_4d(ks, &tmK, &bar[K_FULL + s], 0, kvh, t0, it.x);
-                    tma_load_4d(ks + kHalf, &tmK, &bar[K_FULL + s], 64, kvh, t0, it.x);
-                    mbar_arrive_expect_tx(&bar[V_FULL + s], kTile);
-                    tma_load_4d(ks + kTile, &tmV, &bar[V_FULL + s], 0, kvh, t0, it.x);
-                    tma_load_4d(ks + kTile + kHalf, &tmV, &bar[V_FULL + s], 64, kvh, t0, it.x);
+                    uint8_t *ks = smem + s * C::stage_bytes;
+                    if constexpr (F8) {
+                        if (tcount >= C::stages &&
+                            !wait_or_fail(&bar[R_EMPTY + s], ((tcount / C::stages) - 1) & 1, a, err)) {
+                            ok = false;
+                            break;
+                        }
+                        // one box = 128 tokens x 128 one-byte codes of a head
+                        mbar_arrive_expect_tx(&bar[R_FULL + s], kTile);
+                        tma_load_4d(ks, &tmK, &bar[R_FULL + s], 0, kvh, t0, it.x);
+                        tma_load_4d(ks + kHalf, &tmV, &bar[R_FULL + s], 0, kvh, t0, it.x);
+                    } else {
+                        if (tcount >= C::stages &&
+                            !wait_or_fail(&bar[KV_EMPTY + s], ((tcount / C::stages) - 1) & 1, a, err)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&bar[K_FULL + s], kTile);
+                        tma_load_4d(ks, &tmK, &bar[K_FULL + s], 0, kvh, t0, it.x);
+                        tma_load_4d(ks + kHalf, &tmK, &bar[K_FULL + s], 64, kvh, t0, it.x);
+                        mbar_arrive_expect_tx(&bar[V_FULL + s], kTile);
+                        tma_load_4d(ks + kTile, &tmV, &bar[V_FULL + s], 0, kvh, t0, it.x);
+                        tma_load_4d(ks + kTile + kHalf, &tmV, &bar[V_FULL + s], 64, kvh, t0, it.x);
+                    }
                     issued_tiles = tcount + 1;
                 }
                 ++icount;
@@ -407,8 +471,12 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             // leave no copy in flight
             for (int t = issued_tiles - 1; t >= 0 && t >= issued_tiles - C::stages; --t) {
                 const uint32_t ph = (t / C::stages) & 1;
-                mbar_wait(&bar[K_FULL + t % C::stages], ph, a.wait_budget_ns);
-                mbar_wait(&bar[V_FULL + t % C::stages], ph, a.wait_budget_ns);
+                if constexpr (F8) {
+                    mbar_wait(&bar[R_FULL + t % C::stages], ph, a.wait_budget_ns);
+                } else {
+                    mbar_wait(&bar[K_FULL + t % C::stages], ph, a.wait_budget_ns);
+                    mbar_wait(&bar[V_FULL + t % C::stages], ph, a.wait_budget_ns);
+                }
             }
             for (int i = icount - 1; i >= 0 && i >= icount - 2; --i)
                 mbar_wait(&bar[Q_FULL + (i & 1)], (i >> 1) & 1, a.wait_budget_ns);
@@ -416,8 +484,9 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     } else if (warp == mma_warp) {
         // ---------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_s = umma_idesc_bf16(kTok, N, 0, 0);   // K (K-major) . Q^T (K-major)
-            const uint32_t idesc_o = umma_idesc_bf16(kD, 2 * N, 1, 1); // V^T (MN-major) . [P_hi | P_lo]^T (MN-major)
+            // S^T = K (K-major) . Q^T (K-major); [O_hi | O_lo] = V^T (MN-major) . [P_hi | P_lo]^T (MN-major)
+            const uint32_t idesc_s = F8 ? umma_idesc_f16(kTok, N, 0, 0) : umma_idesc_bf16(kTok, N, 0, 0);
+            const uint32_t idesc_o = F8 ? umma_idesc_f16(kD, 2 * N, 1, 1) : umma_idesc_bf16(kD, 2 * N, 1, 1);
             const uint32_t p_addr = smem_u32(ps);
             int tcount = 0, icount = 0;
             bool ok = true;
@@ -430,48 +499,70 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 if (t_end < 0) break;
                 const int ntl = (t_end - t_begin + kTok - 1) / kTok;
                 const int qb = icount & 1, ob = icount & 1;
-                if (!wait_or_fail(&bar[Q_FULL + qb], (icount >> 1) & 1, a, err)) break;
+                if (!wait_or_fail(&bar[(F8 ? QC_FULL : Q_FULL) + qb], (icount >> 1) & 1, a, err)) break;
                 if (icount >= 2 && !wait_or_fail(&bar[O_FREE + ob], ((icount >> 1) - 1) & 1, a, err)) break;
                 const uint32_t q_addr = smem_u32(smem + C::q_off + qb * C::q_bytes);
                 for (int jj = 0; jj <= ntl; ++jj) {
                     if (jj < ntl) {
                         const int T = tcount + jj;
                         const int s = T % C::stages;
-                        if (!wait_or_fail(&bar[K_FULL + s], (T / C::stages) & 1, a, err)) { ok = false; break; }
+                        if (!wait_or_fail(&bar[(F8 ? KT_FULL + (T & 1) : K_FULL + s)],
+                                          F8 ? ((T >> 1) & 1) : ((T / C::stages) & 1), a, err)) {
+                            ok = false;
+                            break;
+                        }
                         if (T >= 2 && !wait_or_fail(&bar[S_FREE + (T & 1)], ((T >> 1) - 1) & 1, a, err)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t k_addr = smem_u32(smem + s * C::stage_bytes);
+                        if constexpr (F8) {
+                            // A = the converted keys in tensor memory: 16 head coordinates = 8 columns
+                            const uint32_t k_tmem = tmem + (T & 1) * 64;
 #pragma unroll
-                        for (int ks = 0; ks < kD / 16; ++ks) {
-                            const uint32_t ka = k_addr + (ks >> 2) * kHalf + (ks & 3) * 32;
-                            const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
-                            umma_bf16_ss(tS[T & 1], umma_smem_desc(ka, 16, 1024, 2), umma_smem_desc(qa, 16, 1024, 2),
-                                         idesc_s, ks > 0 ? 1u : 0u);
+                            for (int ks = 0; ks < kD / 16; ++ks) {
+                                const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
+                                umma_ts(tS[T & 1], k_tmem + ks * 8, umma_smem_desc(qa, 16, 1024, 2), idesc_s,
+                                            ks > 0 ? 1u : 0u);
+                            }
+                            umma_commit(&bar[S_FULL + (T & 1)]);
+                            umma_commit(&bar[KT_FREE + (T & 1)]);
+                        } else {
+                            const uint32_t k_addr = smem_u32(smem + s * C::stage_bytes);
+#pragma unroll
+                            for (int ks = 0; ks < kD / 16; ++ks) {
+                                const uint32_t ka = k_addr + (ks >> 2) * kHalf + (ks & 3) * 32;
+                                const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
+                                umma_ss(tS[T & 1], umma_smem_desc(ka, 16, 1024, 2),
+                                             umma_smem_desc(qa, 16, 1024, 2), idesc_s, ks > 0 ? 1u : 0u);
+                            }
+                            umma_commit(&bar[S_FULL + (T & 1)]);
                         }
-                        umma_commit(&bar[S_FULL + (T & 1)]);
                     }
                     if (jj >= 1) {
                         const int T = tcount + jj - 1;
                         const int s = T % C::stages;
                         if (!wait_or_fail(&bar[P_FULL], T & 1, a, err)) { ok = false; break; }
-                        if (!wait_or_fail(&bar[V_FULL + s], (T / C::stages) & 1, a, err)) { ok = false; break; }
+                        if (!wait_or_fail(&bar[(F8 ? VC_FULL + (T & 1) : V_FULL + s)],
+                                          F8 ? ((T >> 1) & 1) : ((T / C::stages) & 1), a, err)) {
+                            ok = false;
+                            break;
+                        }
                         tc_fence_after();
-                        const uint32_t v_addr = smem_u32(smem + s * C::stage_bytes + kTile);
+                        const uint32_t v_addr = F8 ? smem_u32(smem + C::vc_off + (T & 1) * kTile)
+                                                   : smem_u32(smem + s * C::stage_bytes + kTile);
                         // [O_hi | O_lo] += V^T [P_hi | P_lo]^T in one product of width 2N: the lo blocks
                         // follow the hi blocks at the same 2048-byte stride, so they are simply more columns
 #pragma unroll
                         for (int ks = 0; ks < kTok / 16; ++ks) {
                             // A = V^T: 16 tokens (two 8-row groups, 1024 B apart), 64-column blocks kHalf apart
                             // B = P^T: 16 tokens (two 128-byte core-matrix groups), 8-head blocks 2048 B apart
-                            umma_bf16_ss(tO[ob], umma_smem_desc(v_addr + ks * 2048, kHalf, 1024, 2),
+                            umma_ss(tO[ob], umma_smem_desc(v_addr + ks * 2048, kHalf, 1024, 2),
                                          umma_smem_desc(p_addr + ks * 256, 128, 2048, 0), idesc_o,
                                          (jj > 1 || ks > 0) ? 1u : 0u);
                         }
                         umma_commit(&bar[P_FREE]);
-                        umma_commit(&bar[KV_EMPTY + s]);
+                        umma_commit(&bar[(F8 ? VC_FREE + (T & 1) : KV_EMPTY + s)]);
                     }
                 }
                 if (!ok) break;
@@ -482,6 +573,125 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             }
             umma_commit(&bar[DRAIN]);
             mbar_wait(&bar[DRAIN], 0, a.wait_budget_ns);
+        }
+    } else if (F8 && warp >= conv_warp0) {
+        // ---------------- FP8 converter: thread ct owns token ct of each tile (TMEM lane ct of K)
+        const int ct = threadIdx.x - kWG * C::nwg;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        int tcount = 0, icount = 0;
+        while (true) {
+            const int slot = icount % kQD;
+            if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
+            volatile int *qq = queue + slot * 8;
+            const int t_begin = qq[3], t_end = qq[4];
+            mbar_arrive(&bar[I_EMPTY + slot]);
+            if (t_end < 0) break;
+            // the group's query rows, in place: bf16 -> f16 times 2^e per head, e putting the head's
+            // largest |q| in [2^14, 2^15); the softmax undoes 2^e in its score factor
+            const int qb = icount & 1;
+            if (!wait_or_fail(&bar[Q_FULL + qb], (icount >> 1) & 1, a, err)) break;
+            {
+                constexpr int tpr = kWG / N;         // threads per query row
+                constexpr int cpt = 16 / tpr;        // 16-byte chunks per thread (16 per row: 2 halves x 8)
+                const int row = ct / tpr, j0 = ct % tpr;
+                uint8_t *qs = smem + C::q_off + qb * C::q_bytes;
+                uint4 v[cpt];
+                float mx = 0.f;
+#pragma unroll
+                for (int i = 0; i < cpt; ++i) {
+                    const int k = j0 + i * tpr;
+                    v[i] = *reinterpret_cast<const uint4 *>(qs + (k >> 3) * C::q_half + row * 128 + (k & 7) * 16);
+                    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        mx = fmaxf(mx, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
+                }
+#pragma unroll
+                for (int o = tpr / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                const int ex = (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127;
+                const int e = min(14 - ex, 100);      // e in [-114, 100]: both 2^e and 2^-e are normal floats
+                const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+                const float down = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+                for (int i = 0; i < cpt; ++i) {
+                    const int k = j0 + i * tpr;
+                    uint4 o;
+                    o.x = pack_f16x2(bf16_lo(v[i].x) * up, bf16_hi(v[i].x) * up);
+                    o.y = pack_f16x2(bf16_lo(v[i].y) * up, bf16_hi(v[i].y) * up);
+                    o.z = pack_f16x2(bf16_lo(v[i].z) * up, bf16_hi(v[i].z) * up);
+                    o.w = pack_f16x2(bf16_lo(v[i].w) * up, bf16_hi(v[i].w) * up);
+                    *reinterpret_cast<uint4 *>(qs + (k >> 3) * C::q_half + row * 128 + (k & 7) * 16) = o;
+                }
+                if (j0 == 0) qfac[qb * N + row] = a.qk_factor * down;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar[QC_FULL + qb]);
+            const int ntl = (t_end - t_begin + kTok - 1) / kTok;
+            bool ok = true;
+            for (int jj = 0; jj < ntl; ++jj) {
+                const int T = tcount + jj;
+                const int s = T % C::stages, cb = T & 1;
+                if (!wait_or_fail(&bar[R_FULL + s], (T / C::stages) & 1, a, err)) { ok = false; break; }
+                // the raw tiles were stored with the 128-byte swizzle: chunk c of row ct at c ^ (ct & 7)
+                const uint8_t *krow = smem + s * C::stage_bytes + ct * 128;
+                uint4 kr[8], vr[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    kr[c] = *reinterpret_cast<const uint4 *>(krow + ((c ^ (ct & 7)) << 4));
+                    vr[c] = *reinterpret_cast<const uint4 *>(krow + kHalf + ((c ^ (ct & 7)) << 4));
+                }
+                mbar_arrive(&bar[R_EMPTY + s]);
+                // tokens past the piece's end may hold anything (NaN codes included): they become zeros,
+                // so that no 0 * NaN reaches an accumulator
+                const bool valid = (t_begin + jj * kTok + ct) < t_end;
+                // keys -> tensor memory, row ct: column j holds head coordinates 2j, 2j+1
+                if (T >= 2 && !wait_or_fail(&bar[KT_FREE + cb], ((T >> 1) - 1) & 1, a, err)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t w[32];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint4 r = kr[h * 4 + c];
+                        e4m3x4_to_f16x4(r.x, w[c * 8 + 0], w[c * 8 + 1]);
+                        e4m3x4_to_f16x4(r.y, w[c * 8 + 2], w[c * 8 + 3]);
+                        e4m3x4_to_f16x4(r.z, w[c * 8 + 4], w[c * 8 + 5]);
+                        e4m3x4_to_f16x4(r.w, w[c * 8 + 6], w[c * 8 + 7]);
+                    }
+                    if (!valid) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) w[i] = 0u;
+                    }
+                    tmem_st32(tmem + cb * 64 + lane_off + h * 32, w);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bar[KT_FULL + cb]);
+                // values -> f16 tile [2 halves][128 rows][128 B], 128-byte swizzle, row ct
+                if (T >= 2 && !wait_or_fail(&bar[VC_FREE + cb], ((T >> 1) - 1) & 1, a, err)) { ok = false; break; }
+                uint8_t *vt = smem + C::vc_off + cb * kTile + ct * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint4 lo4, hi4;
+                    e4m3x4_to_f16x4(vr[c].x, lo4.x, lo4.y);
+                    e4m3x4_to_f16x4(vr[c].y, lo4.z, lo4.w);
+                    e4m3x4_to_f16x4(vr[c].z, hi4.x, hi4.y);
+                    e4m3x4_to_f16x4(vr[c].w, hi4.z, hi4.w);
+                    if (!valid) {
+                        lo4 = make_uint4(0, 0, 0, 0);
+                        hi4 = lo4;
+                    }
+                    const int j = 2 * (c & 3);   // 16 codes = two 16-byte f16 chunks of half c / 4
+                    uint8_t *half = vt + (c >> 2) * kHalf;
+                    *reinterpret_cast<uint4 *>(half + ((j ^ (ct & 7)) << 4)) = lo4;
+                    *reinterpret_cast<uint4 *>(half + (((j + 1) ^ (ct & 7)) << 4)) = hi4;
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&bar[VC_FULL + cb]);
+            }
+            if (!ok) break;
+            tcount += ntl;
+            ++icount;
         }
     } else {
         // ---------------- softmax warpgroup wg: heads 16*wg .. 16*wg+15; thread t owns token t of
@@ -499,6 +709,8 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         bool pend = false;
         int pb = 0, pkvh = 0, psplit = 0, pob = 0;
         float pm[kHPW];
+        // FP8: O carries 128 p v_code; the value scale and 1/128 are applied here
+        const float ofac = F8 ? a.o_factor : 1.f;
         auto epilogue = [&]() -> bool {
             if (!group_sync(&bar[GRP + wg], uses, a, err)) return false;      // lsum[pob] complete
             if (!wait_or_fail(&bar[O_FULL + pob], (((icount - 1) >> 1)) & 1, a, err)) return false;
@@ -508,7 +720,8 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             tmem_ld16(tO[pob] + lane_off + N + hs, olo);
             tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < kHPW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) + __uint_as_float(olo[h]));
+            for (int h = 0; h < kHPW; ++h)
+                o[h] = __float_as_uint((__uint_as_float(o[h]) + __uint_as_float(olo[h])) * ofac);
             const float *ls = lsum + pob * 4 * N;
             const int d = t;
             const int npieces = a.nsplit_b[pb];
@@ -554,6 +767,16 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             }
             const int ntl = (t_end - t_begin + kTok - 1) / kTok;
             const int ob = icount & 1;
+            // score factor per head: log2(e) * scale (FP8: times k_scale and the head's 2^-e)
+            float qf[kHPW];
+            if constexpr (F8) {
+                if (!wait_or_fail(&bar[QC_FULL + (icount & 1)], (icount >> 1) & 1, a, err)) break;
+#pragma unroll
+                for (int h = 0; h < kHPW; ++h) qf[h] = qfac[(icount & 1) * N + hs + h];
+            } else {
+#pragma unroll
+                for (int h = 0; h < kHPW; ++h) qf[h] = a.qscale;
+            }
             float m_use[kHPW], l_part[kHPW];
 #pragma unroll
             for (int h = 0; h < kHPW; ++h) {
@@ -576,7 +799,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 bool over = false;
 #pragma unroll
                 for (int h = 0; h < kHPW; ++h) {
-                    x[h] = valid ? __uint_as_float(raw[h]) * a.qscale : -INFINITY;
+                    x[h] = valid ? __uint_as_float(raw[h]) * qf[h] : -INFINITY;
                     over |= x[h] > m_use[h] + kMoveThreshold;
                 }
                 const int wflag = __any_sync(0xffffffffu, over) ? 1 : 0;
@@ -638,29 +861,38 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                         tmem_wait_st();
                     }
                 }
-                // Rows past the history may hold anything (NaN included) and the tensor cores would form
-                // 0 * NaN: in a partial tile the masked tokens zero their own V row once it has landed.
-                if (wg == 0 && t_end - (t_begin + jj * kTok) < kTok && !valid) {
-                    const int st = T % C::stages;
-                    if (!wait_or_fail(&bar[V_FULL + st], (T / C::stages) & 1, a, err)) { ok = false; break; }
-                    uint8_t *vrow = smem + st * C::stage_bytes + kTile + t * 128;
-                    const uint4 z = make_uint4(0, 0, 0, 0);
+                if constexpr (!F8) {
+                    // Rows past the history may hold anything (NaN included) and the tensor cores would
+                    // form 0 * NaN: in a partial tile the masked tokens zero their own V row once it has
+                    // landed.  (The FP8 converter writes zeros for them instead.)
+                    if (wg == 0 && t_end - (t_begin + jj * kTok) < kTok && !valid) {
+                        const int st = T % C::stages;
+                        if (!wait_or_fail(&bar[V_FULL + st], (T / C::stages) & 1, a, err)) { ok = false; break; }
+                        uint8_t *vrow = smem + st * C::stage_bytes + kTile + t * 128;
+                        const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        *reinterpret_cast<uint4 *>(vrow + c * 16) = z;
-                        *reinterpret_cast<uint4 *>(vrow + kHalf + c * 16) = z;
+                        for (int c = 0; c < 8; ++c) {
+                            *reinterpret_cast<uint4 *>(vrow + c * 16) = z;
+                            *reinterpret_cast<uint4 *>(vrow + kHalf + c * 16) = z;
+                        }
                     }
                 }
                 // P^T, MN-major without swizzle: core matrices of 8 tokens x 8 heads (128 B), each weight
-                // as hi = bf16(p) plus lo = bf16(p - hi)
+                // as hi plus lo = (p - hi) in the products' 16-bit type (FP8: f16 terms of 128 p)
 #pragma unroll
                 for (int hb = 0; hb < kHPW / 8; ++hb) {
                     uint32_t hi[4], lo[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float a0 = p[hb * 8 + 2 * e], a1 = p[hb * 8 + 2 * e + 1];
-                        hi[e] = pack2(a0, a1);
-                        lo[e] = pack2(a0 - bf16_lo(hi[e]), a1 - bf16_hi(hi[e]));
+                        if constexpr (F8) {
+                            const float a0 = p[hb * 8 + 2 * e] * 128.f, a1 = p[hb * 8 + 2 * e + 1] * 128.f;
+                            hi[e] = pack_f16x2(a0, a1);
+                            lo[e] = pack_f16x2(a0 - f16_lo(hi[e]), a1 - f16_hi(hi[e]));
+                        } else {
+                            const float a0 = p[hb * 8 + 2 * e], a1 = p[hb * 8 + 2 * e + 1];
+                            hi[e] = pack2(a0, a1);
+                            lo[e] = pack2(a0 - bf16_lo(hi[e]), a1 - bf16_hi(hi[e]));
+                        }
                     }
                     uint8_t *dst = ps + (hs / 8 + hb) * 2048 + (t >> 3) * 128 + (t & 7) * 16;
                     *reinterpret_cast<uint4 *>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -705,17 +937,17 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     }
 }
 
-template <int N>
+template <int N, bool F8>
 cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, const CUtensorMap &tmQ,
                               const DecodeArgs &a, cudaStream_t stream)
 {
-    const int smem = TcCfg<N>::bytes;
+    const int smem = TcCfg<N, F8>::bytes;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(decode_persistent_kernel<N>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaFuncSetAttribute(decode_persistent_kernel<N, F8>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
     }
@@ -723,7 +955,7 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
     // waits for (griddepcontrol.wait) before reading the plan
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.num_ctas);
-    cfg.blockDim = dim3(TcCfg<N>::threads);
+    cfg.blockDim = dim3(TcCfg<N, F8>::threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -731,7 +963,7 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_persistent_kernel<N>, tmK, tmV, tmQ, a);
+    return cudaLaunchKernelEx(&cfg, decode_persistent_kernel<N, F8>, tmK, tmV, tmQ, a);
 }
 
 }  // namespace
@@ -743,10 +975,15 @@ cudaError_t launch_decode_plan(const DecodeArgs &a, cudaStream_t stream)
 }
 
 cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, const CUtensorMap &tmQ,
-                             const DecodeArgs &a, cudaStream_t stream)
+                             const DecodeArgs &a, cudaStream_t stream, bool fp8)
 {
-    if (a.group <= 16) return launch_persistent<16>(tmK, tmV, tmQ, a, stream);
-    if (a.group <= 32) return launch_persistent<32>(tmK, tmV, tmQ, a, stream);
+    if (fp8) {
+        if (a.group <= 16) return launch_persistent<16, true>(tmK, tmV, tmQ, a, stream);
+        if (a.group <= 32) return launch_persistent<32, true>(tmK, tmV, tmQ, a, stream);
+        return cudaErrorInvalidValue;
+    }
+    if (a.group <= 16) return launch_persistent<16, false>(tmK, tmV, tmQ, a, stream);
+    if (a.group <= 32) return launch_persistent<32, false>(tmK, tmV, tmQ, a, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -24,6 +24,8 @@ struct DecodeArgs {
     int *status;              // device status word
     int B, Hq, Hkv, Tmax, group, chunk, nsplit, nhb;
     float qscale;             // scale * log2(e)
+    float qk_factor;          // FP8 cache: scale * log2(e) * k_scale
+    float o_factor;           // FP8 cache: v_scale / 128 (the weights enter the PV product as 128 p)
     unsigned long long wait_budget_ns;
     // device-planned schedule (tensor-core path): see decode_tc.cu
     int *plan_hdr;            // {claim counter, pieces, C}
@@ -40,13 +42,21 @@ struct DecodePlan {
     size_t off_hdr, off_nsb, off_items, off_po, off_pml, ws_bytes;
 };
 // ws_budget bounds the split partials of the tensor-core path (more pieces per sequence when it allows).
-DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_t ws_budget);
+// fp8: the plan of the FP8-cache decode, which always takes the tensor-core path (group sizes <= 32).
+DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_t ws_budget, bool fp8 = false);
 
-// Enqueues one decode (all kernels) on `stream` with the workspace `ws` laid out by `p`.
+// Per-tensor scales of an FP8 (E4M3) cache: a key is e4m3(code) * k_scale, a value e4m3(code) * v_scale.
+struct Fp8Scales {
+    float k_scale, v_scale;
+};
+
+// Enqueues one decode (all kernels) on `stream` with the workspace `ws` laid out by `p`; `fp8` non-null:
+// the caches hold E4M3 codes with those scales (p must then come from decode_plan_host(..., true)).
 // Returns 0 or a gqa_status code; adds the kernels launched to *launches.
 int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *seqlens, int B, int Hq, int Hkv,
                    int Tmax, float scale, void *out, void *ws, const DecodePlan &p, int num_sms, int *status,
-                   cudaStream_t stream, int *launches, cudaEvent_t ev_before, cudaEvent_t ev_after);
+                   cudaStream_t stream, int *launches, cudaEvent_t ev_before, cudaEvent_t ev_after,
+                   const Fp8Scales *fp8 = nullptr);
 
 // How the decode of group size g is laid out: the kernel family (tensor cores for
 // 3 <= g <= 32, CUDA cores otherwise), its token tile (TMA box rows and split
@@ -64,8 +74,9 @@ int decode_heads_per_cta(int g);   // CUDA-core kernel only
 // Launches the CUDA-core decode kernel (group sizes outside the tensor-core range).
 cudaError_t launch_decode_split(const CUtensorMap &tmK, const CUtensorMap &tmV, const DecodeArgs &a,
                                 cudaStream_t stream);
+// fp8: tmK / tmV map E4M3 code tiles (128 tokens x 128 bytes) instead of bf16 halves.
 cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, const CUtensorMap &tmQ,
-                             const DecodeArgs &a, cudaStream_t stream);
+                             const DecodeArgs &a, cudaStream_t stream, bool fp8);
 cudaError_t launch_decode_plan(const DecodeArgs &a, cudaStream_t stream);
 // pdl: launched as a programmatic dependent of the previous kernel on the stream
 cudaError_t launch_decode_combine(const DecodeArgs &a, cudaStream_t stream, bool pdl = false);

@@ -93,30 +93,6 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr, uint32_t lbo)
     return umma_smem_desc(saddr, lbo, 1024, 2);
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t *r)
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r)
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
 // max of three floats in one instruction (PTX max.f32 with three sources, sm_100)
 __device__ __forceinline__ float fmax3(float a, float b, float c)
 {
@@ -233,7 +209,7 @@ prefill_causal_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks) {
                         const uint32_t off = (ks >> 2) * kHalfTile + (ks & 3) * 32;
-                        umma_bf16_ss(tS[s], desc_kmajor(q_addr + off), desc_kmajor(k_addr + off), idesc_s,
+                        umma_ss(tS[s], desc_kmajor(q_addr + off), desc_kmajor(k_addr + off), idesc_s,
                                      ks > 0 ? 1u : 0u);
                     }
                     umma_commit(&bar[S_FULL + s]);
@@ -248,7 +224,7 @@ prefill_causal_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
 #pragma unroll
                     for (int ks = 0; ks < kBN / 16; ++ks) {
                         const uint32_t poff = (ks >> 2) * kHalfTile + (ks & 3) * 32;
-                        umma_bf16_ss(tO, desc_kmajor(p_addr + poff), desc_mnmajor(v_addr + ks * 2048, kHalfTile),
+                        umma_ss(tO, desc_kmajor(p_addr + poff), desc_mnmajor(v_addr + ks * 2048, kHalfTile),
                                      idesc_o, (jp > 0 || ks > 0) ? 1u : 0u);
                     }
                     umma_commit(&bar[P_FREE]);
@@ -414,17 +390,6 @@ struct PairSmem {
 enum PairBar { PQ_FULL = 0, PK_FULL = 1, PV_FULL = 3, PKV_EMPTY = 5, PS_FULL = 7, PP_FULL = 9, PO_FULL = 11,
                PDRAIN = 12 };
 
-// D[tmem] (+)= A[tmem] * B[smem]: A (M x K, K-major, 16-bit pairs per column) read from tensor memory.
-__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 __global__ void __launch_bounds__(kPairThreads, 1)
 prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const PrefillArgs a)
@@ -520,7 +485,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * kHalfTile + (ks & 3) * 32;
-                    umma_bf16_ss(tmem + w * 128, desc_kmajor(qa + off), desc_kmajor(k_addr + off), idesc_s,
+                    umma_ss(tmem + w * 128, desc_kmajor(qa + off), desc_kmajor(k_addr + off), idesc_s,
                                  ks > 0 ? 1u : 0u);
                 }
                 umma_commit(&bar[PS_FULL + w]);
@@ -541,7 +506,7 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                     for (int ks = 0; ks < kBN / 16; ++ks) {
                         // A = P: 16 keys = 8 columns of packed bf16 pairs; B = V rows ks*16 .. +16
-                        umma_bf16_ts(tmem + 256 + w * 128, tmem + w * 128 + ks * 8,
+                        umma_ts(tmem + 256 + w * 128, tmem + w * 128 + ks * 8,
                                      desc_mnmajor(v_addr + ks * 2048, kHalfTile), idesc_o,
                                      (j > 0 || ks > 0) ? 1u : 0u);
                     }

@@ -136,7 +136,8 @@ def make_decode_fp8(B: int, Hq: int, Hkv: int, d: int, Tmax: int, seqlens=None, 
                     seed: int = 0, scale: float | None = None, poison: bool = False, q_gain: float = 1.0,
                     seqlen_range=None, k_scale: float = 0.0135, v_scale: float = 0.0142) -> DecodeFp8Inputs:
     """Decode inputs over an FP8 (E4M3) cache with per-tensor scales; ``seqlens`` as in make_decode.
-    The default scales map about six standard deviations onto the largest E4M3 value."""
+    The default scales map about six standard deviations onto the largest E4M3 value.  The codes are
+    N(0,1) / scale; a zero scale draws them with the default scale (its keys or values are all zero)."""
     if seqlen_range is not None:
         sl = seqlens_uniform(B, seqlen_range[0], seqlen_range[1], seed + 3)
     elif seqlens is None:
@@ -146,8 +147,8 @@ def make_decode_fp8(B: int, Hq: int, Hkv: int, d: int, Tmax: int, seqlens=None, 
     else:
         sl = torch.as_tensor(seqlens, dtype=torch.int32).cpu()
     q = _normal((B, Hq, d), seed + 0, device, q_gain)
-    k = _normal_e4m3((B, Tmax, Hkv, d), seed + 1, device, 1.0 / k_scale)
-    v = _normal_e4m3((B, Tmax, Hkv, d), seed + 2, device, 1.0 / v_scale)
+    k = _normal_e4m3((B, Tmax, Hkv, d), seed + 1, device, 1.0 / (k_scale or 0.0135))
+    v = _normal_e4m3((B, Tmax, Hkv, d), seed + 2, device, 1.0 / (v_scale or 0.0142))
     if poison:
         for b in range(B):
             t = int(sl[b])

@@ -78,6 +78,35 @@ gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache, c
                       int B, int Hq, int Hkv, int d, int Tmax, float scale, void *out, void *stream);
 
 /*
+ * gqa_decode_fp8 -- one decode step over an FP8 (E4M3) KV cache with
+ * per-tensor scales, the cache quantisation that "Other ways to shrink the KV
+ * cache" (anrans.github.io attention-variants) lists: K and V stored in FP8,
+ * half the bytes of bf16.
+ *
+ *   q        [B, Hq, d]        bf16, as in gqa_decode
+ *   k_cache  [B, Tmax, Hkv, d] one-byte E4M3 codes (the "fn" variant: no
+ *                              infinities, 0x7F / 0xFF are NaN, largest finite 448)
+ *   v_cache  [B, Tmax, Hkv, d] E4M3 codes, same layout
+ *   k_scale, v_scale           a key element is e4m3(code) * k_scale, a value
+ *                              element e4m3(code) * v_scale (finite floats)
+ *   seqlens, scale, out, stream: as in gqa_decode
+ *
+ *   out[b,h] = sum_{t < seqlens[b]} softmax_t(scale q[b,h].K[b,t,h/g]) V[b,t,h/g]
+ *   with K = e4m3(k_cache) * k_scale and V = e4m3(v_cache) * v_scale.
+ *
+ * Group sizes g = Hq / Hkv up to 32 (GQA_ERR_UNSUPPORTED above).  The codes
+ * are widened to f16 on the SM, exactly, after one TMA read of each tile;
+ * the query is carried in f16 with a power-of-two scale per head (elements
+ * below 2^-24 of the head's largest |q| flush to zero), the products run on
+ * the tensor cores with fp32 accumulation.  NaN codes inside the history
+ * propagate to the output; rows past seqlens[b] are never used.  Same
+ * workspace, stream and error rules as gqa_decode.
+ */
+gqa_status gqa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, const int32_t *seqlens, int B,
+                          int Hq, int Hkv, int d, int Tmax, float scale, float k_scale, float v_scale, void *out,
+                          void *stream);
+
+/*
  * gqa_decode_noalloc -- gqa_decode for callers that cannot let a library
  * allocate device memory.  (This entry point is an engineering addition; the
  * pages describe no counterpart.)

@@ -126,3 +126,21 @@ def test_plan_argument_checks(lib):
     assert lib.gqa_decode_plan(1, 8, 3, 128, 64, 148, ctypes.byref(c), ctypes.byref(n), ctypes.byref(w)) == INVALID
     assert lib.gqa_decode_plan(1, 8, 2, 128, 64, 0, ctypes.byref(c), ctypes.byref(n), ctypes.byref(w)) == INVALID
     assert lib.gqa_decode_plan(1, 8, 2, 64, 64, 148, ctypes.byref(c), ctypes.byref(n), ctypes.byref(w)) == UNSUPPORTED
+
+
+def _decode_fp8(lib, q=A, k=A, v=A, sl=A, B=2, Hq=8, Hkv=2, d=128, T=64, out=A, scale=0.088, ks=0.01, vs=0.02):
+    return lib.gqa_decode_fp8(q, k, v, sl, B, Hq, Hkv, d, T, ctypes.c_float(scale), ctypes.c_float(ks),
+                              ctypes.c_float(vs), out, None)
+
+
+def test_fp8_decode_argument_checks(lib):
+    assert _decode_fp8(lib, k=None) == INVALID
+    assert _decode_fp8(lib, B=0) == INVALID
+    assert _decode_fp8(lib, Hq=6, Hkv=4) == INVALID
+    assert _decode_fp8(lib, ks=float("nan")) == INVALID
+    assert _decode_fp8(lib, vs=float("inf")) == INVALID
+    assert _decode_fp8(lib, scale=float("inf")) == INVALID
+    assert _decode_fp8(lib, d=64) == UNSUPPORTED
+    assert _decode_fp8(lib, Hq=64, Hkv=1) == UNSUPPORTED     # groups above 32
+    assert _decode_fp8(lib, v=U) == MISALIGNED
+    assert gqa.gqa_last_launch_count() == 0
