@@ -11,7 +11,8 @@ tokens/s (sequences decoded per second, one layer) rides along.
 
 The JSON line also carries the other hot-path rows measured the same way
 (tiny decode, variable-length sweep, extreme grouping, the expanded repeat-KV
-baseline, causal prefill), the roofline of the dominant kernel, the clocks
+baseline, FP8 (E4M3) caches of the headline, two variable-length and the
+extreme-grouping shapes, causal prefill), the roofline of the dominant kernel, the clocks
 seen during the timed region, an end-to-end figure with host buffers, and the
 fp64 CPU oracle timed on a bounded sample of the same workload.
 
@@ -40,9 +41,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # ---------------------------------------------------------------- host helpers (no GPU needed)
 
-def unique_kv_bytes(seqlens, Hkv: int, d: int) -> int:
-    """K and V rows actually cached: 2 * sum(T) * Hkv * d * 2 bytes (bf16)."""
-    return 2 * int(sum(int(t) for t in seqlens)) * Hkv * d * 2
+def unique_kv_bytes(seqlens, Hkv: int, d: int, elem_bytes: int = 2) -> int:
+    """K and V rows actually cached: 2 * sum(T) * Hkv * d * elem_bytes (2 for bf16, 1 for FP8)."""
+    return 2 * int(sum(int(t) for t in seqlens)) * Hkv * d * elem_bytes
 
 
 def decode_flops(seqlens, Hq: int, d: int) -> int:
@@ -175,9 +176,14 @@ def _events(torch):
 def time_decode(gqa, torch, x, steps: int, warmup: int, expanded=None):
     """Mean step time and mean split-kernel time (ms) over `steps` timed decode steps."""
     out = torch.empty_like(x.q)
-    call = (lambda: gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out)) if expanded is None else \
-        (lambda: gqa.gqa_decode_expanded(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out,
-                                         k_rep=expanded[0], v_rep=expanded[1]))
+    if hasattr(x, "k_scale"):      # an FP8 cache
+        call = lambda: gqa.gqa_decode_fp8(x.q, x.k_cache, x.v_cache, x.seqlens, x.k_scale, x.v_scale, x.scale,
+                                          out=out)
+    elif expanded is None:
+        call = lambda: gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out)
+    else:
+        call = lambda: gqa.gqa_decode_expanded(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out,
+                                               k_rep=expanded[0], v_rep=expanded[1])
     for _ in range(warmup):
         call()
     torch.cuda.synchronize()
@@ -497,6 +503,21 @@ def main():
             "slowdown_vs_grouped": st_ms / step_ms}
         del k_rep, v_rep
         torch.cuda.empty_cache()
+        # FP8 (E4M3) caches: half the bytes per token
+        for ww in (w, workloads.VARLEN_DECODE[1], workloads.VARLEN_DECODE[3], workloads.EXTREME_GROUP_DECODE):
+            xx = inputs.make_decode_fp8(ww.B, ww.Hq, ww.Hkv, ww.d, ww.Tmax, device="cuda", seed=0,
+                                        seqlen_range=ww.seqlen_range)
+            uu = unique_kv_bytes(xx.seqlens.cpu().tolist(), ww.Hkv, ww.d, elem_bytes=1)
+            st_ms, k_ms, n, _ = time_decode(gqa, torch, xx, 20, 3)
+            rows["FP8 KV cache, " + ww.name] = {
+                "ms_per_step": st_ms, "kernel_ms": k_ms, "unique_kv_GBps": uu / (st_ms * 1e-3) / 1e9,
+                "kernel_frac_hbm": uu / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "frac_hbm": uu / (st_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "tokens_per_s": ww.B / (st_ms * 1e-3), "launches_per_step": n / 20,
+                "speedup_vs_bf16_cache": (rows.get(ww.name, {}).get("ms_per_step") or
+                                          (step_ms if ww is w else float("nan"))) / st_ms}
+            del xx
+            torch.cuda.empty_cache()
         # causal prefill
         pw = workloads.CAUSAL_PREFILL
         try:

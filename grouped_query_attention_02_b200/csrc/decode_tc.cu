@@ -31,9 +31,11 @@
 // of each head only moves when some score exceeds it by more than 8 (log2
 // units); in the common case a tile costs one warp vote and one group barrier.
 //
-// Warps: 0..4*nwg-1 softmax + epilogue (nwg = N/16), then the TMA producer
-// (it also claims units and loads the group's query rows), then the TMEM
-// allocator + MMA issuer.
+// Warps: 0..4*nwg-1 softmax + epilogue (nwg = N/16), then (FP8 cache) the
+// converter warpgroup, the TMA producer (it also claims units and loads the
+// group's query rows), the TMEM allocator + S^T issuer, and the PV issuer.  The
+// two products are issued by different threads so that S^T runs up to four
+// tiles ahead instead of queueing behind the previous tile's PV product.
 #include <cuda_fp16.h>
 
 #include "internal.h"
@@ -48,7 +50,6 @@ constexpr int kTok = 128;                 // tokens per tile (the M of S^T)
 constexpr int kTile = kTok * kD * 2;      // 32 KB: one K or V tile
 constexpr int kHalf = kTile / 2;          // one 64-column half
 constexpr int kWG = 128;                  // threads of one softmax warpgroup (one token each)
-constexpr int kHPW = 16;                  // heads per softmax warpgroup
 constexpr int kQD = 4;                    // depth of the unit queue in shared memory
 constexpr float kMoveThreshold = 8.0f;
 constexpr int kPlanThreads = 1024;
@@ -57,46 +58,58 @@ constexpr int kPlanMaxC = 4096;           // remainder sizes sorted by a shared-
 // F8 = false: bf16 cache; the K and V tiles go from TMA straight to the tensor cores.
 // F8 = true: FP8 (E4M3) cache.  TMA brings the raw code tiles (16 KB each) into a ring; one converter
 // warpgroup widens them exactly to f16 (every E4M3 value is an f16 value): the keys into tensor
-// memory, where they are the A operand of S^T, the values into a 128-byte-swizzled f16 tile in shared
-// memory.  Q is converted in place to f16 with a power-of-two scale per head, and P enters the second
+// memory, where they are the A operand of S^T, the values into a 128-byte-swizzled f16 tile that
+// takes the place of the stage's two code tiles (each thread rewrites only the two 128-byte rows it
+// has just read, so no thread waits for another).  Q is converted in place to f16 with a power-of-two scale per head, and P enters the second
 // product as f16 hi + lo terms (of 128 p, so that small weights stay normal), with f16 MMAs throughout.
-template <int N, bool F8>
+// HW: heads one softmax warpgroup handles (4, 8 or 16): groups of up to 4 or 8 heads only compute
+// their own columns of the N = 16 wide products.
+template <int N, bool F8, int HW>
 struct TcCfg {
-    static constexpr int nwg = N / kHPW;                      // softmax warpgroups, 16 heads each
+    static_assert(HW == 16 || N == 16, "narrow softmax only with N = 16");
+    static constexpr int nwg = HW == 16 ? N / 16 : 1;         // softmax warpgroups
+    static constexpr int nb = HW <= 8 ? 1 : N / 8;            // 8-head blocks of P^T / O^T that carry heads
     static constexpr int conv_warps = F8 ? 4 : 0;             // FP8: the converter warpgroup
-    static constexpr int threads = kWG * nwg + 32 * conv_warps + 64;   // + TMA warp + MMA warp
-    static constexpr int stages = F8 ? 4 : 3;
-    static constexpr int stage_bytes = F8 ? kTile : 2 * kTile;   // K then V (FP8: two 16 KB code tiles)
-    static constexpr int vc_off = stages * stage_bytes;       // FP8: two converted f16 V tiles
-    static constexpr int vc_bytes = F8 ? 2 * kTile : 0;
-    static constexpr int q_off = vc_off + vc_bytes;           // Q[2 buffers]: [2 halves][N rows][128 B], swizzled
+    // + TMA warp + S^T issuer warp + PV issuer warp
+    static constexpr int threads = kWG * nwg + 32 * conv_warps + 96;
+    static constexpr int sbufs = 4;                            // S^T buffers: QK^T runs up to four tiles ahead
+    static constexpr int pbufs = (F8 || N == 16) ? 2 : 1;      // P^T buffers (2: the softmax runs a tile ahead)
+    static constexpr int stages = F8 ? (N == 32 ? 5 : 6) : 3;
+    // K then V (FP8: two 16 KB code tiles, then the f16 V tile in their place)
+    static constexpr int stage_bytes = F8 ? kTile : 2 * kTile;
+    static constexpr int q_off = stages * stage_bytes;        // Q[2 buffers]: [2 halves][N rows][128 B], swizzled
     static constexpr int q_half = N * 128;
     static constexpr int q_bytes = 2 * q_half;
-    static constexpr int p_off = q_off + 2 * q_bytes;         // P^T hi, then lo: [N/8][16 token groups][8][8] 16-bit
-    static constexpr int p_bytes = N * kTok * 2;
-    static constexpr int red_off = p_off + 2 * p_bytes;       // [2][4][N] floats: tile maxima per warp
+    static constexpr int p_off = q_off + 2 * q_bytes;         // P^T[pbufs]: hi blocks, then lo blocks,
+    static constexpr int p_half = nb * 2048;                  //   each [16 token groups][8 tokens][8 heads] 16-bit
+    static constexpr int red_off = p_off + pbufs * 2 * p_half; // [2][4][N] floats: tile maxima per warp
     static constexpr int lsum_off = red_off + 2 * 4 * N * 4;  // [2 O buffers][4][N] floats: l partials per warp
-    static constexpr int qfac_off = lsum_off + 2 * 4 * N * 4; // FP8: [2 Q buffers][N] score factors per head
-    static constexpr int vote_off = qfac_off + (F8 ? 2 * N * 4 : 0);   // [nwg][2][4] ints
+    static constexpr int qfac_off = lsum_off + 2 * 4 * N * 4; // FP8: [kQD unit slots][N] score factors per head
+    static constexpr int vote_off = qfac_off + (F8 ? kQD * N * 4 : 0);   // [nwg][2][4] ints
     static constexpr int queue_off = vote_off + nwg * 32;     // kQD units of 8 ints
     static constexpr int bar_off = queue_off + kQD * 32;
-    static constexpr int nbars = F8 ? 52 : 32 + nwg;
+    static constexpr int nbars = F8 ? 69 : 41;
     static constexpr int tmem_off = bar_off + nbars * 8;
     static constexpr int err_off = tmem_off + 8;
     static constexpr int bytes = err_off + 8;
     // FP8: K[2] (64 columns each: 128 f16 keys per token, packed in pairs) first, then as below.
-    // S[2] (N columns each) and O[2] (2N columns each: the hi and lo products side by side)
+    // S[sbufs] (N columns each) and O[2] (2N columns each: the hi and lo products side by side; the lo
+    // columns start 8 * nb columns after the hi ones)
     static constexpr uint32_t s_base = F8 ? 128 : 0;
-    static constexpr uint32_t tmem_used = s_base + 6 * N;
+    static constexpr uint32_t o_base = s_base + sbufs * N;
+    static constexpr uint32_t tmem_used = o_base + 4 * N;
     static constexpr uint32_t tmem_cols = tmem_used <= 128 ? 128 : (tmem_used <= 256 ? 256 : 512);
     static_assert(bytes <= 227 * 1024, "shared memory budget");
 };
 
 // barrier slots
-enum : int { K_FULL = 0, V_FULL = 3, KV_EMPTY = 6, S_FULL = 9, S_FREE = 11, P_FULL = 13, P_FREE = 14, O_FULL = 15,
-             O_FREE = 17, Q_FULL = 19, Q_EMPTY = 21, I_FULL = 23, I_EMPTY = 27, DRAIN = 31, GRP = 32,
-             // FP8 only: raw code ring, converted K (tensor memory), converted V (shared memory), converted Q
-             R_FULL = 34, R_EMPTY = 38, KT_FULL = 42, KT_FREE = 44, VC_FULL = 46, VC_FREE = 48, QC_FULL = 50 };
+enum : int { K_FULL = 0, V_FULL = 3, KV_EMPTY = 6, S_FULL = 9, S_FREE = 13, P_FULL = 17, P_FREE = 19, O_FULL = 21,
+             O_FREE = 23, Q_FULL = 25, Q_EMPTY = 27, I_FULL = 29, I_EMPTY = 33, DRAIN = 37, DRAIN_PV = 38, GRP = 39,
+             // FP8 only: code ring (R_EMPTY: the stage's PV product is done), converted K (tensor memory),
+             // converted V (in the stage), converted Q
+             R_FULL = 41, R_EMPTY = 47, KT_FULL = 53, KT_FREE = 55, VC_FULL = 57, QC_FULL = 63,
+             // FP8: the unit slot's score factors are written (the softmax releases the slot after reading)
+             QF_FULL = 65 };
 
 __device__ __forceinline__ void record_status(int *status, int code)
 {
@@ -315,13 +328,49 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
 __device__ __forceinline__ float f16_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
 __device__ __forceinline__ float f16_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
+// 32 lanes x 32 bits, NC (4, 8 or 16) consecutive columns per thread.
+template <int NC>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, uint32_t (&r)[NC])
+{
+    if constexpr (NC == 16) {
+        tmem_ld16(taddr, r);
+    } else if constexpr (NC == 8) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                       "=r"(r[7])
+                     : "r"(taddr));
+    } else {
+        static_assert(NC == 4, "4, 8 or 16 columns");
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                     : "r"(taddr));
+    }
+}
+
+template <int NC>
+__device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t (&r)[NC])
+{
+    if constexpr (NC == 16) {
+        tmem_st16(taddr, r);
+    } else if constexpr (NC == 8) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+                     "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                     : "memory");
+    } else {
+        static_assert(NC == 4, "4, 8 or 16 columns");
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]),
+                     "r"(r[1]), "r"(r[2]), "r"(r[3])
+                     : "memory");
+    }
+}
+
 // ---------------------------------------------------------------------------------------------
-template <int N, bool F8>
-__global__ void __launch_bounds__(TcCfg<N, F8>::threads, 1)
+template <int N, bool F8, int HW>
+__global__ void __launch_bounds__(TcCfg<N, F8, HW>::threads, 1)
 decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a)
 {
-    using C = TcCfg<N, F8>;
+    using C = TcCfg<N, F8, HW>;
     // the 128-byte swizzle needs 1024-byte aligned tiles; the whole budget is used, so there is no room
     // to realign: a misaligned window is reported and the CTA does nothing
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -345,21 +394,21 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     uint8_t *ps = smem + C::p_off;
 
     const int conv_warp0 = 4 * C::nwg;
-    const int producer_warp = conv_warp0 + C::conv_warps, mma_warp = producer_warp + 1;
-    constexpr int unit_readers = 1 + kWG * C::nwg + 32 * C::conv_warps;   // MMA + softmax + converter
+    const int producer_warp = conv_warp0 + C::conv_warps, mma_warp = producer_warp + 1, pv_warp = mma_warp + 1;
+    constexpr int unit_readers = 2 + kWG * C::nwg + 32 * C::conv_warps;   // 2 MMA issuers + softmax + converter
     if (threadIdx.x == 0) {
         if constexpr (F8) {
             for (int s = 0; s < C::stages; ++s) {
                 mbar_init(&bar[R_FULL + s], 1);
-                mbar_init(&bar[R_EMPTY + s], kWG);
+                mbar_init(&bar[R_EMPTY + s], 1);
+                mbar_init(&bar[VC_FULL + s], kWG);
             }
             for (int s = 0; s < 2; ++s) {
                 mbar_init(&bar[KT_FULL + s], kWG);
                 mbar_init(&bar[KT_FREE + s], 1);
-                mbar_init(&bar[VC_FULL + s], kWG);
-                mbar_init(&bar[VC_FREE + s], 1);
                 mbar_init(&bar[QC_FULL + s], kWG);
             }
+            for (int s = 0; s < kQD; ++s) mbar_init(&bar[QF_FULL + s], kWG);
         } else {
             for (int s = 0; s < C::stages; ++s) {
                 mbar_init(&bar[K_FULL + s], 1);
@@ -367,21 +416,26 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 mbar_init(&bar[KV_EMPTY + s], 1);
             }
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < C::sbufs; ++s) {
             mbar_init(&bar[S_FULL + s], 1);
             mbar_init(&bar[S_FREE + s], kWG * C::nwg);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&bar[O_FULL + s], 1);
             mbar_init(&bar[O_FREE + s], kWG * C::nwg);
             mbar_init(&bar[Q_FULL + s], 1);
             mbar_init(&bar[Q_EMPTY + s], 1);
         }
-        mbar_init(&bar[P_FULL], kWG * C::nwg);
-        mbar_init(&bar[P_FREE], 1);
+        for (int s = 0; s < C::pbufs; ++s) {
+            mbar_init(&bar[P_FULL + s], kWG * C::nwg);
+            mbar_init(&bar[P_FREE + s], 1);
+        }
         for (int s = 0; s < kQD; ++s) {
             mbar_init(&bar[I_FULL + s], 1);
             mbar_init(&bar[I_EMPTY + s], unit_readers);
         }
         mbar_init(&bar[DRAIN], 1);
+        mbar_init(&bar[DRAIN_PV], 1);
         for (int w = 0; w < C::nwg; ++w) mbar_init(&bar[GRP + w], kWG);
         *err = 0;
         fence_barrier_init();
@@ -398,9 +452,9 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS[2] = {tmem + C::s_base, tmem + C::s_base + N};
-    // columns [0,N): V^T P_hi^T, [N,2N): V^T P_lo^T
-    const uint32_t tO[2] = {tmem + C::s_base + 2 * N, tmem + C::s_base + 4 * N};
+    const uint32_t tS0 = tmem + C::s_base;   // S buffer i at tS0 + i * N
+    // O buffer i at tO0 + 2N i: V^T P_hi^T, then (8 nb columns later) V^T P_lo^T
+    const uint32_t tO0 = tmem + C::o_base;
 
     if (warp == producer_warp) {
         // ---------------- claims units, loads the group's query rows and streams the K/V tiles
@@ -482,12 +536,10 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 mbar_wait(&bar[Q_FULL + (i & 1)], (i >> 1) & 1, a.wait_budget_ns);
         }
     } else if (warp == mma_warp) {
-        // ---------------- MMA issuer
+        // ---------------- S^T issuer: S^T = K (K-major) . Q^T (K-major), as soon as the keys and a free
+        // S buffer allow (up to four tiles ahead of the softmax)
         if (lane == 0) {
-            // S^T = K (K-major) . Q^T (K-major); [O_hi | O_lo] = V^T (MN-major) . [P_hi | P_lo]^T (MN-major)
             const uint32_t idesc_s = F8 ? umma_idesc_f16(kTok, N, 0, 0) : umma_idesc_bf16(kTok, N, 0, 0);
-            const uint32_t idesc_o = F8 ? umma_idesc_f16(kD, 2 * N, 1, 1) : umma_idesc_bf16(kD, 2 * N, 1, 1);
-            const uint32_t p_addr = smem_u32(ps);
             int tcount = 0, icount = 0;
             bool ok = true;
             while (ok) {
@@ -498,81 +550,105 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 mbar_arrive(&bar[I_EMPTY + slot]);
                 if (t_end < 0) break;
                 const int ntl = (t_end - t_begin + kTok - 1) / kTok;
-                const int qb = icount & 1, ob = icount & 1;
+                const int qb = icount & 1;
                 if (!wait_or_fail(&bar[(F8 ? QC_FULL : Q_FULL) + qb], (icount >> 1) & 1, a, err)) break;
-                if (icount >= 2 && !wait_or_fail(&bar[O_FREE + ob], ((icount >> 1) - 1) & 1, a, err)) break;
                 const uint32_t q_addr = smem_u32(smem + C::q_off + qb * C::q_bytes);
-                for (int jj = 0; jj <= ntl; ++jj) {
-                    if (jj < ntl) {
-                        const int T = tcount + jj;
-                        const int s = T % C::stages;
-                        if (!wait_or_fail(&bar[(F8 ? KT_FULL + (T & 1) : K_FULL + s)],
-                                          F8 ? ((T >> 1) & 1) : ((T / C::stages) & 1), a, err)) {
-                            ok = false;
-                            break;
-                        }
-                        if (T >= 2 && !wait_or_fail(&bar[S_FREE + (T & 1)], ((T >> 1) - 1) & 1, a, err)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        if constexpr (F8) {
-                            // A = the converted keys in tensor memory: 16 head coordinates = 8 columns
-                            const uint32_t k_tmem = tmem + (T & 1) * 64;
-#pragma unroll
-                            for (int ks = 0; ks < kD / 16; ++ks) {
-                                const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
-                                umma_ts(tS[T & 1], k_tmem + ks * 8, umma_smem_desc(qa, 16, 1024, 2), idesc_s,
-                                            ks > 0 ? 1u : 0u);
-                            }
-                            umma_commit(&bar[S_FULL + (T & 1)]);
-                            umma_commit(&bar[KT_FREE + (T & 1)]);
-                        } else {
-                            const uint32_t k_addr = smem_u32(smem + s * C::stage_bytes);
-#pragma unroll
-                            for (int ks = 0; ks < kD / 16; ++ks) {
-                                const uint32_t ka = k_addr + (ks >> 2) * kHalf + (ks & 3) * 32;
-                                const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
-                                umma_ss(tS[T & 1], umma_smem_desc(ka, 16, 1024, 2),
-                                             umma_smem_desc(qa, 16, 1024, 2), idesc_s, ks > 0 ? 1u : 0u);
-                            }
-                            umma_commit(&bar[S_FULL + (T & 1)]);
-                        }
+                for (int jj = 0; jj < ntl; ++jj) {
+                    const int T = tcount + jj;
+                    const int s = T % C::stages, sb = T % C::sbufs;
+                    if (!wait_or_fail(&bar[(F8 ? KT_FULL + (T & 1) : K_FULL + s)],
+                                      F8 ? ((T >> 1) & 1) : ((T / C::stages) & 1), a, err)) {
+                        ok = false;
+                        break;
                     }
-                    if (jj >= 1) {
-                        const int T = tcount + jj - 1;
-                        const int s = T % C::stages;
-                        if (!wait_or_fail(&bar[P_FULL], T & 1, a, err)) { ok = false; break; }
-                        if (!wait_or_fail(&bar[(F8 ? VC_FULL + (T & 1) : V_FULL + s)],
-                                          F8 ? ((T >> 1) & 1) : ((T / C::stages) & 1), a, err)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint32_t v_addr = F8 ? smem_u32(smem + C::vc_off + (T & 1) * kTile)
-                                                   : smem_u32(smem + s * C::stage_bytes + kTile);
-                        // [O_hi | O_lo] += V^T [P_hi | P_lo]^T in one product of width 2N: the lo blocks
-                        // follow the hi blocks at the same 2048-byte stride, so they are simply more columns
+                    if (T >= C::sbufs &&
+                        !wait_or_fail(&bar[S_FREE + sb], ((T / C::sbufs) - 1) & 1, a, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tS0 + sb * N;
+                    if constexpr (F8) {
+                        // A = the converted keys in tensor memory: 16 head coordinates = 8 columns
+                        const uint32_t k_tmem = tmem + (T & 1) * 64;
 #pragma unroll
-                        for (int ks = 0; ks < kTok / 16; ++ks) {
-                            // A = V^T: 16 tokens (two 8-row groups, 1024 B apart), 64-column blocks kHalf apart
-                            // B = P^T: 16 tokens (two 128-byte core-matrix groups), 8-head blocks 2048 B apart
-                            umma_ss(tO[ob], umma_smem_desc(v_addr + ks * 2048, kHalf, 1024, 2),
-                                         umma_smem_desc(p_addr + ks * 256, 128, 2048, 0), idesc_o,
-                                         (jj > 1 || ks > 0) ? 1u : 0u);
+                        for (int ks = 0; ks < kD / 16; ++ks) {
+                            const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
+                            umma_ts(d_tmem, k_tmem + ks * 8, umma_smem_desc(qa, 16, 1024, 2), idesc_s,
+                                    ks > 0 ? 1u : 0u);
                         }
-                        umma_commit(&bar[P_FREE]);
-                        umma_commit(&bar[(F8 ? VC_FREE + (T & 1) : KV_EMPTY + s)]);
+                        umma_commit(&bar[S_FULL + sb]);
+                        umma_commit(&bar[KT_FREE + (T & 1)]);
+                    } else {
+                        const uint32_t k_addr = smem_u32(smem + s * C::stage_bytes);
+#pragma unroll
+                        for (int ks = 0; ks < kD / 16; ++ks) {
+                            const uint32_t ka = k_addr + (ks >> 2) * kHalf + (ks & 3) * 32;
+                            const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
+                            umma_ss(d_tmem, umma_smem_desc(ka, 16, 1024, 2), umma_smem_desc(qa, 16, 1024, 2),
+                                    idesc_s, ks > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&bar[S_FULL + sb]);
                     }
                 }
                 if (!ok) break;
-                umma_commit(&bar[O_FULL + ob]);
-                umma_commit(&bar[Q_EMPTY + qb]);
+                umma_commit(&bar[Q_EMPTY + qb]);   // the unit's query rows are no longer read
                 tcount += ntl;
                 ++icount;
             }
             umma_commit(&bar[DRAIN]);
             mbar_wait(&bar[DRAIN], 0, a.wait_budget_ns);
+        }
+    } else if (warp == pv_warp) {
+        // ---------------- PV issuer: [O_hi | O_lo] += V^T (MN-major) . [P_hi | P_lo]^T (MN-major)
+        if (lane == 0) {
+            constexpr int npv = 16 * C::nb;   // the hi and lo blocks that carry heads
+            const uint32_t idesc_o = F8 ? umma_idesc_f16(kD, npv, 1, 1) : umma_idesc_bf16(kD, npv, 1, 1);
+            int tcount = 0, icount = 0;
+            bool ok = true;
+            while (ok) {
+                const int slot = icount % kQD;
+                if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
+                volatile int *q = queue + slot * 8;
+                const int t_begin = q[3], t_end = q[4];
+                mbar_arrive(&bar[I_EMPTY + slot]);
+                if (t_end < 0) break;
+                const int ntl = (t_end - t_begin + kTok - 1) / kTok;
+                const int ob = icount & 1;
+                if (icount >= 2 && !wait_or_fail(&bar[O_FREE + ob], ((icount >> 1) - 1) & 1, a, err)) break;
+                const uint32_t d_tmem = tO0 + ob * 2 * N;
+                for (int jj = 0; jj < ntl; ++jj) {
+                    const int T = tcount + jj;
+                    const int s = T % C::stages;
+                    const int pb = T % C::pbufs;
+                    if (!wait_or_fail(&bar[P_FULL + pb], (T / C::pbufs) & 1, a, err)) { ok = false; break; }
+                    if (!wait_or_fail(&bar[(F8 ? VC_FULL : V_FULL) + s], (T / C::stages) & 1, a, err)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t v_addr = smem_u32(smem + s * C::stage_bytes + (F8 ? 0 : kTile));
+                    // one product of width 16 nb: the lo blocks follow the hi blocks at the same 2048-byte
+                    // stride, so they are simply more columns
+                    const uint32_t p_addr = smem_u32(ps + pb * 2 * C::p_half);
+#pragma unroll
+                    for (int ks = 0; ks < kTok / 16; ++ks) {
+                        // A = V^T: 16 tokens (two 8-row groups, 1024 B apart), 64-column blocks kHalf apart
+                        // B = P^T: 16 tokens (two 128-byte core-matrix groups), 8-head blocks 2048 B apart
+                        umma_ss(d_tmem, umma_smem_desc(v_addr + ks * 2048, kHalf, 1024, 2),
+                                umma_smem_desc(p_addr + ks * 256, 128, 2048, 0), idesc_o, (jj > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&bar[P_FREE + pb]);
+                    // the stage's keys were read by an S^T product that completed before this P existed
+                    umma_commit(&bar[(F8 ? R_EMPTY : KV_EMPTY) + s]);
+                }
+                if (!ok) break;
+                umma_commit(&bar[O_FULL + ob]);
+                tcount += ntl;
+                ++icount;
+            }
+            umma_commit(&bar[DRAIN_PV]);
+            mbar_wait(&bar[DRAIN_PV], 0, a.wait_budget_ns);
         }
     } else if (F8 && warp >= conv_warp0) {
         // ---------------- FP8 converter: thread ct owns token ct of each tile (TMEM lane ct of K)
@@ -622,25 +698,26 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     o.w = pack_f16x2(bf16_lo(v[i].w) * up, bf16_hi(v[i].w) * up);
                     *reinterpret_cast<uint4 *>(qs + (k >> 3) * C::q_half + row * 128 + (k & 7) * 16) = o;
                 }
-                if (j0 == 0) qfac[qb * N + row] = a.qk_factor * down;
+                if (j0 == 0) qfac[slot * N + row] = a.qk_factor * down;
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar[QC_FULL + qb]);
+            mbar_arrive(&bar[QF_FULL + slot]);
             const int ntl = (t_end - t_begin + kTok - 1) / kTok;
             bool ok = true;
             for (int jj = 0; jj < ntl; ++jj) {
                 const int T = tcount + jj;
                 const int s = T % C::stages, cb = T & 1;
                 if (!wait_or_fail(&bar[R_FULL + s], (T / C::stages) & 1, a, err)) { ok = false; break; }
-                // the raw tiles were stored with the 128-byte swizzle: chunk c of row ct at c ^ (ct & 7)
-                const uint8_t *krow = smem + s * C::stage_bytes + ct * 128;
+                // the raw tiles were stored with the 128-byte swizzle: chunk c of row ct at c ^ (ct & 7).
+                // This thread's key row and value row, into registers.
+                uint8_t *krow = smem + s * C::stage_bytes + ct * 128;
                 uint4 kr[8], vr[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     kr[c] = *reinterpret_cast<const uint4 *>(krow + ((c ^ (ct & 7)) << 4));
                     vr[c] = *reinterpret_cast<const uint4 *>(krow + kHalf + ((c ^ (ct & 7)) << 4));
                 }
-                mbar_arrive(&bar[R_EMPTY + s]);
                 // tokens past the piece's end may hold anything (NaN codes included): they become zeros,
                 // so that no 0 * NaN reaches an accumulator
                 const bool valid = (t_begin + jj * kTok + ct) < t_end;
@@ -667,9 +744,9 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bar[KT_FULL + cb]);
-                // values -> f16 tile [2 halves][128 rows][128 B], 128-byte swizzle, row ct
-                if (T >= 2 && !wait_or_fail(&bar[VC_FREE + cb], ((T >> 1) - 1) & 1, a, err)) { ok = false; break; }
-                uint8_t *vt = smem + C::vc_off + cb * kTile + ct * 128;
+                // values -> f16 tile [2 halves][128 rows][128 B] with the 128-byte swizzle over the stage:
+                // row ct of half 0 is where this thread's key codes were, row ct of half 1 where its value
+                // codes were
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint4 lo4, hi4;
@@ -682,12 +759,12 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                         hi4 = lo4;
                     }
                     const int j = 2 * (c & 3);   // 16 codes = two 16-byte f16 chunks of half c / 4
-                    uint8_t *half = vt + (c >> 2) * kHalf;
-                    *reinterpret_cast<uint4 *>(half + ((j ^ (ct & 7)) << 4)) = lo4;
-                    *reinterpret_cast<uint4 *>(half + (((j + 1) ^ (ct & 7)) << 4)) = hi4;
+                    uint8_t *row = krow + (c >> 2) * kHalf;
+                    *reinterpret_cast<uint4 *>(row + ((j ^ (ct & 7)) << 4)) = lo4;
+                    *reinterpret_cast<uint4 *>(row + (((j + 1) ^ (ct & 7)) << 4)) = hi4;
                 }
                 fence_proxy_async_smem();
-                mbar_arrive(&bar[VC_FULL + cb]);
+                mbar_arrive(&bar[VC_FULL + s]);
             }
             if (!ok) break;
             tcount += ntl;
@@ -699,7 +776,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         const int wg = warp >> 2;
         const int quarter = warp & 3;              // TMEM lane quarter this warp may access
         const int t = quarter * 32 + lane;
-        const int hs = wg * kHPW;                  // first head (column) of this warpgroup
+        const int hs = wg * HW;                  // first head (column) of this warpgroup
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         volatile int *myvote = vote + wg * 8;
         int tcount = 0, icount = 0, uses = 0;
@@ -708,19 +785,19 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         // tile, so that waiting for the unit's last PV product overlaps useful work.
         bool pend = false;
         int pb = 0, pkvh = 0, psplit = 0, pob = 0;
-        float pm[kHPW];
+        float pm[HW];
         // FP8: O carries 128 p v_code; the value scale and 1/128 are applied here
         const float ofac = F8 ? a.o_factor : 1.f;
         auto epilogue = [&]() -> bool {
             if (!group_sync(&bar[GRP + wg], uses, a, err)) return false;      // lsum[pob] complete
             if (!wait_or_fail(&bar[O_FULL + pob], (((icount - 1) >> 1)) & 1, a, err)) return false;
             tc_fence_after();
-            uint32_t o[kHPW], olo[kHPW];
-            tmem_ld16(tO[pob] + lane_off + hs, o);
-            tmem_ld16(tO[pob] + lane_off + N + hs, olo);
+            uint32_t o[HW], olo[HW];
+            tmem_ldn<HW>(tO0 + pob * 2 * N + lane_off + hs, o);
+            tmem_ldn<HW>(tO0 + pob * 2 * N + lane_off + 8 * C::nb + hs, olo);
             tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < kHPW; ++h)
+            for (int h = 0; h < HW; ++h)
                 o[h] = __float_as_uint((__uint_as_float(o[h]) + __uint_as_float(olo[h])) * ofac);
             const float *ls = lsum + pob * 4 * N;
             const int d = t;
@@ -728,7 +805,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             if (npieces == 1) {
                 // the whole history in one unit: normalise and write the output
 #pragma unroll
-                for (int h = 0; h < kHPW; ++h) {
+                for (int h = 0; h < HW; ++h) {
                     const int hg = hs + h;
                     if (hg >= g) break;
                     const float L = ls[hg] + ls[N + hg] + ls[2 * N + hg] + ls[3 * N + hg];
@@ -738,7 +815,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             } else {
                 // one piece of several: a partial (o, m, l) for decode_combine_kernel
 #pragma unroll
-                for (int h = 0; h < kHPW; ++h) {
+                for (int h = 0; h < HW; ++h) {
                     const int hg = hs + h;
                     if (hg >= g) break;
                     const float L = ls[hg] + ls[N + hg] + ls[2 * N + hg] + ls[3 * N + hg];
@@ -760,45 +837,48 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
             volatile int *qq = queue + slot * 8;
             const int b = qq[0], kvh = qq[1], split = qq[2], t_begin = qq[3], t_end = qq[4];
-            mbar_arrive(&bar[I_EMPTY + slot]);
             if (t_end < 0) {
+                mbar_arrive(&bar[I_EMPTY + slot]);
                 if (pend) epilogue();   // the pending unit is icount - 1, as in the loop
                 break;
             }
-            const int ntl = (t_end - t_begin + kTok - 1) / kTok;
-            const int ob = icount & 1;
-            // score factor per head: log2(e) * scale (FP8: times k_scale and the head's 2^-e)
-            float qf[kHPW];
+            // score factor per head: log2(e) * scale (FP8: times k_scale and the head's 2^-e, which the
+            // converter leaves in the unit's slot; the slot is released only after reading them)
+            float qf[HW];
             if constexpr (F8) {
-                if (!wait_or_fail(&bar[QC_FULL + (icount & 1)], (icount >> 1) & 1, a, err)) break;
+                if (!wait_or_fail(&bar[QF_FULL + slot], (icount / kQD) & 1, a, err)) break;
 #pragma unroll
-                for (int h = 0; h < kHPW; ++h) qf[h] = qfac[(icount & 1) * N + hs + h];
+                for (int h = 0; h < HW; ++h) qf[h] = qfac[slot * N + hs + h];
             } else {
 #pragma unroll
-                for (int h = 0; h < kHPW; ++h) qf[h] = a.qscale;
+                for (int h = 0; h < HW; ++h) qf[h] = a.qscale;
             }
-            float m_use[kHPW], l_part[kHPW];
+            mbar_arrive(&bar[I_EMPTY + slot]);
+            const int ntl = (t_end - t_begin + kTok - 1) / kTok;
+            const int ob = icount & 1;
+            float m_use[HW], l_part[HW];
 #pragma unroll
-            for (int h = 0; h < kHPW; ++h) {
+            for (int h = 0; h < HW; ++h) {
                 m_use[h] = -INFINITY;
                 l_part[h] = 0.f;
             }
             for (int jj = 0; jj < ntl; ++jj) {
                 const int T = tcount + jj;
-                const int sb = T & 1;
-                if (!wait_or_fail(&bar[S_FULL + sb], (T >> 1) & 1, a, err)) { ok = false; break; }
+                const int sb = T & 1;                  // vote and maxima buffers
+                const int sbuf = T % C::sbufs;         // S buffer
+                if (!wait_or_fail(&bar[S_FULL + sbuf], (T / C::sbufs) & 1, a, err)) { ok = false; break; }
                 tc_fence_after();
-                uint32_t raw[kHPW];
-                tmem_ld16(tS[sb] + lane_off + hs, raw);
+                uint32_t raw[HW];
+                tmem_ldn<HW>(tS0 + sbuf * N + lane_off + hs, raw);
                 tmem_wait_ld();
                 tc_fence_before();
-                mbar_arrive(&bar[S_FREE + sb]);
+                mbar_arrive(&bar[S_FREE + sbuf]);
 
                 const bool valid = (t_begin + jj * kTok + t) < t_end;
-                float x[kHPW];
+                float x[HW];
                 bool over = false;
 #pragma unroll
-                for (int h = 0; h < kHPW; ++h) {
+                for (int h = 0; h < HW; ++h) {
                     x[h] = valid ? __uint_as_float(raw[h]) * qf[h] : -INFINITY;
                     over |= x[h] > m_use[h] + kMoveThreshold;
                 }
@@ -807,14 +887,14 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 if (!group_sync(&bar[GRP + wg], uses, a, err)) { ok = false; break; }
                 const bool any_move = (myvote[sb * 4 + 0] | myvote[sb * 4 + 1] | myvote[sb * 4 + 2] |
                                        myvote[sb * 4 + 3]) != 0;
-                float alpha[kHPW];
+                float alpha[HW];
                 bool rescale_o = false;
 #pragma unroll
-                for (int h = 0; h < kHPW; ++h) alpha[h] = 1.f;
+                for (int h = 0; h < HW; ++h) alpha[h] = 1.f;
                 if (any_move) {
                     // this tile's maximum over all 128 tokens, per head
 #pragma unroll
-                    for (int h = 0; h < kHPW; ++h) {
+                    for (int h = 0; h < HW; ++h) {
                         float mx = x[h];
                         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
                         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
@@ -825,7 +905,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     }
                     if (!group_sync(&bar[GRP + wg], uses, a, err)) { ok = false; break; }
 #pragma unroll
-                    for (int h = 0; h < kHPW; ++h) {
+                    for (int h = 0; h < HW; ++h) {
                         const float *rr = red + sb * 4 * N + hs + h;
                         const float tm = fmaxf(fmaxf(rr[0], rr[N]), fmaxf(rr[2 * N], rr[3 * N]));
                         const float m_new = fmaxf(m_use[h], tm);
@@ -838,28 +918,31 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     }
                     rescale_o = rescale_o && (jj > 0);          // uniform: the warpgroup saw the same maxima
                 }
-                float p[kHPW];
+                float p[HW];
 #pragma unroll
-                for (int h = 0; h < kHPW; ++h) {
+                for (int h = 0; h < HW; ++h) {
                     p[h] = ex2(x[h] - m_use[h]);
                     l_part[h] += p[h];
                 }
-                if (T >= 1) {
-                    // previous PV done: P buffer free and this unit's O stable
-                    if (!wait_or_fail(&bar[P_FREE], (T - 1) & 1, a, err)) { ok = false; break; }
-                    tc_fence_after();
-                    if (rescale_o) {
+                // this tile's P buffer must have been read by its last PV product; a rescale of O also
+                // needs the previous tile's PV finished
+                const int pbuf = T % C::pbufs;
+                if (T >= C::pbufs &&
+                    !wait_or_fail(&bar[P_FREE + pbuf], ((T / C::pbufs) - 1) & 1, a, err)) { ok = false; break; }
+                if (rescale_o && C::pbufs == 2 &&
+                    !wait_or_fail(&bar[P_FREE + ((T - 1) & 1)], ((T - 1) >> 1) & 1, a, err)) { ok = false; break; }
+                tc_fence_after();
+                if (rescale_o) {
 #pragma unroll
-                        for (int part = 0; part < 2; ++part) {   // the hi and the lo columns
-                            uint32_t o[kHPW];
-                            tmem_ld16(tO[ob] + lane_off + part * N + hs, o);
-                            tmem_wait_ld();
+                    for (int part = 0; part < 2; ++part) {   // the hi and the lo columns
+                        uint32_t o[HW];
+                        tmem_ldn<HW>(tO0 + ob * 2 * N + lane_off + part * 8 * C::nb + hs, o);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int h = 0; h < kHPW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-                            tmem_st16(tO[ob] + lane_off + part * N + hs, o);
-                        }
-                        tmem_wait_st();
+                        for (int h = 0; h < HW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+                        tmem_stn<HW>(tO0 + ob * 2 * N + lane_off + part * 8 * C::nb + hs, o);
                     }
+                    tmem_wait_st();
                 }
                 if constexpr (!F8) {
                     // Rows past the history may hold anything (NaN included) and the tensor cores would
@@ -878,12 +961,16 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     }
                 }
                 // P^T, MN-major without swizzle: core matrices of 8 tokens x 8 heads (128 B), each weight
-                // as hi plus lo = (p - hi) in the products' 16-bit type (FP8: f16 terms of 128 p)
+                // as hi plus lo = (p - hi) in the products' 16-bit type (FP8: f16 terms of 128 p).  With
+                // four heads only the first half of each 16-byte core-matrix row is written: the other
+                // four columns of the products are never read.
+                uint8_t *pdst = ps + pbuf * 2 * C::p_half + (t >> 3) * 128 + (t & 7) * 16;
 #pragma unroll
-                for (int hb = 0; hb < kHPW / 8; ++hb) {
+                for (int hb = 0; hb < (HW + 7) / 8; ++hb) {
+                    constexpr int E = HW < 8 ? HW / 2 : 4;   // packed pairs per block
                     uint32_t hi[4], lo[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
+                    for (int e = 0; e < E; ++e) {
                         if constexpr (F8) {
                             const float a0 = p[hb * 8 + 2 * e] * 128.f, a1 = p[hb * 8 + 2 * e + 1] * 128.f;
                             hi[e] = pack_f16x2(a0, a1);
@@ -894,13 +981,18 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                             lo[e] = pack2(a0 - bf16_lo(hi[e]), a1 - bf16_hi(hi[e]));
                         }
                     }
-                    uint8_t *dst = ps + (hs / 8 + hb) * 2048 + (t >> 3) * 128 + (t & 7) * 16;
-                    *reinterpret_cast<uint4 *>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    *reinterpret_cast<uint4 *>(dst + C::p_bytes) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    uint8_t *dst = pdst + (hs / 8 + hb) * 2048;
+                    if constexpr (E == 4) {
+                        *reinterpret_cast<uint4 *>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        *reinterpret_cast<uint4 *>(dst + C::p_half) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                    } else {
+                        *reinterpret_cast<uint2 *>(dst) = make_uint2(hi[0], hi[1]);
+                        *reinterpret_cast<uint2 *>(dst + C::p_half) = make_uint2(lo[0], lo[1]);
+                    }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(&bar[P_FULL]);
+                mbar_arrive(&bar[P_FULL + pbuf]);
                 // the previous unit's epilogue, now that its last PV has long been issued
                 if (jj == 0 && pend && !epilogue()) { ok = false; break; }
             }
@@ -908,7 +1000,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             // this unit's weight sums per head, reduced over each warp's 32 tokens; the CTA-wide sum is
             // finished in the (deferred) epilogue
 #pragma unroll
-            for (int h = 0; h < kHPW; ++h) {
+            for (int h = 0; h < HW; ++h) {
                 float v = l_part[h];
                 v += __shfl_xor_sync(0xffffffffu, v, 16);
                 v += __shfl_xor_sync(0xffffffffu, v, 8);
@@ -923,7 +1015,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             psplit = split;
             pob = ob;
 #pragma unroll
-            for (int h = 0; h < kHPW; ++h) pm[h] = m_use[h];
+            for (int h = 0; h < HW; ++h) pm[h] = m_use[h];
             tcount += ntl;
             ++icount;
         }
@@ -937,16 +1029,16 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     }
 }
 
-template <int N, bool F8>
+template <int N, bool F8, int HW>
 cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, const CUtensorMap &tmQ,
                               const DecodeArgs &a, cudaStream_t stream)
 {
-    const int smem = TcCfg<N, F8>::bytes;
+    const int smem = TcCfg<N, F8, HW>::bytes;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(decode_persistent_kernel<N, F8>,
+        cudaError_t e = cudaFuncSetAttribute(decode_persistent_kernel<N, F8, HW>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
@@ -955,7 +1047,7 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
     // waits for (griddepcontrol.wait) before reading the plan
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.num_ctas);
-    cfg.blockDim = dim3(TcCfg<N, F8>::threads);
+    cfg.blockDim = dim3(TcCfg<N, F8, HW>::threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -963,7 +1055,7 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_persistent_kernel<N, F8>, tmK, tmV, tmQ, a);
+    return cudaLaunchKernelEx(&cfg, decode_persistent_kernel<N, F8, HW>, tmK, tmV, tmQ, a);
 }
 
 }  // namespace
@@ -978,12 +1070,16 @@ cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, con
                              const DecodeArgs &a, cudaStream_t stream, bool fp8)
 {
     if (fp8) {
-        if (a.group <= 16) return launch_persistent<16, true>(tmK, tmV, tmQ, a, stream);
-        if (a.group <= 32) return launch_persistent<32, true>(tmK, tmV, tmQ, a, stream);
+        if (a.group <= 4) return launch_persistent<16, true, 4>(tmK, tmV, tmQ, a, stream);
+        if (a.group <= 8) return launch_persistent<16, true, 8>(tmK, tmV, tmQ, a, stream);
+        if (a.group <= 16) return launch_persistent<16, true, 16>(tmK, tmV, tmQ, a, stream);
+        if (a.group <= 32) return launch_persistent<32, true, 16>(tmK, tmV, tmQ, a, stream);
         return cudaErrorInvalidValue;
     }
-    if (a.group <= 16) return launch_persistent<16, false>(tmK, tmV, tmQ, a, stream);
-    if (a.group <= 32) return launch_persistent<32, false>(tmK, tmV, tmQ, a, stream);
+    if (a.group <= 4) return launch_persistent<16, false, 4>(tmK, tmV, tmQ, a, stream);
+    if (a.group <= 8) return launch_persistent<16, false, 8>(tmK, tmV, tmQ, a, stream);
+    if (a.group <= 16) return launch_persistent<16, false, 16>(tmK, tmV, tmQ, a, stream);
+    if (a.group <= 32) return launch_persistent<32, false, 16>(tmK, tmV, tmQ, a, stream);
     return cudaErrorInvalidValue;
 }
 
