@@ -70,8 +70,12 @@ struct TcCfg {
     static constexpr int nwg = HW == 16 ? N / 16 : 1;         // softmax warpgroups
     static constexpr int nb = HW <= 8 ? 1 : N / 8;            // 8-head blocks of P^T / O^T that carry heads
     static constexpr int conv_warps = F8 ? 4 : 0;             // FP8: the converter warpgroup
-    // + TMA warp + S^T issuer warp + PV issuer warp
-    static constexpr int threads = kWG * nwg + 32 * conv_warps + 96;
+    // + TMA warp + S^T issuer warp + PV issuer warp.  FP8 with 32 heads: the last three warps are padded
+    // to a warpgroup and the registers are redistributed (setmaxnreg): 512 threads launch with 128
+    // registers each, the softmax warpgroups then take 176, the converter 104 and the last warpgroup 56
+    // (2 * 176 + 104 + 56 = 4 * 128, so every increase is covered by the decreases)
+    static constexpr bool regsplit = F8 && N == 32;
+    static constexpr int threads = regsplit ? 512 : kWG * nwg + 32 * conv_warps + 96;
     static constexpr int sbufs = 4;                            // S^T buffers: QK^T runs up to four tiles ahead
     static constexpr int pbufs = (F8 || N == 16) ? 2 : 1;      // P^T buffers (2: the softmax runs a tile ahead)
     static constexpr int stages = F8 ? (N == 32 ? 5 : 6) : 3;
@@ -456,202 +460,210 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     // O buffer i at tO0 + 2N i: V^T P_hi^T, then (8 nb columns later) V^T P_lo^T
     const uint32_t tO0 = tmem + C::o_base;
 
-    if (warp == producer_warp) {
-        // ---------------- claims units, loads the group's query rows and streams the K/V tiles
-        if (lane == 0) {
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            tma_prefetch_desc(&tmQ);
-            const int units = a.plan_hdr[1] * a.Hkv;
-            int tcount = 0, icount = 0, issued_tiles = 0;
-            while (true) {
-                const int u = atomicAdd(&a.plan_hdr[0], 1);
-                const int slot = icount % kQD;
-                if (icount >= kQD && !wait_or_fail(&bar[I_EMPTY + slot], ((icount / kQD) - 1) & 1, a, err)) break;
-                volatile int *q = queue + slot * 8;
-                if (u >= units) {
-                    q[4] = -1;                         // no more work
+    // Register split (FP8, 32 heads): each warpgroup sets its share first thing in its own branch, the
+    // same instruction for all four of its warps; 2 * 176 + 104 + 56 = 4 * 128, the launch's share.
+    static_assert(!C::regsplit || (C::threads == 512 && 2 * 176 + 104 + 56 == 4 * 128), "register split");
+    if (warp >= producer_warp) {
+        // the last warpgroup: producer, S^T issuer, PV issuer (and, with the split, one idle warp)
+        if constexpr (C::regsplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+        if (warp == producer_warp) {
+            // ---------------- claims units, loads the group's query rows and streams the K/V tiles
+            if (lane == 0) {
+                tma_prefetch_desc(&tmK);
+                tma_prefetch_desc(&tmV);
+                tma_prefetch_desc(&tmQ);
+                const int units = a.plan_hdr[1] * a.Hkv;
+                int tcount = 0, icount = 0, issued_tiles = 0;
+                while (true) {
+                    const int u = atomicAdd(&a.plan_hdr[0], 1);
+                    const int slot = icount % kQD;
+                    if (icount >= kQD && !wait_or_fail(&bar[I_EMPTY + slot], ((icount / kQD) - 1) & 1, a, err)) break;
+                    volatile int *q = queue + slot * 8;
+                    if (u >= units) {
+                        q[4] = -1;                         // no more work
+                        mbar_arrive(&bar[I_FULL + slot]);
+                        break;
+                    }
+                    const int4 it = a.items[u / a.Hkv];
+                    const int kvh = u % a.Hkv;
+                    q[0] = it.x;
+                    q[1] = kvh;
+                    q[2] = it.y;
+                    q[3] = it.z;
+                    q[4] = it.w;
                     mbar_arrive(&bar[I_FULL + slot]);
-                    break;
+                    const int qb = icount & 1;
+                    if (icount >= 2 && !wait_or_fail(&bar[Q_EMPTY + qb], ((icount >> 1) - 1) & 1, a, err)) break;
+                    uint8_t *qs = smem + C::q_off + qb * C::q_bytes;
+                    mbar_arrive_expect_tx(&bar[Q_FULL + qb], C::q_bytes);
+                    tma_load_3d(qs, &tmQ, &bar[Q_FULL + qb], 0, kvh * g, it.x);
+                    tma_load_3d(qs + C::q_half, &tmQ, &bar[Q_FULL + qb], 64, kvh * g, it.x);
+                    const int ntl = (it.w - it.z + kTok - 1) / kTok;
+                    bool ok = true;
+                    for (int jj = 0; jj < ntl; ++jj, ++tcount) {
+                        const int s = tcount % C::stages;
+                        const int t0 = it.z + jj * kTok;
+                        uint8_t *ks = smem + s * C::stage_bytes;
+                        if constexpr (F8) {
+                            if (tcount >= C::stages &&
+                                !wait_or_fail(&bar[R_EMPTY + s], ((tcount / C::stages) - 1) & 1, a, err)) {
+                                ok = false;
+                                break;
+                            }
+                            // one box = 128 tokens x 128 one-byte codes of a head
+                            mbar_arrive_expect_tx(&bar[R_FULL + s], kTile);
+                            tma_load_4d(ks, &tmK, &bar[R_FULL + s], 0, kvh, t0, it.x);
+                            tma_load_4d(ks + kHalf, &tmV, &bar[R_FULL + s], 0, kvh, t0, it.x);
+                        } else {
+                            if (tcount >= C::stages &&
+                                !wait_or_fail(&bar[KV_EMPTY + s], ((tcount / C::stages) - 1) & 1, a, err)) {
+                                ok = false;
+                                break;
+                            }
+                            mbar_arrive_expect_tx(&bar[K_FULL + s], kTile);
+                            tma_load_4d(ks, &tmK, &bar[K_FULL + s], 0, kvh, t0, it.x);
+                            tma_load_4d(ks + kHalf, &tmK, &bar[K_FULL + s], 64, kvh, t0, it.x);
+                            mbar_arrive_expect_tx(&bar[V_FULL + s], kTile);
+                            tma_load_4d(ks + kTile, &tmV, &bar[V_FULL + s], 0, kvh, t0, it.x);
+                            tma_load_4d(ks + kTile + kHalf, &tmV, &bar[V_FULL + s], 64, kvh, t0, it.x);
+                        }
+                        issued_tiles = tcount + 1;
+                    }
+                    ++icount;
+                    if (!ok) break;
                 }
-                const int4 it = a.items[u / a.Hkv];
-                const int kvh = u % a.Hkv;
-                q[0] = it.x;
-                q[1] = kvh;
-                q[2] = it.y;
-                q[3] = it.z;
-                q[4] = it.w;
-                mbar_arrive(&bar[I_FULL + slot]);
-                const int qb = icount & 1;
-                if (icount >= 2 && !wait_or_fail(&bar[Q_EMPTY + qb], ((icount >> 1) - 1) & 1, a, err)) break;
-                uint8_t *qs = smem + C::q_off + qb * C::q_bytes;
-                mbar_arrive_expect_tx(&bar[Q_FULL + qb], C::q_bytes);
-                tma_load_3d(qs, &tmQ, &bar[Q_FULL + qb], 0, kvh * g, it.x);
-                tma_load_3d(qs + C::q_half, &tmQ, &bar[Q_FULL + qb], 64, kvh * g, it.x);
-                const int ntl = (it.w - it.z + kTok - 1) / kTok;
+                // leave no copy in flight
+                for (int t = issued_tiles - 1; t >= 0 && t >= issued_tiles - C::stages; --t) {
+                    const uint32_t ph = (t / C::stages) & 1;
+                    if constexpr (F8) {
+                        mbar_wait(&bar[R_FULL + t % C::stages], ph, a.wait_budget_ns);
+                    } else {
+                        mbar_wait(&bar[K_FULL + t % C::stages], ph, a.wait_budget_ns);
+                        mbar_wait(&bar[V_FULL + t % C::stages], ph, a.wait_budget_ns);
+                    }
+                }
+                for (int i = icount - 1; i >= 0 && i >= icount - 2; --i)
+                    mbar_wait(&bar[Q_FULL + (i & 1)], (i >> 1) & 1, a.wait_budget_ns);
+            }
+        } else if (warp == mma_warp) {
+            // ---------------- S^T issuer: S^T = K (K-major) . Q^T (K-major), as soon as the keys and a free
+            // S buffer allow (up to four tiles ahead of the softmax)
+            if (lane == 0) {
+                const uint32_t idesc_s = F8 ? umma_idesc_f16(kTok, N, 0, 0) : umma_idesc_bf16(kTok, N, 0, 0);
+                int tcount = 0, icount = 0;
                 bool ok = true;
-                for (int jj = 0; jj < ntl; ++jj, ++tcount) {
-                    const int s = tcount % C::stages;
-                    const int t0 = it.z + jj * kTok;
-                    uint8_t *ks = smem + s * C::stage_bytes;
-                    if constexpr (F8) {
-                        if (tcount >= C::stages &&
-                            !wait_or_fail(&bar[R_EMPTY + s], ((tcount / C::stages) - 1) & 1, a, err)) {
+                while (ok) {
+                    const int slot = icount % kQD;
+                    if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
+                    volatile int *q = queue + slot * 8;
+                    const int t_begin = q[3], t_end = q[4];
+                    mbar_arrive(&bar[I_EMPTY + slot]);
+                    if (t_end < 0) break;
+                    const int ntl = (t_end - t_begin + kTok - 1) / kTok;
+                    const int qb = icount & 1;
+                    if (!wait_or_fail(&bar[(F8 ? QC_FULL : Q_FULL) + qb], (icount >> 1) & 1, a, err)) break;
+                    const uint32_t q_addr = smem_u32(smem + C::q_off + qb * C::q_bytes);
+                    for (int jj = 0; jj < ntl; ++jj) {
+                        const int T = tcount + jj;
+                        const int s = T % C::stages, sb = T % C::sbufs;
+                        if (!wait_or_fail(&bar[(F8 ? KT_FULL + (T & 1) : K_FULL + s)],
+                                          F8 ? ((T >> 1) & 1) : ((T / C::stages) & 1), a, err)) {
                             ok = false;
                             break;
                         }
-                        // one box = 128 tokens x 128 one-byte codes of a head
-                        mbar_arrive_expect_tx(&bar[R_FULL + s], kTile);
-                        tma_load_4d(ks, &tmK, &bar[R_FULL + s], 0, kvh, t0, it.x);
-                        tma_load_4d(ks + kHalf, &tmV, &bar[R_FULL + s], 0, kvh, t0, it.x);
-                    } else {
-                        if (tcount >= C::stages &&
-                            !wait_or_fail(&bar[KV_EMPTY + s], ((tcount / C::stages) - 1) & 1, a, err)) {
+                        if (T >= C::sbufs &&
+                            !wait_or_fail(&bar[S_FREE + sb], ((T / C::sbufs) - 1) & 1, a, err)) {
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&bar[K_FULL + s], kTile);
-                        tma_load_4d(ks, &tmK, &bar[K_FULL + s], 0, kvh, t0, it.x);
-                        tma_load_4d(ks + kHalf, &tmK, &bar[K_FULL + s], 64, kvh, t0, it.x);
-                        mbar_arrive_expect_tx(&bar[V_FULL + s], kTile);
-                        tma_load_4d(ks + kTile, &tmV, &bar[V_FULL + s], 0, kvh, t0, it.x);
-                        tma_load_4d(ks + kTile + kHalf, &tmV, &bar[V_FULL + s], 64, kvh, t0, it.x);
-                    }
-                    issued_tiles = tcount + 1;
-                }
-                ++icount;
-                if (!ok) break;
-            }
-            // leave no copy in flight
-            for (int t = issued_tiles - 1; t >= 0 && t >= issued_tiles - C::stages; --t) {
-                const uint32_t ph = (t / C::stages) & 1;
-                if constexpr (F8) {
-                    mbar_wait(&bar[R_FULL + t % C::stages], ph, a.wait_budget_ns);
-                } else {
-                    mbar_wait(&bar[K_FULL + t % C::stages], ph, a.wait_budget_ns);
-                    mbar_wait(&bar[V_FULL + t % C::stages], ph, a.wait_budget_ns);
-                }
-            }
-            for (int i = icount - 1; i >= 0 && i >= icount - 2; --i)
-                mbar_wait(&bar[Q_FULL + (i & 1)], (i >> 1) & 1, a.wait_budget_ns);
-        }
-    } else if (warp == mma_warp) {
-        // ---------------- S^T issuer: S^T = K (K-major) . Q^T (K-major), as soon as the keys and a free
-        // S buffer allow (up to four tiles ahead of the softmax)
-        if (lane == 0) {
-            const uint32_t idesc_s = F8 ? umma_idesc_f16(kTok, N, 0, 0) : umma_idesc_bf16(kTok, N, 0, 0);
-            int tcount = 0, icount = 0;
-            bool ok = true;
-            while (ok) {
-                const int slot = icount % kQD;
-                if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
-                volatile int *q = queue + slot * 8;
-                const int t_begin = q[3], t_end = q[4];
-                mbar_arrive(&bar[I_EMPTY + slot]);
-                if (t_end < 0) break;
-                const int ntl = (t_end - t_begin + kTok - 1) / kTok;
-                const int qb = icount & 1;
-                if (!wait_or_fail(&bar[(F8 ? QC_FULL : Q_FULL) + qb], (icount >> 1) & 1, a, err)) break;
-                const uint32_t q_addr = smem_u32(smem + C::q_off + qb * C::q_bytes);
-                for (int jj = 0; jj < ntl; ++jj) {
-                    const int T = tcount + jj;
-                    const int s = T % C::stages, sb = T % C::sbufs;
-                    if (!wait_or_fail(&bar[(F8 ? KT_FULL + (T & 1) : K_FULL + s)],
-                                      F8 ? ((T >> 1) & 1) : ((T / C::stages) & 1), a, err)) {
-                        ok = false;
-                        break;
-                    }
-                    if (T >= C::sbufs &&
-                        !wait_or_fail(&bar[S_FREE + sb], ((T / C::sbufs) - 1) & 1, a, err)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t d_tmem = tS0 + sb * N;
-                    if constexpr (F8) {
-                        // A = the converted keys in tensor memory: 16 head coordinates = 8 columns
-                        const uint32_t k_tmem = tmem + (T & 1) * 64;
-#pragma unroll
-                        for (int ks = 0; ks < kD / 16; ++ks) {
-                            const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
-                            umma_ts(d_tmem, k_tmem + ks * 8, umma_smem_desc(qa, 16, 1024, 2), idesc_s,
-                                    ks > 0 ? 1u : 0u);
+                        tc_fence_after();
+                        const uint32_t d_tmem = tS0 + sb * N;
+                        if constexpr (F8) {
+                            // A = the converted keys in tensor memory: 16 head coordinates = 8 columns
+                            const uint32_t k_tmem = tmem + (T & 1) * 64;
+    #pragma unroll
+                            for (int ks = 0; ks < kD / 16; ++ks) {
+                                const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
+                                umma_ts(d_tmem, k_tmem + ks * 8, umma_smem_desc(qa, 16, 1024, 2), idesc_s,
+                                        ks > 0 ? 1u : 0u);
+                            }
+                            umma_commit(&bar[S_FULL + sb]);
+                            umma_commit(&bar[KT_FREE + (T & 1)]);
+                        } else {
+                            const uint32_t k_addr = smem_u32(smem + s * C::stage_bytes);
+    #pragma unroll
+                            for (int ks = 0; ks < kD / 16; ++ks) {
+                                const uint32_t ka = k_addr + (ks >> 2) * kHalf + (ks & 3) * 32;
+                                const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
+                                umma_ss(d_tmem, umma_smem_desc(ka, 16, 1024, 2), umma_smem_desc(qa, 16, 1024, 2),
+                                        idesc_s, ks > 0 ? 1u : 0u);
+                            }
+                            umma_commit(&bar[S_FULL + sb]);
                         }
-                        umma_commit(&bar[S_FULL + sb]);
-                        umma_commit(&bar[KT_FREE + (T & 1)]);
-                    } else {
-                        const uint32_t k_addr = smem_u32(smem + s * C::stage_bytes);
-#pragma unroll
-                        for (int ks = 0; ks < kD / 16; ++ks) {
-                            const uint32_t ka = k_addr + (ks >> 2) * kHalf + (ks & 3) * 32;
-                            const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
-                            umma_ss(d_tmem, umma_smem_desc(ka, 16, 1024, 2), umma_smem_desc(qa, 16, 1024, 2),
-                                    idesc_s, ks > 0 ? 1u : 0u);
+                    }
+                    if (!ok) break;
+                    umma_commit(&bar[Q_EMPTY + qb]);   // the unit's query rows are no longer read
+                    tcount += ntl;
+                    ++icount;
+                }
+                umma_commit(&bar[DRAIN]);
+                mbar_wait(&bar[DRAIN], 0, a.wait_budget_ns);
+            }
+        } else if (warp == pv_warp) {
+            // ---------------- PV issuer: [O_hi | O_lo] += V^T (MN-major) . [P_hi | P_lo]^T (MN-major)
+            if (lane == 0) {
+                constexpr int npv = 16 * C::nb;   // the hi and lo blocks that carry heads
+                const uint32_t idesc_o = F8 ? umma_idesc_f16(kD, npv, 1, 1) : umma_idesc_bf16(kD, npv, 1, 1);
+                int tcount = 0, icount = 0;
+                bool ok = true;
+                while (ok) {
+                    const int slot = icount % kQD;
+                    if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
+                    volatile int *q = queue + slot * 8;
+                    const int t_begin = q[3], t_end = q[4];
+                    mbar_arrive(&bar[I_EMPTY + slot]);
+                    if (t_end < 0) break;
+                    const int ntl = (t_end - t_begin + kTok - 1) / kTok;
+                    const int ob = icount & 1;
+                    if (icount >= 2 && !wait_or_fail(&bar[O_FREE + ob], ((icount >> 1) - 1) & 1, a, err)) break;
+                    const uint32_t d_tmem = tO0 + ob * 2 * N;
+                    for (int jj = 0; jj < ntl; ++jj) {
+                        const int T = tcount + jj;
+                        const int s = T % C::stages;
+                        const int pb = T % C::pbufs;
+                        if (!wait_or_fail(&bar[P_FULL + pb], (T / C::pbufs) & 1, a, err)) { ok = false; break; }
+                        if (!wait_or_fail(&bar[(F8 ? VC_FULL : V_FULL) + s], (T / C::stages) & 1, a, err)) {
+                            ok = false;
+                            break;
                         }
-                        umma_commit(&bar[S_FULL + sb]);
+                        tc_fence_after();
+                        const uint32_t v_addr = smem_u32(smem + s * C::stage_bytes + (F8 ? 0 : kTile));
+                        // one product of width 16 nb: the lo blocks follow the hi blocks at the same 2048-byte
+                        // stride, so they are simply more columns
+                        const uint32_t p_addr = smem_u32(ps + pb * 2 * C::p_half);
+    #pragma unroll
+                        for (int ks = 0; ks < kTok / 16; ++ks) {
+                            // A = V^T: 16 tokens (two 8-row groups, 1024 B apart), 64-column blocks kHalf apart
+                            // B = P^T: 16 tokens (two 128-byte core-matrix groups), 8-head blocks 2048 B apart
+                            umma_ss(d_tmem, umma_smem_desc(v_addr + ks * 2048, kHalf, 1024, 2),
+                                    umma_smem_desc(p_addr + ks * 256, 128, 2048, 0), idesc_o, (jj > 0 || ks > 0) ? 1u : 0u);
+                        }
+                        umma_commit(&bar[P_FREE + pb]);
+                        // the stage's keys were read by an S^T product that completed before this P existed
+                        umma_commit(&bar[(F8 ? R_EMPTY : KV_EMPTY) + s]);
                     }
+                    if (!ok) break;
+                    umma_commit(&bar[O_FULL + ob]);
+                    tcount += ntl;
+                    ++icount;
                 }
-                if (!ok) break;
-                umma_commit(&bar[Q_EMPTY + qb]);   // the unit's query rows are no longer read
-                tcount += ntl;
-                ++icount;
+                umma_commit(&bar[DRAIN_PV]);
+                mbar_wait(&bar[DRAIN_PV], 0, a.wait_budget_ns);
             }
-            umma_commit(&bar[DRAIN]);
-            mbar_wait(&bar[DRAIN], 0, a.wait_budget_ns);
-        }
-    } else if (warp == pv_warp) {
-        // ---------------- PV issuer: [O_hi | O_lo] += V^T (MN-major) . [P_hi | P_lo]^T (MN-major)
-        if (lane == 0) {
-            constexpr int npv = 16 * C::nb;   // the hi and lo blocks that carry heads
-            const uint32_t idesc_o = F8 ? umma_idesc_f16(kD, npv, 1, 1) : umma_idesc_bf16(kD, npv, 1, 1);
-            int tcount = 0, icount = 0;
-            bool ok = true;
-            while (ok) {
-                const int slot = icount % kQD;
-                if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
-                volatile int *q = queue + slot * 8;
-                const int t_begin = q[3], t_end = q[4];
-                mbar_arrive(&bar[I_EMPTY + slot]);
-                if (t_end < 0) break;
-                const int ntl = (t_end - t_begin + kTok - 1) / kTok;
-                const int ob = icount & 1;
-                if (icount >= 2 && !wait_or_fail(&bar[O_FREE + ob], ((icount >> 1) - 1) & 1, a, err)) break;
-                const uint32_t d_tmem = tO0 + ob * 2 * N;
-                for (int jj = 0; jj < ntl; ++jj) {
-                    const int T = tcount + jj;
-                    const int s = T % C::stages;
-                    const int pb = T % C::pbufs;
-                    if (!wait_or_fail(&bar[P_FULL + pb], (T / C::pbufs) & 1, a, err)) { ok = false; break; }
-                    if (!wait_or_fail(&bar[(F8 ? VC_FULL : V_FULL) + s], (T / C::stages) & 1, a, err)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t v_addr = smem_u32(smem + s * C::stage_bytes + (F8 ? 0 : kTile));
-                    // one product of width 16 nb: the lo blocks follow the hi blocks at the same 2048-byte
-                    // stride, so they are simply more columns
-                    const uint32_t p_addr = smem_u32(ps + pb * 2 * C::p_half);
-#pragma unroll
-                    for (int ks = 0; ks < kTok / 16; ++ks) {
-                        // A = V^T: 16 tokens (two 8-row groups, 1024 B apart), 64-column blocks kHalf apart
-                        // B = P^T: 16 tokens (two 128-byte core-matrix groups), 8-head blocks 2048 B apart
-                        umma_ss(d_tmem, umma_smem_desc(v_addr + ks * 2048, kHalf, 1024, 2),
-                                umma_smem_desc(p_addr + ks * 256, 128, 2048, 0), idesc_o, (jj > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    umma_commit(&bar[P_FREE + pb]);
-                    // the stage's keys were read by an S^T product that completed before this P existed
-                    umma_commit(&bar[(F8 ? R_EMPTY : KV_EMPTY) + s]);
-                }
-                if (!ok) break;
-                umma_commit(&bar[O_FULL + ob]);
-                tcount += ntl;
-                ++icount;
-            }
-            umma_commit(&bar[DRAIN_PV]);
-            mbar_wait(&bar[DRAIN_PV], 0, a.wait_budget_ns);
         }
     } else if (F8 && warp >= conv_warp0) {
         // ---------------- FP8 converter: thread ct owns token ct of each tile (TMEM lane ct of K)
+        if constexpr (C::regsplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 104;" ::: "memory");
         const int ct = threadIdx.x - kWG * C::nwg;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         int tcount = 0, icount = 0;
@@ -709,15 +721,8 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 const int T = tcount + jj;
                 const int s = T % C::stages, cb = T & 1;
                 if (!wait_or_fail(&bar[R_FULL + s], (T / C::stages) & 1, a, err)) { ok = false; break; }
-                // the raw tiles were stored with the 128-byte swizzle: chunk c of row ct at c ^ (ct & 7).
-                // This thread's key row and value row, into registers.
+                // the raw tiles were stored with the 128-byte swizzle: chunk c of row ct at c ^ (ct & 7)
                 uint8_t *krow = smem + s * C::stage_bytes + ct * 128;
-                uint4 kr[8], vr[8];
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    kr[c] = *reinterpret_cast<const uint4 *>(krow + ((c ^ (ct & 7)) << 4));
-                    vr[c] = *reinterpret_cast<const uint4 *>(krow + kHalf + ((c ^ (ct & 7)) << 4));
-                }
                 // tokens past the piece's end may hold anything (NaN codes included): they become zeros,
                 // so that no 0 * NaN reaches an accumulator
                 const bool valid = (t_begin + jj * kTok + ct) < t_end;
@@ -729,7 +734,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     uint32_t w[32];
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        const uint4 r = kr[h * 4 + c];
+                        const uint4 r = *reinterpret_cast<const uint4 *>(krow + (((h * 4 + c) ^ (ct & 7)) << 4));
                         e4m3x4_to_f16x4(r.x, w[c * 8 + 0], w[c * 8 + 1]);
                         e4m3x4_to_f16x4(r.y, w[c * 8 + 2], w[c * 8 + 3]);
                         e4m3x4_to_f16x4(r.z, w[c * 8 + 4], w[c * 8 + 5]);
@@ -745,8 +750,11 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 tc_fence_before();
                 mbar_arrive(&bar[KT_FULL + cb]);
                 // values -> f16 tile [2 halves][128 rows][128 B] with the 128-byte swizzle over the stage:
-                // row ct of half 0 is where this thread's key codes were, row ct of half 1 where its value
-                // codes were
+                // row ct of half 0 is where this thread's key codes were (all read above), row ct of half 1
+                // where its value codes are (read into registers first)
+                uint4 vr[8];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) vr[c] = *reinterpret_cast<const uint4 *>(krow + kHalf + ((c ^ (ct & 7)) << 4));
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint4 lo4, hi4;
@@ -773,6 +781,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     } else {
         // ---------------- softmax warpgroup wg: heads 16*wg .. 16*wg+15; thread t owns token t of
         // each tile (TMEM lane t of S^T) and column d = t of O^T
+        if constexpr (C::regsplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 176;" ::: "memory");
         const int wg = warp >> 2;
         const int quarter = warp & 3;              // TMEM lane quarter this warp may access
         const int t = quarter * 32 + lane;
