@@ -55,6 +55,21 @@ constexpr float kMoveThreshold = 8.0f;
 constexpr int kPlanThreads = 1024;
 constexpr int kPlanMaxC = 4096;           // remainder sizes sorted by a shared-memory histogram up to this
 
+// barrier slots: each name owns a contiguous range (sizes checked against the configuration below)
+enum : int { K_FULL = 0, V_FULL = 3, KV_EMPTY = 6, S_FULL = 9, S_FREE = 13, P_FULL = 17, P_FREE = 21, O_FULL = 25,
+             O_FREE = 27, Q_FULL = 29, Q_EMPTY = 31, I_FULL = 33, I_EMPTY = 37, DRAIN = 41, DRAIN_PV = 42, GRP = 43,
+             // FP8 only: code ring (R_EMPTY: the stage's PV product is done), converted K (tensor memory),
+             // converted V (in the stage), converted Q, and the unit slot's score factors (the softmax
+             // releases the slot after reading them)
+             R_FULL = 45, R_EMPTY = 51, KT_FULL = 57, KT_FREE = 59, VC_FULL = 61, QC_FULL = 67, QF_FULL = 69,
+             kBarSlots = 73 };
+constexpr int kBarSlotsFor(bool f8) { return f8 ? kBarSlots : R_FULL; }
+template <class C, bool F8>
+constexpr bool barrier_ranges_fit()
+{
+    return (F8 ? C::stages <= 6 : C::stages <= 3) && C::sbufs <= 4 && C::pbufs <= 4 && C::nwg <= 2 && kQD <= 4;
+}
+
 // F8 = false: bf16 cache; the K and V tiles go from TMA straight to the tensor cores.
 // F8 = true: FP8 (E4M3) cache.  TMA brings the raw code tiles (16 KB each) into a ring; one converter
 // warpgroup widens them exactly to f16 (every E4M3 value is an f16 value): the keys into tensor
@@ -62,13 +77,14 @@ constexpr int kPlanMaxC = 4096;           // remainder sizes sorted by a shared-
 // takes the place of the stage's two code tiles (each thread rewrites only the two 128-byte rows it
 // has just read, so no thread waits for another).  Q is converted in place to f16 with a power-of-two scale per head, and P enters the second
 // product as f16 hi + lo terms (of 128 p, so that small weights stay normal), with f16 MMAs throughout.
-// HW: heads one softmax warpgroup handles (4, 8 or 16): groups of up to 4 or 8 heads only compute
-// their own columns of the N = 16 wide products.
-template <int N, bool F8, int HW>
+// HW: heads one softmax warpgroup handles (4, 8 or 16), NWG: softmax warpgroups.  Groups of up to 4
+// or 8 heads only compute their own columns of the N = 16 wide products; more warpgroups with fewer
+// heads each shorten the softmax's per-tile chain.
+template <int N, bool F8, int HW, int NWG>
 struct TcCfg {
-    static_assert(HW == 16 || N == 16, "narrow softmax only with N = 16");
-    static constexpr int nwg = HW == 16 ? N / 16 : 1;         // softmax warpgroups
-    static constexpr int nb = HW <= 8 ? 1 : N / 8;            // 8-head blocks of P^T / O^T that carry heads
+    static_assert(NWG * HW <= N && (NWG == 1 || HW % 8 == 0), "softmax heads within the product");
+    static constexpr int nwg = NWG;                           // softmax warpgroups
+    static constexpr int nb = NWG * HW <= 8 ? 1 : NWG * HW / 8;   // 8-head blocks of P^T / O^T that carry heads
     static constexpr int conv_warps = F8 ? 4 : 0;             // FP8: the converter warpgroup
     // + TMA warp + S^T issuer warp + PV issuer warp.  FP8 with 32 heads: the last three warps are padded
     // to a warpgroup and the registers are redistributed (setmaxnreg): 512 threads launch with 128
@@ -92,7 +108,7 @@ struct TcCfg {
     static constexpr int vote_off = qfac_off + (F8 ? kQD * N * 4 : 0);   // [nwg][2][4] ints
     static constexpr int queue_off = vote_off + nwg * 32;     // kQD units of 8 ints
     static constexpr int bar_off = queue_off + kQD * 32;
-    static constexpr int nbars = F8 ? 69 : 41;
+    static constexpr int nbars = kBarSlotsFor(F8);
     static constexpr int tmem_off = bar_off + nbars * 8;
     static constexpr int err_off = tmem_off + 8;
     static constexpr int bytes = err_off + 8;
@@ -106,14 +122,6 @@ struct TcCfg {
     static_assert(bytes <= 227 * 1024, "shared memory budget");
 };
 
-// barrier slots
-enum : int { K_FULL = 0, V_FULL = 3, KV_EMPTY = 6, S_FULL = 9, S_FREE = 13, P_FULL = 17, P_FREE = 19, O_FULL = 21,
-             O_FREE = 23, Q_FULL = 25, Q_EMPTY = 27, I_FULL = 29, I_EMPTY = 33, DRAIN = 37, DRAIN_PV = 38, GRP = 39,
-             // FP8 only: code ring (R_EMPTY: the stage's PV product is done), converted K (tensor memory),
-             // converted V (in the stage), converted Q
-             R_FULL = 41, R_EMPTY = 47, KT_FULL = 53, KT_FREE = 55, VC_FULL = 57, QC_FULL = 63,
-             // FP8: the unit slot's score factors are written (the softmax releases the slot after reading)
-             QF_FULL = 65 };
 
 __device__ __forceinline__ void record_status(int *status, int code)
 {
@@ -369,12 +377,13 @@ __device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t (&r)[NC]
 }
 
 // ---------------------------------------------------------------------------------------------
-template <int N, bool F8, int HW>
-__global__ void __launch_bounds__(TcCfg<N, F8, HW>::threads, 1)
+template <int N, bool F8, int HW, int NWG>
+__global__ void __launch_bounds__(TcCfg<N, F8, HW, NWG>::threads, 1)
 decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                          const __grid_constant__ CUtensorMap tmQ, const DecodeArgs a)
 {
-    using C = TcCfg<N, F8, HW>;
+    using C = TcCfg<N, F8, HW, NWG>;
+    static_assert(barrier_ranges_fit<C, F8>(), "a barrier range is too small for this configuration");
     // the 128-byte swizzle needs 1024-byte aligned tiles; the whole budget is used, so there is no room
     // to realign: a misaligned window is reported and the CTA does nothing
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -779,7 +788,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             ++icount;
         }
     } else {
-        // ---------------- softmax warpgroup wg: heads 16*wg .. 16*wg+15; thread t owns token t of
+        // ---------------- softmax warpgroup wg: heads HW*wg .. HW*wg+HW-1; thread t owns token t of
         // each tile (TMEM lane t of S^T) and column d = t of O^T
         if constexpr (C::regsplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 176;" ::: "memory");
         const int wg = warp >> 2;
@@ -1038,16 +1047,16 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     }
 }
 
-template <int N, bool F8, int HW>
+template <int N, bool F8, int HW, int NWG>
 cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, const CUtensorMap &tmQ,
                               const DecodeArgs &a, cudaStream_t stream)
 {
-    const int smem = TcCfg<N, F8, HW>::bytes;
+    const int smem = TcCfg<N, F8, HW, NWG>::bytes;
     static bool attr_done[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr_done[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(decode_persistent_kernel<N, F8, HW>,
+        cudaError_t e = cudaFuncSetAttribute(decode_persistent_kernel<N, F8, HW, NWG>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_done[dev] = true;
@@ -1056,7 +1065,7 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
     // waits for (griddepcontrol.wait) before reading the plan
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.num_ctas);
-    cfg.blockDim = dim3(TcCfg<N, F8, HW>::threads);
+    cfg.blockDim = dim3(TcCfg<N, F8, HW, NWG>::threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -1064,7 +1073,7 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_persistent_kernel<N, F8, HW>, tmK, tmV, tmQ, a);
+    return cudaLaunchKernelEx(&cfg, decode_persistent_kernel<N, F8, HW, NWG>, tmK, tmV, tmQ, a);
 }
 
 }  // namespace
@@ -1079,16 +1088,16 @@ cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, con
                              const DecodeArgs &a, cudaStream_t stream, bool fp8)
 {
     if (fp8) {
-        if (a.group <= 4) return launch_persistent<16, true, 4>(tmK, tmV, tmQ, a, stream);
-        if (a.group <= 8) return launch_persistent<16, true, 8>(tmK, tmV, tmQ, a, stream);
-        if (a.group <= 16) return launch_persistent<16, true, 16>(tmK, tmV, tmQ, a, stream);
-        if (a.group <= 32) return launch_persistent<32, true, 16>(tmK, tmV, tmQ, a, stream);
+        if (a.group <= 4) return launch_persistent<16, true, 4, 1>(tmK, tmV, tmQ, a, stream);
+        if (a.group <= 8) return launch_persistent<16, true, 8, 1>(tmK, tmV, tmQ, a, stream);
+        if (a.group <= 16) return launch_persistent<16, true, 8, 2>(tmK, tmV, tmQ, a, stream);
+        if (a.group <= 32) return launch_persistent<32, true, 16, 2>(tmK, tmV, tmQ, a, stream);
         return cudaErrorInvalidValue;
     }
-    if (a.group <= 4) return launch_persistent<16, false, 4>(tmK, tmV, tmQ, a, stream);
-    if (a.group <= 8) return launch_persistent<16, false, 8>(tmK, tmV, tmQ, a, stream);
-    if (a.group <= 16) return launch_persistent<16, false, 16>(tmK, tmV, tmQ, a, stream);
-    if (a.group <= 32) return launch_persistent<32, false, 16>(tmK, tmV, tmQ, a, stream);
+    if (a.group <= 4) return launch_persistent<16, false, 4, 1>(tmK, tmV, tmQ, a, stream);
+    if (a.group <= 8) return launch_persistent<16, false, 8, 1>(tmK, tmV, tmQ, a, stream);
+    if (a.group <= 16) return launch_persistent<16, false, 16, 1>(tmK, tmV, tmQ, a, stream);
+    if (a.group <= 32) return launch_persistent<32, false, 16, 2>(tmK, tmV, tmQ, a, stream);
     return cudaErrorInvalidValue;
 }
 
