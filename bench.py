@@ -225,6 +225,17 @@ def time_prefill(gqa, torch, p, steps: int, warmup: int):
     return s0.elapsed_time(s1) / steps, sum(a.elapsed_time(b) for a, b in kev) / steps, launches
 
 
+def decode_call(gqa, x, out, q=None, k=None, v=None, sl=None):
+    """One decode step through the public API: the FP8 entry point when x carries per-tensor scales."""
+    q = x.q if q is None else q
+    k = x.k_cache if k is None else k
+    v = x.v_cache if v is None else v
+    sl = x.seqlens if sl is None else sl
+    if hasattr(x, "k_scale"):
+        return gqa.gqa_decode_fp8(q, k, v, sl, x.k_scale, x.v_scale, x.scale, out=out)
+    return gqa.gqa_decode(q, k, v, sl, x.scale, out=out)
+
+
 def time_e2e(gqa, torch, x, steps: int):
     """Host buffers in, host result out: pinned H2D of q, K, V, seqlens + decode + D2H of out, per step."""
     hq = x.q.cpu().pin_memory()
@@ -240,7 +251,7 @@ def time_e2e(gqa, torch, x, steps: int):
         dk.copy_(hk, non_blocking=True)
         dv.copy_(hv, non_blocking=True)
         ds.copy_(hs, non_blocking=True)
-        gqa.gqa_decode(dq, dk, dv, ds, x.scale, out=dout)
+        decode_call(gqa, x, dout, dq, dk, dv, ds)
         hout.copy_(dout, non_blocking=True)
 
     step()
@@ -274,7 +285,10 @@ def cpu_oracle_sample(x, target_s: float = 12.0):
         kk = x.k_cache[:n, :T].cpu()
         vv = x.v_cache[:n, :T].cpu()
         t0 = time.perf_counter()
-        oracle.decode(q, kk, vv, sl[:n], x.scale, nthreads=cores)
+        if hasattr(x, "k_scale"):
+            oracle.decode_fp8(q, kk, vv, x.k_scale, x.v_scale, sl[:n], x.scale, nthreads=cores)
+        else:
+            oracle.decode(q, kk, vv, sl[:n], x.scale, nthreads=cores)
         return time.perf_counter() - t0
 
     t1 = run(1)
@@ -283,17 +297,20 @@ def cpu_oracle_sample(x, target_s: float = 12.0):
     while spent < target_s and reps < 1000:
         spent += run(n)
         reps += 1
-    ub = unique_kv_bytes(sl[:n], Hkv, d) * reps
+    ub = unique_kv_bytes(sl[:n], Hkv, d, x.k_cache.element_size()) * reps
     return {"value": ub / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"first {n} of {B} sequences (every query head, {sum(sl[:n])} cached tokens) "
                       f"x {reps} repetitions; {spent:.1f} s wall on {cores} threads",
             "seconds": spent, "tokens_per_s": n * reps / spent}
 
 
-def decode_kernel_name(g: int) -> str:
-    """Which decode kernel the library launches for group size g (label only)."""
-    if 3 <= g <= 32:
-        return f"decode_persistent_kernel<{16 if g <= 16 else 32}>"
+def decode_kernel_name(g: int, fp8: bool = False) -> str:
+    """Which decode kernel the library launches for group size g (label only): template arguments
+    <product width N, FP8 cache, heads per softmax warpgroup, softmax warpgroups>."""
+    if fp8 or 3 <= g <= 32:
+        n, hw, nwg = (16, 4, 1) if g <= 4 else (16, 8, 1) if g <= 8 else \
+            ((16, 8, 2) if fp8 else (16, 16, 1)) if g <= 16 else (32, 16, 2)
+        return f"decode_persistent_kernel<{n}, {str(fp8).lower()}, {hw}, {nwg}>"
     return f"decode_split_kernel<{1 if g <= 1 else 2 if g <= 2 else 4 if g <= 4 else 8}>"
 
 
@@ -328,6 +345,8 @@ def main():
     ap.add_argument("--prefill-batch", type=int, default=4, help="sequences in --mode prefill")
     ap.add_argument("--decode-workload", default="Qwen3-8B",
                     help="name prefix of the decode workload timed as the headline (profiling other rows)")
+    ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
+                    help="fp8: the headline decode over an FP8 (E4M3) cache with per-tensor scales")
     args = ap.parse_args()
 
     import torch
@@ -341,9 +360,11 @@ def main():
     from grouped_query_attention_02_b200 import inputs, workloads
 
     w = next(x for x in workloads.DECODE_WORKLOADS if x.name.startswith(args.decode_workload))
+    fp8 = args.kv == "fp8"
     base_cfg = {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.Tmax,
                 "global_batch": w.B * max(world, 1), "parallelism": f"dp{max(world, 1)} (batch-sharded, no collective)",
-                "l2": "inputs larger than L2 (1.64 GB cache vs 126 MB); no flush"}
+                "kv_cache": "fp8 e4m3, per-tensor scales" if fp8 else "bf16",
+                "l2": "inputs larger than L2 (cache of at least 0.8 GB vs 126 MB); no flush"}
 
     if args.impl == "reference":
         # the reference arm is the fp64 CPU oracle, on rank 0 only
@@ -392,16 +413,16 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
 
     peaks = load_peaks()
-    x = inputs.make_decode(w.B, w.Hq, w.Hkv, w.d, w.Tmax, device="cuda", seed=rank_seed(rank),
-                           seqlen_range=w.seqlen_range)
+    make = inputs.make_decode_fp8 if fp8 else inputs.make_decode
+    x = make(w.B, w.Hq, w.Hkv, w.d, w.Tmax, device="cuda", seed=rank_seed(rank), seqlen_range=w.seqlen_range)
     sl = x.seqlens.cpu().tolist()
-    U = unique_kv_bytes(sl, w.Hkv, w.d)
+    U = unique_kv_bytes(sl, w.Hkv, w.d, x.k_cache.element_size())
     alg_bytes = U + 2 * x.q.numel() * 2   # cache + q in + out
 
     # warm-up + barrier, then the timed steps bracketed by barrier + synchronize
     out = torch.empty_like(x.q)
     for _ in range(args.warmup):
-        gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out)
+        decode_call(gqa, x, out)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -411,7 +432,7 @@ def main():
         time.sleep(0.25)
         s0.record()
         for i in range(args.steps):
-            gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out)
+            decode_call(gqa, x, out)
             launches += gqa.gqa_last_launch_count()
         s1.record()
         torch.cuda.synchronize()
@@ -423,7 +444,7 @@ def main():
     kev = [_events(torch) for _ in range(args.steps)]
     for i in range(args.steps):
         gqa.gqa_set_profile_events(*kev[i])
-        gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out)
+        decode_call(gqa, x, out)
     gqa.gqa_set_profile_events(None, None)
     torch.cuda.synchronize()
     kern_ms = sum(a.elapsed_time(b) for a, b in kev) / args.steps
@@ -461,12 +482,16 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": max(world, 1), "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "accumulate": "fp32", "data": "synthetic", "config": base_cfg,
+        "vs_baseline": None, "dtype": "fp8 e4m3 cache, f16 products" if fp8 else "bf16", "accumulate": "fp32",
+        "data": "synthetic", "config": base_cfg,
         "tokens_per_s": tokens_per_s, "frac_of_hbm_peak_step": value / max(world, 1) / peaks["hbm_gbs"],
         "gpu_launches": launches, "device_status": status,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": profile_traffic("decode_persistent_qwen3_8b.md"),
-                     "kernel": decode_kernel_name(w.group), "kernel_ms": kern_ms, "algorithmic_bytes": alg_bytes,
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": profile_traffic("decode_persistent_fp8_qwen3_8b.md" if fp8 and w is workloads.QWEN3_8B_DECODE
+                                                else "decode_persistent_qwen3_8b.md" if w is workloads.QWEN3_8B_DECODE
+                                                else "-"),
+                     "kernel": decode_kernel_name(w.group, fp8), "kernel_ms": kern_ms, "algorithmic_bytes": alg_bytes,
                      "peak_source": f"{peaks.get('source')} hbm_gbs (copy bandwidth)"},
         "clocks": clk.summary(),
     }
@@ -478,7 +503,7 @@ def main():
         line["e2e"]["error"] = e2e_err
 
     # ---- the other rows of the hot path
-    if args.rows == "all" and max(world, 1) == 1:
+    if args.rows == "all" and max(world, 1) == 1 and not fp8:
         rows = {}
         del out
         for ww in (workloads.TINY_DECODE,) + workloads.VARLEN_DECODE + (workloads.EXTREME_GROUP_DECODE,):
