@@ -12,9 +12,10 @@
  * head, read once, never copied; causal mask as a lower triangle).
  *
  * Conventions shared by every entry point.
- *  - Tensors are bf16 (IEEE binary32 with the low 16 bits dropped), dense and
- *    row-major in the layouts named below; all device pointers must be
- *    16-byte aligned.  Accumulation is fp32; outputs are rounded to bf16.
+ *  - Tensors are bf16 (IEEE binary32 with the low 16 bits dropped), except the
+ *    one-byte E4M3 caches of gqa_decode_fp8, dense and row-major in the layouts
+ *    named below; all device pointers must be 16-byte aligned.  Accumulation
+ *    is fp32; outputs are rounded to bf16.
  *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy
  *    default stream.  Every call only enqueues work on `stream` and returns;
  *    no call synchronises the host, and the caller owns every tensor and the
@@ -201,10 +202,11 @@ gqa_status gqa_selftest_wait_timeout(int timeout_us, void *stream);
 
 /*
  * gqa_set_profile_events -- measurement hook.  When both are non-NULL
- * (cudaEvent_t passed as void*), every later gqa_decode / gqa_prefill_causal /
- * gqa_decode_expanded records `before` on its stream immediately before its
- * dominant kernel (the split-KV decode kernel; the prefill kernel) and
- * `after` immediately after it.  NULL, NULL turns the hook off.
+ * (cudaEvent_t passed as void*), every later gqa_decode / gqa_decode_fp8 /
+ * gqa_prefill_causal / gqa_decode_expanded records `before` on its stream
+ * immediately before its dominant kernel (the decode kernel; the prefill
+ * kernel) and `after` immediately after it (gqa_decode_noalloc records
+ * nothing).  NULL, NULL turns the hook off.
  */
 gqa_status gqa_set_profile_events(void *before, void *after);
 
