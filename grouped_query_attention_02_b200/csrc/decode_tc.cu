@@ -1059,6 +1059,14 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
         cudaError_t e = cudaFuncSetAttribute(decode_persistent_kernel<N, F8, HW, NWG>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
+        if constexpr (TcCfg<N, F8, HW, NWG>::regsplit) {
+            // setmaxnreg.inc waits until the decreases have freed enough of the registers the block was
+            // launched with: refuse to launch unless the launch holds the whole split
+            cudaFuncAttributes fa;
+            if ((e = cudaFuncGetAttributes(&fa, decode_persistent_kernel<N, F8, HW, NWG>)) != cudaSuccess) return e;
+            if ((long long)fa.numRegs * TcCfg<N, F8, HW, NWG>::threads < 4LL * 128 * 128)
+                return cudaErrorInvalidConfiguration;
+        }
         attr_done[dev] = true;
     }
     // programmatic dependent launch: the prologue overlaps decode_plan_kernel, which the kernel
