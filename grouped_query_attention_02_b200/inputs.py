@@ -10,7 +10,8 @@ attention arithmetic.  Recipe (the same for every workload):
   ``base+3`` on a CPU generator (so every device sees the same lengths);
 * cache rows at or past ``seqlens[b]`` hold random values too, or NaN when
   ``poison=True`` (a read past the end then shows up as NaN in the output);
-* ``q_gain`` multiplies q before rounding (a "peaky" softmax when > 1).
+* ``q_gain`` multiplies q before rounding (a "peaky" softmax when > 1);
+* the backward's incoming gradient dO: N(0, 1) in bf16 from seed ``base+4``.
 
 FP8 caches (``make_decode_fp8``): the same N(0, 1) draws divided by a
 per-tensor scale, clamped to the largest finite E4M3 value (448) and stored as
@@ -174,3 +175,8 @@ def make_prefill(B: int, S: int, Hq: int, Hkv: int, d: int, *, device="cpu", see
     k = _normal((B, S, Hkv, d), seed + 1, device)
     v = _normal((B, S, Hkv, d), seed + 2, device)
     return PrefillInputs(q, k, v, 1.0 / float(d) ** 0.5)
+
+
+def make_dout(B: int, S: int, Hq: int, d: int, *, device="cpu", seed: int = 0) -> torch.Tensor:
+    """Incoming gradient dO [B,S,Hq,d] of the causal prefill's output (seed ``seed+4``)."""
+    return _normal((B, S, Hq, d), seed + 4, device)

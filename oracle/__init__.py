@@ -90,6 +90,9 @@ class Oracle:
         lib.gqa_oracle_decode.restype = ctypes.c_int
         lib.gqa_oracle_decode.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 5 + [
             ctypes.c_double, ctypes.c_void_p, ctypes.c_int]
+        lib.gqa_oracle_prefill_backward.restype = ctypes.c_int
+        lib.gqa_oracle_prefill_backward.argtypes = [ctypes.c_void_p] * 4 + [ctypes.c_int] * 5 + [
+            ctypes.c_double] + [ctypes.c_void_p] * 5 + [ctypes.c_int]
         lib.gqa_oracle_e4m3_to_f64.restype = None
         lib.gqa_oracle_e4m3_to_f64.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_longlong]
         lib.gqa_oracle_decode_fp8.restype = ctypes.c_int
@@ -111,6 +114,34 @@ class Oracle:
         out = np.empty(b.shape, dtype=np.float64)
         self.lib.gqa_oracle_bf16_to_f64(b.ctypes.data, out.ctypes.data, b.size)
         return out
+
+    def prefill_backward(self, q, k, v, dout, scale: float, row_sel=None, key_sel=None,
+                         nthreads: int | None = None):
+        """Causal prefill backward: q, dout [B,S,Hq,d], k, v [B,S,Hkv,d] (bf16) -> (dq, dk, dv) fp64.
+        row_sel / key_sel: optional iterables of positions whose dq / dk, dv are computed (others 0)."""
+        qb, kb, vb, ob = _bits(q), _bits(k), _bits(v), _bits(dout)
+        B, S, Hq, d = qb.shape
+        Hkv = kb.shape[2]
+        assert kb.shape == (B, S, Hkv, d) and vb.shape == kb.shape and ob.shape == qb.shape
+
+        def flags(sel):
+            if sel is None:
+                return None
+            f = np.zeros(S, dtype=np.int32)
+            f[np.asarray(list(sel), dtype=np.int64)] = 1
+            return f
+
+        rf, kf = flags(row_sel), flags(key_sel)
+        dq = np.empty((B, S, Hq, d), dtype=np.float64)
+        dk = np.empty((B, S, Hkv, d), dtype=np.float64)
+        dv = np.empty((B, S, Hkv, d), dtype=np.float64)
+        st = self.lib.gqa_oracle_prefill_backward(
+            qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, ob.ctypes.data, B, S, Hq, Hkv, d, float(scale),
+            None if rf is None else rf.ctypes.data, None if kf is None else kf.ctypes.data,
+            dq.ctypes.data, dk.ctypes.data, dv.ctypes.data, nthreads or default_threads())
+        if st != 0:
+            raise ValueError(f"oracle backward rejected its arguments (status {st})")
+        return dq, dk, dv
 
     def e4m3_to_f64(self, bytes_: np.ndarray) -> np.ndarray:
         b = np.ascontiguousarray(bytes_, dtype=np.uint8)
@@ -204,6 +235,10 @@ def decode(q, k_cache, v_cache, seqlens, scale, nthreads=None):
 
 def e4m3_to_f64(bytes_):
     return _get().e4m3_to_f64(bytes_)
+
+
+def prefill_backward(q, k, v, dout, scale, row_sel=None, key_sel=None, nthreads=None):
+    return _get().prefill_backward(q, k, v, dout, scale, row_sel, key_sel, nthreads)
 
 
 def decode_fp8(q, k8, v8, k_scale, v_scale, seqlens, scale, nthreads=None):

@@ -27,6 +27,10 @@
  *  - Causal prefill: row r attends to tokens t <= r (lower triangle including
  *    the diagonal), masked scores excluded from the softmax: same section,
  *    the tril mask of its example.
+ *  - Causal prefill backward: dq, and dk / dv summed over the group's query
+ *    heads (study.greatitself.com, grouped-query and multi-query attention,
+ *    training paragraph: the shared tensors receive every head's gradient,
+ *    as differentiation of the explicitly repeated form gives).
  *  - FP8 KV cache: the cache stored in FP8 instead of bf16 ("Other ways to
  *    shrink the KV cache", anrans.github.io attention-variants: K and V in
  *    FP8, as serving engines support); every element is the E4M3 value of its
@@ -359,6 +363,164 @@ int gqa_oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
     }
     for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, prefill_worker, &jobs[i]);
     prefill_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    int st = ORACLE_OK;
+    for (int i = 0; i < nthreads; ++i) if (jobs[i].status != ORACLE_OK) st = jobs[i].status;
+    free(jobs); free(th);
+    return st;
+}
+
+/* ---- causal prefill backward ----------------------------------------------
+ *
+ * Gradients of a scalar loss through the causal prefill, given dO = dL/dout:
+ * "During training, a shared key or value tensor receives gradient
+ * contributions from every query head in its group" (study.greatitself.com,
+ * grouped-query and multi-query attention, training paragraph).  Written out
+ * per query head h of KV head kvh, with s_rt = scale q_r.k_t for t <= r,
+ * P_rt = exp(s_rt - lse_r), lse_r = log sum_{t<=r} exp(s_rt):
+ *
+ *   dP_rt = dO_r . v_t
+ *   D_r   = sum_t P_rt dP_rt
+ *   dS_rt = P_rt (dP_rt - D_r)
+ *   dq_r  = scale sum_{t<=r} dS_rt k_t
+ *   dk_t += scale sum_{r>=t} dS_rt q_r      (summed over the group's heads)
+ *   dv_t += sum_{r>=t} P_rt dO_r            (summed over the group's heads)
+ *
+ * Each (b, kvh) is one job (so the group sums have a single writer); within
+ * it every head of the group works on its own explicit copy of K and V.
+ * row_sel / key_sel (S flags, or NULL for all): which query rows get dq and
+ * which keys get dk / dv; the others are left zero.  The row statistics
+ * (lse_r, D_r) are always computed for every row, since dk and dv of one key
+ * need them for every later row. */
+
+typedef struct {
+    const uint16_t *q, *k, *v, *dout;
+    int B, S, Hq, Hkv, d;
+    double scale;
+    const int32_t *row_sel, *key_sel;
+    double *dq, *dk, *dv;
+    int tid, nthreads;
+    int status;
+} backward_job;
+
+static void *backward_worker(void *arg)
+{
+    backward_job *J = (backward_job *)arg;
+    const int S = J->S, d = J->d, g = J->Hq / J->Hkv;
+    double *Kh = (double *)malloc(sizeof(double) * (size_t)S * (size_t)d);
+    double *Vh = (double *)malloc(sizeof(double) * (size_t)S * (size_t)d);
+    double *Qh = (double *)malloc(sizeof(double) * (size_t)S * (size_t)d);
+    double *dOh = (double *)malloc(sizeof(double) * (size_t)S * (size_t)d);
+    double *lse = (double *)malloc(sizeof(double) * (size_t)S);
+    double *Dr = (double *)malloc(sizeof(double) * (size_t)S);
+    double *sc = (double *)malloc(sizeof(double) * (size_t)S);
+    if (!Kh || !Vh || !Qh || !dOh || !lse || !Dr || !sc) {
+        J->status = ORACLE_NO_MEMORY;
+        free(Kh); free(Vh); free(Qh); free(dOh); free(lse); free(Dr); free(sc);
+        return NULL;
+    }
+    const long long jobs = (long long)J->B * J->Hkv;
+    for (long long jb = J->tid; jb < jobs; jb += J->nthreads) {
+        const int b = (int)(jb / J->Hkv), kvh = (int)(jb % J->Hkv);
+        for (int hh = 0; hh < g; ++hh) {
+            const int h = kvh * g + hh;
+            if (gqa_oracle_kv_head(h, J->Hq, J->Hkv) != kvh) { J->status = ORACLE_BAD_ARG; break; }
+            /* this head's own copies: q, dO rows of head h; K, V rows of its KV head */
+            for (int t = 0; t < S; ++t) {
+                const size_t kv = (((size_t)b * S + (size_t)t) * J->Hkv + (size_t)kvh) * (size_t)d;
+                const size_t qo = (((size_t)b * S + (size_t)t) * J->Hq + (size_t)h) * (size_t)d;
+                for (int j = 0; j < d; ++j) {
+                    Kh[(size_t)t * d + j] = bf16_to_double(J->k[kv + j]);
+                    Vh[(size_t)t * d + j] = bf16_to_double(J->v[kv + j]);
+                    Qh[(size_t)t * d + j] = bf16_to_double(J->q[qo + j]);
+                    dOh[(size_t)t * d + j] = bf16_to_double(J->dout[qo + j]);
+                }
+            }
+            /* row statistics: lse_r and D_r for every row */
+            for (int r = 0; r < S; ++r) {
+                double m = -INFINITY;
+                for (int t = 0; t <= r; ++t) {
+                    double s = 0.0;
+                    for (int j = 0; j < d; ++j) s += Qh[(size_t)r * d + j] * Kh[(size_t)t * d + j];
+                    s *= J->scale;
+                    sc[t] = s;
+                    if (s > m) m = s;
+                }
+                double z = 0.0;
+                for (int t = 0; t <= r; ++t) z += exp(sc[t] - m);
+                lse[r] = m + log(z);
+                double Dsum = 0.0;
+                for (int t = 0; t <= r; ++t) {
+                    double dP = 0.0;
+                    for (int j = 0; j < d; ++j) dP += dOh[(size_t)r * d + j] * Vh[(size_t)t * d + j];
+                    Dsum += exp(sc[t] - lse[r]) * dP;
+                }
+                Dr[r] = Dsum;
+            }
+            /* dq for the selected rows */
+            for (int r = 0; r < S; ++r) {
+                if (J->row_sel && !J->row_sel[r]) continue;
+                double *dq = J->dq + (((size_t)b * S + (size_t)r) * J->Hq + (size_t)h) * (size_t)d;
+                for (int t = 0; t <= r; ++t) {
+                    double s = 0.0, dP = 0.0;
+                    for (int j = 0; j < d; ++j) {
+                        s += Qh[(size_t)r * d + j] * Kh[(size_t)t * d + j];
+                        dP += dOh[(size_t)r * d + j] * Vh[(size_t)t * d + j];
+                    }
+                    const double P = exp(s * J->scale - lse[r]);
+                    const double dS = P * (dP - Dr[r]);
+                    for (int j = 0; j < d; ++j) dq[j] += J->scale * dS * Kh[(size_t)t * d + j];
+                }
+            }
+            /* dk, dv for the selected keys, accumulated over the group's heads */
+            for (int t = 0; t < S; ++t) {
+                if (J->key_sel && !J->key_sel[t]) continue;
+                const size_t kv = (((size_t)b * S + (size_t)t) * J->Hkv + (size_t)kvh) * (size_t)d;
+                double *dk = J->dk + kv, *dv = J->dv + kv;
+                for (int r = t; r < S; ++r) {
+                    double s = 0.0, dP = 0.0;
+                    for (int j = 0; j < d; ++j) {
+                        s += Qh[(size_t)r * d + j] * Kh[(size_t)t * d + j];
+                        dP += dOh[(size_t)r * d + j] * Vh[(size_t)t * d + j];
+                    }
+                    const double P = exp(s * J->scale - lse[r]);
+                    const double dS = P * (dP - Dr[r]);
+                    for (int j = 0; j < d; ++j) {
+                        dv[j] += P * dOh[(size_t)r * d + j];
+                        dk[j] += J->scale * dS * Qh[(size_t)r * d + j];
+                    }
+                }
+            }
+        }
+    }
+    free(Kh); free(Vh); free(Qh); free(dOh); free(lse); free(Dr); free(sc);
+    return NULL;
+}
+
+/* q, dout [B,S,Hq,d], k, v [B,S,Hkv,d] bf16 bits; dq [B,S,Hq,d], dk, dv [B,S,Hkv,d] fp64, zeroed
+ * here.  row_sel / key_sel: NULL or S int32 flags.  Returns 0 on success. */
+int gqa_oracle_prefill_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                                int B, int S, int Hq, int Hkv, int d, double scale, const int32_t *row_sel,
+                                const int32_t *key_sel, double *dq, double *dk, double *dv, int nthreads)
+{
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return ORACLE_BAD_ARG;
+    if (B <= 0 || S <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return ORACLE_BAD_ARG;
+    if (Hq % Hkv != 0) return ORACLE_BAD_ARG;
+    memset(dq, 0, sizeof(double) * (size_t)B * S * Hq * d);
+    memset(dk, 0, sizeof(double) * (size_t)B * S * Hkv * d);
+    memset(dv, 0, sizeof(double) * (size_t)B * S * Hkv * d);
+    if (nthreads < 1) nthreads = 1;
+    if ((long long)nthreads > (long long)B * Hkv) nthreads = B * Hkv;
+    backward_job *jobs = (backward_job *)calloc((size_t)nthreads, sizeof(backward_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) { free(jobs); free(th); return ORACLE_NO_MEMORY; }
+    for (int i = 0; i < nthreads; ++i) {
+        backward_job J = {q, k, v, dout, B, S, Hq, Hkv, d, scale, row_sel, key_sel, dq, dk, dv, i, nthreads,
+                          ORACLE_OK};
+        jobs[i] = J;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, backward_worker, &jobs[i]);
+    backward_worker(&jobs[0]);
     for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
     int st = ORACLE_OK;
     for (int i = 0; i < nthreads; ++i) if (jobs[i].status != ORACLE_OK) st = jobs[i].status;

@@ -43,6 +43,13 @@ MUTANTS = {
     "e4m3 NaN code read as a number": ("if (e == 15 && m == 7) return NAN;", "if (e == 16) return NAN;"),
     "fp8 key scale dropped": ("Kh[t * d + j] = e4m3_to_double(J->k8[src + j]) * J->k_scale;",
                               "Kh[t * d + j] = e4m3_to_double(J->k8[src + j]);"),
+    "backward drops the D term": ("const double dS = P * (dP - Dr[r]);\n                    for (int j = 0; j < d; ++j) dq[j]",
+                                  "const double dS = P * dP;\n                    for (int j = 0; j < d; ++j) dq[j]"),
+    "backward dk without scale": ("dk[j] += J->scale * dS * Qh[(size_t)r * d + j];", "dk[j] += dS * Qh[(size_t)r * d + j];"),
+    "backward dv weighted by dS": ("dv[j] += P * dOh[(size_t)r * d + j];", "dv[j] += dS * dOh[(size_t)r * d + j];"),
+    "backward keys skip their own row": ("for (int r = t; r < S; ++r) {", "for (int r = t + 1; r < S; ++r) {"),
+    "backward group gradient from one head": ("if (J->key_sel && !J->key_sel[t]) continue;",
+                                              "if ((J->key_sel && !J->key_sel[t]) || hh > 0) continue;"),
     "fp8 values scaled by the key scale": ("Vh[t * d + j] = e4m3_to_double(J->v8[src + j]) * J->v_scale;",
                                            "Vh[t * d + j] = e4m3_to_double(J->v8[src + j]) * J->k_scale;"),
 }

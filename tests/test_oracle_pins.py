@@ -382,3 +382,98 @@ def test_fp8_rows_past_the_history_are_never_read(oracle_mod):
     b = oracle_mod.decode_fp8(y.q, y.k_cache, y.v_cache, y.k_scale, y.v_scale, y.seqlens, y.scale)
     assert np.isfinite(a).all()
     np.testing.assert_array_equal(a, b)
+
+
+# ---------------------------------------------------------------- causal prefill backward
+
+
+def test_backward_equals_autograd_of_the_repeated_form(oracle_mod):
+    """The pages' reference for the backward: repeat K and V along the query-head axis, run plain
+    attention, and let differentiation sum the repeats back (torch autograd in fp64), at the pages'
+    12/3 equivalence shape with distinct heads."""
+    B, S, Hq, Hkv, d = 2, 9, 12, 3, 16
+    x = inputs.make_prefill(B, S, Hq, Hkv, d, seed=61)
+    dout = inputs.make_dout(B, S, Hq, d, seed=61)
+    dq, dk, dv = oracle_mod.prefill_backward(x.q, x.k, x.v, dout, x.scale)
+    q = x.q.double().requires_grad_()
+    k = x.k.double().requires_grad_()
+    v = x.v.double().requires_grad_()
+    g = Hq // Hkv
+    out = _sdpa(q.transpose(1, 2), k.repeat_interleave(g, dim=2).transpose(1, 2),
+                v.repeat_interleave(g, dim=2).transpose(1, 2), x.scale, causal=True).transpose(1, 2)
+    out.backward(dout.double())
+    np.testing.assert_allclose(dq, q.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk, k.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv, v.grad.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def _causal_gqa_forward_np(q, k, v, scale):
+    """Plain float64 restatement of the causal grouped forward for finite differences."""
+    B, S, Hq, d = q.shape
+    Hkv = k.shape[2]
+    g = Hq // Hkv
+    out = np.zeros_like(q)
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // g
+            for r in range(S):
+                s = np.array([scale * q[b, r, h] @ k[b, t, kv] for t in range(r + 1)])
+                w = np.exp(s - s.max())
+                out[b, r, h] = (w[:, None] * v[b, :r + 1, kv]).sum(0) / w.sum()
+    return out
+
+
+def test_backward_finite_differences(oracle_mod):
+    """Central differences of L = sum(dO * out) with respect to every input element."""
+    B, S, Hq, Hkv, d = 1, 5, 4, 2, 3
+    x = inputs.make_prefill(B, S, Hq, Hkv, d, seed=62)
+    dout = inputs.make_dout(B, S, Hq, d, seed=62)
+    dq, dk, dv = oracle_mod.prefill_backward(x.q, x.k, x.v, dout, x.scale)
+    q0, k0, v0, w = (t.double().numpy() for t in (x.q, x.k, x.v, dout))
+    h = 1e-6
+
+    def loss(qq, kk, vv):
+        return float((w * _causal_gqa_forward_np(qq, kk, vv, x.scale)).sum())
+
+    for name, arr, grad in (("q", q0, dq), ("k", k0, dk), ("v", v0, dv)):
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            a1, a2 = arr.copy(), arr.copy()
+            a1[idx] += h
+            a2[idx] -= h
+            args1 = {"q": q0, "k": k0, "v": v0}
+            args2 = dict(args1)
+            args1[name], args2[name] = a1, a2
+            num[idx] = (loss(args1["q"], args1["k"], args1["v"]) - loss(args2["q"], args2["k"], args2["v"])) / (2 * h)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+def test_backward_shared_head_gradient_is_the_group_sum(oracle_mod):
+    """dK, dV of a shared head = the sum, over its group, of the per-head gradients of the same
+    computation written as MHA on explicitly repeated K and V."""
+    B, S, Hq, Hkv, d = 2, 7, 8, 2, 16
+    x = inputs.make_prefill(B, S, Hq, Hkv, d, seed=63)
+    dout = inputs.make_dout(B, S, Hq, d, seed=63)
+    g = Hq // Hkv
+    dq, dk, dv = oracle_mod.prefill_backward(x.q, x.k, x.v, dout, x.scale)
+    kr = x.k.repeat_interleave(g, dim=2).contiguous()
+    vr = x.v.repeat_interleave(g, dim=2).contiguous()
+    dq1, dk1, dv1 = oracle_mod.prefill_backward(x.q, kr, vr, dout, x.scale)
+    np.testing.assert_allclose(dq, dq1, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dk, dk1.reshape(B, S, Hkv, g, d).sum(3), rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dv, dv1.reshape(B, S, Hkv, g, d).sum(3), rtol=1e-12, atol=1e-14)
+    # a group of distinct heads does not give g times one head's gradient
+    assert not np.allclose(dk, g * dk1.reshape(B, S, Hkv, g, d)[:, :, :, 0])
+
+
+def test_backward_selected_rows_and_keys_match_the_full_gradient(oracle_mod):
+    B, S, Hq, Hkv, d = 1, 11, 6, 2, 8
+    x = inputs.make_prefill(B, S, Hq, Hkv, d, seed=64)
+    dout = inputs.make_dout(B, S, Hq, d, seed=64)
+    full = oracle_mod.prefill_backward(x.q, x.k, x.v, dout, x.scale)
+    rows, keys = [0, 5, 10], [0, 3, 10]
+    part = oracle_mod.prefill_backward(x.q, x.k, x.v, dout, x.scale, row_sel=rows, key_sel=keys)
+    np.testing.assert_array_equal(part[0][:, rows], full[0][:, rows])
+    np.testing.assert_array_equal(part[1][:, keys], full[1][:, keys])
+    np.testing.assert_array_equal(part[2][:, keys], full[2][:, keys])
+    assert not part[0][:, 1].any() and not part[1][:, 1].any()
