@@ -12,7 +12,8 @@ import ctypes
 import os
 
 __all__ = [
-    "GQAError", "gqa_decode", "gqa_decode_fp8", "gqa_decode_noalloc", "gqa_prefill_causal", "gqa_decode_expanded", "gqa_decode_expanded_bytes",
+    "GQAError", "gqa_decode", "gqa_decode_fp8", "gqa_decode_noalloc", "gqa_prefill_causal",
+    "gqa_prefill_causal_fwd", "gqa_prefill_causal_bwd", "gqa_decode_expanded", "gqa_decode_expanded_bytes",
     "gqa_decode_plan", "gqa_get_last_device_status", "gqa_selftest_wait_timeout", "gqa_set_profile_events",
     "gqa_last_launch_count", "gqa_release", "gqa_status_string", "gqa_version", "library_path", "load",
 ]
@@ -31,6 +32,8 @@ EXPORTS = {
                             _vp, _vp]),
     "gqa_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp]),
     "gqa_prefill_causal": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp]),
+    "gqa_prefill_causal_fwd": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "gqa_prefill_causal_bwd": (_i, [_vp] * 6 + [_i] * 5 + [_vp] * 4),
     "gqa_decode_expanded": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp, _vp, _vp]),
     "gqa_decode_expanded_bytes": (ctypes.c_size_t, [_i, _i, _i, _i]),
     "gqa_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
@@ -248,6 +251,60 @@ def gqa_prefill_causal(q, k, v, out=None, stream=None):
                                    _stream_ptr(stream))
     _check(st, "gqa_prefill_causal")
     return out
+
+
+def gqa_prefill_causal_fwd(q, k, v, out=None, lse=None, stream=None):
+    """gqa_prefill_causal that also returns lse [B,Hq,S] fp32 (natural log-sum-exp of each row's scaled
+    scores), for the backward.  Returns (out, lse)."""
+    import torch
+
+    _need(q, "q", torch.bfloat16, 4)
+    B, S, Hq, d = q.shape
+    _need(k, "k", torch.bfloat16, 4, q.device)
+    _need(v, "v", torch.bfloat16, 4, q.device)
+    Bk, Sk, Hkv, dk = k.shape
+    if (Bk, Sk, dk) != (B, S, d) or v.shape != k.shape:
+        raise ValueError("shape mismatch between q, k and v")
+    out = torch.empty_like(q) if out is None else out
+    _need(out, "out", torch.bfloat16, 4, q.device)
+    lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(lse, "lse", torch.float32, 3, q.device)
+    if out.shape != q.shape or lse.shape != (B, Hq, S):
+        raise ValueError("out must have q's shape and lse [B,Hq,S]")
+    st = load().gqa_prefill_causal_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, S, Hq, Hkv, d, out.data_ptr(),
+                                       lse.data_ptr(), _stream_ptr(stream))
+    _check(st, "gqa_prefill_causal_fwd")
+    return out, lse
+
+
+def gqa_prefill_causal_bwd(q, k, v, out, lse, dout, dq=None, dk=None, dv=None, stream=None):
+    """Gradients through gqa_prefill_causal: (dq [B,S,Hq,d], dk, dv [B,S,Hkv,d]) bf16; dk and dv are summed
+    over each KV head's group of query heads."""
+    import torch
+
+    _need(q, "q", torch.bfloat16, 4)
+    B, S, Hq, d = q.shape
+    _need(k, "k", torch.bfloat16, 4, q.device)
+    _need(v, "v", torch.bfloat16, 4, q.device)
+    _need(out, "out", torch.bfloat16, 4, q.device)
+    _need(dout, "dout", torch.bfloat16, 4, q.device)
+    _need(lse, "lse", torch.float32, 3, q.device)
+    Hkv = k.shape[2]
+    if k.shape != (B, S, Hkv, d) or v.shape != k.shape or out.shape != q.shape or dout.shape != q.shape \
+            or lse.shape != (B, Hq, S):
+        raise ValueError("shape mismatch between q, k, v, out, lse and dout")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, n, torch.bfloat16, 4, q.device)
+    if dq.shape != q.shape or dk.shape != k.shape or dv.shape != v.shape:
+        raise ValueError("gradient buffers must have the shapes of q, k and v")
+    st = load().gqa_prefill_causal_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                       dout.data_ptr(), B, S, Hq, Hkv, d, dq.data_ptr(), dk.data_ptr(),
+                                       dv.data_ptr(), _stream_ptr(stream))
+    _check(st, "gqa_prefill_causal_bwd")
+    return dq, dk, dv
 
 
 def gqa_decode_expanded_bytes(B, Tmax, Hq, d):

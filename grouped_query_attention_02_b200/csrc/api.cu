@@ -384,16 +384,25 @@ gqa_status gqa_decode_plan(int B, int Hq, int Hkv, int d, int Tmax, int num_sms,
     return GQA_OK;
 }
 
-gqa_status gqa_prefill_causal(const void *q, const void *k, const void *v, int B, int S, int Hq, int Hkv, int d,
-                              void *out, void *stream)
+}  // extern "C"
+
+namespace {
+
+gqa_status check_prefill_args(const void *q, const void *k, const void *v, int B, int S, int Hq, int Hkv, int d,
+                              const void *out)
 {
-    g_last_launches = 0;
     if (!q || !k || !v || !out) return GQA_ERR_INVALID_ARG;
     if (B <= 0 || S <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return GQA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
     if (d != kHeadDim) return GQA_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return GQA_ERR_MISALIGNED;
     if (B > 65535 || S > (1 << 30)) return GQA_ERR_UNSUPPORTED;
+    return GQA_OK;
+}
+
+gqa_status run_prefill(const void *q, const void *k, const void *v, int B, int S, int Hq, int Hkv, int d, void *out,
+                       float *lse, void *stream)
+{
     std::lock_guard<std::mutex> lk(g_mu);
     DeviceState *st = nullptr;
     gqa_status s = device_state(&st);
@@ -405,6 +414,7 @@ gqa_status gqa_prefill_causal(const void *q, const void *k, const void *v, int B
     if ((s = encode_4d(&tmV, v, kHeadDim, Hkv, S, B, 128)) != GQA_OK) return s;
     PrefillArgs a;
     a.out = static_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
     a.status = st->status;
     a.B = B;
     a.S = S;
@@ -419,6 +429,77 @@ gqa_status gqa_prefill_causal(const void *q, const void *k, const void *v, int B
     if (g_ev_after) cudaEventRecord(g_ev_after, cs);
     g_last_launches = 1;
     return GQA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gqa_status gqa_prefill_causal(const void *q, const void *k, const void *v, int B, int S, int Hq, int Hkv, int d,
+                              void *out, void *stream)
+{
+    g_last_launches = 0;
+    gqa_status s = check_prefill_args(q, k, v, B, S, Hq, Hkv, d, out);
+    if (s != GQA_OK) return s;
+    return run_prefill(q, k, v, B, S, Hq, Hkv, d, out, nullptr, stream);
+}
+
+gqa_status gqa_prefill_causal_fwd(const void *q, const void *k, const void *v, int B, int S, int Hq, int Hkv,
+                                  int d, void *out, float *lse, void *stream)
+{
+    g_last_launches = 0;
+    gqa_status s = check_prefill_args(q, k, v, B, S, Hq, Hkv, d, out);
+    if (s != GQA_OK) return s;
+    if (!lse) return GQA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(lse) & 3u) return GQA_ERR_MISALIGNED;
+    return run_prefill(q, k, v, B, S, Hq, Hkv, d, out, lse, stream);
+}
+
+gqa_status gqa_prefill_causal_bwd(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                                  const void *dout, int B, int S, int Hq, int Hkv, int d, void *dq, void *dk,
+                                  void *dv, void *stream)
+{
+    g_last_launches = 0;
+    gqa_status s = check_prefill_args(q, k, v, B, S, Hq, Hkv, d, out);
+    if (s != GQA_OK) return s;
+    if (!lse || !dout || !dq || !dk || !dv) return GQA_ERR_INVALID_ARG;
+    if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return GQA_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(lse) & 3u) return GQA_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState *st = nullptr;
+    if ((s = device_state(&st)) != GQA_OK) return s;
+    if ((s = get_encoder()) != GQA_OK) return s;
+    const size_t dbytes = (size_t)B * Hq * S * sizeof(float);
+    if ((s = ensure_workspace(st, dbytes)) != GQA_OK) return s;
+    CUtensorMap tmQ, tmK, tmV, tmDO;
+    if ((s = encode_4d(&tmQ, q, kHeadDim, Hq, S, B, 128)) != GQA_OK) return s;
+    if ((s = encode_4d(&tmK, k, kHeadDim, Hkv, S, B, 128)) != GQA_OK) return s;
+    if ((s = encode_4d(&tmV, v, kHeadDim, Hkv, S, B, 128)) != GQA_OK) return s;
+    if ((s = encode_4d(&tmDO, dout, kHeadDim, Hq, S, B, 128)) != GQA_OK) return s;
+    BackwardArgs a;
+    a.out = static_cast<const __nv_bfloat16 *>(out);
+    a.dout = static_cast<const __nv_bfloat16 *>(dout);
+    a.lse = lse;
+    a.dsum = static_cast<float *>(st->ws);
+    a.dq = static_cast<__nv_bfloat16 *>(dq);
+    a.dk = static_cast<__nv_bfloat16 *>(dk);
+    a.dv = static_cast<__nv_bfloat16 *>(dv);
+    a.status = st->status;
+    a.B = B;
+    a.S = S;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.group = Hq / Hkv;
+    a.scale = 1.0f / std::sqrt((float)d);
+    a.qscale = 1.4426950408889634f * a.scale;
+    a.wait_budget_ns = kWaitBudgetNs;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    int n = 0;
+    if (g_ev_before) cudaEventRecord(g_ev_before, cs);
+    s = cuda_status(launch_prefill_backward(tmQ, tmK, tmV, tmDO, a, cs, &n));
+    if (g_ev_after) cudaEventRecord(g_ev_after, cs);
+    g_last_launches = n;
+    return s;
 }
 
 gqa_status gqa_get_last_device_status(void *stream)

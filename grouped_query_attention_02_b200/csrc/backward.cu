@@ -1,0 +1,571 @@
+// backward.cu -- causal GQA prefill backward on the tcgen05 tensor cores.
+//
+// The gradients of a loss through O = softmax(scale Q K^T + causal mask) V, per query head h and its
+// KV head h / g ("grouped-query and multi-query attention", study.greatitself.com, training
+// paragraph: a shared key or value tensor receives the gradient of every query head of its group):
+//
+//   P = exp(scale q.k - lse)            (lse: the forward's log-sum-exp of the row)
+//   dP = dO V^T,  D = rowsum(dO * O),   dS = P * (dP - D)
+//   dV = sum over the group of P^T dO,  dK = scale * sum over the group of dS^T Q,  dQ = scale * dS K
+//
+// Three kernels:
+//   bwd_rowdot_kernel   D = rowsum(dO * O) in fp32, one warp per (sequence, row, head)
+//   bwd_dkdv_kernel     one CTA per (sequence, KV head, 128-key tile): loops over the g query heads
+//                       of the group and over the query tiles at or after the key tile; S^T = K Q^T and
+//                       dP^T = V dO^T into tensor memory, P^T and dS^T back into tensor memory as bf16,
+//                       then dV += P^T dO and dK += dS^T Q with the accumulators resident in tensor
+//                       memory for the whole loop, so the group sum costs nothing extra
+//   bwd_dq_kernel       one CTA per (sequence, query head, 128-row tile): loops over the key tiles up
+//                       to the diagonal; S = Q K^T and dP = dO V^T, dS back into tensor memory, then
+//                       dQ += dS K
+//
+// Roles in both tensor-core kernels (192 threads): warps 0..3 elementwise (one TMEM lane each: a key
+// row of S^T in the dK/dV kernel, a query row of S in the dQ kernel), warp 4 TMA producer, warp 5
+// TMEM allocator + MMA issuer.  The probabilities and dS are rounded to bf16 for the products, as the
+// forward rounds P.  Every wait is bounded; a kernel that gives up records GQA_ERR_DEVICE_TIMEOUT.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace gqa {
+
+namespace {
+
+constexpr int kD = kHeadDim;
+constexpr int kB = 128;                    // rows of a query tile and of a key tile
+constexpr int kTile = kB * kD * 2;         // 32 KB: one 128 x 128 bf16 tile
+constexpr int kHalf = kTile / 2;           // one 64-column half (128-byte rows, 128-byte swizzle)
+constexpr int kThreads = 192;
+constexpr int kEw = 128;                   // elementwise threads
+constexpr uint32_t kTmemCols = 512;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ void record_status(int *status, int code)
+{
+    if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ bool wait_or_fail(uint64_t *bar, uint32_t parity, const BackwardArgs &a,
+                                             volatile int *err)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*err) return false;
+        if (global_timer_ns() - t0 > a.wait_budget_ns) {
+            *err = 1;
+            record_status(a.status, kStatusTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t saddr) { return umma_smem_desc(saddr, 16, 1024, 2); }
+__device__ __forceinline__ uint64_t desc_mnmajor(uint32_t saddr) { return umma_smem_desc(saddr, kHalf, 1024, 2); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// D[b][h][r] = sum_j dO[b,r,h,j] * O[b,r,h,j]: one warp per row, four elements per lane.
+__global__ void bwd_rowdot_kernel(const BackwardArgs a)
+{
+    const long long rows = (long long)a.B * a.S * a.Hq;
+    const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (wid >= rows) return;
+    const int h = (int)(wid % a.Hq);
+    const long long br = wid / a.Hq;
+    const int r = (int)(br % a.S), b = (int)(br / a.S);
+    const uint2 o = *reinterpret_cast<const uint2 *>(a.out + wid * kD + lane * 4);
+    const uint2 g = *reinterpret_cast<const uint2 *>(a.dout + wid * kD + lane * 4);
+    float s = bf16_lo(o.x) * bf16_lo(g.x) + bf16_hi(o.x) * bf16_hi(g.x) + bf16_lo(o.y) * bf16_lo(g.y) +
+              bf16_hi(o.y) * bf16_hi(g.y);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) a.dsum[((size_t)b * a.Hq + h) * a.S + r] = s;
+}
+
+// ------------------------------------------------------------------------------------------------
+// dK, dV
+struct KvSmem {
+    static constexpr int k = 0;                      // K tile of this CTA's keys
+    static constexpr int v = k + kTile;              // V tile
+    static constexpr int q = v + kTile;              // Q[2] tiles of the current / next query tile
+    static constexpr int dout = q + 2 * kTile;       // dO[2]
+    static constexpr int lse = dout + 2 * kTile;     // [2][128] floats: lse * log2(e) (+inf past the end)
+    static constexpr int dsum = lse + 2 * kB * 4;    // [2][128] floats: D
+    static constexpr int bars = dsum + 2 * kB * 4;
+    static constexpr int nbars = 16;
+    static constexpr int tmem_slot = bars + nbars * 8;
+    static constexpr int err = tmem_slot + 8;
+    static constexpr int bytes = err + 8;
+};
+enum KvBar { KV_FULL = 0, QD_FULL = 1, QD_EMPTY = 3, RS_FULL = 5, RS_EMPTY = 7, SD_FULL = 9, PS_READY = 10,
+             MM_DONE = 11, ACC_FULL = 12, KDRAIN = 13 };
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                const BackwardArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + KvSmem::bars);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + KvSmem::tmem_slot);
+    volatile int *err = reinterpret_cast<volatile int *>(smem + KvSmem::err);
+
+    // the key tiles near the start of a sequence have the most query tiles after them: first
+    const int nt = (a.S + kB - 1) / kB;
+    const int bk_count = a.B * a.Hkv;
+    const int kt = blockIdx.x / bk_count;
+    const int bk = blockIdx.x % bk_count;
+    const int b = bk / a.Hkv, kvh = bk % a.Hkv;
+    const int g = a.group;
+    const int nq = nt - kt;                 // query tiles kt .. nt-1
+    const int n_it = g * nq;                // (head, query tile) iterations
+    const int k0 = kt * kB;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[KV_FULL], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar[QD_FULL + s], 1);
+            mbar_init(&bar[QD_EMPTY + s], 1);
+            mbar_init(&bar[RS_FULL + s], 32);
+            mbar_init(&bar[RS_EMPTY + s], kEw);
+        }
+        mbar_init(&bar[SD_FULL], 1);
+        mbar_init(&bar[PS_READY], kEw);
+        mbar_init(&bar[MM_DONE], 1);
+        mbar_init(&bar[ACC_FULL], 1);
+        mbar_init(&bar[KDRAIN], 1);
+        *err = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+
+    if (warp == 4) {
+        // ---------------- producer: K, V once; then Q, dO tiles (TMA) and lse, D rows (lane loads)
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmDO);
+            mbar_arrive_expect_tx(&bar[KV_FULL], 2 * kTile);
+            tma_load_4d(smem + KvSmem::k, &tmK, &bar[KV_FULL], 0, kvh, k0, b);
+            tma_load_4d(smem + KvSmem::k + kHalf, &tmK, &bar[KV_FULL], 64, kvh, k0, b);
+            tma_load_4d(smem + KvSmem::v, &tmV, &bar[KV_FULL], 0, kvh, k0, b);
+            tma_load_4d(smem + KvSmem::v + kHalf, &tmV, &bar[KV_FULL], 64, kvh, k0, b);
+        }
+        int issued = 0;
+        for (int n = 0; n < n_it; ++n) {
+            const int h = kvh * g + n / nq, q0 = (kt + n % nq) * kB, s = n & 1;
+            bool ok = true;
+            if (lane == 0) {
+                // lane 0 does every wait of the warp and tells the others, so that no lane leaves the loop
+                // alone (the warp meets again in __shfl_sync)
+                if (n >= 2 && !wait_or_fail(&bar[QD_EMPTY + s], ((n >> 1) - 1) & 1, a, err)) ok = false;
+                if (ok && n >= 2 && !wait_or_fail(&bar[RS_EMPTY + s], ((n >> 1) - 1) & 1, a, err)) ok = false;
+                if (ok) {
+                    mbar_arrive_expect_tx(&bar[QD_FULL + s], 2 * kTile);
+                    uint8_t *qs = smem + KvSmem::q + s * kTile, *ds = smem + KvSmem::dout + s * kTile;
+                    tma_load_4d(qs, &tmQ, &bar[QD_FULL + s], 0, h, q0, b);
+                    tma_load_4d(qs + kHalf, &tmQ, &bar[QD_FULL + s], 64, h, q0, b);
+                    tma_load_4d(ds, &tmDO, &bar[QD_FULL + s], 0, h, q0, b);
+                    tma_load_4d(ds + kHalf, &tmDO, &bar[QD_FULL + s], 64, h, q0, b);
+                    issued = n + 1;
+                }
+            }
+            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
+            // the row statistics of this query tile: rows past the sequence get lse = +inf (P = 0), D = 0
+            float *ls = reinterpret_cast<float *>(smem + KvSmem::lse) + s * kB;
+            float *dd = reinterpret_cast<float *>(smem + KvSmem::dsum) + s * kB;
+            const size_t row0 = ((size_t)b * a.Hq + h) * a.S;
+#pragma unroll
+            for (int i = 0; i < kB / 32; ++i) {
+                const int r = q0 + lane + 32 * i;
+                ls[lane + 32 * i] = r < a.S ? a.lse[row0 + r] * kLog2e : INFINITY;
+                dd[lane + 32 * i] = r < a.S ? a.dsum[row0 + r] : 0.f;
+            }
+            mbar_arrive(&bar[RS_FULL + s]);
+        }
+        if (lane == 0) {
+            // leave no copy in flight
+            mbar_wait(&bar[KV_FULL], 0, a.wait_budget_ns);
+            for (int n = issued - 1; n >= 0 && n >= issued - 2; --n)
+                mbar_wait(&bar[QD_FULL + (n & 1)], (n >> 1) & 1, a.wait_budget_ns);
+        }
+    } else if (warp == 5) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = umma_idesc_bf16(kB, kB, 0, 0);   // K (K-major) x Q (K-major) -> S^T
+            const uint32_t idesc_g = umma_idesc_bf16(kB, kD, 0, 1);   // P^T / dS^T (TMEM) x dO / Q (MN-major)
+            const uint32_t k_addr = smem_u32(smem + KvSmem::k), v_addr = smem_u32(smem + KvSmem::v);
+            bool ok = wait_or_fail(&bar[KV_FULL], 0, a, err);
+            int done = 0;
+            for (int n = 0; ok && n < n_it; ++n) {
+                const int s = n & 1;
+                if (!wait_or_fail(&bar[QD_FULL + s], (n >> 1) & 1, a, err)) break;
+                // the previous iteration's products read P^T and dS^T out of the S^T and dP^T columns
+                if (n >= 1 && !wait_or_fail(&bar[MM_DONE], (n - 1) & 1, a, err)) break;
+                tc_fence_after();
+                const uint32_t q_addr = smem_u32(smem + KvSmem::q + s * kTile);
+                const uint32_t o_addr = smem_u32(smem + KvSmem::dout + s * kTile);
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                    umma_ss(tS, desc_kmajor(k_addr + off), desc_kmajor(q_addr + off), idesc_s, ks > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                    umma_ss(tdP, desc_kmajor(v_addr + off), desc_kmajor(o_addr + off), idesc_s, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(&bar[SD_FULL]);
+                if (!wait_or_fail(&bar[PS_READY], n & 1, a, err)) break;
+                tc_fence_after();
+                // dV += P^T dO, dK += dS^T Q: A from tensor memory (16 query columns = 8 packed columns)
+#pragma unroll
+                for (int ks = 0; ks < kB / 16; ++ks)
+                    umma_ts(tdV, tS + ks * 8, desc_mnmajor(o_addr + ks * 2048), idesc_g, (n > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+                for (int ks = 0; ks < kB / 16; ++ks)
+                    umma_ts(tdK, tdP + ks * 8, desc_mnmajor(q_addr + ks * 2048), idesc_g, (n > 0 || ks > 0) ? 1u : 0u);
+                umma_commit(&bar[MM_DONE]);
+                umma_commit(&bar[QD_EMPTY + s]);
+                done = n + 1;
+            }
+            if (done == n_it) umma_commit(&bar[ACC_FULL]);
+            umma_commit(&bar[KDRAIN]);
+            mbar_wait(&bar[KDRAIN], 0, a.wait_budget_ns);
+        }
+    } else {
+        // ---------------- elementwise: thread t owns key k0 + t (TMEM lane t of S^T, dP^T, dV, dK)
+        const int quarter = warp & 3;
+        const int t = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        bool ok = true;
+        for (int n = 0; n < n_it; ++n) {
+            const int s = n & 1;
+            const bool diag = (n % nq) == 0;      // the query tile that holds this CTA's keys
+            if (!wait_or_fail(&bar[SD_FULL], n & 1, a, err)) { ok = false; break; }
+            if (!wait_or_fail(&bar[RS_FULL + s], (n >> 1) & 1, a, err)) { ok = false; break; }
+            tc_fence_after();
+            const float *ls = reinterpret_cast<const float *>(smem + KvSmem::lse) + s * kB;
+            const float *dd = reinterpret_cast<const float *>(smem + KvSmem::dsum) + s * kB;
+#pragma unroll 1
+            for (int c0 = 0; c0 < kB / 32; ++c0) {
+                uint32_t sr[32], pr[32];
+                tmem_ld32(tS + lane_off + c0 * 32, sr);
+                tmem_ld32(tdP + lane_off + c0 * 32, pr);
+                tmem_wait_ld();
+                uint32_t pw[16], dw[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const int c = c0 * 32 + i;
+                    // query c of the tile sees key t only when c >= t on the diagonal tile
+                    float p0 = ex2(__uint_as_float(sr[i]) * a.qscale - ls[c]);
+                    float p1 = ex2(__uint_as_float(sr[i + 1]) * a.qscale - ls[c + 1]);
+                    if (diag && c < t) p0 = 0.f;
+                    if (diag && c + 1 < t) p1 = 0.f;
+                    const float s0 = p0 * (__uint_as_float(pr[i]) - dd[c]);
+                    const float s1 = p1 * (__uint_as_float(pr[i + 1]) - dd[c + 1]);
+                    pw[i >> 1] = pack_bf16x2(p0, p1);
+                    dw[i >> 1] = pack_bf16x2(s0, s1);
+                }
+                // packed in place: 32 columns in, 16 columns out, at or before what was just read
+                tmem_st16(tS + lane_off + c0 * 16, pw);
+                tmem_st16(tdP + lane_off + c0 * 16, dw);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bar[RS_EMPTY + s]);
+            mbar_arrive(&bar[PS_READY]);
+        }
+        if (ok && wait_or_fail(&bar[ACC_FULL], 0, a, err)) {
+            tc_fence_after();
+            const int key = k0 + t;
+            __nv_bfloat16 *dvg = a.dv + (((size_t)b * a.S + key) * a.Hkv + kvh) * kD;
+            __nv_bfloat16 *dkg = a.dk + (((size_t)b * a.S + key) * a.Hkv + kvh) * kD;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t vr[32], kr[32];
+                tmem_ld32(tdV + lane_off + c * 32, vr);
+                tmem_ld32(tdK + lane_off + c * 32, kr);
+                tmem_wait_ld();
+                if (key < a.S) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(vr[i + 0]), __uint_as_float(vr[i + 1]));
+                        w.y = pack_bf16x2(__uint_as_float(vr[i + 2]), __uint_as_float(vr[i + 3]));
+                        w.z = pack_bf16x2(__uint_as_float(vr[i + 4]), __uint_as_float(vr[i + 5]));
+                        w.w = pack_bf16x2(__uint_as_float(vr[i + 6]), __uint_as_float(vr[i + 7]));
+                        *reinterpret_cast<uint4 *>(dvg + c * 32 + i) = w;
+                        w.x = pack_bf16x2(__uint_as_float(kr[i + 0]) * a.scale, __uint_as_float(kr[i + 1]) * a.scale);
+                        w.y = pack_bf16x2(__uint_as_float(kr[i + 2]) * a.scale, __uint_as_float(kr[i + 3]) * a.scale);
+                        w.z = pack_bf16x2(__uint_as_float(kr[i + 4]) * a.scale, __uint_as_float(kr[i + 5]) * a.scale);
+                        w.w = pack_bf16x2(__uint_as_float(kr[i + 6]) * a.scale, __uint_as_float(kr[i + 7]) * a.scale);
+                        *reinterpret_cast<uint4 *>(dkg + c * 32 + i) = w;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// dQ
+struct QSmem {
+    static constexpr int q = 0;                      // this CTA's Q tile
+    static constexpr int dout = q + kTile;           // and its dO tile
+    static constexpr int k = dout + kTile;           // K[2] tiles
+    static constexpr int v = k + 2 * kTile;          // V[2] tiles
+    static constexpr int bars = v + 2 * kTile;
+    static constexpr int nbars = 12;
+    static constexpr int tmem_slot = bars + nbars * 8;
+    static constexpr int err = tmem_slot + 8;
+    static constexpr int bytes = err + 8;
+};
+enum QBar { QO_FULL = 0, K2_FULL = 1, K2_EMPTY = 3, S2_FULL = 5, DS_READY = 6, MQ_DONE = 7, DQ_FULL = 8, QDRAIN = 9 };
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+              const BackwardArgs a)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + QSmem::bars);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + QSmem::tmem_slot);
+    volatile int *err = reinterpret_cast<volatile int *>(smem + QSmem::err);
+
+    // the last query tiles see the most key tiles: first
+    const int nt = (a.S + kB - 1) / kB;
+    const int bh_count = a.B * a.Hq;
+    const int qt = nt - 1 - blockIdx.x / bh_count;
+    const int bh = blockIdx.x % bh_count;
+    const int b = bh / a.Hq, h = bh % a.Hq;
+    const int kvh = h / a.group;
+    const int q0 = qt * kB;
+    const int ntiles = qt + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar[QO_FULL], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar[K2_FULL + s], 1);
+            mbar_init(&bar[K2_EMPTY + s], 1);
+        }
+        mbar_init(&bar[S2_FULL], 1);
+        mbar_init(&bar[DS_READY], kEw);
+        mbar_init(&bar[MQ_DONE], 1);
+        mbar_init(&bar[DQ_FULL], 1);
+        mbar_init(&bar[QDRAIN], 1);
+        *err = 0;
+        fence_barrier_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+
+    if (warp == 4) {
+        // ---------------- producer: Q, dO once; K_j, V_j into a two-stage ring
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmDO);
+            mbar_arrive_expect_tx(&bar[QO_FULL], 2 * kTile);
+            tma_load_4d(smem + QSmem::q, &tmQ, &bar[QO_FULL], 0, h, q0, b);
+            tma_load_4d(smem + QSmem::q + kHalf, &tmQ, &bar[QO_FULL], 64, h, q0, b);
+            tma_load_4d(smem + QSmem::dout, &tmDO, &bar[QO_FULL], 0, h, q0, b);
+            tma_load_4d(smem + QSmem::dout + kHalf, &tmDO, &bar[QO_FULL], 64, h, q0, b);
+            int issued = 0;
+            for (int j = 0; j < ntiles; ++j) {
+                const int s = j & 1;
+                if (j >= 2 && !wait_or_fail(&bar[K2_EMPTY + s], ((j >> 1) - 1) & 1, a, err)) break;
+                uint8_t *ks = smem + QSmem::k + s * kTile, *vs = smem + QSmem::v + s * kTile;
+                mbar_arrive_expect_tx(&bar[K2_FULL + s], 2 * kTile);
+                tma_load_4d(ks, &tmK, &bar[K2_FULL + s], 0, kvh, j * kB, b);
+                tma_load_4d(ks + kHalf, &tmK, &bar[K2_FULL + s], 64, kvh, j * kB, b);
+                tma_load_4d(vs, &tmV, &bar[K2_FULL + s], 0, kvh, j * kB, b);
+                tma_load_4d(vs + kHalf, &tmV, &bar[K2_FULL + s], 64, kvh, j * kB, b);
+                issued = j + 1;
+            }
+            for (int j = issued - 1; j >= 0 && j >= issued - 2; --j)
+                mbar_wait(&bar[K2_FULL + (j & 1)], (j >> 1) & 1, a.wait_budget_ns);
+            mbar_wait(&bar[QO_FULL], 0, a.wait_budget_ns);
+        }
+    } else if (warp == 5) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = umma_idesc_bf16(kB, kB, 0, 0);   // Q / dO (K-major) x K / V (K-major)
+            const uint32_t idesc_q = umma_idesc_bf16(kB, kD, 0, 1);   // dS (TMEM) x K (MN-major)
+            const uint32_t q_addr = smem_u32(smem + QSmem::q), o_addr = smem_u32(smem + QSmem::dout);
+            bool ok = wait_or_fail(&bar[QO_FULL], 0, a, err);
+            int done = 0;
+            for (int j = 0; ok && j < ntiles; ++j) {
+                const int s = j & 1;
+                if (!wait_or_fail(&bar[K2_FULL + s], (j >> 1) & 1, a, err)) break;
+                if (j >= 1 && !wait_or_fail(&bar[MQ_DONE], (j - 1) & 1, a, err)) break;
+                tc_fence_after();
+                const uint32_t k_addr = smem_u32(smem + QSmem::k + s * kTile);
+                const uint32_t v_addr = smem_u32(smem + QSmem::v + s * kTile);
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                    umma_ss(tS, desc_kmajor(q_addr + off), desc_kmajor(k_addr + off), idesc_s, ks > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int ks = 0; ks < kD / 16; ++ks) {
+                    const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                    umma_ss(tdP, desc_kmajor(o_addr + off), desc_kmajor(v_addr + off), idesc_s, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(&bar[S2_FULL]);
+                if (!wait_or_fail(&bar[DS_READY], j & 1, a, err)) break;
+                tc_fence_after();
+                // dQ += dS K: A = dS from tensor memory (16 keys = 8 packed columns), B = K rows (MN-major)
+#pragma unroll
+                for (int ks = 0; ks < kB / 16; ++ks)
+                    umma_ts(tdQ, tS + ks * 8, desc_mnmajor(k_addr + ks * 2048), idesc_q, (j > 0 || ks > 0) ? 1u : 0u);
+                umma_commit(&bar[MQ_DONE]);
+                umma_commit(&bar[K2_EMPTY + s]);
+                done = j + 1;
+            }
+            if (done == ntiles) umma_commit(&bar[DQ_FULL]);
+            umma_commit(&bar[QDRAIN]);
+            mbar_wait(&bar[QDRAIN], 0, a.wait_budget_ns);
+        }
+    } else {
+        // ---------------- elementwise: thread r owns query row q0 + r (TMEM lane r of S, dP, dQ)
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int qrow = q0 + r;
+        const size_t rs = ((size_t)b * a.Hq + h) * a.S + qrow;
+        const float lse2 = qrow < a.S ? a.lse[rs] * kLog2e : INFINITY;
+        const float dsum = qrow < a.S ? a.dsum[rs] : 0.f;
+        bool ok = true;
+        for (int j = 0; j < ntiles; ++j) {
+            if (!wait_or_fail(&bar[S2_FULL], j & 1, a, err)) { ok = false; break; }
+            tc_fence_after();
+            const bool diag = (j == qt);
+            const int kend = a.S - j * kB;        // keys of this tile that exist
+#pragma unroll 1
+            for (int c0 = 0; c0 < kB / 32; ++c0) {
+                uint32_t sr[32], pr[32];
+                tmem_ld32(tS + lane_off + c0 * 32, sr);
+                tmem_ld32(tdP + lane_off + c0 * 32, pr);
+                tmem_wait_ld();
+                uint32_t dw[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const int c = c0 * 32 + i;
+                    float p0 = ex2(__uint_as_float(sr[i]) * a.qscale - lse2);
+                    float p1 = ex2(__uint_as_float(sr[i + 1]) * a.qscale - lse2);
+                    // key c of the tile: after the row on the diagonal tile, or past the sequence
+                    if ((diag && c > r) || c >= kend) p0 = 0.f;
+                    if ((diag && c + 1 > r) || c + 1 >= kend) p1 = 0.f;
+                    dw[i >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[i]) - dsum),
+                                             p1 * (__uint_as_float(pr[i + 1]) - dsum));
+                }
+                tmem_st16(tS + lane_off + c0 * 16, dw);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bar[DS_READY]);
+        }
+        if (ok && wait_or_fail(&bar[DQ_FULL], 0, a, err)) {
+            tc_fence_after();
+            __nv_bfloat16 *dqg = a.dq + (((size_t)b * a.S + qrow) * a.Hq + h) * kD;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t qr[32];
+                tmem_ld32(tdQ + lane_off + c * 32, qr);
+                tmem_wait_ld();
+                if (qrow < a.S) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(qr[i + 0]) * a.scale, __uint_as_float(qr[i + 1]) * a.scale);
+                        w.y = pack_bf16x2(__uint_as_float(qr[i + 2]) * a.scale, __uint_as_float(qr[i + 3]) * a.scale);
+                        w.z = pack_bf16x2(__uint_as_float(qr[i + 4]) * a.scale, __uint_as_float(qr[i + 5]) * a.scale);
+                        w.w = pack_bf16x2(__uint_as_float(qr[i + 6]) * a.scale, __uint_as_float(qr[i + 7]) * a.scale);
+                        *reinterpret_cast<uint4 *>(dqg + c * 32 + i) = w;
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_backward(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                                    const CUtensorMap &tmDO, const BackwardArgs &a, cudaStream_t stream,
+                                    int *launches)
+{
+    static bool attr_done[64] = {};
+    const int smem_kv = KvSmem::bytes + 1024, smem_q = QSmem::bytes + 1024;
+    static_assert(KvSmem::bytes + 1024 <= 227 * 1024 && QSmem::bytes + 1024 <= 227 * 1024, "shared memory budget");
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_kv);
+        if (e != cudaSuccess) return e;
+        if ((e = cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q)) !=
+            cudaSuccess)
+            return e;
+        attr_done[dev] = true;
+    }
+    const long long rows = (long long)a.B * a.S * a.Hq;
+    const long long blocks = (rows * 32 + 255) / 256;
+    const long long nt = (a.S + kB - 1) / kB;
+    const long long grid_kv = nt * a.B * a.Hkv, grid_q = nt * a.B * a.Hq;
+    if (blocks > 0x7fffffffLL || grid_q > 0x7fffffffLL) return cudaErrorInvalidValue;
+    bwd_rowdot_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ++*launches;
+    bwd_dkdv_kernel<<<(unsigned)grid_kv, kThreads, smem_kv, stream>>>(tmQ, tmK, tmV, tmDO, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ++*launches;
+    bwd_dq_kernel<<<(unsigned)grid_q, kThreads, smem_q, stream>>>(tmQ, tmK, tmV, tmDO, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ++*launches;
+    return cudaSuccess;
+}
+
+}  // namespace gqa

@@ -86,11 +86,30 @@ cudaError_t launch_wait_timeout_selftest(int *status, unsigned long long budget_
 
 struct PrefillArgs {
     __nv_bfloat16 *out;       // [B,S,Hq,d]
+    float *lse;               // [B,Hq,S] natural log-sum-exp of each row's scaled scores, or null
     int *status;
     int B, S, Hq, Hkv, group;
     float qscale;             // log2(e) / sqrt(d)
     unsigned long long wait_budget_ns;
 };
+
+// Causal prefill backward (backward.cu): D = rowsum(dO * O), then dK/dV per key tile (summed over the
+// group's heads), then dQ per query tile.
+struct BackwardArgs {
+    const __nv_bfloat16 *out, *dout;   // [B,S,Hq,d]
+    const float *lse;                  // [B,Hq,S] natural log-sum-exp from the forward
+    float *dsum;                       // [B,Hq,S] workspace: D = rowsum(dO * O)
+    __nv_bfloat16 *dq;                 // [B,S,Hq,d]
+    __nv_bfloat16 *dk, *dv;            // [B,S,Hkv,d]
+    int *status;
+    int B, S, Hq, Hkv, group;
+    float qscale;                      // log2(e) / sqrt(d)
+    float scale;                       // 1 / sqrt(d)
+    unsigned long long wait_budget_ns;
+};
+cudaError_t launch_prefill_backward(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV,
+                                    const CUtensorMap &tmDO, const BackwardArgs &a, cudaStream_t stream,
+                                    int *launches);
 
 // The current device's status word (address of the library's device variable), or null.
 int *device_status_word();

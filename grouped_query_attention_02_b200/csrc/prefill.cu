@@ -331,6 +331,9 @@ prefill_causal_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         if (ok && wait_or_fail(&bar[O_FULL], 0, a, err)) {
             tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            // log-sum-exp of the row's scaled scores, natural log: (m + log2 l) ln 2
+            if (a.lse && qrow < a.S)
+                a.lse[((size_t)b * a.Hq + h) * a.S + qrow] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
             __nv_bfloat16 *orow_g = a.out + (((size_t)b * a.S + qrow) * a.Hq + h) * kD;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -622,6 +625,9 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         if (ok && wait_or_fail(&bar[PO_FULL], 0, a, err)) {
             tc_fence_after();
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            // log-sum-exp of the row's scaled scores, natural log: (m + log2 l) ln 2
+            if (a.lse && qrow < a.S)
+                a.lse[((size_t)b * a.Hq + hA + w) * a.S + qrow] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
             __nv_bfloat16 *orow_g = a.out + (((size_t)b * a.S + qrow) * a.Hq + hA + w) * kD;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {

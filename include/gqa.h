@@ -155,6 +155,39 @@ gqa_status gqa_prefill_causal(const void *q, const void *k, const void *v, int B
                               int d, void *out, void *stream);
 
 /*
+ * gqa_prefill_causal_fwd -- gqa_prefill_causal that also returns, per query
+ * row, the log-sum-exp of its scaled scores, which the backward needs:
+ *
+ *   lse  [B, Hq, S] fp32, device: lse[b,h,r] = log sum_{t <= r} exp(q[b,r,h].k[b,t,h/g] / sqrt(d))
+ *        (natural log; 4-byte aligned)
+ *
+ * out as in gqa_prefill_causal.
+ */
+gqa_status gqa_prefill_causal_fwd(const void *q, const void *k, const void *v, int B, int S, int Hq, int Hkv,
+                                  int d, void *out, float *lse, void *stream);
+
+/*
+ * gqa_prefill_causal_bwd -- gradients of a loss through gqa_prefill_causal.
+ * During training a shared key or value head receives the gradient of every
+ * query head of its group (study.greatitself.com "grouped-query and
+ * multi-query attention", training paragraph); dk and dv are those sums.
+ *
+ *   q, k, v, out, lse  the forward's inputs, output and log-sum-exp (gqa_prefill_causal_fwd)
+ *   dout  [B, S, Hq, d]   dL/dout
+ *   dq    [B, S, Hq, d]   dL/dq, written
+ *   dk, dv [B, S, Hkv, d] dL/dk, dL/dv, written (each the sum over the group's query heads)
+ *
+ * With P = exp(q.k / sqrt(d) - lse) (causal), dP = dout v^T, D = rowsum(dout * out),
+ * dS = P (dP - D): dv = sum_h P^T dout, dk = sum_h dS^T q / sqrt(d), dq = dS k / sqrt(d).
+ * P and dS are rounded to bf16 for the tensor-core products (fp32 accumulation); D is
+ * computed from the bf16 out.  Uses B*Hq*S*4 bytes of the library workspace; three
+ * kernels.  Same layouts, alignment and error rules as gqa_prefill_causal.
+ */
+gqa_status gqa_prefill_causal_bwd(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                                  const void *dout, int B, int S, int Hq, int Hkv, int d, void *dq, void *dk,
+                                  void *dv, void *stream);
+
+/*
  * gqa_decode_expanded -- the same decode computed the wasteful way, kept as a
  * baseline: every KV head is first physically repeated g times into the
  * caller's buffers k_rep/v_rep [B, Tmax, Hq, d] (rows t < seqlens[b] are
@@ -203,10 +236,11 @@ gqa_status gqa_selftest_wait_timeout(int timeout_us, void *stream);
 /*
  * gqa_set_profile_events -- measurement hook.  When both are non-NULL
  * (cudaEvent_t passed as void*), every later gqa_decode / gqa_decode_fp8 /
- * gqa_prefill_causal / gqa_decode_expanded records `before` on its stream
+ * gqa_prefill_causal(_fwd) / gqa_decode_expanded records `before` on its stream
  * immediately before its dominant kernel (the decode kernel; the prefill
- * kernel) and `after` immediately after it (gqa_decode_noalloc records
- * nothing).  NULL, NULL turns the hook off.
+ * kernel) and `after` immediately after it; gqa_prefill_causal_bwd records
+ * them around its three kernels; gqa_decode_noalloc records nothing.  NULL,
+ * NULL turns the hook off.
  */
 gqa_status gqa_set_profile_events(void *before, void *after);
 

@@ -390,14 +390,16 @@ int gqa_oracle_prefill(const uint16_t *q, const uint16_t *k, const uint16_t *v, 
  * it every head of the group works on its own explicit copy of K and V.
  * row_sel / key_sel (S flags, or NULL for all): which query rows get dq and
  * which keys get dk / dv; the others are left zero.  The row statistics
- * (lse_r, D_r) are always computed for every row, since dk and dv of one key
- * need them for every later row. */
+ * (lse_r, D_r) are computed for the selected rows and for every row at or
+ * after the first selected key, since dk and dv of a key need them for every
+ * later row. */
 
 typedef struct {
     const uint16_t *q, *k, *v, *dout;
     int B, S, Hq, Hkv, d;
     double scale;
     const int32_t *row_sel, *key_sel;
+    int first_key;        /* first selected key (key_sel given) */
     double *dq, *dk, *dv;
     int tid, nthreads;
     int status;
@@ -436,8 +438,10 @@ static void *backward_worker(void *arg)
                     dOh[(size_t)t * d + j] = bf16_to_double(J->dout[qo + j]);
                 }
             }
-            /* row statistics: lse_r and D_r for every row */
+            /* row statistics lse_r and D_r: for the selected rows and every row at or after the first
+             * selected key (the rows whose weights reach a selected key) */
             for (int r = 0; r < S; ++r) {
+                if (J->row_sel && J->key_sel && !J->row_sel[r] && r < J->first_key) continue;
                 double m = -INFINITY;
                 for (int t = 0; t <= r; ++t) {
                     double s = 0.0;
@@ -514,9 +518,13 @@ int gqa_oracle_prefill_backward(const uint16_t *q, const uint16_t *k, const uint
     backward_job *jobs = (backward_job *)calloc((size_t)nthreads, sizeof(backward_job));
     pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
     if (!jobs || !th) { free(jobs); free(th); return ORACLE_NO_MEMORY; }
+    int first_key = S;
+    if (key_sel)
+        for (int t = S - 1; t >= 0; --t)
+            if (key_sel[t]) first_key = t;
     for (int i = 0; i < nthreads; ++i) {
-        backward_job J = {q, k, v, dout, B, S, Hq, Hkv, d, scale, row_sel, key_sel, dq, dk, dv, i, nthreads,
-                          ORACLE_OK};
+        backward_job J = {q, k, v, dout, B, S, Hq, Hkv, d, scale, row_sel, key_sel, first_key, dq, dk, dv, i,
+                          nthreads, ORACLE_OK};
         jobs[i] = J;
     }
     for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, backward_worker, &jobs[i]);

@@ -144,3 +144,18 @@ def test_fp8_decode_argument_checks(lib):
     assert _decode_fp8(lib, Hq=64, Hkv=1) == UNSUPPORTED     # groups above 32
     assert _decode_fp8(lib, v=U) == MISALIGNED
     assert gqa.gqa_last_launch_count() == 0
+
+
+def test_prefill_fwd_and_bwd_argument_checks(lib):
+    assert lib.gqa_prefill_causal_fwd(A, A, A, 2, 64, 8, 2, 128, A, None, None) == INVALID
+    assert lib.gqa_prefill_causal_fwd(A, A, A, 2, 64, 8, 2, 128, A, A + 2, None) == MISALIGNED
+    assert lib.gqa_prefill_causal_fwd(A, A, A, 2, 64, 8, 3, 128, A, A, None) == INVALID
+    bwd = lambda **kw: lib.gqa_prefill_causal_bwd(
+        kw.get("q", A), A, A, A, kw.get("lse", A), kw.get("dout", A), 2, 64, 8, kw.get("Hkv", 2), kw.get("d", 128),
+        kw.get("dq", A), A, A, None)
+    assert bwd(dout=None) == INVALID
+    assert bwd(lse=None) == INVALID
+    assert bwd(Hkv=3) == INVALID
+    assert bwd(d=96) == UNSUPPORTED
+    assert bwd(dq=U) == MISALIGNED
+    assert gqa.gqa_last_launch_count() == 0

@@ -477,3 +477,9 @@ def test_backward_selected_rows_and_keys_match_the_full_gradient(oracle_mod):
     np.testing.assert_array_equal(part[1][:, keys], full[1][:, keys])
     np.testing.assert_array_equal(part[2][:, keys], full[2][:, keys])
     assert not part[0][:, 1].any() and not part[1][:, 1].any()
+    # late keys only: the row statistics are then taken for the selected rows and the rows after the keys
+    rows, keys = [1, 4], [7, 10]
+    part = oracle_mod.prefill_backward(x.q, x.k, x.v, dout, x.scale, row_sel=rows, key_sel=keys)
+    np.testing.assert_array_equal(part[0][:, rows], full[0][:, rows])
+    np.testing.assert_array_equal(part[1][:, keys], full[1][:, keys])
+    np.testing.assert_array_equal(part[2][:, keys], full[2][:, keys])
