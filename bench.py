@@ -225,6 +225,33 @@ def time_prefill(gqa, torch, p, steps: int, warmup: int):
     return s0.elapsed_time(s1) / steps, sum(a.elapsed_time(b) for a, b in kev) / steps, launches
 
 
+def prefill_backward_flops(B: int, S: int, Hq: int, d: int) -> int:
+    """10 * d per unmasked (query, key) pair per head: the five products of the backward
+    (S, dP, dV, dK, dQ), the minimal count (recomputation is not counted)."""
+    return 10 * d * B * Hq * S * (S + 1) // 2
+
+
+def time_backward(gqa, torch, inputs, p, steps: int, warmup: int):
+    """Mean time (ms) of gqa_prefill_causal_bwd (its three kernels) on the forward's outputs."""
+    B, S, Hq, d = p.q.shape
+    dout = inputs.make_dout(B, S, Hq, d, device="cuda", seed=0)
+    out, lse = gqa.gqa_prefill_causal_fwd(p.q, p.k, p.v)
+    dq, dk, dv = torch.empty_like(p.q), torch.empty_like(p.k), torch.empty_like(p.v)
+    call = lambda: gqa.gqa_prefill_causal_bwd(p.q, p.k, p.v, out, lse, dout, dq, dk, dv)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    s0, s1 = _events(torch)
+    launches = 0
+    s0.record()
+    for _ in range(steps):
+        call()
+        launches += gqa.gqa_last_launch_count()
+    s1.record()
+    torch.cuda.synchronize()
+    return s0.elapsed_time(s1) / steps, launches
+
+
 def decode_call(gqa, x, out, q=None, k=None, v=None, sl=None):
     """One decode step through the public API: the FP8 entry point when x carries per-tensor scales."""
     q = x.q if q is None else q
@@ -340,8 +367,9 @@ def main():
     ap.add_argument("--rows", choices=["all", "none"], default="all")
     ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the host-buffer measurement")
     ap.add_argument("--cpu-baseline", choices=["on", "off"], default="on")
-    ap.add_argument("--mode", choices=["decode", "prefill"], default="decode",
-                    help="prefill: time only the causal prefill workload (used for its ncu captures)")
+    ap.add_argument("--mode", choices=["decode", "prefill", "backward"], default="decode",
+                    help="prefill / backward: time only the causal prefill workload's forward / backward "
+                         "(used for their ncu captures)")
     ap.add_argument("--prefill-batch", type=int, default=4, help="sequences in --mode prefill")
     ap.add_argument("--decode-workload", default="Qwen3-8B",
                     help="name prefix of the decode workload timed as the headline (profiling other rows)")
@@ -402,6 +430,19 @@ def main():
     torch.cuda.set_device(local_rank)
     if args.mode == "prefill":
         prefill_only(gqa, torch, inputs, workloads, args)
+        return
+    if args.mode == "backward":
+        pw = workloads.CAUSAL_PREFILL
+        p = inputs.make_prefill(args.prefill_batch, pw.S, pw.Hq, pw.Hkv, pw.d, device="cuda", seed=0)
+        st_ms, n = time_backward(gqa, torch, inputs, p, args.steps, args.warmup)
+        fl = prefill_backward_flops(args.prefill_batch, pw.S, pw.Hq, pw.d)
+        peaks = load_peaks()
+        print(json.dumps({"metric": "causal GQA prefill backward TFLOP/s", "value": fl / (st_ms * 1e-3) / 1e12,
+                          "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": st_ms, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                          "config": {"workload": pw.name, "B": args.prefill_batch},
+                          "frac_bf16_peak": fl / (st_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                          "gpu_launches": n, "device_status": gqa.gqa_get_last_device_status()}))
         return
     dist = None
     if world > 1:
@@ -559,6 +600,20 @@ def main():
                                           "peak_source": f"{peaks.get('source')} bf16_tflops (cuBLAS burst)"}}
         except gqa.GQAError as e:
             rows[pw.name] = {"error": str(e)}
+        # causal prefill backward (dq, and dk / dv summed over each group)
+        try:
+            p = inputs.make_prefill(pw.B, pw.S, pw.Hq, pw.Hkv, pw.d, device="cuda", seed=0)
+            st_ms, n = time_backward(gqa, torch, inputs, p, 5, 2)
+            fl = prefill_backward_flops(pw.B, pw.S, pw.Hq, pw.d)
+            rows["backward, " + pw.name] = {
+                "ms_per_step": st_ms, "TFLOPs": fl / (st_ms * 1e-3) / 1e12,
+                "frac_bf16_peak": fl / (st_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                "flop_count": "10 d per unmasked pair per head (five products; recomputed S, dP not counted)",
+                "launches_per_step": n / 5}
+            del p
+            torch.cuda.empty_cache()
+        except gqa.GQAError as e:
+            rows["backward, " + pw.name] = {"error": str(e)}
         line["rows"] = rows
 
     # ---- the fp64 oracle on a bounded sample, host cores of this machine
