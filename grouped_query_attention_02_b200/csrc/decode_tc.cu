@@ -17,8 +17,8 @@
 //
 // Scheduling.  The host cannot see the lengths (they live on the device), so
 // decode_plan_kernel reads them and cuts every history into pieces of C tiles,
-// C chosen from the total work so that there are about eight rounds of pieces,
-// and lists the pieces longest first.  decode_persistent_kernel then runs one
+// C chosen from the total work so that there are about eight rounds of pieces
+// (two for groups above 16), and lists the pieces longest first.  decode_persistent_kernel then runs one
 // CTA per SM; each CTA claims (piece, KV head) units from an atomic counter
 // and keeps its TMA / MMA / softmax pipeline running across units.  A unit
 // that covers its whole history writes the output; otherwise it writes a
@@ -269,8 +269,10 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
             T += red_ll[i];
             M = max(M, red_i[i]);
         }
-        // about eight rounds of (piece, KV head) units per persistent CTA, never more than nsplit pieces
-        long long C = (T * a.Hkv + 8LL * slots - 1) / (8LL * slots);
+        // about eight rounds of (piece, KV head) units per persistent CTA (two for groups above 16, whose
+        // units of up to 32 heads carry a larger fixed cost each), never more than nsplit pieces
+        const long long rounds = a.group > 16 ? 2 : 8;
+        long long C = (T * a.Hkv + rounds * slots - 1) / (rounds * slots);
         const long long cmin = (M + a.nsplit - 1) / a.nsplit;
         if (C < cmin) C = cmin;
         if (C > M) C = M;
