@@ -98,13 +98,15 @@ struct KvSmem {
     static constexpr int lse = dout + 2 * kTile;     // [2][128] floats: lse * log2(e) (+inf past the end)
     static constexpr int dsum = lse + 2 * kB * 4;    // [2][128] floats: D
     static constexpr int bars = dsum + 2 * kB * 4;
-    static constexpr int nbars = 16;
+    static constexpr int nbars = 18;
     static constexpr int tmem_slot = bars + nbars * 8;
     static constexpr int err = tmem_slot + 8;
     static constexpr int bytes = err + 8;
 };
-enum KvBar { KV_FULL = 0, QD_FULL = 1, QD_EMPTY = 3, RS_FULL = 5, RS_EMPTY = 7, SD_FULL = 9, PS_READY = 10,
-             MM_DONE = 11, ACC_FULL = 12, KDRAIN = 13 };
+// S^T and dP^T products complete (ST_FULL, DPT_FULL); P^T written (P_READY); dS^T written (DST_READY);
+// the dV and dK products that read them complete (DV_DONE, DK_DONE)
+enum KvBar { KV_FULL = 0, QD_FULL = 1, QD_EMPTY = 3, RS_FULL = 5, RS_EMPTY = 7, ST_FULL = 9, DPT_FULL = 10,
+             P_READY = 11, DST_READY = 12, DV_DONE = 13, DK_DONE = 14, ACC_FULL = 15, KDRAIN = 16 };
 
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -137,9 +139,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_init(&bar[RS_FULL + s], 32);
             mbar_init(&bar[RS_EMPTY + s], kEw);
         }
-        mbar_init(&bar[SD_FULL], 1);
-        mbar_init(&bar[PS_READY], kEw);
-        mbar_init(&bar[MM_DONE], 1);
+        mbar_init(&bar[ST_FULL], 1);
+        mbar_init(&bar[DPT_FULL], 1);
+        mbar_init(&bar[P_READY], kEw);
+        mbar_init(&bar[DST_READY], kEw);
+        mbar_init(&bar[DV_DONE], 1);
+        mbar_init(&bar[DK_DONE], 1);
         mbar_init(&bar[ACC_FULL], 1);
         mbar_init(&bar[KDRAIN], 1);
         *err = 0;
@@ -207,7 +212,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 mbar_wait(&bar[QD_FULL + (n & 1)], (n >> 1) & 1, a.wait_budget_ns);
         }
     } else if (warp == 5) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer.  The elementwise pass hands over P^T before it computes dS^T, so
+        // dV += P^T dO runs while dS^T is being formed, and the next S^T once dV has read P^T.
         if (lane == 0) {
             const uint32_t idesc_s = umma_idesc_bf16(kB, kB, 0, 0);   // K (K-major) x Q (K-major) -> S^T
             const uint32_t idesc_g = umma_idesc_bf16(kB, kD, 0, 1);   // P^T / dS^T (TMEM) x dO / Q (MN-major)
@@ -217,32 +223,40 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             for (int n = 0; ok && n < n_it; ++n) {
                 const int s = n & 1;
                 if (!wait_or_fail(&bar[QD_FULL + s], (n >> 1) & 1, a, err)) break;
-                // the previous iteration's products read P^T and dS^T out of the S^T and dP^T columns
-                if (n >= 1 && !wait_or_fail(&bar[MM_DONE], (n - 1) & 1, a, err)) break;
-                tc_fence_after();
                 const uint32_t q_addr = smem_u32(smem + KvSmem::q + s * kTile);
                 const uint32_t o_addr = smem_u32(smem + KvSmem::dout + s * kTile);
+                // S^T: its columns held the previous P^T, read by the previous dV product
+                if (n >= 1 && !wait_or_fail(&bar[DV_DONE], (n - 1) & 1, a, err)) break;
+                tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
                     umma_ss(tS, desc_kmajor(k_addr + off), desc_kmajor(q_addr + off), idesc_s, ks > 0 ? 1u : 0u);
                 }
+                umma_commit(&bar[ST_FULL]);
+                // dP^T: its columns held the previous dS^T, read by the previous dK product
+                if (n >= 1 && !wait_or_fail(&bar[DK_DONE], (n - 1) & 1, a, err)) break;
+                tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
                     umma_ss(tdP, desc_kmajor(v_addr + off), desc_kmajor(o_addr + off), idesc_s, ks > 0 ? 1u : 0u);
                 }
-                umma_commit(&bar[SD_FULL]);
-                if (!wait_or_fail(&bar[PS_READY], n & 1, a, err)) break;
+                umma_commit(&bar[DPT_FULL]);
+                // dV += P^T dO: A from tensor memory (16 query columns = 8 packed columns)
+                if (!wait_or_fail(&bar[P_READY], n & 1, a, err)) break;
                 tc_fence_after();
-                // dV += P^T dO, dK += dS^T Q: A from tensor memory (16 query columns = 8 packed columns)
 #pragma unroll
                 for (int ks = 0; ks < kB / 16; ++ks)
                     umma_ts(tdV, tS + ks * 8, desc_mnmajor(o_addr + ks * 2048), idesc_g, (n > 0 || ks > 0) ? 1u : 0u);
+                umma_commit(&bar[DV_DONE]);
+                // dK += dS^T Q
+                if (!wait_or_fail(&bar[DST_READY], n & 1, a, err)) break;
+                tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < kB / 16; ++ks)
                     umma_ts(tdK, tdP + ks * 8, desc_mnmajor(q_addr + ks * 2048), idesc_g, (n > 0 || ks > 0) ? 1u : 0u);
-                umma_commit(&bar[MM_DONE]);
+                umma_commit(&bar[DK_DONE]);
                 umma_commit(&bar[QD_EMPTY + s]);
                 done = n + 1;
             }
@@ -256,42 +270,81 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int t = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         bool ok = true;
+        const float2 qs2 = make_float2(a.qscale, a.qscale);
         for (int n = 0; n < n_it; ++n) {
             const int s = n & 1;
             const bool diag = (n % nq) == 0;      // the query tile that holds this CTA's keys
-            if (!wait_or_fail(&bar[SD_FULL], n & 1, a, err)) { ok = false; break; }
             if (!wait_or_fail(&bar[RS_FULL + s], (n >> 1) & 1, a, err)) { ok = false; break; }
+            if (!wait_or_fail(&bar[ST_FULL], n & 1, a, err)) { ok = false; break; }
             tc_fence_after();
             const float *ls = reinterpret_cast<const float *>(smem + KvSmem::lse) + s * kB;
             const float *dd = reinterpret_cast<const float *>(smem + KvSmem::dsum) + s * kB;
-#pragma unroll 1
-            for (int c0 = 0; c0 < kB / 32; ++c0) {
-                uint32_t sr[32], pr[32];
-                tmem_ld32(tS + lane_off + c0 * 32, sr);
-                tmem_ld32(tdP + lane_off + c0 * 32, pr);
-                tmem_wait_ld();
-                uint32_t pw[16], dw[16];
+            // pass 1: P^T row t = 2^(s qscale - lse2), kept in registers and written back as bf16
+            float p[kB];
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
+            for (int c0 = 0; c0 < kB / 32; ++c0) {
+                uint32_t sr[32];
+                tmem_ld32(tS + lane_off + c0 * 32, sr);
+                tmem_wait_ld();
+                const float4 *ls4 = reinterpret_cast<const float4 *>(ls + c0 * 32);
+                uint32_t pw[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    const float4 l = ls4[i >> 2];
+                    const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])),
+                                                  qs2, make_float2(-l.x, -l.y));
+                    const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3])),
+                                                  qs2, make_float2(-l.z, -l.w));
                     const int c = c0 * 32 + i;
-                    // query c of the tile sees key t only when c >= t on the diagonal tile
-                    float p0 = ex2(__uint_as_float(sr[i]) * a.qscale - ls[c]);
-                    float p1 = ex2(__uint_as_float(sr[i + 1]) * a.qscale - ls[c + 1]);
-                    if (diag && c < t) p0 = 0.f;
-                    if (diag && c + 1 < t) p1 = 0.f;
-                    const float s0 = p0 * (__uint_as_float(pr[i]) - dd[c]);
-                    const float s1 = p1 * (__uint_as_float(pr[i + 1]) - dd[c + 1]);
-                    pw[i >> 1] = pack_bf16x2(p0, p1);
-                    dw[i >> 1] = pack_bf16x2(s0, s1);
+                    p[c] = ex2(x01.x);
+                    p[c + 1] = ex2(x01.y);
+                    p[c + 2] = ex2(x23.x);
+                    p[c + 3] = ex2(x23.y);
+                    if (diag) {
+                        // query c of the tile sees key t only when c >= t on the diagonal tile
+                        if (c < t) p[c] = 0.f;
+                        if (c + 1 < t) p[c + 1] = 0.f;
+                        if (c + 2 < t) p[c + 2] = 0.f;
+                        if (c + 3 < t) p[c + 3] = 0.f;
+                    }
+                    pw[i >> 1] = pack_bf16x2(p[c], p[c + 1]);
+                    pw[(i >> 1) + 1] = pack_bf16x2(p[c + 2], p[c + 3]);
                 }
                 // packed in place: 32 columns in, 16 columns out, at or before what was just read
                 tmem_st16(tS + lane_off + c0 * 16, pw);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bar[P_READY]);
+            // pass 2: dS^T = P^T (dP^T - D), written back as bf16 over dP^T
+            if (!wait_or_fail(&bar[DPT_FULL], n & 1, a, err)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int c0 = 0; c0 < kB / 32; ++c0) {
+                uint32_t pr[32];
+                tmem_ld32(tdP + lane_off + c0 * 32, pr);
+                tmem_wait_ld();
+                const float4 *dd4 = reinterpret_cast<const float4 *>(dd + c0 * 32);
+                uint32_t dw[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    const float4 dv = dd4[i >> 2];
+                    const int c = c0 * 32 + i;
+                    const float2 s01 = __fmul2_rn(make_float2(p[c], p[c + 1]),
+                                                  __fadd2_rn(make_float2(__uint_as_float(pr[i]), __uint_as_float(pr[i + 1])),
+                                                             make_float2(-dv.x, -dv.y)));
+                    const float2 s23 = __fmul2_rn(make_float2(p[c + 2], p[c + 3]),
+                                                  __fadd2_rn(make_float2(__uint_as_float(pr[i + 2]), __uint_as_float(pr[i + 3])),
+                                                             make_float2(-dv.z, -dv.w)));
+                    dw[i >> 1] = pack_bf16x2(s01.x, s01.y);
+                    dw[(i >> 1) + 1] = pack_bf16x2(s23.x, s23.y);
+                }
                 tmem_st16(tdP + lane_off + c0 * 16, dw);
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bar[RS_EMPTY + s]);
-            mbar_arrive(&bar[PS_READY]);
+            mbar_arrive(&bar[DST_READY]);
         }
         if (ok && wait_or_fail(&bar[ACC_FULL], 0, a, err)) {
             tc_fence_after();
@@ -340,12 +393,15 @@ struct QSmem {
     static constexpr int k = dout + kTile;           // K[2] tiles
     static constexpr int v = k + 2 * kTile;          // V[2] tiles
     static constexpr int bars = v + 2 * kTile;
-    static constexpr int nbars = 12;
+    static constexpr int nbars = 16;
     static constexpr int tmem_slot = bars + nbars * 8;
     static constexpr int err = tmem_slot + 8;
     static constexpr int bytes = err + 8;
 };
-enum QBar { QO_FULL = 0, K2_FULL = 1, K2_EMPTY = 3, S2_FULL = 5, DS_READY = 6, MQ_DONE = 7, DQ_FULL = 8, QDRAIN = 9 };
+// S2_FULL / S2_FREE / DS_READY: per S buffer (the pass of tile j + 1 can finish before the issuer has
+// seen tile j's, so DS_READY alternates like the buffers); DP_FREE: the pass has dP in registers
+enum QBar { QO_FULL = 0, K2_FULL = 1, K2_EMPTY = 3, S2_FULL = 5, S2_FREE = 7, DP_FULL = 9, DP_FREE = 10,
+            DS_READY = 11, DQ_FULL = 13, QDRAIN = 14 };
 
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -375,9 +431,14 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_init(&bar[K2_FULL + s], 1);
             mbar_init(&bar[K2_EMPTY + s], 1);
         }
-        mbar_init(&bar[S2_FULL], 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar[S2_FULL + s], 1);
+            mbar_init(&bar[S2_FREE + s], 1);
+        }
+        mbar_init(&bar[DP_FULL], 1);
+        mbar_init(&bar[DP_FREE], kEw);
         mbar_init(&bar[DS_READY], kEw);
-        mbar_init(&bar[MQ_DONE], 1);
+        mbar_init(&bar[DS_READY + 1], kEw);
         mbar_init(&bar[DQ_FULL], 1);
         mbar_init(&bar[QDRAIN], 1);
         *err = 0;
@@ -391,7 +452,8 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+    // S[2] (dS is packed into the S buffer it came from), dP, the dQ accumulator
+    const uint32_t tS0 = tmem, tdP = tmem + 256, tdQ = tmem + 384;
 
     if (warp == 4) {
         // ---------------- producer: Q, dO once; K_j, V_j into a two-stage ring
@@ -422,40 +484,54 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_wait(&bar[QO_FULL], 0, a.wait_budget_ns);
         }
     } else if (warp == 5) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer.  S is double-buffered and dP is released as soon as the elementwise
+        // pass holds it in registers, so the next tile's S and dP products run during this tile's pass.
         if (lane == 0) {
             const uint32_t idesc_s = umma_idesc_bf16(kB, kB, 0, 0);   // Q / dO (K-major) x K / V (K-major)
             const uint32_t idesc_q = umma_idesc_bf16(kB, kD, 0, 1);   // dS (TMEM) x K (MN-major)
             const uint32_t q_addr = smem_u32(smem + QSmem::q), o_addr = smem_u32(smem + QSmem::dout);
             bool ok = wait_or_fail(&bar[QO_FULL], 0, a, err);
             int done = 0;
-            for (int j = 0; ok && j < ntiles; ++j) {
-                const int s = j & 1;
-                if (!wait_or_fail(&bar[K2_FULL + s], (j >> 1) & 1, a, err)) break;
-                if (j >= 1 && !wait_or_fail(&bar[MQ_DONE], (j - 1) & 1, a, err)) break;
-                tc_fence_after();
-                const uint32_t k_addr = smem_u32(smem + QSmem::k + s * kTile);
-                const uint32_t v_addr = smem_u32(smem + QSmem::v + s * kTile);
+            for (int j = 0; ok && j <= ntiles; ++j) {
+                if (j < ntiles) {
+                    const int s = j & 1;
+                    if (!wait_or_fail(&bar[K2_FULL + s], (j >> 1) & 1, a, err)) break;
+                    // this S buffer's previous dS was read by the dQ product of tile j - 2
+                    if (j >= 2 && !wait_or_fail(&bar[S2_FREE + s], ((j >> 1) - 1) & 1, a, err)) break;
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(smem + QSmem::k + s * kTile);
+                    const uint32_t v_addr = smem_u32(smem + QSmem::v + s * kTile);
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-                    umma_ss(tS, desc_kmajor(q_addr + off), desc_kmajor(k_addr + off), idesc_s, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                        umma_ss(tS0 + s * 128, desc_kmajor(q_addr + off), desc_kmajor(k_addr + off), idesc_s,
+                                ks > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&bar[S2_FULL + s]);
+                    // the previous tile's dP is in the elementwise threads' registers by now
+                    if (j >= 1 && !wait_or_fail(&bar[DP_FREE], (j - 1) & 1, a, err)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < kD / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
+                        umma_ss(tdP, desc_kmajor(o_addr + off), desc_kmajor(v_addr + off), idesc_s, ks > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&bar[DP_FULL]);
                 }
+                if (j >= 1) {
+                    const int jp = j - 1, s = jp & 1;
+                    if (!wait_or_fail(&bar[DS_READY + s], (jp >> 1) & 1, a, err)) break;
+                    tc_fence_after();
+                    const uint32_t k_addr = smem_u32(smem + QSmem::k + s * kTile);
+                    // dQ += dS K: A = dS from tensor memory (16 keys = 8 packed columns), B = K rows (MN-major)
 #pragma unroll
-                for (int ks = 0; ks < kD / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-                    umma_ss(tdP, desc_kmajor(o_addr + off), desc_kmajor(v_addr + off), idesc_s, ks > 0 ? 1u : 0u);
+                    for (int ks = 0; ks < kB / 16; ++ks)
+                        umma_ts(tdQ, tS0 + s * 128 + ks * 8, desc_mnmajor(k_addr + ks * 2048), idesc_q,
+                                (jp > 0 || ks > 0) ? 1u : 0u);
+                    umma_commit(&bar[S2_FREE + s]);
+                    umma_commit(&bar[K2_EMPTY + s]);
+                    done = j;
                 }
-                umma_commit(&bar[S2_FULL]);
-                if (!wait_or_fail(&bar[DS_READY], j & 1, a, err)) break;
-                tc_fence_after();
-                // dQ += dS K: A = dS from tensor memory (16 keys = 8 packed columns), B = K rows (MN-major)
-#pragma unroll
-                for (int ks = 0; ks < kB / 16; ++ks)
-                    umma_ts(tdQ, tS + ks * 8, desc_mnmajor(k_addr + ks * 2048), idesc_q, (j > 0 || ks > 0) ? 1u : 0u);
-                umma_commit(&bar[MQ_DONE]);
-                umma_commit(&bar[K2_EMPTY + s]);
-                done = j + 1;
             }
             if (done == ntiles) umma_commit(&bar[DQ_FULL]);
             umma_commit(&bar[QDRAIN]);
@@ -472,33 +548,48 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const float dsum = qrow < a.S ? a.dsum[rs] : 0.f;
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
-            if (!wait_or_fail(&bar[S2_FULL], j & 1, a, err)) { ok = false; break; }
+            const int s = j & 1;
+            // dP into registers first, then release it for the next tile's product
+            if (!wait_or_fail(&bar[DP_FULL], j & 1, a, err)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t pr[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tdP + lane_off + c * 32, pr + c * 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&bar[DP_FREE]);
+            if (!wait_or_fail(&bar[S2_FULL + s], (j >> 1) & 1, a, err)) { ok = false; break; }
             tc_fence_after();
             const bool diag = (j == qt);
             const int kend = a.S - j * kB;        // keys of this tile that exist
-#pragma unroll 1
+            const bool edge = diag || kend < kB;  // masks only on the diagonal tile and at the sequence's end
+#pragma unroll
             for (int c0 = 0; c0 < kB / 32; ++c0) {
-                uint32_t sr[32], pr[32];
-                tmem_ld32(tS + lane_off + c0 * 32, sr);
-                tmem_ld32(tdP + lane_off + c0 * 32, pr);
+                uint32_t sr[32];
+                tmem_ld32(tS0 + s * 128 + lane_off + c0 * 32, sr);
                 tmem_wait_ld();
                 uint32_t dw[16];
+                const float2 qs2 = make_float2(a.qscale, a.qscale), nl2 = make_float2(-lse2, -lse2);
+                const float2 nd2 = make_float2(-dsum, -dsum);
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     const int c = c0 * 32 + i;
-                    float p0 = ex2(__uint_as_float(sr[i]) * a.qscale - lse2);
-                    float p1 = ex2(__uint_as_float(sr[i + 1]) * a.qscale - lse2);
-                    // key c of the tile: after the row on the diagonal tile, or past the sequence
-                    if ((diag && c > r) || c >= kend) p0 = 0.f;
-                    if ((diag && c + 1 > r) || c + 1 >= kend) p1 = 0.f;
-                    dw[i >> 1] = pack_bf16x2(p0 * (__uint_as_float(pr[i]) - dsum),
-                                             p1 * (__uint_as_float(pr[i + 1]) - dsum));
+                    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), qs2, nl2);
+                    float2 p = make_float2(ex2(x.x), ex2(x.y));
+                    if (edge) {
+                        // key c of the tile: after the row on the diagonal tile, or past the sequence
+                        if ((diag && c > r) || c >= kend) p.x = 0.f;
+                        if ((diag && c + 1 > r) || c + 1 >= kend) p.y = 0.f;
+                    }
+                    const float2 d = __fmul2_rn(p, __fadd2_rn(make_float2(__uint_as_float(pr[c]), __uint_as_float(pr[c + 1])), nd2));
+                    dw[i >> 1] = pack_bf16x2(d.x, d.y);
                 }
-                tmem_st16(tS + lane_off + c0 * 16, dw);
+                // packed in place: 32 columns in, 16 columns out, at or before what was just read
+                tmem_st16(tS0 + s * 128 + lane_off + c0 * 16, dw);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bar[DS_READY]);
+            mbar_arrive(&bar[DS_READY + s]);
         }
         if (ok && wait_or_fail(&bar[DQ_FULL], 0, a, err)) {
             tc_fence_after();
