@@ -34,8 +34,9 @@ constexpr int kD = kHeadDim;
 constexpr int kB = 128;                    // rows of a query tile and of a key tile
 constexpr int kTile = kB * kD * 2;         // 32 KB: one 128 x 128 bf16 tile
 constexpr int kHalf = kTile / 2;           // one 64-column half (128-byte rows, 128-byte swizzle)
-constexpr int kThreads = 192;
-constexpr int kEw = 128;                   // elementwise threads
+constexpr int kThreads = 320;
+constexpr int kEw = 256;                   // elementwise threads: two warpgroups, 64 columns each
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -96,17 +97,23 @@ struct KvSmem {
     static constexpr int q = v + kTile;              // Q[2] tiles of the current / next query tile
     static constexpr int dout = q + 2 * kTile;       // dO[2]
     static constexpr int lse = dout + 2 * kTile;     // [2][128] floats: lse * log2(e) (+inf past the end)
+    // (written by the first elementwise warpgroup; D below by the second)
     static constexpr int dsum = lse + 2 * kB * 4;    // [2][128] floats: D
     static constexpr int bars = dsum + 2 * kB * 4;
-    static constexpr int nbars = 18;
+    static constexpr int nbars = 20;
     static constexpr int tmem_slot = bars + nbars * 8;
     static constexpr int err = tmem_slot + 8;
     static constexpr int bytes = err + 8;
 };
 // S^T and dP^T products complete (ST_FULL, DPT_FULL); P^T written (P_READY); dS^T written (DST_READY);
 // the dV and dK products that read them complete (DV_DONE, DK_DONE)
-enum KvBar { KV_FULL = 0, QD_FULL = 1, QD_EMPTY = 3, RS_FULL = 5, RS_EMPTY = 7, ST_FULL = 9, DPT_FULL = 10,
-             P_READY = 11, DST_READY = 12, DV_DONE = 13, DK_DONE = 14, ACC_FULL = 15, KDRAIN = 16 };
+// ST_READ / DPT_READ: the first elementwise warpgroup has read the raw columns the second one's packed
+// output lands on
+// RS_FULL: the row statistics of an iteration are in shared memory (the elementwise threads load them one
+// iteration ahead, so their global-memory latency hides behind a whole iteration)
+enum KvBar { KV_FULL = 0, QD_FULL = 1, QD_EMPTY = 3, RS_FULL = 5, ST_FULL = 9, DPT_FULL = 10,
+             P_READY = 11, DST_READY = 12, DV_DONE = 13, DK_DONE = 14, ACC_FULL = 15, KDRAIN = 16, ST_READ = 17,
+             DPT_READ = 18 };
 
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -136,8 +143,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar[QD_FULL + s], 1);
             mbar_init(&bar[QD_EMPTY + s], 1);
-            mbar_init(&bar[RS_FULL + s], 32);
-            mbar_init(&bar[RS_EMPTY + s], kEw);
+            mbar_init(&bar[RS_FULL + s], kEw);
         }
         mbar_init(&bar[ST_FULL], 1);
         mbar_init(&bar[DPT_FULL], 1);
@@ -147,10 +153,12 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_init(&bar[DK_DONE], 1);
         mbar_init(&bar[ACC_FULL], 1);
         mbar_init(&bar[KDRAIN], 1);
+        mbar_init(&bar[ST_READ], kEw / 2);
+        mbar_init(&bar[DPT_READ], kEw / 2);
         *err = 0;
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -160,8 +168,8 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
 
-    if (warp == 4) {
-        // ---------------- producer: K, V once; then Q, dO tiles (TMA) and lse, D rows (lane loads)
+    if (warp == kProducerWarp) {
+        // ---------------- producer: K, V once; then the Q, dO tiles of every iteration (TMA)
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
@@ -172,46 +180,24 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tma_load_4d(smem + KvSmem::k + kHalf, &tmK, &bar[KV_FULL], 64, kvh, k0, b);
             tma_load_4d(smem + KvSmem::v, &tmV, &bar[KV_FULL], 0, kvh, k0, b);
             tma_load_4d(smem + KvSmem::v + kHalf, &tmV, &bar[KV_FULL], 64, kvh, k0, b);
-        }
-        int issued = 0;
-        for (int n = 0; n < n_it; ++n) {
-            const int h = kvh * g + n / nq, q0 = (kt + n % nq) * kB, s = n & 1;
-            bool ok = true;
-            if (lane == 0) {
-                // lane 0 does every wait of the warp and tells the others, so that no lane leaves the loop
-                // alone (the warp meets again in __shfl_sync)
-                if (n >= 2 && !wait_or_fail(&bar[QD_EMPTY + s], ((n >> 1) - 1) & 1, a, err)) ok = false;
-                if (ok && n >= 2 && !wait_or_fail(&bar[RS_EMPTY + s], ((n >> 1) - 1) & 1, a, err)) ok = false;
-                if (ok) {
-                    mbar_arrive_expect_tx(&bar[QD_FULL + s], 2 * kTile);
-                    uint8_t *qs = smem + KvSmem::q + s * kTile, *ds = smem + KvSmem::dout + s * kTile;
-                    tma_load_4d(qs, &tmQ, &bar[QD_FULL + s], 0, h, q0, b);
-                    tma_load_4d(qs + kHalf, &tmQ, &bar[QD_FULL + s], 64, h, q0, b);
-                    tma_load_4d(ds, &tmDO, &bar[QD_FULL + s], 0, h, q0, b);
-                    tma_load_4d(ds + kHalf, &tmDO, &bar[QD_FULL + s], 64, h, q0, b);
-                    issued = n + 1;
-                }
+            int issued = 0;
+            for (int n = 0; n < n_it; ++n) {
+                const int h = kvh * g + n / nq, q0 = (kt + n % nq) * kB, s = n & 1;
+                if (n >= 2 && !wait_or_fail(&bar[QD_EMPTY + s], ((n >> 1) - 1) & 1, a, err)) break;
+                mbar_arrive_expect_tx(&bar[QD_FULL + s], 2 * kTile);
+                uint8_t *qs = smem + KvSmem::q + s * kTile, *ds = smem + KvSmem::dout + s * kTile;
+                tma_load_4d(qs, &tmQ, &bar[QD_FULL + s], 0, h, q0, b);
+                tma_load_4d(qs + kHalf, &tmQ, &bar[QD_FULL + s], 64, h, q0, b);
+                tma_load_4d(ds, &tmDO, &bar[QD_FULL + s], 0, h, q0, b);
+                tma_load_4d(ds + kHalf, &tmDO, &bar[QD_FULL + s], 64, h, q0, b);
+                issued = n + 1;
             }
-            if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) break;
-            // the row statistics of this query tile: rows past the sequence get lse = +inf (P = 0), D = 0
-            float *ls = reinterpret_cast<float *>(smem + KvSmem::lse) + s * kB;
-            float *dd = reinterpret_cast<float *>(smem + KvSmem::dsum) + s * kB;
-            const size_t row0 = ((size_t)b * a.Hq + h) * a.S;
-#pragma unroll
-            for (int i = 0; i < kB / 32; ++i) {
-                const int r = q0 + lane + 32 * i;
-                ls[lane + 32 * i] = r < a.S ? a.lse[row0 + r] * kLog2e : INFINITY;
-                dd[lane + 32 * i] = r < a.S ? a.dsum[row0 + r] : 0.f;
-            }
-            mbar_arrive(&bar[RS_FULL + s]);
-        }
-        if (lane == 0) {
             // leave no copy in flight
             mbar_wait(&bar[KV_FULL], 0, a.wait_budget_ns);
             for (int n = issued - 1; n >= 0 && n >= issued - 2; --n)
                 mbar_wait(&bar[QD_FULL + (n & 1)], (n >> 1) & 1, a.wait_budget_ns);
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer.  The elementwise pass hands over P^T before it computes dS^T, so
         // dV += P^T dO runs while dS^T is being formed, and the next S^T once dV has read P^T.
         if (lane == 0) {
@@ -265,53 +251,70 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             mbar_wait(&bar[KDRAIN], 0, a.wait_budget_ns);
         }
     } else {
-        // ---------------- elementwise: thread t owns key k0 + t (TMEM lane t of S^T, dP^T, dV, dK)
+        // ---------------- elementwise: thread t owns key k0 + t (TMEM lane t of S^T, dP^T, dV, dK);
+        // warpgroup w takes query columns 64w .. 64w + 63
+        const int w = warp >> 2;
         const int quarter = warp & 3;
         const int t = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         bool ok = true;
         const float2 qs2 = make_float2(a.qscale, a.qscale);
+        // row statistic t of iteration n's query tile: lse * log2(e) (warpgroup 0) or D (warpgroup 1); rows
+        // past the sequence get lse = +inf (P = 0) and D = 0
+        auto row_stat = [&](int n) -> float {
+            const int h = kvh * g + n / nq, r = (kt + n % nq) * kB + t;
+            const size_t i = ((size_t)b * a.Hq + h) * a.S + r;
+            return w == 0 ? (r < a.S ? a.lse[i] * kLog2e : INFINITY) : (r < a.S ? a.dsum[i] : 0.f);
+        };
+        float *stat_smem = reinterpret_cast<float *>(smem + (w == 0 ? KvSmem::lse : KvSmem::dsum));
+        stat_smem[t] = row_stat(0);
+        mbar_arrive(&bar[RS_FULL]);
         for (int n = 0; n < n_it; ++n) {
             const int s = n & 1;
             const bool diag = (n % nq) == 0;      // the query tile that holds this CTA's keys
             if (!wait_or_fail(&bar[RS_FULL + s], (n >> 1) & 1, a, err)) { ok = false; break; }
+            // the next iteration's statistic, in flight during this iteration
+            const float next_stat = n + 1 < n_it ? row_stat(n + 1) : 0.f;
             if (!wait_or_fail(&bar[ST_FULL], n & 1, a, err)) { ok = false; break; }
             tc_fence_after();
-            const float *ls = reinterpret_cast<const float *>(smem + KvSmem::lse) + s * kB;
-            const float *dd = reinterpret_cast<const float *>(smem + KvSmem::dsum) + s * kB;
-            // pass 1: P^T row t = 2^(s qscale - lse2), kept in registers and written back as bf16
-            float p[kB];
-#pragma unroll
-            for (int c0 = 0; c0 < kB / 32; ++c0) {
-                uint32_t sr[32];
-                tmem_ld32(tS + lane_off + c0 * 32, sr);
+            const float *ls = reinterpret_cast<const float *>(smem + KvSmem::lse) + s * kB + w * 64;
+            const float *dd = reinterpret_cast<const float *>(smem + KvSmem::dsum) + s * kB + w * 64;
+            // pass 1: P^T = 2^(s qscale - lse2) over this warpgroup's 64 columns, kept in registers and
+            // written back as bf16 (packed: columns 64w.. land on packed columns 32w..)
+            float p[64];
+            {
+                uint32_t sr[64];
+                tmem_ld32(tS + lane_off + w * 64, sr);
+                tmem_ld32(tS + lane_off + w * 64 + 32, sr + 32);
                 tmem_wait_ld();
-                const float4 *ls4 = reinterpret_cast<const float4 *>(ls + c0 * 32);
-                uint32_t pw[16];
+                if (w == 0) mbar_arrive(&bar[ST_READ]);
+                const float4 *ls4 = reinterpret_cast<const float4 *>(ls);
+                uint32_t pw[32];
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) {
+                for (int i = 0; i < 64; i += 4) {
                     const float4 l = ls4[i >> 2];
                     const float2 x01 = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])),
                                                   qs2, make_float2(-l.x, -l.y));
                     const float2 x23 = __ffma2_rn(make_float2(__uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3])),
                                                   qs2, make_float2(-l.z, -l.w));
-                    const int c = c0 * 32 + i;
-                    p[c] = ex2(x01.x);
-                    p[c + 1] = ex2(x01.y);
-                    p[c + 2] = ex2(x23.x);
-                    p[c + 3] = ex2(x23.y);
+                    p[i] = ex2(x01.x);
+                    p[i + 1] = ex2(x01.y);
+                    p[i + 2] = ex2(x23.x);
+                    p[i + 3] = ex2(x23.y);
                     if (diag) {
                         // query c of the tile sees key t only when c >= t on the diagonal tile
-                        if (c < t) p[c] = 0.f;
-                        if (c + 1 < t) p[c + 1] = 0.f;
-                        if (c + 2 < t) p[c + 2] = 0.f;
-                        if (c + 3 < t) p[c + 3] = 0.f;
+                        const int c = w * 64 + i;
+                        if (c < t) p[i] = 0.f;
+                        if (c + 1 < t) p[i + 1] = 0.f;
+                        if (c + 2 < t) p[i + 2] = 0.f;
+                        if (c + 3 < t) p[i + 3] = 0.f;
                     }
-                    pw[i >> 1] = pack_bf16x2(p[c], p[c + 1]);
-                    pw[(i >> 1) + 1] = pack_bf16x2(p[c + 2], p[c + 3]);
+                    pw[i >> 1] = pack_bf16x2(p[i], p[i + 1]);
+                    pw[(i >> 1) + 1] = pack_bf16x2(p[i + 2], p[i + 3]);
                 }
-                // packed in place: 32 columns in, 16 columns out, at or before what was just read
-                tmem_st16(tS + lane_off + c0 * 16, pw);
+                // the second warpgroup's packed columns 32..63 are raw columns the first one reads
+                if (w == 1 && !wait_or_fail(&bar[ST_READ], n & 1, a, err)) { ok = false; break; }
+                tmem_st32(tS + lane_off + w * 32, pw);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -319,32 +322,38 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             // pass 2: dS^T = P^T (dP^T - D), written back as bf16 over dP^T
             if (!wait_or_fail(&bar[DPT_FULL], n & 1, a, err)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
-            for (int c0 = 0; c0 < kB / 32; ++c0) {
-                uint32_t pr[32];
-                tmem_ld32(tdP + lane_off + c0 * 32, pr);
+            {
+                uint32_t pr[64];
+                tmem_ld32(tdP + lane_off + w * 64, pr);
+                tmem_ld32(tdP + lane_off + w * 64 + 32, pr + 32);
                 tmem_wait_ld();
-                const float4 *dd4 = reinterpret_cast<const float4 *>(dd + c0 * 32);
-                uint32_t dw[16];
+                if (w == 0) mbar_arrive(&bar[DPT_READ]);
+                const float4 *dd4 = reinterpret_cast<const float4 *>(dd);
+                uint32_t dw[32];
 #pragma unroll
-                for (int i = 0; i < 32; i += 4) {
+                for (int i = 0; i < 64; i += 4) {
                     const float4 dv = dd4[i >> 2];
-                    const int c = c0 * 32 + i;
-                    const float2 s01 = __fmul2_rn(make_float2(p[c], p[c + 1]),
+                    const float2 s01 = __fmul2_rn(make_float2(p[i], p[i + 1]),
                                                   __fadd2_rn(make_float2(__uint_as_float(pr[i]), __uint_as_float(pr[i + 1])),
                                                              make_float2(-dv.x, -dv.y)));
-                    const float2 s23 = __fmul2_rn(make_float2(p[c + 2], p[c + 3]),
+                    const float2 s23 = __fmul2_rn(make_float2(p[i + 2], p[i + 3]),
                                                   __fadd2_rn(make_float2(__uint_as_float(pr[i + 2]), __uint_as_float(pr[i + 3])),
                                                              make_float2(-dv.z, -dv.w)));
                     dw[i >> 1] = pack_bf16x2(s01.x, s01.y);
                     dw[(i >> 1) + 1] = pack_bf16x2(s23.x, s23.y);
                 }
-                tmem_st16(tdP + lane_off + c0 * 16, dw);
+                if (w == 1 && !wait_or_fail(&bar[DPT_READ], n & 1, a, err)) { ok = false; break; }
+                tmem_st32(tdP + lane_off + w * 32, dw);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bar[RS_EMPTY + s]);
             mbar_arrive(&bar[DST_READY]);
+            // the other buffer was read in iteration n - 1, which both warpgroups have left: the dP^T of
+            // this iteration needed the dK product of n - 1, which needed every thread's dS^T of n - 1
+            if (n + 1 < n_it) {
+                stat_smem[(s ^ 1) * kB + t] = next_stat;
+                mbar_arrive(&bar[RS_FULL + (s ^ 1)]);
+            }
         }
         if (ok && wait_or_fail(&bar[ACC_FULL], 0, a, err)) {
             tc_fence_after();
@@ -352,7 +361,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             __nv_bfloat16 *dvg = a.dv + (((size_t)b * a.S + key) * a.Hkv + kvh) * kD;
             __nv_bfloat16 *dkg = a.dk + (((size_t)b * a.S + key) * a.Hkv + kvh) * kD;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * w; c < 2 * w + 2; ++c) {
                 uint32_t vr[32], kr[32];
                 tmem_ld32(tdV + lane_off + c * 32, vr);
                 tmem_ld32(tdK + lane_off + c * 32, kr);
@@ -360,17 +369,17 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 if (key < a.S) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(vr[i + 0]), __uint_as_float(vr[i + 1]));
-                        w.y = pack_bf16x2(__uint_as_float(vr[i + 2]), __uint_as_float(vr[i + 3]));
-                        w.z = pack_bf16x2(__uint_as_float(vr[i + 4]), __uint_as_float(vr[i + 5]));
-                        w.w = pack_bf16x2(__uint_as_float(vr[i + 6]), __uint_as_float(vr[i + 7]));
-                        *reinterpret_cast<uint4 *>(dvg + c * 32 + i) = w;
-                        w.x = pack_bf16x2(__uint_as_float(kr[i + 0]) * a.scale, __uint_as_float(kr[i + 1]) * a.scale);
-                        w.y = pack_bf16x2(__uint_as_float(kr[i + 2]) * a.scale, __uint_as_float(kr[i + 3]) * a.scale);
-                        w.z = pack_bf16x2(__uint_as_float(kr[i + 4]) * a.scale, __uint_as_float(kr[i + 5]) * a.scale);
-                        w.w = pack_bf16x2(__uint_as_float(kr[i + 6]) * a.scale, __uint_as_float(kr[i + 7]) * a.scale);
-                        *reinterpret_cast<uint4 *>(dkg + c * 32 + i) = w;
+                        uint4 v4;
+                        v4.x = pack_bf16x2(__uint_as_float(vr[i + 0]), __uint_as_float(vr[i + 1]));
+                        v4.y = pack_bf16x2(__uint_as_float(vr[i + 2]), __uint_as_float(vr[i + 3]));
+                        v4.z = pack_bf16x2(__uint_as_float(vr[i + 4]), __uint_as_float(vr[i + 5]));
+                        v4.w = pack_bf16x2(__uint_as_float(vr[i + 6]), __uint_as_float(vr[i + 7]));
+                        *reinterpret_cast<uint4 *>(dvg + c * 32 + i) = v4;
+                        v4.x = pack_bf16x2(__uint_as_float(kr[i + 0]) * a.scale, __uint_as_float(kr[i + 1]) * a.scale);
+                        v4.y = pack_bf16x2(__uint_as_float(kr[i + 2]) * a.scale, __uint_as_float(kr[i + 3]) * a.scale);
+                        v4.z = pack_bf16x2(__uint_as_float(kr[i + 4]) * a.scale, __uint_as_float(kr[i + 5]) * a.scale);
+                        v4.w = pack_bf16x2(__uint_as_float(kr[i + 6]) * a.scale, __uint_as_float(kr[i + 7]) * a.scale);
+                        *reinterpret_cast<uint4 *>(dkg + c * 32 + i) = v4;
                     }
                 }
             }
@@ -379,7 +388,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
@@ -401,7 +410,8 @@ struct QSmem {
 // S2_FULL / S2_FREE / DS_READY: per S buffer (the pass of tile j + 1 can finish before the issuer has
 // seen tile j's, so DS_READY alternates like the buffers); DP_FREE: the pass has dP in registers
 enum QBar { QO_FULL = 0, K2_FULL = 1, K2_EMPTY = 3, S2_FULL = 5, S2_FREE = 7, DP_FULL = 9, DP_FREE = 10,
-            DS_READY = 11, DQ_FULL = 13, QDRAIN = 14 };
+            DS_READY = 11, DQ_FULL = 13, QDRAIN = 14, S2_READ = 15 };   // S2_READ: see the dK/dV kernel's ST_READ
+static_assert(S2_READ < QSmem::nbars && DPT_READ < KvSmem::nbars, "barrier slots");
 
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -441,10 +451,11 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(&bar[DS_READY + 1], kEw);
         mbar_init(&bar[DQ_FULL], 1);
         mbar_init(&bar[QDRAIN], 1);
+        mbar_init(&bar[S2_READ], kEw / 2);
         *err = 0;
         fence_barrier_init();
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -455,7 +466,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     // S[2] (dS is packed into the S buffer it came from), dP, the dQ accumulator
     const uint32_t tS0 = tmem, tdP = tmem + 256, tdQ = tmem + 384;
 
-    if (warp == 4) {
+    if (warp == kProducerWarp) {
         // ---------------- producer: Q, dO once; K_j, V_j into a two-stage ring
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
@@ -483,7 +494,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 mbar_wait(&bar[K2_FULL + (j & 1)], (j >> 1) & 1, a.wait_budget_ns);
             mbar_wait(&bar[QO_FULL], 0, a.wait_budget_ns);
         }
-    } else if (warp == 5) {
+    } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer.  S is double-buffered and dP is released as soon as the elementwise
         // pass holds it in registers, so the next tile's S and dP products run during this tile's pass.
         if (lane == 0) {
@@ -538,7 +549,9 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             mbar_wait(&bar[QDRAIN], 0, a.wait_budget_ns);
         }
     } else {
-        // ---------------- elementwise: thread r owns query row q0 + r (TMEM lane r of S, dP, dQ)
+        // ---------------- elementwise: thread r owns query row q0 + r (TMEM lane r of S, dP, dQ);
+        // warpgroup w takes key columns 64w .. 64w + 63
+        const int w = warp >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
@@ -546,15 +559,17 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const size_t rs = ((size_t)b * a.Hq + h) * a.S + qrow;
         const float lse2 = qrow < a.S ? a.lse[rs] * kLog2e : INFINITY;
         const float dsum = qrow < a.S ? a.dsum[rs] : 0.f;
+        const float2 qs2 = make_float2(a.qscale, a.qscale), nl2 = make_float2(-lse2, -lse2);
+        const float2 nd2 = make_float2(-dsum, -dsum);
         bool ok = true;
         for (int j = 0; j < ntiles; ++j) {
             const int s = j & 1;
             // dP into registers first, then release it for the next tile's product
             if (!wait_or_fail(&bar[DP_FULL], j & 1, a, err)) { ok = false; break; }
             tc_fence_after();
-            uint32_t pr[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tdP + lane_off + c * 32, pr + c * 32);
+            uint32_t pr[64];
+            tmem_ld32(tdP + lane_off + w * 64, pr);
+            tmem_ld32(tdP + lane_off + w * 64 + 32, pr + 32);
             tmem_wait_ld();
             tc_fence_before();
             mbar_arrive(&bar[DP_FREE]);
@@ -563,30 +578,29 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const bool diag = (j == qt);
             const int kend = a.S - j * kB;        // keys of this tile that exist
             const bool edge = diag || kend < kB;  // masks only on the diagonal tile and at the sequence's end
+            uint32_t sr[64];
+            tmem_ld32(tS0 + s * 128 + lane_off + w * 64, sr);
+            tmem_ld32(tS0 + s * 128 + lane_off + w * 64 + 32, sr + 32);
+            tmem_wait_ld();
+            if (w == 0) mbar_arrive(&bar[S2_READ]);
+            uint32_t dw[32];
 #pragma unroll
-            for (int c0 = 0; c0 < kB / 32; ++c0) {
-                uint32_t sr[32];
-                tmem_ld32(tS0 + s * 128 + lane_off + c0 * 32, sr);
-                tmem_wait_ld();
-                uint32_t dw[16];
-                const float2 qs2 = make_float2(a.qscale, a.qscale), nl2 = make_float2(-lse2, -lse2);
-                const float2 nd2 = make_float2(-dsum, -dsum);
-#pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const int c = c0 * 32 + i;
-                    const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), qs2, nl2);
-                    float2 p = make_float2(ex2(x.x), ex2(x.y));
-                    if (edge) {
-                        // key c of the tile: after the row on the diagonal tile, or past the sequence
-                        if ((diag && c > r) || c >= kend) p.x = 0.f;
-                        if ((diag && c + 1 > r) || c + 1 >= kend) p.y = 0.f;
-                    }
-                    const float2 d = __fmul2_rn(p, __fadd2_rn(make_float2(__uint_as_float(pr[c]), __uint_as_float(pr[c + 1])), nd2));
-                    dw[i >> 1] = pack_bf16x2(d.x, d.y);
+            for (int i = 0; i < 64; i += 2) {
+                const int c = w * 64 + i;
+                const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), qs2, nl2);
+                float2 p = make_float2(ex2(x.x), ex2(x.y));
+                if (edge) {
+                    // key c of the tile: after the row on the diagonal tile, or past the sequence
+                    if ((diag && c > r) || c >= kend) p.x = 0.f;
+                    if ((diag && c + 1 > r) || c + 1 >= kend) p.y = 0.f;
                 }
-                // packed in place: 32 columns in, 16 columns out, at or before what was just read
-                tmem_st16(tS0 + s * 128 + lane_off + c0 * 16, dw);
+                const float2 d = __fmul2_rn(p, __fadd2_rn(make_float2(__uint_as_float(pr[i]), __uint_as_float(pr[i + 1])), nd2));
+                dw[i >> 1] = pack_bf16x2(d.x, d.y);
             }
+            // packed: key columns 64w.. land on packed columns 32w.., which for w = 1 are raw columns the
+            // first warpgroup reads
+            if (w == 1 && !wait_or_fail(&bar[S2_READ], j & 1, a, err)) { ok = false; break; }
+            tmem_st32(tS0 + s * 128 + lane_off + w * 32, dw);
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bar[DS_READY + s]);
@@ -595,19 +609,19 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tc_fence_after();
             __nv_bfloat16 *dqg = a.dq + (((size_t)b * a.S + qrow) * a.Hq + h) * kD;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 2 * w; c < 2 * w + 2; ++c) {
                 uint32_t qr[32];
                 tmem_ld32(tdQ + lane_off + c * 32, qr);
                 tmem_wait_ld();
                 if (qrow < a.S) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(qr[i + 0]) * a.scale, __uint_as_float(qr[i + 1]) * a.scale);
-                        w.y = pack_bf16x2(__uint_as_float(qr[i + 2]) * a.scale, __uint_as_float(qr[i + 3]) * a.scale);
-                        w.z = pack_bf16x2(__uint_as_float(qr[i + 4]) * a.scale, __uint_as_float(qr[i + 5]) * a.scale);
-                        w.w = pack_bf16x2(__uint_as_float(qr[i + 6]) * a.scale, __uint_as_float(qr[i + 7]) * a.scale);
-                        *reinterpret_cast<uint4 *>(dqg + c * 32 + i) = w;
+                        uint4 v4;
+                        v4.x = pack_bf16x2(__uint_as_float(qr[i + 0]) * a.scale, __uint_as_float(qr[i + 1]) * a.scale);
+                        v4.y = pack_bf16x2(__uint_as_float(qr[i + 2]) * a.scale, __uint_as_float(qr[i + 3]) * a.scale);
+                        v4.z = pack_bf16x2(__uint_as_float(qr[i + 4]) * a.scale, __uint_as_float(qr[i + 5]) * a.scale);
+                        v4.w = pack_bf16x2(__uint_as_float(qr[i + 6]) * a.scale, __uint_as_float(qr[i + 7]) * a.scale);
+                        *reinterpret_cast<uint4 *>(dqg + c * 32 + i) = v4;
                     }
                 }
             }
@@ -616,7 +630,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
