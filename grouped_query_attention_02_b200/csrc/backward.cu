@@ -399,19 +399,23 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 struct QSmem {
     static constexpr int q = 0;                      // this CTA's Q tile
     static constexpr int dout = q + kTile;           // and its dO tile
-    static constexpr int k = dout + kTile;           // K[2] tiles
-    static constexpr int v = k + 2 * kTile;          // V[2] tiles
-    static constexpr int bars = v + 2 * kTile;
-    static constexpr int nbars = 16;
+    // separate rings: K is read by S and by the dQ product, V only by dP, which frees it much earlier
+    static constexpr int kstages = 3, vstages = 2;
+    static constexpr int k = dout + kTile;           // K[3] tiles
+    static constexpr int v = k + kstages * kTile;    // V[2] tiles
+    static constexpr int bars = v + vstages * kTile;
+    static constexpr int nbars = 22;
     static constexpr int tmem_slot = bars + nbars * 8;
     static constexpr int err = tmem_slot + 8;
     static constexpr int bytes = err + 8;
 };
 // S2_FULL / S2_FREE / DS_READY: per S buffer (the pass of tile j + 1 can finish before the issuer has
 // seen tile j's, so DS_READY alternates like the buffers); DP_FREE: the pass has dP in registers
-enum QBar { QO_FULL = 0, K2_FULL = 1, K2_EMPTY = 3, S2_FULL = 5, S2_FREE = 7, DP_FULL = 9, DP_FREE = 10,
-            DS_READY = 11, DQ_FULL = 13, QDRAIN = 14, S2_READ = 15 };   // S2_READ: see the dK/dV kernel's ST_READ
-static_assert(S2_READ < QSmem::nbars && DPT_READ < KvSmem::nbars, "barrier slots");
+enum QBar { QO_FULL = 0, K2_FULL = 1, K2_EMPTY = 4, S2_FULL = 7, S2_FREE = 9, DP_FULL = 11, DP_FREE = 12,
+            DS_READY = 13, DQ_FULL = 15, QDRAIN = 16, S2_READ = 17,   // S2_READ: see the dK/dV kernel's ST_READ
+            V2_FULL = 18, V2_EMPTY = 20 };
+static_assert(V2_EMPTY + QSmem::vstages <= QSmem::nbars && K2_FULL + QSmem::kstages <= K2_EMPTY &&
+                  K2_EMPTY + QSmem::kstages <= S2_FULL && DPT_READ < KvSmem::nbars, "barrier slots");
 
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -437,9 +441,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         mbar_init(&bar[QO_FULL], 1);
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < QSmem::kstages; ++s) {
             mbar_init(&bar[K2_FULL + s], 1);
             mbar_init(&bar[K2_EMPTY + s], 1);
+        }
+        for (int s = 0; s < QSmem::vstages; ++s) {
+            mbar_init(&bar[V2_FULL + s], 1);
+            mbar_init(&bar[V2_EMPTY + s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&bar[S2_FULL + s], 1);
@@ -467,7 +475,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const uint32_t tS0 = tmem, tdP = tmem + 256, tdQ = tmem + 384;
 
     if (warp == kProducerWarp) {
-        // ---------------- producer: Q, dO once; K_j, V_j into a two-stage ring
+        // ---------------- producer: Q, dO once; K_j into a three-stage ring, V_j into a two-stage ring
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
@@ -478,20 +486,31 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tma_load_4d(smem + QSmem::q + kHalf, &tmQ, &bar[QO_FULL], 64, h, q0, b);
             tma_load_4d(smem + QSmem::dout, &tmDO, &bar[QO_FULL], 0, h, q0, b);
             tma_load_4d(smem + QSmem::dout + kHalf, &tmDO, &bar[QO_FULL], 64, h, q0, b);
-            int issued = 0;
+            int issued_k = 0, issued_v = 0;
             for (int j = 0; j < ntiles; ++j) {
-                const int s = j & 1;
-                if (j >= 2 && !wait_or_fail(&bar[K2_EMPTY + s], ((j >> 1) - 1) & 1, a, err)) break;
-                uint8_t *ks = smem + QSmem::k + s * kTile, *vs = smem + QSmem::v + s * kTile;
-                mbar_arrive_expect_tx(&bar[K2_FULL + s], 2 * kTile);
-                tma_load_4d(ks, &tmK, &bar[K2_FULL + s], 0, kvh, j * kB, b);
-                tma_load_4d(ks + kHalf, &tmK, &bar[K2_FULL + s], 64, kvh, j * kB, b);
-                tma_load_4d(vs, &tmV, &bar[K2_FULL + s], 0, kvh, j * kB, b);
-                tma_load_4d(vs + kHalf, &tmV, &bar[K2_FULL + s], 64, kvh, j * kB, b);
-                issued = j + 1;
+                const int sk = j % QSmem::kstages, sv = j % QSmem::vstages;
+                if (j >= QSmem::kstages &&
+                    !wait_or_fail(&bar[K2_EMPTY + sk], ((j / QSmem::kstages) - 1) & 1, a, err))
+                    break;
+                uint8_t *ks = smem + QSmem::k + sk * kTile;
+                mbar_arrive_expect_tx(&bar[K2_FULL + sk], kTile);
+                tma_load_4d(ks, &tmK, &bar[K2_FULL + sk], 0, kvh, j * kB, b);
+                tma_load_4d(ks + kHalf, &tmK, &bar[K2_FULL + sk], 64, kvh, j * kB, b);
+                issued_k = j + 1;
+                if (j >= QSmem::vstages &&
+                    !wait_or_fail(&bar[V2_EMPTY + sv], ((j / QSmem::vstages) - 1) & 1, a, err))
+                    break;
+                uint8_t *vs = smem + QSmem::v + sv * kTile;
+                mbar_arrive_expect_tx(&bar[V2_FULL + sv], kTile);
+                tma_load_4d(vs, &tmV, &bar[V2_FULL + sv], 0, kvh, j * kB, b);
+                tma_load_4d(vs + kHalf, &tmV, &bar[V2_FULL + sv], 64, kvh, j * kB, b);
+                issued_v = j + 1;
             }
-            for (int j = issued - 1; j >= 0 && j >= issued - 2; --j)
-                mbar_wait(&bar[K2_FULL + (j & 1)], (j >> 1) & 1, a.wait_budget_ns);
+            // leave no copy in flight
+            for (int j = issued_k - 1; j >= 0 && j >= issued_k - QSmem::kstages; --j)
+                mbar_wait(&bar[K2_FULL + j % QSmem::kstages], (j / QSmem::kstages) & 1, a.wait_budget_ns);
+            for (int j = issued_v - 1; j >= 0 && j >= issued_v - QSmem::vstages; --j)
+                mbar_wait(&bar[V2_FULL + j % QSmem::vstages], (j / QSmem::vstages) & 1, a.wait_budget_ns);
             mbar_wait(&bar[QO_FULL], 0, a.wait_budget_ns);
         }
     } else if (warp == kMmaWarp) {
@@ -505,13 +524,13 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             int done = 0;
             for (int j = 0; ok && j <= ntiles; ++j) {
                 if (j < ntiles) {
-                    const int s = j & 1;
-                    if (!wait_or_fail(&bar[K2_FULL + s], (j >> 1) & 1, a, err)) break;
+                    const int s = j & 1, sk = j % QSmem::kstages, sv = j % QSmem::vstages;
+                    if (!wait_or_fail(&bar[K2_FULL + sk], (j / QSmem::kstages) & 1, a, err)) break;
                     // this S buffer's previous dS was read by the dQ product of tile j - 2
                     if (j >= 2 && !wait_or_fail(&bar[S2_FREE + s], ((j >> 1) - 1) & 1, a, err)) break;
                     tc_fence_after();
-                    const uint32_t k_addr = smem_u32(smem + QSmem::k + s * kTile);
-                    const uint32_t v_addr = smem_u32(smem + QSmem::v + s * kTile);
+                    const uint32_t k_addr = smem_u32(smem + QSmem::k + sk * kTile);
+                    const uint32_t v_addr = smem_u32(smem + QSmem::v + sv * kTile);
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks) {
                         const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
@@ -521,6 +540,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     umma_commit(&bar[S2_FULL + s]);
                     // the previous tile's dP is in the elementwise threads' registers by now
                     if (j >= 1 && !wait_or_fail(&bar[DP_FREE], (j - 1) & 1, a, err)) break;
+                    if (!wait_or_fail(&bar[V2_FULL + sv], (j / QSmem::vstages) & 1, a, err)) break;
                     tc_fence_after();
 #pragma unroll
                     for (int ks = 0; ks < kD / 16; ++ks) {
@@ -528,19 +548,20 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         umma_ss(tdP, desc_kmajor(o_addr + off), desc_kmajor(v_addr + off), idesc_s, ks > 0 ? 1u : 0u);
                     }
                     umma_commit(&bar[DP_FULL]);
+                    umma_commit(&bar[V2_EMPTY + sv]);
                 }
                 if (j >= 1) {
-                    const int jp = j - 1, s = jp & 1;
+                    const int jp = j - 1, s = jp & 1, sk = jp % QSmem::kstages;
                     if (!wait_or_fail(&bar[DS_READY + s], (jp >> 1) & 1, a, err)) break;
                     tc_fence_after();
-                    const uint32_t k_addr = smem_u32(smem + QSmem::k + s * kTile);
+                    const uint32_t k_addr = smem_u32(smem + QSmem::k + sk * kTile);
                     // dQ += dS K: A = dS from tensor memory (16 keys = 8 packed columns), B = K rows (MN-major)
 #pragma unroll
                     for (int ks = 0; ks < kB / 16; ++ks)
                         umma_ts(tdQ, tS0 + s * 128 + ks * 8, desc_mnmajor(k_addr + ks * 2048), idesc_q,
                                 (jp > 0 || ks > 0) ? 1u : 0u);
                     umma_commit(&bar[S2_FREE + s]);
-                    umma_commit(&bar[K2_EMPTY + s]);
+                    umma_commit(&bar[K2_EMPTY + sk]);
                     done = j;
                 }
             }
