@@ -296,7 +296,8 @@ decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         }
         const size_t row = (size_t)b * a.Hq + h0 + hh;
         if (a.nsplit == 1) {
-            a.out[row * kD + j] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+            // a zero sum only for an empty history (output 0); a NaN sum (a NaN in the cache) stays NaN
+            a.out[row * kD + j] = __float2bfloat16_rn(Lsum != 0.f ? O / Lsum : 0.f);
         } else {
             const size_t prow = row * a.nsplit + split;
             a.part_o[prow * kD + j] = O;
@@ -356,7 +357,8 @@ __global__ void __launch_bounds__(kD) decode_combine_kernel(const DecodeArgs a)
             Lsum += ml[2 * (c + s) + 1] * wgt[s];
         }
     }
-    a.out[row * kD + j] = __float2bfloat16_rn(Lsum > 0.f ? O / Lsum : 0.f);
+    // a zero sum only for an empty history (output 0); a NaN sum (a NaN in the cache) stays NaN
+    a.out[row * kD + j] = __float2bfloat16_rn(Lsum != 0.f ? O / Lsum : 0.f);
 }
 
 // The deliberately expanded baseline: physically repeat each KV head for its g

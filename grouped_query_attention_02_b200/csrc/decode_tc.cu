@@ -830,7 +830,8 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     if (hg >= g) break;
                     const float L = ls[hg] + ls[N + hg] + ls[2 * N + hg] + ls[3 * N + hg];
                     const float O = __uint_as_float(o[h]);
-                    a.out[((size_t)pb * a.Hq + pkvh * g + hg) * kD + d] = __float2bfloat16_rn(L > 0.f ? O / L : 0.f);
+                    // a zero sum only for an empty history (output 0); a NaN sum (a NaN in the cache) stays NaN
+                    a.out[((size_t)pb * a.Hq + pkvh * g + hg) * kD + d] = __float2bfloat16_rn(L != 0.f ? O / L : 0.f);
                 }
             } else {
                 // one piece of several: a partial (o, m, l) for decode_combine_kernel

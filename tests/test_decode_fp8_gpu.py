@@ -137,6 +137,78 @@ def test_fp8_accepts_float8_tensors(oracle_mod):
     assert torch.equal(a, b)
 
 
+def _e4m3_values():
+    return torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).double()
+
+
+def test_fp8_every_value_code_reaches_the_output_exactly(oracle_mod):
+    """One cached token per sequence: the output is v_scale times the widened value codes, so every one
+    of the 256 codes (subnormals, both zeros and the two NaNs included) is checked to bf16 rounding."""
+    x = inputs.make_decode_fp8(2, 2, 1, 128, 1, device=DEV, seed=12, v_scale=0.37)
+    v = torch.arange(256, dtype=torch.int32).to(torch.uint8).reshape(2, 1, 1, 128)
+    x.v_cache.copy_(v.to(DEV))
+    out = _run(x).double().cpu().numpy()
+    ref = _ref(oracle_mod, x)
+    assert np.array_equal(np.isnan(out), np.isnan(ref)) and int(np.isnan(ref).sum()) == 2 * 2
+    fin = ~np.isnan(ref)
+    assert np.all(np.abs(out[fin] - ref[fin]) <= np.abs(ref[fin]) * 2.0 ** -8)
+
+
+def test_fp8_every_key_code_moves_the_weights_as_its_value(oracle_mod):
+    """Sequence b holds two tokens: key 0 is code b in coordinate 0 (zeros elsewhere), key 1 is zero; the
+    values are +1 and -1, so the output is v_scale * tanh(s / 2) with s the first token's score.  The
+    query is the power of two that puts |s| near 1 for that code, so each key code is checked through
+    the scores to a few bf16 steps."""
+    B = 256
+    x = inputs.make_decode_fp8(B, 1, 1, 128, 2, device=DEV, seed=13, k_scale=1.0 / 64, v_scale=1.0)
+    k = torch.zeros(B, 2, 1, 128, dtype=torch.uint8)
+    k[:, 0, 0, 0] = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    v = torch.empty(B, 2, 1, 128, dtype=torch.uint8)
+    v[:, 0] = 0x38   # +1.0
+    v[:, 1] = 0xB8   # -1.0
+    vals = _e4m3_values()
+    q = torch.zeros(B, 1, 128, dtype=torch.float64)
+    mag = (vals.abs() * x.k_scale * x.scale).clamp_min(1e-30)
+    q[:, 0, 0] = torch.where(torch.isfinite(vals) & (vals != 0), torch.exp2(-torch.round(torch.log2(mag))), 1.0)
+    x.k_cache.copy_(k.to(DEV))
+    x.v_cache.copy_(v.to(DEV))
+    x.q.copy_(q.to(torch.bfloat16).to(DEV))
+    out = _run(x).double().cpu().numpy()
+    ref = _ref(oracle_mod, x)
+    assert np.array_equal(np.isnan(out), np.isnan(ref)) and int(np.isnan(ref[:, 0, 0]).sum()) == 2
+    fin = ~np.isnan(ref)
+    assert np.all(out[fin][np.abs(ref[fin]) == 0] == 0)
+    assert np.all(np.abs(out[fin] - ref[fin]) <= np.abs(ref[fin]) * 2.0 ** -7 + 1e-30)
+
+
+@pytest.mark.parametrize("frac_subnormal", [1.0, 0.5])
+def test_fp8_subnormal_codes(oracle_mod, frac_subnormal):
+    """Caches of E4M3 subnormals (exponent field 0), alone or mixed with normal codes, with scales that
+    make them matter: the keys spread the scores over several units and the values set the output."""
+    x = inputs.make_decode_fp8(3, 8, 2, 128, 400, seqlens=[400, 257, 31], device=DEV, seed=14,
+                               k_scale=64.0, v_scale=64.0, q_gain=4.0)
+    g = torch.Generator().manual_seed(15)
+    for c in (x.k_cache, x.v_cache):
+        sub = torch.randint(0, 8, c.shape, generator=g, dtype=torch.int32) | (torch.randint(0, 2, c.shape, generator=g, dtype=torch.int32) << 7)
+        keep = torch.rand(c.shape, generator=g) >= frac_subnormal
+        c.copy_(torch.where(keep, c.cpu().to(torch.int32), sub).to(torch.uint8).to(DEV))
+    assert_close(_run(x).double().cpu().numpy(), _ref(oracle_mod, x))
+
+
+def test_fp8_nan_codes_inside_the_history_propagate(oracle_mod):
+    """A NaN key code turns its token's scores into NaN for every head of the group (all of their
+    outputs NaN); a NaN value code poisons that coordinate of the group's outputs only, as in the oracle."""
+    x = inputs.make_decode_fp8(2, 8, 2, 128, 300, seqlens=[300, 250], device=DEV, seed=16)
+    x.k_cache[0, 5, 1, 17] = 0x7F
+    x.v_cache[1, 200, 0, 3] = 0xFF
+    out = _run(x).double().cpu().numpy()
+    ref = _ref(oracle_mod, x)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(out), nan)
+    assert nan[0, 4:].all() and nan[1, :4, 3].all() and int(nan.sum()) == 4 * 128 + 4
+    assert_close(np.where(nan, 0.0, out), np.where(nan, 0.0, ref))
+
+
 def test_fp8_rejects_groups_above_32():
     x = inputs.make_decode_fp8(1, 64, 1, 128, 128, device=DEV, seed=12)
     with pytest.raises(gqa.GQAError) as e:

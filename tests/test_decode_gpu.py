@@ -110,6 +110,22 @@ def test_nan_poisoned_padding_is_never_read(oracle_mod):
     _check_all(oracle_mod, x, out)
 
 
+@pytest.mark.parametrize("Hq,Hkv,T", [(8, 2, 300), (8, 2, 20000), (8, 8, 300), (8, 8, 20000), (71, 1, 3000)])
+def test_nan_inside_the_history_reaches_the_output(oracle_mod, Hq, Hkv, T):
+    """A NaN key makes its token's scores NaN for the whole group (all of their outputs NaN); a NaN value
+    coordinate poisons that coordinate of the group's outputs, in one piece or across split pieces."""
+    x = inputs.make_decode(2, Hq, Hkv, 128, T, seqlens=[T, T - 7], device=DEV, seed=21)
+    g = Hq // Hkv
+    x.k_cache[0, T // 3, Hkv - 1, 17] = float("nan")
+    x.v_cache[1, T - 9, 0, 3] = float("nan")
+    out = _run(x).double().cpu().numpy()
+    ref = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens.cpu(), x.scale)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(out), nan)
+    assert nan[0, (Hkv - 1) * g:].all() and nan[1, :g, 3].all() and int(nan.sum()) == g * 128 + g
+    assert_close(np.where(nan, 0.0, out), np.where(nan, 0.0, ref))
+
+
 def test_peaky_softmax(oracle_mod):
     x = inputs.make_decode(4, 32, 8, 128, 2048, seqlens=[2048, 1500, 33, 700], device=DEV, seed=6, q_gain=8.0)
     _check_all(oracle_mod, x, _run(x))
