@@ -65,7 +65,10 @@ typedef enum gqa_status {
  * seqlens[b] are never used (they may hold anything, NaN included).
  * Preconditions not checked on the host (checking needs a device read):
  * 0 <= seqlens[b] <= Tmax; values outside are clamped to [0, Tmax].  A
- * sequence with seqlens[b] == 0 gets an all-zero output row.
+ * sequence with seqlens[b] == 0 gets an all-zero output row.  A NaN inside
+ * the history follows the definition: a NaN key makes the outputs of every
+ * head of its group NaN, a NaN value element makes that output coordinate
+ * NaN for the group's heads.
  *
  * Each K/V tile is fetched once by TMA and shared by the g query heads of its
  * group.  For 3 <= g <= 32 the products run on the tcgen05 tensor cores and
