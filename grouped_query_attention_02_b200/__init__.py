@@ -15,7 +15,8 @@ __all__ = [
     "GQAError", "gqa_decode", "gqa_decode_fp8", "gqa_decode_noalloc", "gqa_prefill_causal",
     "gqa_prefill_causal_fwd", "gqa_prefill_causal_bwd", "gqa_decode_expanded", "gqa_decode_expanded_bytes",
     "gqa_decode_plan", "gqa_get_last_device_status", "gqa_selftest_wait_timeout", "gqa_set_profile_events",
-    "gqa_last_launch_count", "gqa_release", "gqa_status_string", "gqa_version", "library_path", "load",
+    "gqa_last_launch_count", "gqa_release", "gqa_set_workspace_allocator", "gqa_status_string", "gqa_version",
+    "library_path", "load",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -24,6 +25,9 @@ _lib = None
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
+# gqa_alloc_fn / gqa_free_fn of include/gqa.h
+ALLOC_FN = ctypes.CFUNCTYPE(ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p)
+FREE_FN = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_void_p)
 
 EXPORTS = {
     # name: (restype, argtypes)
@@ -43,6 +47,7 @@ EXPORTS = {
     "gqa_set_profile_events": (_i, [_vp, _vp]),
     "gqa_last_launch_count": (_i, []),
     "gqa_release": (None, []),
+    "gqa_set_workspace_allocator": (_i, [_vp, _vp, _vp]),   # ALLOC_FN / FREE_FN pointers or NULL
     "gqa_status_string": (ctypes.c_char_p, [_i]),
     "gqa_version": (ctypes.c_char_p, []),
 }
@@ -343,6 +348,27 @@ def gqa_last_launch_count() -> int:
 
 def gqa_release():
     load().gqa_release()
+
+
+_allocator_refs = None   # the ctypes callbacks the library may call; kept alive while installed
+
+
+def gqa_set_workspace_allocator(alloc=None, free=None):
+    """Take the library's per-device workspace from the caller's pool: ``alloc(nbytes, device)`` returns a
+    256-byte aligned device address (0 when there is none), ``free(ptr, nbytes, device)`` takes it back.
+    Both None restores cudaMalloc / cudaFree.  Must be called with no library work in flight."""
+    global _allocator_refs
+    if (alloc is None) != (free is None):
+        raise ValueError("alloc and free are installed together")
+    if alloc is None:
+        _check(load().gqa_set_workspace_allocator(None, None, None), "gqa_set_workspace_allocator")
+        _allocator_refs = None   # dropped only now: the call handed the blocks back through them
+        return
+    ca = ALLOC_FN(lambda nbytes, dev, ctx: int(alloc(int(nbytes), int(dev)) or 0) or None)
+    cf = FREE_FN(lambda ptr, nbytes, dev, ctx: free(int(ptr or 0), int(nbytes), int(dev)))
+    _check(load().gqa_set_workspace_allocator(ctypes.cast(ca, _vp), ctypes.cast(cf, _vp), None),
+           "gqa_set_workspace_allocator")
+    _allocator_refs = (ca, cf)
 
 
 def gqa_status_string(status: int) -> str:

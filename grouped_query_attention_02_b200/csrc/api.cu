@@ -28,7 +28,15 @@ struct DeviceState {
     int *status = nullptr;
 };
 
+// Where workspaces come from: cudaMalloc / cudaFree, or the caller's pair (gqa_set_workspace_allocator).
+struct WorkspaceAllocator {
+    gqa_alloc_fn alloc = nullptr;
+    gqa_free_fn free_fn = nullptr;
+    void *ctx = nullptr;
+};
+
 std::mutex g_mu;
+WorkspaceAllocator g_alloc;
 std::unordered_map<int, DeviceState> g_devices;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 cudaEvent_t g_ev_before = nullptr, g_ev_after = nullptr;
@@ -55,18 +63,60 @@ gqa_status device_state(DeviceState **out)
     return GQA_OK;
 }
 
+// Hands a workspace block back to whoever allocated it; `dev` is current.  A caller's pool may reuse
+// the block at once, so the device is synchronised first (cudaFree does the same implicitly).
+void workspace_free(void *p, size_t bytes, int dev)
+{
+    if (!p) return;
+    if (g_alloc.free_fn) {
+        cudaDeviceSynchronize();
+        g_alloc.free_fn(p, bytes, dev, g_alloc.ctx);
+    } else {
+        cudaFree(p);
+    }
+}
+
+// Caller holds g_mu; the state's device is current.
 gqa_status ensure_workspace(DeviceState *st, size_t bytes)
 {
     if (bytes <= st->ws_bytes) return GQA_OK;
-    if (st->ws) cudaFree(st->ws);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ERR_CUDA;
+    workspace_free(st->ws, st->ws_bytes, dev);
     st->ws = nullptr;
     st->ws_bytes = 0;
-    if (cudaMalloc(&st->ws, bytes) != cudaSuccess) {
+    void *p = nullptr;
+    if (g_alloc.alloc) {
+        p = g_alloc.alloc(bytes, dev, g_alloc.ctx);
+    } else if (cudaMalloc(&p, bytes) != cudaSuccess) {
         cudaGetLastError();
-        return GQA_ERR_OUT_OF_MEMORY;
+        p = nullptr;
     }
+    if (!p) return GQA_ERR_OUT_OF_MEMORY;
+    if (reinterpret_cast<uintptr_t>(p) & 255u) {   // the partials and the piece list assume 256-byte alignment
+        workspace_free(p, bytes, dev);
+        return GQA_ERR_MISALIGNED;
+    }
+    st->ws = p;
     st->ws_bytes = bytes;
     return GQA_OK;
+}
+
+// Hands back every device's workspace (caller holds g_mu); the current device is restored.
+void release_workspaces()
+{
+    if (g_devices.empty()) return;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    for (auto &kv : g_devices) {
+        if (kv.second.ws) {
+            cudaSetDevice(kv.first);
+            workspace_free(kv.second.ws, kv.second.ws_bytes, kv.first);
+            kv.second.ws = nullptr;
+            kv.second.ws_bytes = 0;
+        }
+    }
+    cudaSetDevice(cur);
 }
 
 gqa_status get_encoder()
@@ -539,16 +589,19 @@ int gqa_last_launch_count(void) { return g_last_launches; }
 void gqa_release(void)
 {
     std::lock_guard<std::mutex> lk(g_mu);
-    int cur = 0;
-    cudaGetDevice(&cur);
-    for (auto &kv : g_devices) {
-        if (kv.second.ws) {
-            cudaSetDevice(kv.first);
-            cudaFree(kv.second.ws);
-        }
-    }
+    release_workspaces();
     g_devices.clear();
-    cudaSetDevice(cur);
+}
+
+gqa_status gqa_set_workspace_allocator(gqa_alloc_fn alloc, gqa_free_fn free_fn, void *ctx)
+{
+    if ((alloc == nullptr) != (free_fn == nullptr)) return GQA_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_mu);
+    release_workspaces();   // each block goes back to the allocator that made it
+    g_alloc.alloc = alloc;
+    g_alloc.free_fn = free_fn;
+    g_alloc.ctx = alloc ? ctx : nullptr;
+    return GQA_OK;
 }
 
 const char *gqa_status_string(gqa_status s)

@@ -24,7 +24,8 @@
  *    check returns its status and enqueues nothing.  A CUDA launch error is
  *    returned as GQA_ERR_CUDA.
  *  - The library keeps, per device, a grow-only workspace for the split-KV
- *    plan and partial results (allocated with cudaMalloc on first need);
+ *    plan and partial results (allocated on first need with cudaMalloc, or
+ *    by the caller's allocator: gqa_set_workspace_allocator);
  *    gqa_release() frees it.  TMA tensor maps are encoded on the host for
  *    every call (kernel parameters, nothing is cached).  Calls that share the
  *    workspace on one device must be ordered on one stream (or otherwise
@@ -250,8 +251,37 @@ gqa_status gqa_set_profile_events(void *before, void *after);
 /* Number of kernels the most recent call on this host thread enqueued. */
 int gqa_last_launch_count(void);
 
-/* Frees the workspace and tensor-map cache of every device the library used. */
+/* Frees (hands back to its allocator) the workspace of every device the
+ * library used.  Call it with no library work in flight. */
 void gqa_release(void);
+
+/*
+ * gqa_set_workspace_allocator -- where the per-device workspace comes from.
+ * By default it is cudaMalloc'd on first need and grown, never shrunk, as
+ * calls need more; an engine that already owns the GPU's memory can hand the
+ * library blocks from its own pool instead.
+ *
+ *   alloc(bytes, device, ctx)          a block of at least `bytes` bytes of
+ *                                      device memory on `device`, 256-byte
+ *                                      aligned, or NULL when there is none
+ *   free_fn(ptr, bytes, device, ctx)   takes back a block alloc returned
+ *                                      (`bytes` as requested)
+ *   ctx                                passed through to both
+ *
+ * Both NULL restores cudaMalloc / cudaFree; exactly one NULL is
+ * GQA_ERR_INVALID_ARG.  The call first hands every current workspace back to
+ * the allocator that made it, so, like gqa_release, it must run with no
+ * library work in flight.  When alloc returns NULL, the call that needed the
+ * workspace returns GQA_ERR_OUT_OF_MEMORY with nothing enqueued; a block that
+ * is not 256-byte aligned is handed back and that call returns
+ * GQA_ERR_MISALIGNED.  Before free_fn receives a block the library
+ * synchronises the block's device (as cudaFree does), so no enqueued kernel
+ * still reads it.  Both functions run with the library's lock held, with the
+ * block's device current, and must not call back into the library.
+ */
+typedef void *(*gqa_alloc_fn)(size_t bytes, int device, void *ctx);
+typedef void (*gqa_free_fn)(void *ptr, size_t bytes, int device, void *ctx);
+gqa_status gqa_set_workspace_allocator(gqa_alloc_fn alloc, gqa_free_fn free_fn, void *ctx);
 
 /* Text for a status code (static storage). */
 const char *gqa_status_string(gqa_status status);

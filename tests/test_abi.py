@@ -159,3 +159,14 @@ def test_prefill_fwd_and_bwd_argument_checks(lib):
     assert bwd(d=96) == UNSUPPORTED
     assert bwd(dq=U) == MISALIGNED
     assert gqa.gqa_last_launch_count() == 0
+
+
+def test_workspace_allocator_comes_in_pairs(lib):
+    keep = (gqa.ALLOC_FN(lambda n, dev, ctx: None), gqa.FREE_FN(lambda p, n, dev, ctx: None))
+    fn, fr = (ctypes.cast(f, ctypes.c_void_p) for f in keep)
+    assert lib.gqa_set_workspace_allocator(fn, None, None) == INVALID
+    assert lib.gqa_set_workspace_allocator(None, fr, None) == INVALID
+    assert lib.gqa_set_workspace_allocator(None, None, None) == OK
+    with pytest.raises(ValueError):
+        gqa.gqa_set_workspace_allocator(lambda n, dev: 0, None)
+
