@@ -18,6 +18,11 @@ per-tensor scale, clamped to the largest finite E4M3 value (448) and stored as
 E4M3 codes (torch's float8_e4m3fn cast, round to nearest even); rows past the
 history hold the NaN code 0x7F when ``poison=True``.
 
+MLA decode (``make_mla_decode``): q [B,Hq,d_c+d_r] (absorbed latent query, then
+RoPE query) from seed ``base+0`` and the cache [B,Tmax,d_c+d_r] (latent, then the
+shared RoPE key) from seed ``base+1``, both N(0, 1) bf16; the default scale is
+1/sqrt(d_h + d_r) with the original per-head width d_h = 128.
+
 Layouts are the ones of the C ABI: decode q [B,Hq,d], caches [B,Tmax,Hkv,d];
 prefill q [B,S,Hq,d], k/v [B,S,Hkv,d].
 """
@@ -180,3 +185,34 @@ def make_prefill(B: int, S: int, Hq: int, Hkv: int, d: int, *, device="cpu", see
 def make_dout(B: int, S: int, Hq: int, d: int, *, device="cpu", seed: int = 0) -> torch.Tensor:
     """Incoming gradient dO [B,S,Hq,d] of the causal prefill's output (seed ``seed+4``)."""
     return _normal((B, S, Hq, d), seed + 4, device)
+
+
+@dataclass
+class MlaDecodeInputs:
+    q: torch.Tensor          # [B,Hq,d_c+d_r] bf16: absorbed latent query, then RoPE query
+    kv_cache: torch.Tensor   # [B,Tmax,d_c+d_r] bf16: latent, then the RoPE key shared by all heads
+    seqlens: torch.Tensor    # [B] int32, same device as q
+    d_c: int
+    scale: float
+
+
+def make_mla_decode(B: int, Hq: int, Tmax: int, d_c: int = 512, d_r: int = 64, seqlens=None, *, device="cpu",
+                    seed: int = 0, scale: float | None = None, q_gain: float = 1.0, seqlen_range=None,
+                    d_h: int = 128) -> MlaDecodeInputs:
+    """MLA decode inputs; ``seqlens`` as in make_decode.  The default scale is 1/sqrt(d_h + d_r)."""
+    if seqlen_range is not None:
+        sl = seqlens_uniform(B, seqlen_range[0], seqlen_range[1], seed + 3)
+    elif seqlens is None:
+        sl = torch.full((B,), Tmax, dtype=torch.int32)
+    elif isinstance(seqlens, int):
+        sl = torch.full((B,), seqlens, dtype=torch.int32)
+    else:
+        sl = torch.as_tensor(seqlens, dtype=torch.int32).cpu()
+    dk = d_c + d_r
+    q = _normal((B, Hq, dk), seed + 0, device, q_gain)
+    mk = _normal_bf16 if B * Tmax * dk > (1 << 26) else _normal
+    kv = mk((B, Tmax, dk), seed + 1, device)
+    if scale is None:
+        scale = 1.0 / float(d_h + d_r) ** 0.5
+    return MlaDecodeInputs(q, kv, sl.to(device), d_c, scale)
+

@@ -15,7 +15,9 @@ through ctypes.  Pages it follows:
 * KV bytes: lihaoran.work/?p=2890 "KV-head count determines the raw cache
   ratio";
 * per-head attention and the causal mask: anrans.github.io attention-variants,
-  "Kernels do not need to copy the KV heads" (the expanded version).
+  "Kernels do not need to copy the KV heads" (the expanded version);
+* MLA decode with absorbed weights: anrans.github.io attention-variants,
+  "MLA: multi-head latent attention" (weight absorption, decoupled RoPE).
 
 Every function is pinned by ``tests/test_oracle_pins.py``.
 """
@@ -98,6 +100,9 @@ class Oracle:
         lib.gqa_oracle_decode_fp8.restype = ctypes.c_int
         lib.gqa_oracle_decode_fp8.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_double] * 2 + [ctypes.c_void_p] + [
             ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_void_p, ctypes.c_int]
+        lib.gqa_oracle_mla_decode.restype = ctypes.c_int
+        lib.gqa_oracle_mla_decode.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 5 + [
+            ctypes.c_double, ctypes.c_void_p, ctypes.c_int]
         lib.gqa_oracle_prefill.restype = ctypes.c_int
         lib.gqa_oracle_prefill.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 5 + [
             ctypes.c_double, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p, ctypes.c_int]
@@ -183,6 +188,23 @@ class Oracle:
             raise ValueError(f"oracle decode rejected its arguments (status {st})")
         return out
 
+    def mla_decode(self, q, kv, seqlens, d_c: int, scale: float, nthreads: int | None = None) -> np.ndarray:
+        """MLA decode with absorbed weights: q [B,Hq,d_c+d_r], kv [B,Tmax,d_c+d_r] (bf16; latent then RoPE
+        part), seqlens [B] -> out [B,Hq,d_c] fp64, the softmax-weighted sum of the rows' latent parts."""
+        qb, kb = _bits(q), _bits(kv)
+        B, Hq, dk = qb.shape
+        B2, Tmax, dk2 = kb.shape
+        assert B2 == B and dk2 == dk and 0 < d_c <= dk
+        sl = np.ascontiguousarray(np.asarray(
+            seqlens.cpu().numpy() if hasattr(seqlens, "cpu") else seqlens, dtype=np.int32))
+        assert sl.shape == (B,)
+        out = np.zeros((B, Hq, d_c), dtype=np.float64)
+        st = self.lib.gqa_oracle_mla_decode(qb.ctypes.data, kb.ctypes.data, sl.ctypes.data, B, Hq, d_c, dk - d_c,
+                                            Tmax, float(scale), out.ctypes.data, nthreads or default_threads())
+        if st != 0:
+            raise ValueError(f"oracle MLA decode rejected its arguments (status {st})")
+        return out
+
     def prefill_causal(self, q, k, v, scale: float, rows=None, nthreads: int | None = None) -> np.ndarray:
         """q [B,S,Hq,d], k/v [B,S,Hkv,d] (bf16).
 
@@ -243,6 +265,10 @@ def prefill_backward(q, k, v, dout, scale, row_sel=None, key_sel=None, nthreads=
 
 def decode_fp8(q, k8, v8, k_scale, v_scale, seqlens, scale, nthreads=None):
     return _get().decode_fp8(q, k8, v8, k_scale, v_scale, seqlens, scale, nthreads)
+
+
+def mla_decode(q, kv, seqlens, d_c, scale, nthreads=None):
+    return _get().mla_decode(q, kv, seqlens, d_c, scale, nthreads)
 
 
 def prefill_causal(q, k, v, scale, rows=None, nthreads=None):

@@ -35,6 +35,15 @@
  *    shrink the KV cache", anrans.github.io attention-variants: K and V in
  *    FP8, as serving engines support); every element is the E4M3 value of its
  *    byte times a per-tensor scale, and the attention is the same as above.
+ *  - MLA decode with absorbed weights ("MLA: multi-head latent attention",
+ *    anrans.github.io attention-variants, the weight-absorption and
+ *    decoupled-RoPE paragraphs): the cache holds one row per token, the
+ *    d_c-dim latent c followed by the d_r-dim RoPE key shared by all heads;
+ *    every query head (its absorbed latent query, then its RoPE query) scores
+ *    the whole row, and its output is the softmax-weighted sum of the latent
+ *    part alone -- an MQA whose value is the key's first d_c entries.  The
+ *    up-projection W_UV applied afterwards belongs to the output projection
+ *    and is not part of it.
  *
  * Everything is done in double precision.  Inputs are the bf16 bit patterns
  * the GPU sees; bf16 is the upper 16 bits of an IEEE-754 binary32, so the
@@ -535,3 +544,93 @@ int gqa_oracle_prefill_backward(const uint16_t *q, const uint16_t *k, const uint
     free(jobs); free(th);
     return st;
 }
+
+/* ---- MLA decode (absorbed weights) ---------------------------------------- */
+
+typedef struct {
+    const uint16_t *q, *kv;
+    const int32_t *seqlens;
+    int B, Hq, dc, dr, Tmax;
+    double scale;
+    double *out;
+    int tid, nthreads;
+    int status;
+} mla_job;
+
+static void *mla_worker(void *arg)
+{
+    mla_job *J = (mla_job *)arg;
+    const int dk = J->dc + J->dr, dv = J->dc;
+    double *qrow = (double *)malloc(sizeof(double) * (size_t)dk);
+    double *Kh = (double *)malloc(sizeof(double) * (size_t)(J->Tmax > 0 ? J->Tmax : 1) * (size_t)dk);
+    double *Vh = (double *)malloc(sizeof(double) * (size_t)(J->Tmax > 0 ? J->Tmax : 1) * (size_t)dv);
+    double *w = (double *)malloc(sizeof(double) * (size_t)(J->Tmax > 0 ? J->Tmax : 1));
+    if (!qrow || !Kh || !Vh || !w) {
+        J->status = ORACLE_NO_MEMORY;
+        free(qrow); free(Kh); free(Vh); free(w);
+        return NULL;
+    }
+    long long pairs = (long long)J->B * J->Hq;
+    for (long long p = J->tid; p < pairs; p += J->nthreads) {
+        int b = (int)(p / J->Hq), h = (int)(p % J->Hq);
+        long long T = J->seqlens[b];
+        /* this head's own copies: the key is the whole cached row, the value its latent part */
+        for (long long t = 0; t < T; ++t) {
+            const uint16_t *row = J->kv + ((size_t)b * J->Tmax + (size_t)t) * (size_t)dk;
+            for (int i = 0; i < dk; ++i) Kh[t * dk + i] = bf16_to_double(row[i]);
+            for (int j = 0; j < dv; ++j) Vh[t * dv + j] = bf16_to_double(row[j]);
+        }
+        const uint16_t *qs = J->q + ((size_t)b * J->Hq + (size_t)h) * (size_t)dk;
+        for (int i = 0; i < dk; ++i) qrow[i] = bf16_to_double(qs[i]);
+        double *o = J->out + ((size_t)b * J->Hq + (size_t)h) * (size_t)dv;
+        for (int j = 0; j < dv; ++j) o[j] = 0.0;
+        if (T <= 0) continue;
+        /* scores over latent and RoPE parts together, then the two-pass softmax */
+        double m = -INFINITY;
+        for (long long t = 0; t < T; ++t) {
+            double s = 0.0;
+            for (int i = 0; i < dk; ++i) s += qrow[i] * Kh[t * dk + i];
+            w[t] = s * J->scale;
+            if (w[t] > m) m = w[t];
+        }
+        double denom = 0.0;
+        for (long long t = 0; t < T; ++t) {
+            w[t] = exp(w[t] - m);
+            denom += w[t];
+        }
+        for (long long t = 0; t < T; ++t)
+            for (int j = 0; j < dv; ++j) o[j] += w[t] * Vh[t * dv + j];
+        for (int j = 0; j < dv; ++j) o[j] /= denom;
+    }
+    free(qrow); free(Kh); free(Vh); free(w);
+    return NULL;
+}
+
+/* q [B,Hq,dc+dr] (absorbed latent query, then RoPE query), kv [B,Tmax,dc+dr] (latent, then the
+ * shared RoPE key) bf16 bits, seqlens [B] (0 <= seqlens <= Tmax), out [B,Hq,dc] fp64:
+ * out[b,h] = sum_{t < seqlens[b]} softmax_t(scale * q[b,h] . kv[b,t]) kv[b,t,0:dc].  Returns 0 on success. */
+int gqa_oracle_mla_decode(const uint16_t *q, const uint16_t *kv, const int32_t *seqlens, int B, int Hq, int dc,
+                          int dr, int Tmax, double scale, double *out, int nthreads)
+{
+    if (!q || !kv || !seqlens || !out) return ORACLE_BAD_ARG;
+    if (B <= 0 || Hq <= 0 || dc <= 0 || dr < 0 || Tmax < 0) return ORACLE_BAD_ARG;
+    for (int b = 0; b < B; ++b)
+        if (seqlens[b] < 0 || seqlens[b] > Tmax) return ORACLE_BAD_ARG;
+    if (nthreads < 1) nthreads = 1;
+    if ((long long)nthreads > (long long)B * Hq) nthreads = B * Hq;
+    mla_job *jobs = (mla_job *)calloc((size_t)nthreads, sizeof(mla_job));
+    pthread_t *th = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) { free(jobs); free(th); return ORACLE_NO_MEMORY; }
+    for (int i = 0; i < nthreads; ++i) {
+        mla_job J = {q, kv, seqlens, B, Hq, dc, dr, Tmax, scale, out, i, nthreads, ORACLE_OK};
+        jobs[i] = J;
+    }
+    for (int i = 1; i < nthreads; ++i) pthread_create(&th[i], NULL, mla_worker, &jobs[i]);
+    mla_worker(&jobs[0]);
+    for (int i = 1; i < nthreads; ++i) pthread_join(th[i], NULL);
+    int st = ORACLE_OK;
+    for (int i = 0; i < nthreads; ++i) if (jobs[i].status != ORACLE_OK) st = jobs[i].status;
+    free(jobs); free(th);
+    return st;
+}
+

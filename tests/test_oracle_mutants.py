@@ -50,6 +50,17 @@ MUTANTS = {
     "backward keys skip their own row": ("for (int r = t; r < S; ++r) {", "for (int r = t + 1; r < S; ++r) {"),
     "backward group gradient from one head": ("if (J->key_sel && !J->key_sel[t]) continue;",
                                               "if ((J->key_sel && !J->key_sel[t]) || hh > 0) continue;"),
+    "MLA value read from the RoPE end of the row": ("for (int j = 0; j < dv; ++j) Vh[t * dv + j] = bf16_to_double(row[j]);",
+                                                   "for (int j = 0; j < dv; ++j) Vh[t * dv + j] = bf16_to_double(row[j + J->dr]);"),
+    "MLA scores drop the RoPE part": ("for (int i = 0; i < dk; ++i) s += qrow[i] * Kh[t * dk + i];",
+                                      "for (int i = 0; i < dv; ++i) s += qrow[i] * Kh[t * dk + i];"),
+    "MLA scale left out": ("w[t] = s * J->scale;", "w[t] = s;"),
+    "MLA every head reads head 0's query": (
+        "const uint16_t *qs = J->q + ((size_t)b * J->Hq + (size_t)h) * (size_t)dk;",
+        "const uint16_t *qs = J->q + ((size_t)b * J->Hq) * (size_t)dk;"),
+    "MLA cache rows strided by the value width": (
+        "const uint16_t *row = J->kv + ((size_t)b * J->Tmax + (size_t)t) * (size_t)dk;",
+        "const uint16_t *row = J->kv + ((size_t)b * J->Tmax + (size_t)t) * (size_t)dv;"),
     "fp8 values scaled by the key scale": ("Vh[t * d + j] = e4m3_to_double(J->v8[src + j]) * J->v_scale;",
                                            "Vh[t * d + j] = e4m3_to_double(J->v8[src + j]) * J->k_scale;"),
 }

@@ -483,3 +483,98 @@ def test_backward_selected_rows_and_keys_match_the_full_gradient(oracle_mod):
     np.testing.assert_array_equal(part[0][:, rows], full[0][:, rows])
     np.testing.assert_array_equal(part[1][:, keys], full[1][:, keys])
     np.testing.assert_array_equal(part[2][:, keys], full[2][:, keys])
+
+
+# ---------------------------------------------------------------- MLA decode (absorbed weights)
+
+
+def test_mla_absorbed_decode_equals_explicit_heads(oracle_mod):
+    """The weight-absorption identity of the MLA page, with its decoupled RoPE part: per head, attention
+    with the key and value rebuilt from the latent (k = c W_uk, v = c W_uv, the RoPE parts appended to
+    query and key) equals the oracle's latent-space decode followed by W_uv.  The up-projection W_uk and
+    the per-head queries are small integers, so the absorbed query W_uk q is exact in bf16 and both sides
+    see the same numbers."""
+    g = torch.Generator().manual_seed(31)
+    T, d_c, d_r, n_h, d_h = 7, 16, 4, 4, 8
+    bf = lambda x: x.to(torch.bfloat16).double()
+    c = bf(torch.randn(T, d_c, generator=g, dtype=torch.float64))            # cached latents
+    k_r = bf(torch.randn(T, d_r, generator=g, dtype=torch.float64))          # shared RoPE key
+    W_uk = torch.randint(-1, 2, (n_h, d_c, d_h), generator=g).double()
+    W_uv = torch.randn(n_h, d_c, d_h, generator=g, dtype=torch.float64) / 4
+    q = torch.randint(-3, 4, (n_h, d_h), generator=g).double()               # the step's query per head
+    q_r = bf(torch.randn(n_h, d_r, generator=g, dtype=torch.float64))
+    scale = 1.0 / math.sqrt(d_h + d_r)
+    # explicit: each head's own key and value rows
+    naive = torch.empty(n_h, d_h, dtype=torch.float64)
+    for i in range(n_h):
+        k_i = torch.cat([c @ W_uk[i], k_r], dim=1)
+        v_i = c @ W_uv[i]
+        p = torch.softmax(k_i @ torch.cat([q[i], q_r[i]]) * scale, dim=0)
+        naive[i] = p @ v_i
+    # absorbed: the latent-space query per head, attention over the cached rows, then W_uv
+    q_lat = torch.einsum("hcd,hd->hc", W_uk, q)
+    assert torch.equal(bf(q_lat), q_lat)
+    qq = torch.cat([q_lat, q_r], dim=1)[None].to(torch.bfloat16)
+    kv = torch.cat([c, k_r], dim=1)[None].to(torch.bfloat16)
+    lat = torch.from_numpy(oracle_mod.mla_decode(qq, kv, [T], d_c, scale))[0]
+    absorbed = torch.einsum("hc,hcd->hd", lat, W_uv)
+    assert torch.allclose(absorbed, naive, rtol=0, atol=1e-12)
+
+
+def test_mla_decode_equals_library_sdpa(oracle_mod):
+    """Every head against the shared rows: key = the whole row, value = its latent part (torch SDPA, fp64)."""
+    x = inputs.make_mla_decode(3, 16, 40, d_c=32, d_r=8, seqlens=[40, 17, 1], seed=32, q_gain=2.0)
+    out = oracle_mod.mla_decode(x.q, x.kv_cache, x.seqlens, x.d_c, x.scale)
+    for b, T in enumerate(x.seqlens.tolist()):
+        Q = x.q[b].double()[None, :, None, :]
+        K = x.kv_cache[b, :T].double()[None, None].expand(1, 16, T, 40)
+        V = x.kv_cache[b, :T, :32].double()[None, None].expand(1, 16, T, 32)
+        ref = torch.nn.functional.scaled_dot_product_attention(Q, K, V, scale=x.scale)[0, :, 0]
+        assert np.allclose(out[b], ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_mla_decode_is_mqa_with_the_latent_as_value(oracle_mod):
+    """The same numbers through the (separately pinned) decode oracle: one KV head whose key is the whole
+    row and whose value is the row with its RoPE part zeroed; the latent part of that output is the MLA
+    output and the rest is zero."""
+    x = inputs.make_mla_decode(2, 8, 30, d_c=24, d_r=8, seqlens=[30, 11], seed=33)
+    out = oracle_mod.mla_decode(x.q, x.kv_cache, x.seqlens, x.d_c, x.scale)
+    k = x.kv_cache[:, :, None, :]
+    v = k.clone()
+    v[..., 24:] = 0
+    mqa = oracle_mod.decode(x.q, k, v, x.seqlens, x.scale)
+    assert np.allclose(mqa[..., :24], out, rtol=0, atol=1e-13)
+    assert np.all(mqa[..., 24:] == 0)
+
+
+def test_mla_decode_closed_forms(oracle_mod):
+    """One cached token returns its latent part; an empty history gives zeros; a zero query averages the
+    latents; the RoPE part of the key moves the weights (two rows alike in the latent, apart in RoPE)."""
+    x = inputs.make_mla_decode(3, 4, 5, d_c=8, d_r=4, seqlens=[1, 0, 5], seed=34)
+    out = oracle_mod.mla_decode(x.q, x.kv_cache, x.seqlens, x.d_c, x.scale)
+    assert np.array_equal(out[0], np.broadcast_to(x.kv_cache[0, 0, :8].double().numpy(), (4, 8)))
+    assert np.all(out[1] == 0)
+    q0 = torch.zeros_like(x.q)
+    z = oracle_mod.mla_decode(q0, x.kv_cache, x.seqlens, x.d_c, x.scale)
+    assert np.allclose(z[2], x.kv_cache[2, :5, :8].double().mean(0).numpy(), rtol=0, atol=1e-14)
+    kv = torch.zeros(1, 2, 12, dtype=torch.bfloat16)
+    kv[0, 0, :8] = 1.0
+    kv[0, 1, :8] = -1.0
+    kv[0, 1, 8] = 4.0                      # only the second row's RoPE key matches the query
+    qq = torch.zeros(1, 1, 12, dtype=torch.bfloat16)
+    qq[0, 0, 8] = 1.0
+    o = oracle_mod.mla_decode(qq, kv, [2], 8, 1.0)
+    w1 = math.exp(4.0) / (1.0 + math.exp(4.0))
+    assert np.allclose(o[0, 0], (1 - w1) * 1.0 + w1 * -1.0, rtol=0, atol=1e-14)
+
+
+def test_mla_cache_bytes_per_token(oracle_mod):
+    """The MLA page's cache sizes: 512 + 64 numbers per token and layer against 2 x 128 heads x 128 for
+    MHA (about 1/57), and DeepSeek-V3's 61 layers of 576 bf16 numbers per token."""
+    mla, mha = 512 + 64, 2 * 128 * 128
+    assert mha == 32768 and round(mha / mla) == 57
+    assert 61 * (512 + 64) * 2 == 70272
+    # with one "KV head" of width 576 and K = V shared, the MLA cache is half the bytes the GQA byte
+    # model would count for a separate K and V of that width
+    assert oracle_mod.kv_bytes(61, 1, 1, 576, 2) == 2 * 70272
+
