@@ -14,7 +14,7 @@ import os
 __all__ = [
     "GQAError", "gqa_decode", "gqa_decode_fp8", "gqa_decode_noalloc", "gqa_prefill_causal",
     "gqa_prefill_causal_fwd", "gqa_prefill_causal_bwd", "gqa_decode_expanded", "gqa_decode_expanded_bytes",
-    "gqa_decode_plan", "gqa_get_last_device_status", "gqa_selftest_wait_timeout", "gqa_set_profile_events",
+    "gqa_decode_plan", "gqa_tp_shard", "gqa_get_last_device_status", "gqa_selftest_wait_timeout", "gqa_set_profile_events",
     "gqa_last_launch_count", "gqa_release", "gqa_set_workspace_allocator", "gqa_status_string", "gqa_version",
     "library_path", "load",
 ]
@@ -42,6 +42,7 @@ EXPORTS = {
     "gqa_decode_expanded_bytes": (ctypes.c_size_t, [_i, _i, _i, _i]),
     "gqa_decode_plan": (_i, [_i, _i, _i, _i, _i, _i, ctypes.POINTER(_i), ctypes.POINTER(_i),
                              ctypes.POINTER(ctypes.c_size_t)]),
+    "gqa_tp_shard": (_i, [_i, _i, _i, _i] + [ctypes.POINTER(_i)] * 4),
     "gqa_get_last_device_status": (_i, [_vp]),
     "gqa_selftest_wait_timeout": (_i, [_i, _vp]),
     "gqa_set_profile_events": (_i, [_vp, _vp]),
@@ -322,6 +323,15 @@ def gqa_decode_plan(B, Hq, Hkv, d, Tmax, num_sms):
     _check(load().gqa_decode_plan(B, Hq, Hkv, d, Tmax, num_sms, ctypes.byref(c), ctypes.byref(n), ctypes.byref(w)),
            "gqa_decode_plan")
     return c.value, n.value, w.value
+
+
+def gqa_tp_shard(Hq, Hkv, tp, rank):
+    """(q_first, q_count, kv_first, kv_count): the query heads and KV heads (partitioned, or one replica when
+    Hkv < tp) that rank `rank` of `tp` tensor-parallel ranks owns."""
+    a, b, c, d = _i(), _i(), _i(), _i()
+    _check(load().gqa_tp_shard(int(Hq), int(Hkv), int(tp), int(rank), ctypes.byref(a), ctypes.byref(b),
+                               ctypes.byref(c), ctypes.byref(d)), "gqa_tp_shard")
+    return a.value, b.value, c.value, d.value
 
 
 def gqa_get_last_device_status(stream=None) -> int:

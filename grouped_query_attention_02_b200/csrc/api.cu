@@ -420,6 +420,33 @@ gqa_status gqa_decode_expanded(const void *q, const void *k_cache, const void *v
     return run_decode(q, k_rep, v_rep, seqlens, B, Hq, Hq, Tmax, scale, out, st, &g_last_launches);
 }
 
+gqa_status gqa_tp_shard(int Hq, int Hkv, int tp, int rank, int *q_first, int *q_count, int *kv_first,
+                        int *kv_count)
+{
+    if (!q_first || !q_count || !kv_first || !kv_count) return GQA_ERR_INVALID_ARG;
+    if (Hq <= 0 || Hkv <= 0 || tp <= 0 || rank < 0 || rank >= tp || Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
+    // ranks own consecutive, equal runs of query heads
+    if (Hq % tp != 0) return GQA_ERR_UNSUPPORTED;
+    const int g = Hq / Hkv, nq = Hq / tp;
+    int kf = 0, kc = 0;
+    if (Hkv >= tp) {
+        // partition: each rank owns Hkv / tp whole KV heads, and with them exactly its query heads' groups
+        if (Hkv % tp != 0) return GQA_ERR_UNSUPPORTED;
+        kc = Hkv / tp;
+        kf = rank * kc;
+    } else {
+        // replication: the rank's query heads lie in one group; it keeps a copy of that group's KV head
+        if (tp % Hkv != 0) return GQA_ERR_UNSUPPORTED;
+        kc = 1;
+        kf = (rank * nq) / g;
+    }
+    *q_first = rank * nq;
+    *q_count = nq;
+    *kv_first = kf;
+    *kv_count = kc;
+    return GQA_OK;
+}
+
 gqa_status gqa_decode_plan(int B, int Hq, int Hkv, int d, int Tmax, int num_sms, int *chunk, int *nsplit,
                            size_t *workspace_bytes)
 {

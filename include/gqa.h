@@ -219,6 +219,29 @@ gqa_status gqa_decode_plan(int B, int Hq, int Hkv, int d, int Tmax, int num_sms,
                            size_t *workspace_bytes);
 
 /*
+ * gqa_tp_shard -- the heads rank `rank` of `tp` tensor-parallel ranks owns
+ * for one attention layer (kv-head-replication glossary entry,
+ * inferencex.semianalysis.com; the tensor-parallelism paragraphs of
+ * deepconcepts.dev Grouped-Query Attention).  Ranks own consecutive, equal
+ * runs of query heads: [*q_first, *q_first + *q_count), Hq / tp each.
+ *  - Hkv >= tp (Hkv a multiple of tp): the KV heads are partitioned, Hkv / tp
+ *    per rank, [*kv_first, *kv_first + *kv_count), exactly the groups of the
+ *    rank's query heads.
+ *  - Hkv < tp (tp a multiple of Hkv): a rank's query heads lie in one group;
+ *    the rank keeps its own replica of that group's KV head (*kv_count = 1),
+ *    tp / Hkv ranks holding the same one.
+ * The rank then runs gqa_decode (or gqa_decode_fp8) on its shard: q
+ * [B, *q_count, d] and caches [B, Tmax, *kv_count, d], whose local group size
+ * is *q_count / *kv_count.  No exchange is needed inside attention; the
+ * output projection that follows is row-parallel over the same heads.
+ * GQA_ERR_INVALID_ARG for null pointers, non-positive sizes, rank outside
+ * [0, tp) or Hq % Hkv != 0; GQA_ERR_UNSUPPORTED when Hq % tp != 0 or neither
+ * of Hkv, tp divides the other.  Pure host arithmetic; touches no device.
+ */
+gqa_status gqa_tp_shard(int Hq, int Hkv, int tp, int rank, int *q_first, int *q_count, int *kv_first,
+                        int *kv_count);
+
+/*
  * gqa_get_last_device_status -- synchronises `stream`, then reads and clears
  * the device's status word.  Kernels never trap: a kernel that gives up a
  * bounded wait (about a second) records GQA_ERR_DEVICE_TIMEOUT there and

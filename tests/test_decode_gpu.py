@@ -126,6 +126,24 @@ def test_nan_inside_the_history_reaches_the_output(oracle_mod, Hq, Hkv, T):
     assert_close(np.where(nan, 0.0, out), np.where(nan, 0.0, ref))
 
 
+@pytest.mark.parametrize("Hq,Hkv,tp", [(32, 8, 2), (32, 8, 8), (32, 2, 8), (8, 2, 4), (8, 1, 8)])
+def test_tensor_parallel_shards_decoded_in_turn(oracle_mod, Hq, Hkv, tp):
+    """Each tensor-parallel rank's shard (gqa_tp_shard: its query heads with its KV heads, or its replica
+    of one) decoded in turn on this GPU -- the shards are independent, no rank waits on another -- and put
+    back in head order: the unsharded decode of the oracle."""
+    x = inputs.make_decode(3, Hq, Hkv, 128, 1500, seqlens=[1500, 700, 129], device=DEV, seed=51)
+    whole = torch.empty_like(x.q)
+    for r in range(tp):
+        qf, qc, kf, kc = gqa.gqa_tp_shard(Hq, Hkv, tp, r)
+        whole[:, qf:qf + qc] = gqa.gqa_decode(x.q[:, qf:qf + qc].contiguous(),
+                                              x.k_cache[:, :, kf:kf + kc].contiguous(),
+                                              x.v_cache[:, :, kf:kf + kc].contiguous(), x.seqlens, x.scale)
+    torch.cuda.synchronize()
+    assert gqa.gqa_get_last_device_status() == 0
+    assert_close(whole.double().cpu().numpy(),
+                 oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens.cpu(), x.scale))
+
+
 def test_peaky_softmax(oracle_mod):
     x = inputs.make_decode(4, 32, 8, 128, 2048, seqlens=[2048, 1500, 33, 700], device=DEV, seed=6, q_gain=8.0)
     _check_all(oracle_mod, x, _run(x))

@@ -6,7 +6,11 @@ decodes its own sequences.  Checked here without a GPU:
 * concatenating the ranks' (oracle) outputs equals decoding the concatenated
   batch in one place: sharding by sequence needs no collective on the data path;
 * the step time reported is the maximum over ranks and the value is all ranks'
-  bytes over that time (bench.aggregate).
+  bytes over that time (bench.aggregate);
+* tensor-parallel head sharding (gqa_tp_shard): each rank decodes its own query
+  heads against its KV heads, or its replica of one, and the ranks' outputs put
+  back in head order equal the unsharded decode -- with KV heads partitioned
+  (2 ranks) and replicated (4 ranks).
 """
 from __future__ import annotations
 
@@ -92,3 +96,49 @@ def test_aggregate_uses_the_slowest_rank():
     assert bench.unique_kv_bytes([8192] * 49, 8, 128) == 1644167168      # the Qwen3-8B-shaped cache
     assert bench.prefill_causal_flops(4, 8192, 32, 128) == 2199291691008     # 2.199 TFLOP causal
     assert bench.decode_flops([8192], 32, 128) == 4 * 36 * 32 * 128 * 8192 // 36   # one layer of the 4.83 GFLOP figure
+
+
+def _tp_worker(rank, world, port, out_dir, Hq, Hkv):
+    import sys
+
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        import grouped_query_attention_02_b200 as gqa
+        from grouped_query_attention_02_b200 import inputs
+
+        # every rank sees the same layer; it keeps only its shard (the CPU oracle stands in for the
+        # rank's GPU decode of that shard)
+        x = inputs.make_decode(2, Hq, Hkv, 16, 20, seqlens=[20, 7], device="cpu", seed=41)
+        qf, qc, kf, kc = gqa.gqa_tp_shard(Hq, Hkv, world, rank)
+        q = x.q[:, qf:qf + qc].contiguous()
+        k = x.k_cache[:, :, kf:kf + kc].contiguous()
+        v = x.v_cache[:, :, kf:kf + kc].contiguous()
+        out = torch.from_numpy(oracle.decode(q, k, v, x.seqlens, x.scale, nthreads=1))
+        parts = [torch.zeros_like(out) for _ in range(world)]
+        dist.all_gather(parts, out)
+        if rank == 0:
+            whole = torch.zeros(2, Hq, 16, dtype=torch.float64)
+            for r in range(world):
+                f, c, _, _ = gqa.gqa_tp_shard(Hq, Hkv, world, r)
+                whole[:, f:f + c] = parts[r]
+            np.save(os.path.join(out_dir, "tp.npy"), whole.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,Hq,Hkv", [(2, 8, 2), (4, 8, 2), (4, 8, 1)])
+def test_tensor_parallel_shards_reassemble_the_decode(tmp_path, world, Hq, Hkv):
+    import oracle
+    from grouped_query_attention_02_b200 import build, inputs
+
+    oracle.build()
+    build.build()
+    port = _free_port()
+    mp.start_processes(_tp_worker, args=(world, port, str(tmp_path), Hq, Hkv), nprocs=world, start_method="spawn")
+    got = np.load(tmp_path / "tp.npy")
+    x = inputs.make_decode(2, Hq, Hkv, 16, 20, seqlens=[20, 7], device="cpu", seed=41)
+    np.testing.assert_array_equal(got, oracle.decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, nthreads=1))
+
