@@ -252,6 +252,37 @@ def time_backward(gqa, torch, inputs, p, steps: int, warmup: int):
     return s0.elapsed_time(s1) / steps, launches
 
 
+def mla_decode_flops(B: int, Hq: int, T: int, d_c: int, d_r: int) -> int:
+    """2 * Hq * ((d_c + d_r) + d_c) per cached token: every head's score over the whole row and its
+    weighted sum of the latent part."""
+    return 2 * Hq * (2 * d_c + d_r) * B * T
+
+
+def time_mla(gqa, torch, x, steps: int, warmup: int):
+    """Mean step time and mean decode-kernel time (ms) of gqa_mla_decode."""
+    B, Hq, _ = x.q.shape
+    out = torch.empty((B, Hq, x.d_c), dtype=torch.bfloat16, device=x.q.device)
+    call = lambda: gqa.gqa_mla_decode(x.q, x.kv_cache, x.seqlens, x.scale, out=out, d_c=x.d_c)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    s0, s1 = _events(torch)
+    launches = 0
+    s0.record()
+    for _ in range(steps):
+        call()
+        launches += gqa.gqa_last_launch_count()
+    s1.record()
+    torch.cuda.synchronize()
+    kev = [_events(torch) for _ in range(steps)]
+    for i in range(steps):
+        gqa.gqa_set_profile_events(*kev[i])
+        call()
+    gqa.gqa_set_profile_events(None, None)
+    torch.cuda.synchronize()
+    return s0.elapsed_time(s1) / steps, sum(a.elapsed_time(b) for a, b in kev) / steps, launches
+
+
 def decode_call(gqa, x, out, q=None, k=None, v=None, sl=None):
     """One decode step through the public API: the FP8 entry point when x carries per-tensor scales."""
     q = x.q if q is None else q
@@ -614,6 +645,26 @@ def main():
             torch.cuda.empty_cache()
         except gqa.GQAError as e:
             rows["backward, " + pw.name] = {"error": str(e)}
+        # MLA decode with absorbed weights (CUDA-core kernel, the row's first correct path)
+        mw = workloads.MLA_DECODE
+        try:
+            xm = inputs.make_mla_decode(mw.B, mw.Hq, mw.Tmax, mw.d_c, mw.d_r, device="cuda", seed=0)
+            st_ms, k_ms, n = time_mla(gqa, torch, xm, 5, 3)
+            fl = mla_decode_flops(mw.B, mw.Hq, mw.Tmax, mw.d_c, mw.d_r)
+            by = mw.B * mw.Tmax * (mw.d_c + mw.d_r) * 2
+            rows[mw.name] = {
+                "ms_per_step": st_ms, "kernel_ms": k_ms, "TFLOPs": fl / (st_ms * 1e-3) / 1e12,
+                "unique_kv_GBps": by / (st_ms * 1e-3) / 1e9, "tokens_per_s": mw.B / (st_ms * 1e-3),
+                "roofline": {"bound": "tensor", "achieved": fl / (k_ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
+                             "unit": "TFLOP/s", "frac": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                             "traffic": None, "hbm_frac": by / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                             "peak_source": f"{peaks.get('source')} bf16_tflops (cuBLAS burst)"},
+                "flop_count": "2 Hq (2 d_c + d_r) per cached token", "kernel": "CUDA cores (first path)",
+                "launches_per_step": n / 5}
+            del xm
+            torch.cuda.empty_cache()
+        except (gqa.GQAError, RuntimeError) as e:   # a row that fails must not cost the line
+            rows[mw.name] = {"error": f"{type(e).__name__}: {e}"}
         line["rows"] = rows
 
     # ---- the fp64 oracle on a bounded sample, host cores of this machine

@@ -9,6 +9,7 @@
 
 #include "../../include/gqa.h"
 #include "internal.h"
+#include "mla.h"
 
 namespace {
 
@@ -418,6 +419,40 @@ gqa_status gqa_decode_expanded(const void *q, const void *k_cache, const void *v
         return s;
     g_last_launches = 1;
     return run_decode(q, k_rep, v_rep, seqlens, B, Hq, Hq, Tmax, scale, out, st, &g_last_launches);
+}
+
+gqa_status gqa_mla_decode(const void *q, const void *kv_cache, const int32_t *seqlens, int B, int Hq, int d_c,
+                          int d_r, int Tmax, float scale, void *out, void *stream)
+{
+    g_last_launches = 0;
+    if (!q || !kv_cache || !seqlens || !out) return GQA_ERR_INVALID_ARG;
+    if (B <= 0 || Hq <= 0 || d_c <= 0 || d_r < 0 || Tmax <= 0) return GQA_ERR_INVALID_ARG;
+    if (d_c != kMlaLatent || d_r != kMlaRope) return GQA_ERR_UNSUPPORTED;
+    if (B > 65535 || Hq > 65535) return GQA_ERR_UNSUPPORTED;   // grid dimensions
+    if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out)) return GQA_ERR_MISALIGNED;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState *st = nullptr;
+    gqa_status s = device_state(&st);
+    if (s != GQA_OK) return s;
+    const MlaPlan p = mla_plan_host(B, Hq, Tmax, st->num_sms);
+    if (p.ws_bytes > 0 && (s = ensure_workspace(st, p.ws_bytes)) != GQA_OK) return s;
+    MlaArgs a;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.kv = static_cast<const __nv_bfloat16 *>(kv_cache);
+    a.seqlens = seqlens;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.part_o = p.nsplit > 1 ? static_cast<float *>(st->ws) : nullptr;
+    a.part_ml = p.nsplit > 1 ? a.part_o + (size_t)B * Hq * p.nsplit * kMlaLatent : nullptr;
+    a.B = B;
+    a.Hq = Hq;
+    a.Tmax = Tmax;
+    a.nsplit = p.nsplit;
+    a.chunk = p.chunk;
+    a.qscale = scale * 1.4426950408889634f;
+    int n = 0;
+    const cudaError_t e = launch_mla_decode(a, static_cast<cudaStream_t>(stream), &n, g_ev_before, g_ev_after);
+    g_last_launches = n;
+    return cuda_status(e);
 }
 
 gqa_status gqa_tp_shard(int Hq, int Hkv, int tp, int rank, int *q_first, int *q_count, int *kv_first,

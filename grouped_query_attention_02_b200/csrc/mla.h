@@ -1,0 +1,48 @@
+// mla.h -- launch interface of the MLA decode kernels (mla.cu), used by api.cu.
+//
+// MLA with absorbed weights ("MLA: multi-head latent attention", anrans.github.io
+// attention-variants: weight absorption and decoupled RoPE): every query head scores one
+// cached row per token, the 512-wide latent followed by the 64-wide RoPE key shared by all
+// heads, and its output is the softmax-weighted sum of the rows' latent parts -- an MQA whose
+// value is the first 512 entries of its key.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace gqa {
+
+constexpr int kMlaLatent = 512;                   // d_c: latent width, also the value width
+constexpr int kMlaRope = 64;                      // d_r: RoPE key width
+constexpr int kMlaRow = kMlaLatent + kMlaRope;    // one cached row, one query row
+constexpr int kMlaHeads = 16;                     // query heads per CTA
+constexpr int kMlaTile = 32;                      // cached tokens per tile
+
+struct MlaArgs {
+    const __nv_bfloat16 *q;    // [B, Hq, 576]: absorbed latent query, then RoPE query
+    const __nv_bfloat16 *kv;   // [B, Tmax, 576]: latent, then RoPE key
+    const int32_t *seqlens;    // [B], device
+    __nv_bfloat16 *out;        // [B, Hq, 512]
+    float *part_o;             // [B, Hq, nsplit, 512] when nsplit > 1
+    float *part_ml;            // [B, Hq, nsplit, 2] (running max in log2 units, weight sum)
+    int B, Hq, Tmax, nsplit, chunk;
+    float qscale;              // scale * log2(e)
+};
+
+struct MlaPlan {
+    int nsplit;       // token ranges per sequence
+    int chunk;        // tokens per range, a multiple of kMlaTile
+    size_t ws_bytes;  // split partials (0 when nsplit == 1)
+};
+
+MlaPlan mla_plan_host(int B, int Hq, int Tmax, int num_sms);
+
+// Enqueues the decode (and, for nsplit > 1, the combine) on `stream`; adds the launches made to
+// *launches.  `before` / `after`, when non-null, are recorded around the decode kernel.
+cudaError_t launch_mla_decode(const MlaArgs &a, cudaStream_t stream, int *launches, cudaEvent_t before,
+                              cudaEvent_t after);
+
+}  // namespace gqa

@@ -47,3 +47,20 @@ EXTREME_GROUP_DECODE = DecodeWorkload(
 CAUSAL_PREFILL = PrefillWorkload("causal GQA prefill B4 S8192 Hq32 Hkv8 d128", 4, 8192, 32, 8, 128)
 
 DECODE_WORKLOADS = (TINY_DECODE, QWEN3_8B_DECODE) + VARLEN_DECODE + (EXTREME_GROUP_DECODE,)
+
+
+@dataclass(frozen=True)
+class MlaWorkload:
+    name: str
+    B: int
+    Hq: int
+    d_c: int
+    d_r: int
+    Tmax: int
+
+
+# MLA decode with absorbed weights in DeepSeek-V3's geometry as the MLA page gives it (128 query heads,
+# a 512-wide latent plus a 64-wide RoPE key per token); the page gives no batch or length, so 32
+# sequences of 8192 tokens (a 302 MB cache, larger than L2) stand in.
+MLA_DECODE = MlaWorkload("MLA absorbed decode (DeepSeek-V3-shaped) B32 Hq128 d_c512 d_r64 T8192", 32, 128, 512, 64,
+                         8192)

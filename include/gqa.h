@@ -219,6 +219,33 @@ gqa_status gqa_decode_plan(int B, int Hq, int Hkv, int d, int Tmax, int num_sms,
                            size_t *workspace_bytes);
 
 /*
+ * gqa_mla_decode -- one decode step of multi-head latent attention with
+ * absorbed weights ("MLA: multi-head latent attention", anrans.github.io
+ * attention-variants: weight absorption and decoupled RoPE).  The cache holds
+ * one row per token, the d_c-wide latent followed by the d_r-wide RoPE key
+ * shared by all heads; the latent is both key and value, so the operator is an
+ * MQA whose value is the first d_c entries of its key.
+ *
+ *   q        [B, Hq, d_c + d_r]   per head: the absorbed latent query (W_UK
+ *                                 folded in), then the RoPE query
+ *   kv_cache [B, Tmax, d_c + d_r] per token: latent, then RoPE key
+ *   seqlens  [B] int32, DEVICE memory
+ *   scale    multiplier of q.kv (the original head's 1/sqrt(d_h + d_r))
+ *   out      [B, Hq, d_c]         out[b,h] = sum_{t < seqlens[b]}
+ *                                 softmax_t(scale q[b,h].kv[b,t]) kv[b,t,0:d_c]
+ *                                 (W_UV is applied by the caller's output projection)
+ *
+ * bf16 in and out, fp32 accumulation; d_c = 512 and d_r = 64 only
+ * (GQA_ERR_UNSUPPORTED otherwise); B and Hq at most 65535.  Lengths, NaN and
+ * empty histories as in gqa_decode.  This is a CUDA-core kernel (16 heads per
+ * CTA, tiles of 32 cached rows through shared memory, split over token ranges
+ * and merged by a combine kernel through the library workspace); the
+ * contraction belongs on the tensor cores, which is the next step for it.
+ */
+gqa_status gqa_mla_decode(const void *q, const void *kv_cache, const int32_t *seqlens, int B, int Hq, int d_c,
+                          int d_r, int Tmax, float scale, void *out, void *stream);
+
+/*
  * gqa_tp_shard -- the heads rank `rank` of `tp` tensor-parallel ranks owns
  * for one attention layer (kv-head-replication glossary entry,
  * inferencex.semianalysis.com; the tensor-parallelism paragraphs of
@@ -263,7 +290,7 @@ gqa_status gqa_selftest_wait_timeout(int timeout_us, void *stream);
 /*
  * gqa_set_profile_events -- measurement hook.  When both are non-NULL
  * (cudaEvent_t passed as void*), every later gqa_decode / gqa_decode_fp8 /
- * gqa_prefill_causal(_fwd) / gqa_decode_expanded records `before` on its stream
+ * gqa_mla_decode / gqa_prefill_causal(_fwd) / gqa_decode_expanded records `before` on its stream
  * immediately before its dominant kernel (the decode kernel; the prefill
  * kernel) and `after` immediately after it; gqa_prefill_causal_bwd records
  * them around its three kernels; gqa_decode_noalloc records nothing.  NULL,

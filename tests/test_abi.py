@@ -170,3 +170,12 @@ def test_workspace_allocator_comes_in_pairs(lib):
     with pytest.raises(ValueError):
         gqa.gqa_set_workspace_allocator(lambda n, dev: 0, None)
 
+
+def test_mla_decode_argument_checks(lib):
+    f = lambda q=A, kv=A, sl=A, B=2, Hq=16, dc=512, dr=64, T=64, out=A: lib.gqa_mla_decode(
+        q, kv, sl, B, Hq, dc, dr, T, ctypes.c_float(0.07), out, None)
+    assert f(q=None) == INVALID and f(kv=None) == INVALID and f(sl=None) == INVALID and f(out=None) == INVALID
+    assert f(B=0) == INVALID and f(Hq=0) == INVALID and f(T=0) == INVALID and f(dr=-1) == INVALID
+    assert f(dc=128) == UNSUPPORTED and f(dr=0) == UNSUPPORTED and f(B=70000) == UNSUPPORTED
+    assert f(q=U) == MISALIGNED and f(kv=U) == MISALIGNED and f(out=U) == MISALIGNED
+
