@@ -569,12 +569,13 @@ def test_mla_decode_closed_forms(oracle_mod):
 
 
 def test_mla_cache_bytes_per_token(oracle_mod):
-    """The MLA page's cache sizes: 512 + 64 numbers per token and layer against 2 x 128 heads x 128 for
-    MHA (about 1/57), and DeepSeek-V3's 61 layers of 576 bf16 numbers per token."""
-    mla, mha = 512 + 64, 2 * 128 * 128
-    assert mha == 32768 and round(mha / mla) == 57
-    assert 61 * (512 + 64) * 2 == 70272
-    # with one "KV head" of width 576 and K = V shared, the MLA cache is half the bytes the GQA byte
-    # model would count for a separate K and V of that width
-    assert oracle_mod.kv_bytes(61, 1, 1, 576, 2) == 2 * 70272
+    """The MLA page's cache sizes (tests/golden/mla.txt): 512 + 64 numbers per token and layer against
+    2 x 128 heads x 128 for MHA (about 1/57), and DeepSeek-V3's 61 layers of 576 bf16 numbers per token.
+    The latent is both key and value, so the cache holds one row where the GQA byte model counts a
+    separate K and V: half of kv_bytes for one KV head of width 576."""
+    g = {ln.split()[0]: int(ln.split()[1]) for ln in _lines("mla.txt")}
+    mha, mla = 2 * 128 * 128, 512 + 64
+    assert g["mha_numbers_per_token_layer"] == mha and g["mla_numbers_per_token_layer"] == mla
+    assert round(mha / mla) == g["mla_fraction_of_mha"]
+    assert 2 * g["deepseek_v3_bytes_per_token"] == oracle_mod.kv_bytes(61, 1, 1, 576, 2)
 
