@@ -327,9 +327,12 @@ def time_e2e(gqa, torch, x, steps: int):
     return s0.elapsed_time(s1) / steps, h2d, d2h, ok
 
 
-def cpu_oracle_sample(x, target_s: float = 12.0):
+def cpu_oracle_sample(x, target_s: float = 12.0, gpu_out=None):
     """Time the fp64 oracle on a bounded sample of the workload: the first n sequences (every
-    query head), repeated until about target_s seconds of wall time have been spent."""
+    query head), repeated until about target_s seconds of wall time have been spent.  With the GPU's
+    output of the same workload (host tensor [B, Hq, d]) the result also carries "parity": the GPU's
+    error on the sampled sequences against the oracle's output from the last timed run."""
+    import numpy as np
     import oracle
 
     sl = x.seqlens.cpu().tolist()
@@ -344,10 +347,14 @@ def cpu_oracle_sample(x, target_s: float = 12.0):
         vv = x.v_cache[:n, :T].cpu()
         t0 = time.perf_counter()
         if hasattr(x, "k_scale"):
-            oracle.decode_fp8(q, kk, vv, x.k_scale, x.v_scale, sl[:n], x.scale, nthreads=cores)
+            r = oracle.decode_fp8(q, kk, vv, x.k_scale, x.v_scale, sl[:n], x.scale, nthreads=cores)
         else:
-            oracle.decode(q, kk, vv, sl[:n], x.scale, nthreads=cores)
-        return time.perf_counter() - t0
+            r = oracle.decode(q, kk, vv, sl[:n], x.scale, nthreads=cores)
+        el = time.perf_counter() - t0
+        last["n"], last["ref"] = n, r
+        return el
+
+    last = {}
 
     t1 = run(1)
     n = max(1, min(B, int(target_s / max(t1, 1e-3))))
@@ -356,10 +363,20 @@ def cpu_oracle_sample(x, target_s: float = 12.0):
         spent += run(n)
         reps += 1
     ub = unique_kv_bytes(sl[:n], Hkv, d, x.k_cache.element_size()) * reps
-    return {"value": ub / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"first {n} of {B} sequences (every query head, {sum(sl[:n])} cached tokens) "
-                      f"x {reps} repetitions; {spent:.1f} s wall on {cores} threads",
-            "seconds": spent, "tokens_per_s": n * reps / spent}
+    res = {"value": ub / spent / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+           "sample": f"first {n} of {B} sequences (every query head, {sum(sl[:n])} cached tokens) "
+                     f"x {reps} repetitions; {spent:.1f} s wall on {cores} threads",
+           "seconds": spent, "tokens_per_s": n * reps / spent}
+    if gpu_out is not None and "ref" in last:
+        ref = last["ref"]
+        got = gpu_out[:last["n"]].double().numpy()
+        err = np.abs(got - ref)
+        rmax = float(np.abs(ref).max())
+        res["parity"] = {"max_abs": float(err.max()), "rel_normwise": float(err.max() / rmax) if rmax > 0 else 0.0,
+                         "bar": {"max_abs": 2e-2, "rel_normwise": 2e-2},
+                         "within_bar": bool(err.max() <= 2e-2 and (rmax == 0 or err.max() / rmax <= 2e-2)),
+                         "sample": f"first {last['n']} of {B} sequences, every query head, against the fp64 oracle"}
+    return res
 
 
 def decode_kernel_name(g: int, fp8: bool = False) -> str:
@@ -574,6 +591,8 @@ def main():
     if e2e_err:
         line["e2e"]["error"] = e2e_err
 
+    out_host = out.float().cpu()   # the headline's output, for the parity figure of the CPU-baseline leg
+
     # ---- the other rows of the hot path
     if args.rows == "all" and max(world, 1) == 1 and not fp8:
         rows = {}
@@ -669,7 +688,11 @@ def main():
 
     # ---- the fp64 oracle on a bounded sample, host cores of this machine
     if max(world, 1) == 1 and args.cpu_baseline == "on":
-        line["cpu_baseline"] = cpu_oracle_sample(x)
+        cb = cpu_oracle_sample(x, gpu_out=out_host)
+        parity = cb.pop("parity", None)
+        line["cpu_baseline"] = cb
+        if parity is not None:
+            line["parity"] = parity
 
     print(json.dumps(line))
     if dist:
