@@ -406,6 +406,38 @@ def prefill_only(gqa, torch, inputs, workloads, args):
                       "gpu_launches": n, "device_status": gqa.gqa_get_last_device_status()}))
 
 
+def mla_roofline(peaks, mw, st_ms, k_ms):
+    """The MLA row: tensor-bound at 128 heads (about 242 FLOP per byte, near the ridge), so the target
+    time is the larger of FLOP / tensor peak and bytes / HBM peak; both fractions are reported."""
+    fl = mla_decode_flops(mw.B, mw.Hq, mw.Tmax, mw.d_c, mw.d_r)
+    by = mw.B * mw.Tmax * (mw.d_c + mw.d_r) * 2 + mw.B * mw.Hq * (2 * (mw.d_c + mw.d_r) + 2 * mw.d_c)
+    t_bound = max(fl / (peaks["bf16_tflops"] * 1e12), by / (peaks["hbm_gbs"] * 1e9))
+    return {
+        "ms_per_step": st_ms, "kernel_ms": k_ms, "TFLOPs": fl / (st_ms * 1e-3) / 1e12,
+        "unique_kv_GBps": by / (st_ms * 1e-3) / 1e9, "tokens_per_s": mw.B / (st_ms * 1e-3),
+        "roofline": {"bound": "tensor", "achieved": fl / (k_ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                     "traffic": None, "hbm_frac": by / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "frac_of_bound": t_bound / (k_ms * 1e-3), "bound_ms": t_bound * 1e3,
+                     "peak_source": f"{peaks.get('source')} bf16_tflops (cuBLAS burst), hbm_gbs"},
+        "flop_count": "2 Hq (2 d_c + d_r) per cached token; bytes: the cache once, q in, out",
+        "kernel": "tcgen05, 64 heads per CTA, persistent, device-planned pieces + combine"}
+
+
+def mla_only(gqa, torch, inputs, workloads, args):
+    """Time the DeepSeek-V3-shaped MLA decode alone (used for its ncu captures)."""
+    mw = workloads.MLA_DECODE
+    peaks = load_peaks()
+    xm = inputs.make_mla_decode(mw.B, mw.Hq, mw.Tmax, mw.d_c, mw.d_r, device="cuda", seed=0)
+    st_ms, k_ms, n = time_mla(gqa, torch, xm, args.steps, args.warmup)
+    row = mla_roofline(peaks, mw, st_ms, k_ms)
+    print(json.dumps({"metric": "MLA absorbed decode TFLOP/s", "value": row["TFLOPs"], "unit": "TFLOP/s",
+                      "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": st_ms,
+                      "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+                      "config": {"workload": mw.name}, "row": row, "gpu_launches": n,
+                      "device_status": gqa.gqa_get_last_device_status()}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -415,9 +447,9 @@ def main():
     ap.add_argument("--rows", choices=["all", "none"], default="all")
     ap.add_argument("--e2e-steps", type=int, default=3, help="0 skips the host-buffer measurement")
     ap.add_argument("--cpu-baseline", choices=["on", "off"], default="on")
-    ap.add_argument("--mode", choices=["decode", "prefill", "backward"], default="decode",
-                    help="prefill / backward: time only the causal prefill workload's forward / backward "
-                         "(used for their ncu captures)")
+    ap.add_argument("--mode", choices=["decode", "prefill", "backward", "mla"], default="decode",
+                    help="prefill / backward / mla: time only the causal prefill workload's forward / backward, "
+                         "or the MLA decode workload (used for their ncu captures)")
     ap.add_argument("--prefill-batch", type=int, default=4, help="sequences in --mode prefill")
     ap.add_argument("--decode-workload", default="Qwen3-8B",
                     help="name prefix of the decode workload timed as the headline (profiling other rows)")
@@ -478,6 +510,9 @@ def main():
     torch.cuda.set_device(local_rank)
     if args.mode == "prefill":
         prefill_only(gqa, torch, inputs, workloads, args)
+        return
+    if args.mode == "mla":
+        mla_only(gqa, torch, inputs, workloads, args)
         return
     if args.mode == "backward":
         pw = workloads.CAUSAL_PREFILL
@@ -664,22 +699,13 @@ def main():
             torch.cuda.empty_cache()
         except gqa.GQAError as e:
             rows["backward, " + pw.name] = {"error": str(e)}
-        # MLA decode with absorbed weights (CUDA-core kernel, the row's first correct path)
+        # MLA decode with absorbed weights (tensor cores)
         mw = workloads.MLA_DECODE
         try:
             xm = inputs.make_mla_decode(mw.B, mw.Hq, mw.Tmax, mw.d_c, mw.d_r, device="cuda", seed=0)
-            st_ms, k_ms, n = time_mla(gqa, torch, xm, 5, 3)
-            fl = mla_decode_flops(mw.B, mw.Hq, mw.Tmax, mw.d_c, mw.d_r)
-            by = mw.B * mw.Tmax * (mw.d_c + mw.d_r) * 2
-            rows[mw.name] = {
-                "ms_per_step": st_ms, "kernel_ms": k_ms, "TFLOPs": fl / (st_ms * 1e-3) / 1e12,
-                "unique_kv_GBps": by / (st_ms * 1e-3) / 1e9, "tokens_per_s": mw.B / (st_ms * 1e-3),
-                "roofline": {"bound": "tensor", "achieved": fl / (k_ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
-                             "unit": "TFLOP/s", "frac": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
-                             "traffic": None, "hbm_frac": by / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                             "peak_source": f"{peaks.get('source')} bf16_tflops (cuBLAS burst)"},
-                "flop_count": "2 Hq (2 d_c + d_r) per cached token", "kernel": "CUDA cores (first path)",
-                "launches_per_step": n / 5}
+            st_ms, k_ms, n = time_mla(gqa, torch, xm, 20, 3)
+            rows[mw.name] = mla_roofline(peaks, mw, st_ms, k_ms)
+            rows[mw.name]["launches_per_step"] = n / 20
             del xm
             torch.cuda.empty_cache()
         except (gqa.GQAError, RuntimeError) as e:   # a row that fails must not cost the line

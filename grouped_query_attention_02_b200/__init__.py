@@ -14,7 +14,7 @@ import os
 __all__ = [
     "GQAError", "gqa_decode", "gqa_decode_fp8", "gqa_decode_noalloc", "gqa_prefill_causal",
     "gqa_prefill_causal_fwd", "gqa_prefill_causal_bwd", "gqa_decode_expanded", "gqa_decode_expanded_bytes",
-    "gqa_decode_plan", "gqa_tp_shard", "gqa_mla_decode", "gqa_get_last_device_status", "gqa_selftest_wait_timeout", "gqa_set_profile_events",
+    "gqa_decode_plan", "gqa_tp_shard", "gqa_mla_decode", "gqa_mla_decode_cudacore", "gqa_get_last_device_status", "gqa_selftest_wait_timeout", "gqa_set_profile_events",
     "gqa_last_launch_count", "gqa_release", "gqa_set_workspace_allocator", "gqa_status_string", "gqa_version",
     "library_path", "load",
 ]
@@ -44,6 +44,7 @@ EXPORTS = {
                              ctypes.POINTER(ctypes.c_size_t)]),
     "gqa_tp_shard": (_i, [_i, _i, _i, _i] + [ctypes.POINTER(_i)] * 4),
     "gqa_mla_decode": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp]),
+    "gqa_mla_decode_cudacore": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _i, ctypes.c_float, _vp, _vp]),
     "gqa_get_last_device_status": (_i, [_vp]),
     "gqa_selftest_wait_timeout": (_i, [_i, _vp]),
     "gqa_set_profile_events": (_i, [_vp, _vp]),
@@ -326,9 +327,7 @@ def gqa_decode_plan(B, Hq, Hkv, d, Tmax, num_sms):
     return c.value, n.value, w.value
 
 
-def gqa_mla_decode(q, kv_cache, seqlens, scale=None, out=None, stream=None, d_c=512):
-    """MLA decode with absorbed weights: q [B,Hq,d_c+d_r], kv_cache [B,Tmax,d_c+d_r] bf16, seqlens [B] int32
-    (device) -> out [B,Hq,d_c] bf16.  scale defaults to 1/sqrt(128 + d_r)."""
+def _mla(fn_name, q, kv_cache, seqlens, scale, out, stream, d_c):
     import torch
 
     _need(q, "q", torch.bfloat16, 3)
@@ -345,10 +344,21 @@ def gqa_mla_decode(q, kv_cache, seqlens, scale=None, out=None, stream=None, d_c=
         out = torch.empty((B, Hq, int(d_c)), dtype=torch.bfloat16, device=q.device)
     else:
         _need(out, "out", torch.bfloat16, 3, q.device)
-    _check(load().gqa_mla_decode(q.data_ptr(), kv_cache.data_ptr(), seqlens.data_ptr(), B, Hq, int(d_c), d_r,
-                                 kv_cache.shape[1], ctypes.c_float(scale), out.data_ptr(), _stream_ptr(stream)),
-           "gqa_mla_decode")
+    _check(getattr(load(), fn_name)(q.data_ptr(), kv_cache.data_ptr(), seqlens.data_ptr(), B, Hq, int(d_c), d_r,
+                                    kv_cache.shape[1], ctypes.c_float(scale), out.data_ptr(), _stream_ptr(stream)),
+           fn_name)
     return out
+
+
+def gqa_mla_decode(q, kv_cache, seqlens, scale=None, out=None, stream=None, d_c=512):
+    """MLA decode with absorbed weights on the tensor cores: q [B,Hq,d_c+d_r], kv_cache [B,Tmax,d_c+d_r] bf16,
+    seqlens [B] int32 (device) -> out [B,Hq,d_c] bf16.  scale defaults to 1/sqrt(128 + d_r)."""
+    return _mla("gqa_mla_decode", q, kv_cache, seqlens, scale, out, stream, d_c)
+
+
+def gqa_mla_decode_cudacore(q, kv_cache, seqlens, scale=None, out=None, stream=None, d_c=512):
+    """The same operator on the CUDA cores (fp32 weights): the independent second path for full-size checks."""
+    return _mla("gqa_mla_decode_cudacore", q, kv_cache, seqlens, scale, out, stream, d_c)
 
 
 def gqa_tp_shard(Hq, Hkv, tp, rank):

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgqa.so")
-SOURCES = ["api.cu", "decode.cu", "decode_tc.cu", "prefill.cu", "backward.cu", "noalloc.cu", "mla.cu"]
+SOURCES = ["api.cu", "decode.cu", "decode_tc.cu", "prefill.cu", "backward.cu", "noalloc.cu", "mla.cu", "mla_tc.cu"]
 HEADERS = ["ptx.cuh", "internal.h", "mla.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

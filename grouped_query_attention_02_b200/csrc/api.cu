@@ -421,19 +421,65 @@ gqa_status gqa_decode_expanded(const void *q, const void *k_cache, const void *v
     return run_decode(q, k_rep, v_rep, seqlens, B, Hq, Hq, Tmax, scale, out, st, &g_last_launches);
 }
 
-gqa_status gqa_mla_decode(const void *q, const void *kv_cache, const int32_t *seqlens, int B, int Hq, int d_c,
-                          int d_r, int Tmax, float scale, void *out, void *stream)
+// Host checks shared by both MLA decode entry points.
+static gqa_status check_mla_args(const void *q, const void *kv_cache, const int32_t *seqlens, int B, int Hq, int d_c,
+                                 int d_r, int Tmax, const void *out)
 {
-    g_last_launches = 0;
     if (!q || !kv_cache || !seqlens || !out) return GQA_ERR_INVALID_ARG;
     if (B <= 0 || Hq <= 0 || d_c <= 0 || d_r < 0 || Tmax <= 0) return GQA_ERR_INVALID_ARG;
     if (d_c != kMlaLatent || d_r != kMlaRope) return GQA_ERR_UNSUPPORTED;
     if (B > 65535 || Hq > 65535) return GQA_ERR_UNSUPPORTED;   // grid dimensions
     if (!aligned16(q) || !aligned16(kv_cache) || !aligned16(out)) return GQA_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return GQA_ERR_MISALIGNED;
+    return GQA_OK;
+}
+
+// 3-D bf16 map over a [n2][n1][n0] row-major tensor, box {64, rows, 1}, 128-byte swizzle.
+static gqa_status encode_3d(CUtensorMap *tm, const void *base, uint64_t n0, uint64_t n1, uint64_t n2,
+                            uint32_t box_rows)
+{
+    cuuint64_t dims[3] = {n0, n1, n2};
+    cuuint64_t strides[2] = {n0 * 2, n0 * n1 * 2};
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_CUDA;
+}
+
+gqa_status gqa_mla_decode(const void *q, const void *kv_cache, const int32_t *seqlens, int B, int Hq, int d_c,
+                          int d_r, int Tmax, float scale, void *out, void *stream)
+{
+    g_last_launches = 0;
+    gqa_status s = check_mla_args(q, kv_cache, seqlens, B, Hq, d_c, d_r, Tmax, out);
+    if (s != GQA_OK) return s;
     std::lock_guard<std::mutex> lk(g_mu);
     DeviceState *st = nullptr;
-    gqa_status s = device_state(&st);
+    if ((s = device_state(&st)) != GQA_OK) return s;
+    if ((s = get_encoder()) != GQA_OK) return s;
+    const MlaTcPlan p = mla_tc_plan_host(B, Hq, Tmax, kWorkspaceBudget);
+    if ((s = ensure_workspace(st, p.ws_bytes)) != GQA_OK) return s;
+    CUtensorMap tmKV, tmQ;
+    if ((s = encode_3d(&tmKV, kv_cache, kMlaRow, Tmax, B, 128)) != GQA_OK) return s;
+    if ((s = encode_3d(&tmQ, q, kMlaRow, Hq, B, 64)) != GQA_OK) return s;
+    int n = 0;
+    const cudaError_t e = launch_mla_decode_tc(tmKV, tmQ, q, seqlens, B, Hq, Tmax, scale, out, st->ws, p,
+                                               st->num_sms, st->status, kWaitBudgetNs,
+                                               static_cast<cudaStream_t>(stream), &n, g_ev_before, g_ev_after);
+    g_last_launches = n;
+    return cuda_status(e);
+}
+
+gqa_status gqa_mla_decode_cudacore(const void *q, const void *kv_cache, const int32_t *seqlens, int B, int Hq,
+                                   int d_c, int d_r, int Tmax, float scale, void *out, void *stream)
+{
+    g_last_launches = 0;
+    gqa_status s = check_mla_args(q, kv_cache, seqlens, B, Hq, d_c, d_r, Tmax, out);
     if (s != GQA_OK) return s;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceState *st = nullptr;
+    if ((s = device_state(&st)) != GQA_OK) return s;
     const MlaPlan p = mla_plan_host(B, Hq, Tmax, st->num_sms);
     if (p.ws_bytes > 0 && (s = ensure_workspace(st, p.ws_bytes)) != GQA_OK) return s;
     MlaArgs a;

@@ -159,16 +159,6 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// 3-D tiled load (d, heads, batch) of the group's query rows.
-__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *tm, uint64_t *bar, int c0, int c1, int c2)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
-            smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(tm)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-
 // ---------------------------------------------------------------------------------------------
 // Exclusive scan of n ints in shared memory by the whole block.
 __device__ void block_exclusive_scan(int *v, int n, int *warp_tot)
@@ -271,7 +261,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         }
         // about eight rounds of (piece, KV head) units per persistent CTA (two for groups above 16, whose
         // units of up to 32 heads carry a larger fixed cost each), never more than nsplit pieces
-        const long long rounds = a.group > 16 ? 2 : 8;
+        const long long rounds = a.plan_rounds > 0 ? a.plan_rounds : (a.group > 16 ? 2 : 8);
         long long C = (T * a.Hkv + rounds * slots - 1) / (rounds * slots);
         const long long cmin = (M + a.nsplit - 1) / a.nsplit;
         if (C < cmin) C = cmin;
@@ -307,8 +297,9 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         const int full = tl / C, rem = tl % C;
         if (tl == 0) {
             // no cached token: no unit will touch this sequence, its output rows are zero
-            uint4 *o = reinterpret_cast<uint4 *>(a.out + (size_t)b * a.Hq * kD);
-            for (int i = 0; i < a.Hq * kD / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
+            const int orow = a.out_row > 0 ? a.out_row : kD;
+            uint4 *o = reinterpret_cast<uint4 *>(a.out + (size_t)b * a.Hq * orow);
+            for (int i = 0; i < a.Hq * orow / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
         }
         for (int s = 0; s < full; ++s)
             a.items[full_off[b] + s] = make_int4(b, s, s * C * kTok, min((s + 1) * C * kTok, T));

@@ -33,6 +33,9 @@ struct DecodeArgs {
     int *plan_scratch;        // [B] planner scratch
     int4 *items;              // [B * nsplit] pieces, longest first
     int num_ctas;             // persistent CTAs (one per SM)
+    // planner options for other operators that reuse decode_plan_kernel (0: the GQA decode's defaults)
+    int out_row;              // output elements per (sequence, query head) row, zeroed for empty histories
+    int plan_rounds;          // rounds of units per persistent CTA the pieces are sized for
 };
 
 // Host plan of a decode call and the layout of its workspace.

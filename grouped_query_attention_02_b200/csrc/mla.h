@@ -10,6 +10,7 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -44,5 +45,24 @@ MlaPlan mla_plan_host(int B, int Hq, int Tmax, int num_sms);
 // *launches.  `before` / `after`, when non-null, are recorded around the decode kernel.
 cudaError_t launch_mla_decode(const MlaArgs &a, cudaStream_t stream, int *launches, cudaEvent_t before,
                               cudaEvent_t after);
+
+// The tensor-core MLA decode (mla_tc.cu): device-planned pieces, one persistent CTA per SM over
+// (piece, 64-head block) units, a combine for split histories.  Workspace layout:
+struct MlaTcPlan {
+    int nsplit;       // most pieces one sequence can get
+    int nhb;          // 64-head blocks
+    size_t off_hdr, off_nsb, off_items, off_po, off_pml, ws_bytes;
+};
+// ws_budget bounds the split partials (fewer pieces per sequence when it is small).
+MlaTcPlan mla_tc_plan_host(int B, int Hq, int Tmax, size_t ws_budget);
+
+// Enqueues the planner, the decode and the combine on `stream` (three launches, added to
+// *launches); tmKV maps kv_cache [B, Tmax, 576] with box {64, 128, 1}, tmQ maps q [B, Hq, 576]
+// with box {64, 64, 1}, both bf16 with the 128-byte swizzle.  `before` / `after`, when non-null,
+// are recorded around the decode kernel.
+cudaError_t launch_mla_decode_tc(const CUtensorMap &tmKV, const CUtensorMap &tmQ, const void *q,
+                                 const int32_t *seqlens, int B, int Hq, int Tmax, float scale, void *out, void *ws,
+                                 const MlaTcPlan &p, int num_sms, int *status, unsigned long long wait_budget_ns,
+                                 cudaStream_t stream, int *launches, cudaEvent_t before, cudaEvent_t after);
 
 }  // namespace gqa

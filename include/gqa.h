@@ -236,14 +236,33 @@ gqa_status gqa_decode_plan(int B, int Hq, int Hkv, int d, int Tmax, int num_sms,
  *                                 (W_UV is applied by the caller's output projection)
  *
  * bf16 in and out, fp32 accumulation; d_c = 512 and d_r = 64 only
- * (GQA_ERR_UNSUPPORTED otherwise); B and Hq at most 65535.  Lengths, NaN and
- * empty histories as in gqa_decode.  This is a CUDA-core kernel (16 heads per
- * CTA, tiles of 32 cached rows through shared memory, split over token ranges
- * and merged by a combine kernel through the library workspace); the
- * contraction belongs on the tensor cores, which is the next step for it.
+ * (GQA_ERR_UNSUPPORTED otherwise); B and Hq at most 65535; q, kv_cache and out
+ * 16-byte aligned, seqlens 4-byte aligned (GQA_ERR_MISALIGNED otherwise).
+ * Lengths, NaN and empty histories as in gqa_decode.
+ *
+ * Runs on the tcgen05 tensor cores: blocks of 64 query heads, tokens as the
+ * 128-row side of S^T = KV.Q^T and of O^T += KV_latent^T.P^T, the cached rows
+ * fetched by TMA once per head block; histories are cut into pieces on the
+ * device from the real lengths and merged by a combine kernel, through the
+ * library workspace (three launches: plan, decode, combine).  The weights
+ * enter the P.V product rounded to bf16, as in the causal prefill, so each
+ * output is a convex combination of latent rows with weights within 2^-8 of
+ * the exact ones.
  */
 gqa_status gqa_mla_decode(const void *q, const void *kv_cache, const int32_t *seqlens, int B, int Hq, int d_c,
                           int d_r, int Tmax, float scale, void *out, void *stream);
+
+/*
+ * gqa_mla_decode_cudacore -- the same operator as gqa_mla_decode, same
+ * arguments, checks and errors, computed on the CUDA cores (16 heads per CTA,
+ * tiles of 32 cached rows through shared memory, fp32 weights and dot
+ * products, split over token ranges and merged by a combine kernel through the
+ * library workspace).  About two orders of magnitude slower; it is kept as an
+ * independent second path that full-size outputs of the tensor-core kernel can
+ * be compared with where the fp64 oracle would take too long.
+ */
+gqa_status gqa_mla_decode_cudacore(const void *q, const void *kv_cache, const int32_t *seqlens, int B, int Hq,
+                                   int d_c, int d_r, int Tmax, float scale, void *out, void *stream);
 
 /*
  * gqa_tp_shard -- the heads rank `rank` of `tp` tensor-parallel ranks owns
