@@ -250,6 +250,8 @@ DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_
         const long long ct = (tiles + s - 1) / s;
         const long long se = (tiles + ct - 1) / ct;
         if (se != s) continue;
+        // split partials must fit the workspace budget; one piece per sequence needs none
+        if (se > 1 && (double)B * Hq * se * (kHeadDim + 2) * 4.0 > (double)ws_budget) continue;
         const long long waves = (base * se + slots - 1) / slots;
         // each CTA also pays a fixed start-up (barriers, query rows, pipeline fill): about one tile
         double cost = (double)waves * ((double)ct + 1.0);

@@ -44,7 +44,7 @@ struct DecodePlan {
     bool tensor_cores;
     size_t off_hdr, off_nsb, off_items, off_po, off_pml, ws_bytes;
 };
-// ws_budget bounds the split partials of the tensor-core path (more pieces per sequence when it allows).
+// ws_budget bounds the split partials (fewer pieces per sequence when they would not fit; one piece needs none).
 // fp8: the plan of the FP8-cache decode, which always takes the tensor-core path (group sizes <= 32).
 DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_t ws_budget, bool fp8 = false);
 

@@ -58,6 +58,7 @@ constexpr int kMmaWarp = kProducerWarp + 1;
 constexpr int kThreads = kWG * kNWG + 64;
 constexpr int kQD = 4;                            // depth of the unit queue
 constexpr float kMoveThreshold = 8.0f;            // the running maximum moves only by more than this
+constexpr int kPrefetch = 2;                      // tiles prefetched into L2 ahead of their load
 
 // barrier slots
 enum : int { CH_FULL = 0, EMPTY_PAIR = CH_FULL + kChunks, EMPTY_P = EMPTY_PAIR + kLatChunks / 2, S_FULL, P_FULL,
@@ -217,8 +218,14 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
                     tma_load_3d(smem + kQOff + c * kQChunkBytes, &tmQ, &bar[Q_FULL], 64 * c, kNh * hb, it.x);
                 ++q_loads;
                 const int ntl = (it.w - it.z + kTok - 1) / kTok;
+                // the unit's first tiles into L2 now, each later one kPrefetch tiles ahead of its load, so
+                // that a load into a freed slot waits for L2 rather than HBM
+                for (int jp = 0; jp < kPrefetch && jp < ntl; ++jp)
+                    for (int c = 0; c < kChunks; ++c) tma_prefetch_l2_3d(&tmKV, 64 * c, it.z + jp * kTok, it.x);
                 for (int jj = 0; jj < ntl && ok; ++jj, ++T) {
                     const int t0 = it.z + jj * kTok;
+                    if (jj + kPrefetch < ntl)
+                        for (int c = 0; c < kChunks; ++c) tma_prefetch_l2_3d(&tmKV, 64 * c, t0 + kPrefetch * kTok, it.x);
                     for (int c = 0; c < kChunks; ++c) {
                         // the previous tile's PV product has finished with this slot (its O^T block,
                         // or for the last slot the whole product that read P^T there)
@@ -357,6 +364,8 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
                 if (lane == 0) vote[sb * 4 + quarter] = wflag;
                 if (!group_sync(&bar[GRP + wg], uses, a, err)) { ok = false; break; }
                 const bool any_move = (vote[sb * 4 + 0] | vote[sb * 4 + 1] | vote[sb * 4 + 2] | vote[sb * 4 + 3]) != 0;
+                float alpha[kHW];
+                bool rescale_o = false;
                 if (any_move) {
                     // this tile's maximum over its 128 tokens, per head
 #pragma unroll
@@ -367,8 +376,6 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
                         if (lane == 0) red[(sb * 4 + quarter) * kNh + hs + h] = mx;
                     }
                     if (!group_sync(&bar[GRP + wg], uses, a, err)) { ok = false; break; }
-                    float alpha[kHW];
-                    bool rescale_o = false;
 #pragma unroll
                     for (int h = 0; h < kHW; ++h) {
                         const float *rr = red + sb * 4 * kNh + hs + h;
@@ -382,21 +389,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
                             rescale_o = true;
                         }
                     }
-                    // uniform: the warpgroup saw the same maxima.  The previous tile's PV product is
-                    // complete here: this tile's RoPE chunk was loaded into the slot that product
-                    // released, and S^T has read it.
-                    if (rescale_o && jj > 0) {
-#pragma unroll 1
-                        for (int j = 0; j < kLatChunks / 2; ++j) {
-                            uint32_t o[kHW];
-                            tmem_ld32(tmem + j * kNh + lane_off + hs, o);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int h = 0; h < kHW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-                            tmem_st32(tmem + j * kNh + lane_off + hs, o);
-                        }
-                        tmem_wait_st();
-                    }
+                    rescale_o = rescale_o && jj > 0;   // uniform: the warpgroup saw the same maxima
                 }
                 // P^T into the RoPE slot (S^T has read it), MN-major without swizzle: core matrices of
                 // 8 tokens x 8 heads (128 B); the weight sum takes the same bf16-rounded values
@@ -412,6 +405,20 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
                         l_part[h + 1] += bf16_hi(w[e]);
                     }
                     *reinterpret_cast<uint4 *>(pdst + (hs / 8 + h8) * 2048) = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                // The previous tile's PV product is complete here: this tile's RoPE chunk was loaded into
+                // the slot that product released, and S^T has read it.
+                if (rescale_o) {
+#pragma unroll 1
+                    for (int j = 0; j < kLatChunks / 2; ++j) {
+                        uint32_t o[kHW];
+                        tmem_ld32(tmem + j * kNh + lane_off + hs, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int h = 0; h < kHW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+                        tmem_st32(tmem + j * kNh + lane_off + hs, o);
+                    }
+                    tmem_wait_st();
                 }
                 if (!valid) {
                     // Rows past the piece may hold anything (NaN included) and the tensor cores would

@@ -74,9 +74,11 @@ extern "C" gqa_status gqa_decode_noalloc(const void *q, const void *k_cache, con
     // partials), so nothing in it has to start at zero.
     const DecodePlan p = decode_plan_host(B, Hq, Hkv, Tmax, num_sms, kScratchBytes - (size_t(1) << 20));
     if (p.ws_bytes > kScratchBytes) return GQA_ERR_UNSUPPORTED;
+    int *status = device_status_word();
+    if (!status) return GQA_ERR_CUDA;
     int launches = 0;
     s = static_cast<gqa_status>(decode_enqueue(q, k_cache, v_cache, seqlens, B, Hq, Hkv, Tmax, scale, out,
-                                               p.ws_bytes ? scratch : nullptr, p, num_sms, device_status_word(),
+                                               p.ws_bytes ? scratch : nullptr, p, num_sms, status,
                                                static_cast<cudaStream_t>(stream), &launches, nullptr, nullptr));
     set_last_launch_count(launches);
     return s;

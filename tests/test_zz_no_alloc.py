@@ -31,27 +31,69 @@ def _call_noalloc(lib, x, out):
                                   ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-@pytest.mark.parametrize("shape", [
+SHAPES = [
     # (B, Hq, Hkv, Tmax, seqlens): the second splits the history, so the scratch really holds partials
     (1, 8, 2, 256, None),
     (8, 32, 8, 8192, [8192, 8000, 4097, 64, 1, 0, 3000, 8191]),
     (3, 32, 2, 20000, [20000, 12345, 777]),
-], ids=["tiny", "split-8x8192", "group16-split"])
-def test_matches_gqa_decode_on_two_calls_in_a_row(shape):
+    # the CUDA-core kernel's group sizes: MHA and groups of two, each split over several pieces
+    (2, 16, 16, 12000, [12000, 5000]),
+    (2, 16, 8, 12000, [11999, 130]),
+]
+IDS = ["tiny", "split-8x8192", "group16-split", "mha-split", "group2-split"]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=IDS)
+def test_matches_gqa_decode_and_the_oracle_on_two_calls_in_a_row(oracle_mod, shape):
     B, Hq, Hkv, Tmax, lens = shape
     lib = gqa.load()
     x = inputs.make_decode(B, Hq, Hkv, 128, Tmax, seqlens=lens, device=DEV, seed=77)
     ref = gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
     torch.cuda.synchronize()
     ref64 = ref.double().cpu().numpy()
+    exact = oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens.cpu(), x.scale)
     for call in range(2):
         out = torch.full_like(x.q, float("nan"))
         assert _call_noalloc(lib, x, out) == 0
         torch.cuda.synchronize()
         assert gqa.gqa_get_last_device_status() == 0
-        assert_close(out.double().cpu().numpy(), ref64)
+        got = out.double().cpu().numpy()
+        assert_close(got, ref64)      # the existing entry point, at the decode gates
+        assert_close(got, exact)      # and the fp64 oracle directly
     if B == 8:
         assert gqa.gqa_decode_plan(B, Hq, Hkv, 128, Tmax, torch.cuda.get_device_properties(0).multi_processor_count)[1] > 1
+
+
+def test_allocates_nothing(oracle_mod):
+    """With the library's workspace handed back and an allocator installed that refuses every request,
+    the call still succeeds (it never asks), device memory does not change, and the result is right."""
+    lib = gqa.load()
+    x = inputs.make_decode(4, 32, 4, 128, 9000, seqlens=[9000, 8191, 33, 4500], device=DEV, seed=78)
+    out = torch.full_like(x.q, float("nan"))
+    torch.cuda.synchronize()
+    gqa.gqa_release()
+    asked = []
+    gqa.gqa_set_workspace_allocator(lambda n, dev: asked.append(n) or 0, lambda p, n, dev: None)
+    try:
+        # the first call of a fresh process also loads the kernels' code (the driver's doing, not an
+        # allocation by the library), so free memory is sampled after it
+        assert _call_noalloc(lib, x, out) == 0
+        torch.cuda.synchronize()
+        free0, _ = torch.cuda.mem_get_info()
+        for _ in range(2):
+            assert _call_noalloc(lib, x, out) == 0
+            torch.cuda.synchronize()
+        free1, _ = torch.cuda.mem_get_info()
+        assert asked == []
+        assert free1 == free0
+        assert gqa.gqa_get_last_device_status() == 0
+        # the library's own entry point does ask, and is refused
+        with pytest.raises(gqa.GQAError):
+            gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale)
+        assert asked
+    finally:
+        gqa.gqa_set_workspace_allocator(None, None)
+    assert_close(out.double().cpu().numpy(), oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens.cpu(), x.scale))
 
 
 def test_rejects_partials_larger_than_the_fixed_scratch():
