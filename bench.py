@@ -438,6 +438,70 @@ def mla_only(gqa, torch, inputs, workloads, args):
                       "device_status": gqa.gqa_get_last_device_status()}))
 
 
+def tp_bench(gqa, torch, inputs, args, w, world: int, rank: int, local_rank: int):
+    """Tensor-parallel decode of one layer over `world` ranks (one per GPU, NCCL): each rank keeps its head
+    shard (a replica of its KV head when Hkv < world), decodes it and all-gathers the outputs in head order.
+    Total work is fixed as ranks are added ("strong"); value = the layer's unique KV bytes over the slowest
+    rank's step time.  Ranks that hold replicas read the same KV head, so bytes read over all ranks exceed
+    the unique bytes; both are reported."""
+    import datetime
+
+    import torch.distributed as dist
+
+    from grouped_query_attention_02_b200 import tp as tpmod
+
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        # every rank draws the same layer and keeps its shard, as a rank of a deployment holds only its own
+        x = inputs.make_decode(w.B, w.Hq, w.Hkv, w.d, w.Tmax, device="cuda", seed=0, seqlen_range=w.seqlen_range)
+        shard = tpmod.tp_shard(w.Hq, w.Hkv, world, rank)
+        qs, ks, vs = tpmod.take_shard(x.q, x.k_cache, x.v_cache, shard)
+        sl, scale = x.seqlens, x.scale
+        lens = sl.cpu().tolist()
+        del x
+        torch.cuda.empty_cache()
+        U = unique_kv_bytes(lens, w.Hkv, w.d)
+        read_all = unique_kv_bytes(lens, shard.kv_count, w.d) * world
+        step = lambda: tpmod.tp_decode(qs, ks, vs, sl, scale, world)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0, s1 = _events(torch)
+        with ClockSampler(local_rank) as clk:
+            time.sleep(0.25)
+            s0.record()
+            for _ in range(args.steps):
+                out = step()
+            s1.record()
+            torch.cuda.synchronize()
+        ms = s0.elapsed_time(s1) / args.steps
+        if world > 1:
+            dist.barrier()
+            t = torch.tensor([ms], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        ms_max = ms
+        if rank == 0:
+            print(json.dumps({
+                "metric": METRIC + " (tensor-parallel)", "value": U / (ms_max * 1e-3) / 1e9, "unit": "GB/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+                "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic",
+                "config": {"workload": w.name, "parallelism": f"tp{world} (head shards; KV heads replicated when "
+                                                              f"Hkv < tp; outputs all-gathered over NCCL)",
+                           "q_heads_per_rank": shard.q_count, "kv_heads_per_rank": shard.kv_count},
+                "bytes_read_all_ranks": read_all, "unique_kv_bytes": U,
+                "tokens_per_s": w.B / (ms_max * 1e-3), "out_shape": list(out.shape),
+                "clocks": clk.summary(), "device_status": gqa.gqa_get_last_device_status()}))
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -453,6 +517,9 @@ def main():
     ap.add_argument("--prefill-batch", type=int, default=4, help="sequences in --mode prefill")
     ap.add_argument("--decode-workload", default="Qwen3-8B",
                     help="name prefix of the decode workload timed as the headline (profiling other rows)")
+    ap.add_argument("--tp", action="store_true",
+                    help="tensor-parallel decode of the workload over WORLD_SIZE ranks (head shards, outputs "
+                         "all-gathered) instead of the batch-sharded default")
     ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16",
                     help="fp8: the headline decode over an FP8 (E4M3) cache with per-tensor scales")
     args = ap.parse_args()
@@ -513,6 +580,9 @@ def main():
         return
     if args.mode == "mla":
         mla_only(gqa, torch, inputs, workloads, args)
+        return
+    if args.tp:
+        tp_bench(gqa, torch, inputs, args, w, max(world, 1), rank, local_rank)
         return
     if args.mode == "backward":
         pw = workloads.CAUSAL_PREFILL

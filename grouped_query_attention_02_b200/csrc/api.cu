@@ -450,6 +450,22 @@ static gqa_status encode_3d(CUtensorMap *tm, const void *base, uint64_t n0, uint
     return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_CUDA;
 }
 
+// A [n2][rows][576] bf16 tensor viewed as (64 columns, rows, 9 column chunks, n2): the chunk index is
+// outside the row index, so one box {64, box_rows, chunks, 1} lands in shared memory as `chunks`
+// consecutive tiles of box_rows x 64 columns (128-byte swizzle), the layout the MMA descriptors read.
+static gqa_status encode_chunk_view(CUtensorMap *tm, const void *base, uint64_t rows, uint64_t n2, uint32_t box_rows,
+                                    uint32_t chunks)
+{
+    cuuint64_t dims[4] = {64, rows, (cuuint64_t)(kMlaRow / 64), n2};
+    cuuint64_t strides[3] = {(cuuint64_t)kMlaRow * 2, 128, rows * kMlaRow * 2};
+    cuuint32_t box[4] = {64, box_rows, chunks, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? GQA_OK : GQA_ERR_CUDA;
+}
+
 gqa_status gqa_mla_decode(const void *q, const void *kv_cache, const int32_t *seqlens, int B, int Hq, int d_c,
                           int d_r, int Tmax, float scale, void *out, void *stream)
 {
@@ -462,11 +478,12 @@ gqa_status gqa_mla_decode(const void *q, const void *kv_cache, const int32_t *se
     if ((s = get_encoder()) != GQA_OK) return s;
     const MlaTcPlan p = mla_tc_plan_host(B, Hq, Tmax, kWorkspaceBudget);
     if ((s = ensure_workspace(st, p.ws_bytes)) != GQA_OK) return s;
-    CUtensorMap tmKV, tmQ;
-    if ((s = encode_3d(&tmKV, kv_cache, kMlaRow, Tmax, B, 128)) != GQA_OK) return s;
-    if ((s = encode_3d(&tmQ, q, kMlaRow, Hq, B, 64)) != GQA_OK) return s;
+    CUtensorMap tmKV2, tmKV1, tmQ;
+    if ((s = encode_chunk_view(&tmKV2, kv_cache, Tmax, B, 128, 2)) != GQA_OK) return s;
+    if ((s = encode_3d(&tmKV1, kv_cache, kMlaRow, Tmax, B, 128)) != GQA_OK) return s;
+    if ((s = encode_chunk_view(&tmQ, q, Hq, B, 64, kMlaRow / 64)) != GQA_OK) return s;
     int n = 0;
-    const cudaError_t e = launch_mla_decode_tc(tmKV, tmQ, q, seqlens, B, Hq, Tmax, scale, out, st->ws, p,
+    const cudaError_t e = launch_mla_decode_tc(tmKV2, tmKV1, tmQ, q, seqlens, B, Hq, Tmax, scale, out, st->ws, p,
                                                st->num_sms, st->status, kWaitBudgetNs,
                                                static_cast<cudaStream_t>(stream), &n, g_ev_before, g_ev_after);
     g_last_launches = n;

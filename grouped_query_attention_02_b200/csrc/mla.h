@@ -57,10 +57,14 @@ struct MlaTcPlan {
 MlaTcPlan mla_tc_plan_host(int B, int Hq, int Tmax, size_t ws_budget);
 
 // Enqueues the planner, the decode and the combine on `stream` (three launches, added to
-// *launches); tmKV maps kv_cache [B, Tmax, 576] with box {64, 128, 1}, tmQ maps q [B, Hq, 576]
-// with box {64, 64, 1}, both bf16 with the 128-byte swizzle.  `before` / `after`, when non-null,
-// are recorded around the decode kernel.
-cudaError_t launch_mla_decode_tc(const CUtensorMap &tmKV, const CUtensorMap &tmQ, const void *q,
+// *launches).  Tensor maps, all bf16 with the 128-byte swizzle:
+//   tmKV2: kv_cache [B, Tmax, 576] viewed as (64 columns, Tmax, 9 column chunks, B), box {64, 128, 2, 1}
+//          (two consecutive 128-token x 64-column chunk tiles);
+//   tmKV1: kv_cache as (576, Tmax, B), box {64, 128, 1} (one chunk tile: the RoPE key);
+//   tmQ:   q [B, Hq, 576] viewed as (64 columns, Hq, 9 column chunks, B), box {64, 64, 9, 1}.
+// `before` / `after`, when non-null, are recorded around the decode kernel.
+cudaError_t launch_mla_decode_tc(const CUtensorMap &tmKV2, const CUtensorMap &tmKV1, const CUtensorMap &tmQ,
+                                 const void *q,
                                  const int32_t *seqlens, int B, int Hq, int Tmax, float scale, void *out, void *ws,
                                  const MlaTcPlan &p, int num_sms, int *status, unsigned long long wait_budget_ns,
                                  cudaStream_t stream, int *launches, cudaEvent_t before, cudaEvent_t after);

@@ -55,13 +55,15 @@ constexpr int kNWG = 2;                           // softmax / epilogue warpgrou
 constexpr int kHW = kNh / kNWG;                   // heads per warpgroup (32)
 constexpr int kProducerWarp = 4 * kNWG;
 constexpr int kMmaWarp = kProducerWarp + 1;
-constexpr int kThreads = kWG * kNWG + 64;
+constexpr int kPrefetchWarp = kMmaWarp + 1;       // keeps the tiles kAhead ahead of the producer in L2
+constexpr int kThreads = kWG * kNWG + 96;
+constexpr int kAhead = 2;
 constexpr int kQD = 4;                            // depth of the unit queue
 constexpr float kMoveThreshold = 8.0f;            // the running maximum moves only by more than this
-constexpr int kPrefetch = 2;                      // tiles prefetched into L2 ahead of their load
+constexpr int kGroups = kLatChunks / 2 + 1;       // loads per tile: four latent chunk pairs, then the RoPE chunk
 
 // barrier slots
-enum : int { CH_FULL = 0, EMPTY_PAIR = CH_FULL + kChunks, EMPTY_P = EMPTY_PAIR + kLatChunks / 2, S_FULL, P_FULL,
+enum : int { CH_FULL = 0, EMPTY_PAIR = CH_FULL + kGroups, EMPTY_P = EMPTY_PAIR + kLatChunks / 2, S_FULL, P_FULL,
              Q_FULL, Q_EMPTY, O_FULL, O_FREE, I_FULL, I_EMPTY = I_FULL + kQD, DRAIN = I_EMPTY + kQD, GRP,
              kBars = GRP + kNWG };
 
@@ -75,6 +77,7 @@ constexpr int kQueueOff = kVoteOff + kNWG * 8 * 4;           // kQD units of 8 i
 constexpr int kBarOff = kQueueOff + kQD * 32;
 constexpr int kTmemOff = kBarOff + kBars * 8;
 constexpr int kErrOff = kTmemOff + 8;
+constexpr int kIssuedOff = kErrOff + 4;                      // tiles the producer has issued (for the prefetcher)
 constexpr int kSmemBytes = kErrOff + 8;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 static_assert(kNh * kTok * 2 == kChunkBytes, "P^T fills the RoPE chunk's slot exactly");
@@ -134,8 +137,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_constant__ CUtensorMap tmQ,
-                     const MlaTcArgs a)
+mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV2, const __grid_constant__ CUtensorMap tmKV1,
+                     const __grid_constant__ CUtensorMap tmQ, const MlaTcArgs a)
 {
     // the 128-byte swizzle needs 1024-byte aligned chunks; a misaligned window is reported
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -151,7 +154,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
     volatile int *queue = reinterpret_cast<volatile int *>(smem + kQueueOff);
 
     if (threadIdx.x == 0) {
-        for (int c = 0; c < kChunks; ++c) mbar_init(&bar[CH_FULL + c], 1);
+        for (int g = 0; g < kGroups; ++g) mbar_init(&bar[CH_FULL + g], 1);
         for (int j = 0; j < kLatChunks / 2; ++j) mbar_init(&bar[EMPTY_PAIR + j], 1);
         mbar_init(&bar[EMPTY_P], 1);
         mbar_init(&bar[S_FULL], 1);
@@ -162,11 +165,12 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
         mbar_init(&bar[O_FREE], kWG * kNWG);
         for (int s = 0; s < kQD; ++s) {
             mbar_init(&bar[I_FULL + s], 1);
-            mbar_init(&bar[I_EMPTY + s], 1 + kWG * kNWG);   // the MMA issuer and the softmax threads
+            mbar_init(&bar[I_EMPTY + s], 2 + kWG * kNWG);   // the MMA issuer, the prefetcher, the softmax threads
         }
         mbar_init(&bar[DRAIN], 1);
         for (int w = 0; w < kNWG; ++w) mbar_init(&bar[GRP + w], kWG);
         *err = 0;
+        *reinterpret_cast<volatile int *>(smem + kIssuedOff) = 0;
         fence_barrier_init();
     }
     if (warp == kMmaWarp) {
@@ -186,12 +190,13 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
     if (warp == kProducerWarp) {
         // ---------------- claims units, loads the block's query rows, streams the tiles chunk by chunk
         if (lane == 0) {
-            tma_prefetch_desc(&tmKV);
+            tma_prefetch_desc(&tmKV2);
+            tma_prefetch_desc(&tmKV1);
             tma_prefetch_desc(&tmQ);
             const int units = a.plan_hdr[1] * a.nhb;
             int icount = 0, T = 0;
-            // for the drain: tiles whose chunks were all issued, chunks issued of the tile after them
-            int full_tiles = 0, part_chunks = 0, q_loads = 0;
+            // for the drain: tiles whose loads were all issued, loads issued of the tile after them
+            int full_tiles = 0, part_groups = 0, q_loads = 0;
             bool ok = true;
             while (ok) {
                 const int u = atomicAdd(a.claim, 1);
@@ -213,44 +218,80 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
                 mbar_arrive(&bar[I_FULL + slot]);
                 // the previous unit's last S^T product has read the query rows
                 if (icount >= 1 && !wait_or_fail(&bar[Q_EMPTY], (icount - 1) & 1, a, err)) break;
+                // one box: the block's 64 query rows as 9 chunk tiles of 64 columns
                 mbar_arrive_expect_tx(&bar[Q_FULL], kChunks * kQChunkBytes);
-                for (int c = 0; c < kChunks; ++c)
-                    tma_load_3d(smem + kQOff + c * kQChunkBytes, &tmQ, &bar[Q_FULL], 64 * c, kNh * hb, it.x);
+                tma_load_4d(smem + kQOff, &tmQ, &bar[Q_FULL], 0, kNh * hb, 0, it.x);
                 ++q_loads;
                 const int ntl = (it.w - it.z + kTok - 1) / kTok;
-                // the unit's first tiles into L2 now, each later one kPrefetch tiles ahead of its load, so
-                // that a load into a freed slot waits for L2 rather than HBM
-                for (int jp = 0; jp < kPrefetch && jp < ntl; ++jp)
-                    for (int c = 0; c < kChunks; ++c) tma_prefetch_l2_3d(&tmKV, 64 * c, it.z + jp * kTok, it.x);
                 for (int jj = 0; jj < ntl && ok; ++jj, ++T) {
                     const int t0 = it.z + jj * kTok;
-                    if (jj + kPrefetch < ntl)
-                        for (int c = 0; c < kChunks; ++c) tma_prefetch_l2_3d(&tmKV, 64 * c, t0 + kPrefetch * kTok, it.x);
-                    for (int c = 0; c < kChunks; ++c) {
-                        // the previous tile's PV product has finished with this slot (its O^T block,
-                        // or for the last slot the whole product that read P^T there)
-                        const int e = c < kLatChunks ? EMPTY_PAIR + c / 2 : EMPTY_P;
-                        if (T >= 1 && !wait_or_fail(&bar[e], (T - 1) & 1, a, err)) {
+                    for (int g = 0; g < kGroups; ++g) {
+                        // the previous tile's PV product has finished with these slots (its O^T block, or
+                        // for the last slot the whole product that read P^T there)
+                        if (T >= 1 && !wait_or_fail(&bar[g < kGroups - 1 ? EMPTY_PAIR + g : EMPTY_P], (T - 1) & 1,
+                                                    a, err)) {
                             ok = false;
                             break;
                         }
-                        mbar_arrive_expect_tx(&bar[CH_FULL + c], kChunkBytes);
-                        tma_load_3d(smem + kSlotOff + c * kChunkBytes, &tmKV, &bar[CH_FULL + c], 64 * c, t0, it.x);
-                        part_chunks = c + 1;
+                        // TMA costs about the same per instruction up to 32 KB, so the latent chunks come in
+                        // pairs (one box of the chunk-outer view); the RoPE chunk alone
+                        uint8_t *dst = smem + kSlotOff + 2 * g * kChunkBytes;
+                        if (g < kGroups - 1) {
+                            mbar_arrive_expect_tx(&bar[CH_FULL + g], 2 * kChunkBytes);
+                            tma_load_4d(dst, &tmKV2, &bar[CH_FULL + g], 0, t0, 2 * g, it.x);
+                        } else {
+                            mbar_arrive_expect_tx(&bar[CH_FULL + g], kChunkBytes);
+                            tma_load_3d(dst, &tmKV1, &bar[CH_FULL + g], kMlaLatent, t0, it.x);
+                        }
+                        part_groups = g + 1;
                     }
-                    if (part_chunks == kChunks) {
+                    if (part_groups == kGroups) {
                         ++full_tiles;
-                        part_chunks = 0;
+                        part_groups = 0;
+                        *reinterpret_cast<volatile int *>(smem + kIssuedOff) = full_tiles;
                     }
                 }
                 ++icount;
             }
             // leave no copy in flight
-            for (int c = 0; c < kChunks; ++c) {
-                const int n = full_tiles + (c < part_chunks ? 1 : 0);   // loads issued into slot c
-                if (n >= 1) mbar_wait(&bar[CH_FULL + c], (n - 1) & 1, a.wait_budget_ns);
+            for (int g = 0; g < kGroups; ++g) {
+                const int n = full_tiles + (g < part_groups ? 1 : 0);   // loads issued for group g
+                if (n >= 1) mbar_wait(&bar[CH_FULL + g], (n - 1) & 1, a.wait_budget_ns);
             }
             if (q_loads >= 1) mbar_wait(&bar[Q_FULL], (q_loads - 1) & 1, a.wait_budget_ns);
+        }
+    } else if (warp == kPrefetchWarp) {
+        // ---------------- L2 prefetcher: tile T of the CTA's stream goes to L2 once the producer has issued
+        // tile T - kAhead, so that the producer's loads find their tiles in L2 rather than HBM.  It only
+        // reads the unit queue and the producer's count; nothing waits for it.
+        if (lane == 0) {
+            volatile int *issued = reinterpret_cast<volatile int *>(smem + kIssuedOff);
+            int icount = 0, T = 0;
+            bool ok = true;
+            while (ok) {
+                const int slot = icount % kQD;
+                if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
+                volatile int *q = queue + slot * 8;
+                const int b = q[0], t_begin = q[3], t_end = q[4];
+                mbar_arrive(&bar[I_EMPTY + slot]);
+                if (t_end < 0) break;
+                const int ntl = (t_end - t_begin + kTok - 1) / kTok;
+                for (int jj = 0; jj < ntl; ++jj, ++T) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (*issued < T - kAhead + 1) {
+                        if (*err || global_timer_ns() - t0 > a.wait_budget_ns) {
+                            ok = false;   // the producer stopped: nothing more to prefetch
+                            break;
+                        }
+                        __nanosleep(200);
+                    }
+                    if (!ok) break;
+                    const int tt = t_begin + jj * kTok;
+                    for (int g = 0; g < kGroups - 1; ++g) tma_prefetch_l2_4d(&tmKV2, 0, tt, 2 * g, b);
+                    tma_prefetch_l2_3d(&tmKV1, kMlaLatent, tt, b);
+                }
+                ++icount;
+            }
         }
     } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer: S^T over the 9 chunks, then (once P^T is written) the PV blocks
@@ -274,7 +315,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
                 for (int jj = 0; jj < ntl; ++jj, ++T) {
                     // S^T = KV . Q^T, K = 576 in 36 steps of 16, chunk by chunk as they land
                     for (int c = 0; c < kChunks && ok; ++c) {
-                        if (!wait_or_fail(&bar[CH_FULL + c], T & 1, a, err)) {
+                        if ((c & 1) == 0 && !wait_or_fail(&bar[CH_FULL + c / 2], T & 1, a, err)) {
                             ok = false;
                             break;
                         }
@@ -427,7 +468,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV, const __grid_cons
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const int ch = wg * 4 + c;
-                        if (!wait_or_fail(&bar[CH_FULL + ch], T & 1, a, err)) { ok = false; break; }
+                        if (!wait_or_fail(&bar[CH_FULL + ch / 2], T & 1, a, err)) { ok = false; break; }
                         uint4 *row = reinterpret_cast<uint4 *>(smem + kSlotOff + ch * kChunkBytes + t * 128);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) row[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -556,7 +597,8 @@ MlaTcPlan mla_tc_plan_host(int B, int Hq, int Tmax, size_t ws_budget)
     return p;
 }
 
-cudaError_t launch_mla_decode_tc(const CUtensorMap &tmKV, const CUtensorMap &tmQ, const void *q,
+cudaError_t launch_mla_decode_tc(const CUtensorMap &tmKV2, const CUtensorMap &tmKV1, const CUtensorMap &tmQ,
+                                 const void *q,
                                  const int32_t *seqlens, int B, int Hq, int Tmax, float scale, void *out, void *ws,
                                  const MlaTcPlan &p, int num_sms, int *status, unsigned long long wait_budget_ns,
                                  cudaStream_t stream, int *launches, cudaEvent_t before, cudaEvent_t after)
@@ -621,7 +663,7 @@ cudaError_t launch_mla_decode_tc(const CUtensorMap &tmKV, const CUtensorMap &tmQ
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (before) cudaEventRecord(before, stream);
-    if ((e = cudaLaunchKernelEx(&cfg, mla_decode_tc_kernel, tmKV, tmQ, a)) != cudaSuccess) return e;
+    if ((e = cudaLaunchKernelEx(&cfg, mla_decode_tc_kernel, tmKV2, tmKV1, tmQ, a)) != cudaSuccess) return e;
     if (after) cudaEventRecord(after, stream);
     ++*launches;
 

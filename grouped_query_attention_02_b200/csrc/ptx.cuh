@@ -122,6 +122,15 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *tm, int c0
                  : "memory");
 }
 
+// Prefetch of one 4-D box into L2.
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap *tm, int c0, int c1, int c2, int c3)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
 // 4-D tiled load of one box into shared memory, completing `bytes` on bar.
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *tm, uint64_t *bar, int c0, int c1, int c2,
                                             int c3)

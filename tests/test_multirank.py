@@ -7,10 +7,11 @@ decodes its own sequences.  Checked here without a GPU:
   batch in one place: sharding by sequence needs no collective on the data path;
 * the step time reported is the maximum over ranks and the value is all ranks'
   bytes over that time (bench.aggregate);
-* tensor-parallel head sharding (gqa_tp_shard): each rank decodes its own query
-  heads against its KV heads, or its replica of one, and the ranks' outputs put
-  back in head order equal the unsharded decode -- with KV heads partitioned
-  (2 ranks) and replicated (4 ranks).
+* tensor-parallel head sharding (tp.py over gqa_tp_shard, the rank logic of
+  bench.py --tp): each rank decodes its own query heads against its KV heads, or
+  its replica of one, and the all-gather puts the outputs back in head order,
+  equal to the unsharded decode -- with KV heads partitioned (2 and 4 ranks, MHA
+  included) and replicated (4 ranks).
 """
 from __future__ import annotations
 
@@ -106,30 +107,28 @@ def _tp_worker(rank, world, port, out_dir, Hq, Hkv):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         import oracle
-        import grouped_query_attention_02_b200 as gqa
-        from grouped_query_attention_02_b200 import inputs
+        from grouped_query_attention_02_b200 import inputs, tp
 
-        # every rank sees the same layer; it keeps only its shard (the CPU oracle stands in for the
-        # rank's GPU decode of that shard)
+        # the rank logic of bench.py --tp: every rank draws the same layer, keeps only its shard, decodes
+        # it and all-gathers the outputs in head order (the CPU oracle stands in for the rank's GPU decode)
         x = inputs.make_decode(2, Hq, Hkv, 16, 20, seqlens=[20, 7], device="cpu", seed=41)
-        qf, qc, kf, kc = gqa.gqa_tp_shard(Hq, Hkv, world, rank)
-        q = x.q[:, qf:qf + qc].contiguous()
-        k = x.k_cache[:, :, kf:kf + kc].contiguous()
-        v = x.v_cache[:, :, kf:kf + kc].contiguous()
-        out = torch.from_numpy(oracle.decode(q, k, v, x.seqlens, x.scale, nthreads=1))
-        parts = [torch.zeros_like(out) for _ in range(world)]
-        dist.all_gather(parts, out)
+        shard = tp.tp_shard(Hq, Hkv, world, rank)
+        qs, ks, vs = tp.take_shard(x.q, x.k_cache, x.v_cache, shard)
+        assert ks.shape[2] == shard.kv_count and qs.shape[1] == Hq // world
+
+        def cpu_decode(q, k, v, seqlens, scale):
+            return torch.from_numpy(oracle.decode(q, k, v, seqlens, scale, nthreads=1))
+
+        whole = tp.tp_decode(qs, ks, vs, x.seqlens, x.scale, world, decode=cpu_decode)
         if rank == 0:
-            whole = torch.zeros(2, Hq, 16, dtype=torch.float64)
-            for r in range(world):
-                f, c, _, _ = gqa.gqa_tp_shard(Hq, Hkv, world, r)
-                whole[:, f:f + c] = parts[r]
             np.save(os.path.join(out_dir, "tp.npy"), whole.numpy())
+            np.save(os.path.join(out_dir, "shards.npy"),
+                    np.array([tuple(tp.tp_shard(Hq, Hkv, world, r)) for r in range(world)]))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,Hq,Hkv", [(2, 8, 2), (4, 8, 2), (4, 8, 1)])
+@pytest.mark.parametrize("world,Hq,Hkv", [(2, 8, 2), (4, 8, 2), (4, 8, 1), (4, 16, 8), (2, 8, 8)])
 def test_tensor_parallel_shards_reassemble_the_decode(tmp_path, world, Hq, Hkv):
     import oracle
     from grouped_query_attention_02_b200 import build, inputs
@@ -141,4 +140,8 @@ def test_tensor_parallel_shards_reassemble_the_decode(tmp_path, world, Hq, Hkv):
     got = np.load(tmp_path / "tp.npy")
     x = inputs.make_decode(2, Hq, Hkv, 16, 20, seqlens=[20, 7], device="cpu", seed=41)
     np.testing.assert_array_equal(got, oracle.decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, nthreads=1))
+    shards = np.load(tmp_path / "shards.npy")
+    # every query head owned once, in rank order; replicas when there are fewer KV heads than ranks
+    assert shards[:, 0].tolist() == list(range(0, Hq, Hq // world))
+    assert (shards[:, 3] == max(1, Hkv // world)).all()
 
