@@ -83,6 +83,7 @@ def load_peaks():
 
 DECODE_SOURCES = ("decode.cu", "decode_tc.cu", "ptx.cuh", "internal.h")
 PREFILL_SOURCES = ("prefill.cu", "ptx.cuh", "internal.h")
+MLA_SOURCES = ("mla_tc.cu", "ptx.cuh", "internal.h", "mla.h")
 
 
 def kernel_source_digest(files=DECODE_SOURCES) -> str:
@@ -393,13 +394,14 @@ def prefill_only(gqa, torch, inputs, workloads, args):
     """Time the causal prefill workload alone (B sequences of 8192 tokens, 32/8 heads, d=128)."""
     pw = workloads.CAUSAL_PREFILL
     peaks = load_peaks()
-    p = inputs.make_prefill(args.prefill_batch, pw.S, pw.Hq, pw.Hkv, pw.d, device="cuda", seed=0)
+    hq, hkv = (int(v) for v in args.prefill_heads.split(":"))
+    p = inputs.make_prefill(args.prefill_batch, pw.S, hq, hkv, pw.d, device="cuda", seed=0)
     st_ms, k_ms, n = time_prefill(gqa, torch, p, args.steps, args.warmup)
-    fl = prefill_causal_flops(args.prefill_batch, pw.S, pw.Hq, pw.d)
+    fl = prefill_causal_flops(args.prefill_batch, pw.S, hq, pw.d)
     print(json.dumps({"metric": "causal GQA prefill TFLOP/s", "value": fl / (st_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                       "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": st_ms,
                       "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
-                      "config": {"workload": pw.name, "B": args.prefill_batch},
+                      "config": {"workload": pw.name, "B": args.prefill_batch, "Hq": hq, "Hkv": hkv},
                       "roofline": {"bound": "tensor", "achieved": fl / (k_ms * 1e-3) / 1e12,
                                    "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                    "frac": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]},
@@ -417,7 +419,8 @@ def mla_roofline(peaks, mw, st_ms, k_ms):
         "unique_kv_GBps": by / (st_ms * 1e-3) / 1e9, "tokens_per_s": mw.B / (st_ms * 1e-3),
         "roofline": {"bound": "tensor", "achieved": fl / (k_ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
-                     "traffic": None, "hbm_frac": by / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                     "traffic": profile_traffic("mla_decode_deepseek_b32.md", MLA_SOURCES),
+                     "hbm_frac": by / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                      "frac_of_bound": t_bound / (k_ms * 1e-3), "bound_ms": t_bound * 1e3,
                      "peak_source": f"{peaks.get('source')} bf16_tflops (cuBLAS burst), hbm_gbs"},
         "flop_count": "2 Hq (2 d_c + d_r) per cached token; bytes: the cache once, q in, out",
@@ -515,6 +518,7 @@ def main():
                     help="prefill / backward / mla: time only the causal prefill workload's forward / backward, "
                          "or the MLA decode workload (used for their ncu captures)")
     ap.add_argument("--prefill-batch", type=int, default=4, help="sequences in --mode prefill")
+    ap.add_argument("--prefill-heads", default="32:8", help="Hq:Hkv of --mode prefill (e.g. 24:8 for an odd group)")
     ap.add_argument("--decode-workload", default="Qwen3-8B",
                     help="name prefix of the decode workload timed as the headline (profiling other rows)")
     ap.add_argument("--tp", action="store_true",
@@ -755,6 +759,22 @@ def main():
                                           "peak_source": f"{peaks.get('source')} bf16_tflops (cuBLAS burst)"}}
         except gqa.GQAError as e:
             rows[pw.name] = {"error": str(e)}
+        # the same prefill with an odd group (24 query / 8 KV heads, g = 3): the single-head kernel
+        try:
+            name = "causal GQA prefill, odd group B4 S8192 Hq24 Hkv8 d128"
+            p = inputs.make_prefill(pw.B, pw.S, 24, 8, pw.d, device="cuda", seed=0)
+            st_ms, k_ms, n = time_prefill(gqa, torch, p, 10, 3)
+            fl = prefill_causal_flops(pw.B, pw.S, 24, pw.d)
+            rows[name] = {"ms_per_step": st_ms, "kernel_ms": k_ms, "TFLOPs": fl / (st_ms * 1e-3) / 1e12,
+                          "kernel": "prefill_causal_kernel (one head per CTA)",
+                          "roofline": {"bound": "tensor", "achieved": fl / (k_ms * 1e-3) / 1e12,
+                                       "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                       "frac": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], "traffic": None,
+                                       "peak_source": f"{peaks.get('source')} bf16_tflops (cuBLAS burst)"}}
+            del p
+            torch.cuda.empty_cache()
+        except gqa.GQAError as e:
+            rows["causal GQA prefill, odd group"] = {"error": str(e)}
         # causal prefill backward (dq, and dk / dv summed over each group)
         try:
             p = inputs.make_prefill(pw.B, pw.S, pw.Hq, pw.Hkv, pw.d, device="cuda", seed=0)
