@@ -759,14 +759,14 @@ def main():
                                           "peak_source": f"{peaks.get('source')} bf16_tflops (cuBLAS burst)"}}
         except gqa.GQAError as e:
             rows[pw.name] = {"error": str(e)}
-        # the same prefill with an odd group (24 query / 8 KV heads, g = 3): the single-head kernel
+        # the same prefill with an odd group (24 query / 8 KV heads, g = 3): query tiles 2k, 2k+1 of one head per CTA
         try:
             name = "causal GQA prefill, odd group B4 S8192 Hq24 Hkv8 d128"
             p = inputs.make_prefill(pw.B, pw.S, 24, 8, pw.d, device="cuda", seed=0)
             st_ms, k_ms, n = time_prefill(gqa, torch, p, 10, 3)
             fl = prefill_causal_flops(pw.B, pw.S, 24, pw.d)
             rows[name] = {"ms_per_step": st_ms, "kernel_ms": k_ms, "TFLOPs": fl / (st_ms * 1e-3) / 1e12,
-                          "kernel": "prefill_causal_kernel (one head per CTA)",
+                          "kernel": "prefill_pair_kernel, query-tile pairs (odd group)",
                           "roofline": {"bound": "tensor", "achieved": fl / (k_ms * 1e-3) / 1e12,
                                        "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                                        "frac": fl / (k_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], "traffic": None,

@@ -1,33 +1,19 @@
 // prefill.cu -- causal GQA prefill on the tcgen05 tensor cores.
 //
-// One CTA computes one 128-row query tile of one (sequence, query head).  The
+// One CTA computes two 128-row query tiles that read the same KV head: the
 // query head h reads KV head h / g ("grouped-query and multi-query attention",
-// study.greatitself.com: consecutive groups); K/V tiles are fetched by TMA and
-// the g query heads of a group run as neighbouring CTAs so that a tile read
-// from HBM serves the whole group out of L2.  The causal mask of
-// anrans.github.io attention-variants ("Kernels do not need to copy the KV
-// heads": lower triangle, diagonal included) is applied inside the diagonal
-// tile only; tiles above the diagonal are never visited.
-//
-// Warp roles (192 threads):
-//   warp 0      TMA producer: the Q tile once, then K_j / V_j into a two-stage ring
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
-//               S_j = Q K_j^T into one of two TMEM buffers, O += P_j V_j into TMEM
-//   warps 2..5  softmax: one query row per thread, read straight from TMEM
-//               (warp w may touch TMEM lanes 32*(w%4) .. +31), online softmax in
-//               base 2 with fp32 state, P_j rounded to bf16 into shared memory,
-//               then the epilogue O / l -> bf16 -> global.
+// study.greatitself.com: consecutive groups), K/V tiles are fetched by TMA once
+// for both, and the CTAs of one group are neighbours so that a tile read from
+// HBM serves the whole group out of L2.  The causal mask of anrans.github.io
+// attention-variants ("Kernels do not need to copy the KV heads": lower
+// triangle, diagonal included) is applied inside the diagonal tile only; tiles
+// above the diagonal are never visited.
 //
 // The running maximum is only moved when a row's new maximum exceeds it by
 // more than 8 (in log2 units); otherwise the weights are taken against the old
 // maximum (they stay below 2^8, exact in fp32) and the O accumulator in TMEM
 // needs no rescale.  The final division by l uses the same maximum, so the
 // result is the same softmax.
-//
-// Shared memory (1024-byte aligned, 128-byte swizzle everywhere):
-//   Q [2 halves][128 rows][128 B]  32 KB
-//   K [2 stages][2 halves][128][128 B]  64 KB,  V likewise 64 KB
-//   P [2 halves][128 rows][128 B]  32 KB
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -40,28 +26,9 @@ constexpr int kBM = 128;                   // query rows per CTA
 constexpr int kBN = 128;                   // keys per KV tile
 constexpr int kTileBytes = kBM * kD * 2;   // 32 KB: one 128 x 128 bf16 tile
 constexpr int kHalfTile = kTileBytes / 2;  // one 64-column half
-constexpr int kThreads = 192;
 constexpr int kSoftmaxThreads = 128;
 constexpr uint32_t kTmemCols = 512;        // S0, S1, O (128 columns each), rounded to a power of two
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-
-struct Smem {
-    static constexpr int q = 0;
-    static constexpr int k = q + kTileBytes;
-    static constexpr int v = k + 2 * kTileBytes;
-    static constexpr int p = v + 2 * kTileBytes;
-    static constexpr int bars = p + kTileBytes;
-    // barriers: q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], s_free[2], p_full, p_free, o_full, drain
-    static constexpr int nbars = 15;
-    static constexpr int tmem_slot = bars + nbars * 8;
-    static constexpr int err = tmem_slot + 8;
-    static constexpr int bytes = err + 8;
-};
-
-enum Bar {
-    Q_FULL = 0, K_FULL = 1, V_FULL = 3, KV_EMPTY = 5, S_FULL = 7, S_FREE = 9,
-    P_FULL = 11, P_FREE = 12, O_FULL = 13, DRAIN = 14
-};
 
 __device__ __forceinline__ void record_status(int *status, int code)
 {
@@ -107,274 +74,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
-prefill_causal_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, const PrefillArgs a)
-{
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + Smem::bars);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Smem::tmem_slot);
-    volatile int *err = reinterpret_cast<volatile int *>(smem + Smem::err);
-
-    // heaviest query tiles first over the whole grid; a group's heads are neighbours
-    const int nqt = (a.S + kBM - 1) / kBM;
-    const int bh_count = a.B * a.Hq;
-    const int id = blockIdx.x;
-    const int qt = nqt - 1 - id / bh_count;
-    const int bh = id % bh_count;
-    const int b = bh / a.Hq;
-    const int h = bh % a.Hq;
-    const int kvh = h / a.group;
-    const int q0 = qt * kBM;
-    const int ntiles = qt + 1;             // KV tiles 0..qt (causal)
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-
-    if (threadIdx.x == 0) {
-        mbar_init(&bar[Q_FULL], 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&bar[K_FULL + s], 1);
-            mbar_init(&bar[V_FULL + s], 1);
-            mbar_init(&bar[KV_EMPTY + s], 1);
-            mbar_init(&bar[S_FULL + s], 1);
-            mbar_init(&bar[S_FREE + s], kSoftmaxThreads);
-        }
-        mbar_init(&bar[P_FULL], kSoftmaxThreads);
-        mbar_init(&bar[P_FREE], 1);
-        mbar_init(&bar[O_FULL], 1);
-        mbar_init(&bar[DRAIN], 1);
-        *err = 0;
-        fence_barrier_init();
-    }
-    if (warp == 1) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const uint32_t tS[2] = {tmem, tmem + 128};
-    const uint32_t tO = tmem + 256;
-
-    if (warp == 0) {
-        // ---------------- TMA producer
-        if (lane == 0) {
-            tma_prefetch_desc(&tmQ);
-            tma_prefetch_desc(&tmK);
-            tma_prefetch_desc(&tmV);
-            mbar_arrive_expect_tx(&bar[Q_FULL], kTileBytes);
-            tma_load_4d(smem + Smem::q, &tmQ, &bar[Q_FULL], 0, h, q0, b);
-            tma_load_4d(smem + Smem::q + kHalfTile, &tmQ, &bar[Q_FULL], 64, h, q0, b);
-            int issued = 0;
-            for (int j = 0; j < ntiles; ++j) {
-                const int s = j & 1;
-                if (j >= 2 && !wait_or_fail(&bar[KV_EMPTY + s], ((j >> 1) - 1) & 1, a, err)) break;
-                uint8_t *ks = smem + Smem::k + s * kTileBytes;
-                uint8_t *vs = smem + Smem::v + s * kTileBytes;
-                mbar_arrive_expect_tx(&bar[K_FULL + s], kTileBytes);
-                tma_load_4d(ks, &tmK, &bar[K_FULL + s], 0, kvh, j * kBN, b);
-                tma_load_4d(ks + kHalfTile, &tmK, &bar[K_FULL + s], 64, kvh, j * kBN, b);
-                mbar_arrive_expect_tx(&bar[V_FULL + s], kTileBytes);
-                tma_load_4d(vs, &tmV, &bar[V_FULL + s], 0, kvh, j * kBN, b);
-                tma_load_4d(vs + kHalfTile, &tmV, &bar[V_FULL + s], 64, kvh, j * kBN, b);
-                ++issued;
-            }
-            // leave no copy in flight: the last loads of each stage and the Q tile must have landed
-            for (int j = issued - 1; j >= 0 && j >= issued - 2; --j) {
-                const uint32_t ph = (j >> 1) & 1;
-                mbar_wait(&bar[K_FULL + (j & 1)], ph, a.wait_budget_ns);
-                mbar_wait(&bar[V_FULL + (j & 1)], ph, a.wait_budget_ns);
-            }
-            mbar_wait(&bar[Q_FULL], 0, a.wait_budget_ns);
-        }
-    } else if (warp == 1) {
-        // ---------------- MMA issuer (one thread)
-        if (lane == 0) {
-            const uint32_t idesc_s = umma_idesc_bf16(kBM, kBN, 0, 0);   // Q (K-major) x K (K-major)
-            const uint32_t idesc_o = umma_idesc_bf16(kBM, kD, 0, 1);    // P (K-major) x V (MN-major)
-            const uint32_t q_addr = smem_u32(smem + Smem::q);
-            const uint32_t p_addr = smem_u32(smem + Smem::p);
-            bool ok = wait_or_fail(&bar[Q_FULL], 0, a, err);
-            int pv_done = 0;
-            for (int j = 0; ok && j <= ntiles; ++j) {
-                if (j < ntiles) {
-                    const int s = j & 1;
-                    if (!wait_or_fail(&bar[K_FULL + s], (j >> 1) & 1, a, err)) { ok = false; break; }
-                    if (j >= 2 && !wait_or_fail(&bar[S_FREE + s], ((j >> 1) - 1) & 1, a, err)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t k_addr = smem_u32(smem + Smem::k + s * kTileBytes);
-#pragma unroll
-                    for (int ks = 0; ks < kD / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * kHalfTile + (ks & 3) * 32;
-                        umma_ss(tS[s], desc_kmajor(q_addr + off), desc_kmajor(k_addr + off), idesc_s,
-                                     ks > 0 ? 1u : 0u);
-                    }
-                    umma_commit(&bar[S_FULL + s]);
-                }
-                if (j >= 1) {
-                    const int jp = j - 1;      // PV of the previous tile
-                    const int s = jp & 1;
-                    if (!wait_or_fail(&bar[P_FULL], jp & 1, a, err)) { ok = false; break; }
-                    if (!wait_or_fail(&bar[V_FULL + s], (jp >> 1) & 1, a, err)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint32_t v_addr = smem_u32(smem + Smem::v + s * kTileBytes);
-#pragma unroll
-                    for (int ks = 0; ks < kBN / 16; ++ks) {
-                        const uint32_t poff = (ks >> 2) * kHalfTile + (ks & 3) * 32;
-                        umma_ss(tO, desc_kmajor(p_addr + poff), desc_mnmajor(v_addr + ks * 2048, kHalfTile),
-                                     idesc_o, (jp > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    umma_commit(&bar[P_FREE]);
-                    umma_commit(&bar[KV_EMPTY + s]);
-                    ++pv_done;
-                }
-            }
-            if (ok && pv_done == ntiles) umma_commit(&bar[O_FULL]);
-            // no MMA may still run when TMEM is released
-            umma_commit(&bar[DRAIN]);
-            mbar_wait(&bar[DRAIN], 0, a.wait_budget_ns);
-        }
-    } else {
-        // ---------------- softmax warps: thread owns query row r of the tile
-        const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
-        const int r = quarter * 32 + lane;            // row within the tile
-        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const int qrow = q0 + r;
-        uint8_t *prow = smem + Smem::p + r * 128;
-        float m_run = -INFINITY, l_run = 0.f;
-        bool ok = true;
-        for (int j = 0; j < ntiles; ++j) {
-            const int s = j & 1;
-            if (!wait_or_fail(&bar[S_FULL + s], (j >> 1) & 1, a, err)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t sr[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tS[s] + lane_off + c * 32, sr + c * 32);
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&bar[S_FREE + s]);
-
-            // raw scores; the diagonal tile hides keys after the row.  Eight independent partial maxima
-            // keep the reduction off a 128-long dependency chain.
-            const bool diag = (j == qt);
-            float pm[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) pm[i] = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 128; ++c) {
-                if (diag && c > r) sr[c] = __float_as_uint(-INFINITY);
-                pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(sr[c]));
-            }
-            const float mraw = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                     fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
-            // in log2 units: qscale = log2(e)/sqrt(d) > 0, so max(raw)*qscale is the scaled maximum
-            const float m_new = fmaxf(m_run, mraw * a.qscale);
-            const bool move = (m_new > m_run + kRescaleThreshold);
-            const float m_use = move ? m_new : m_run;
-            const float alpha = move ? ex2(m_run - m_new) : 1.f;   // ex2(-inf) = 0 on the first tile
-            // p = 2^(raw*qscale - m_use): one packed FMA per two elements, then the exp unit
-            const float2 sc2 = make_float2(a.qscale, a.qscale);
-            const float2 nm2 = make_float2(-m_use, -m_use);
-            float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                            make_float2(0.f, 0.f)};
-            float x[128];
-#pragma unroll
-            for (int c = 0; c < 128; c += 2) {
-                const float2 e = __ffma2_rn(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
-                const float2 pe = make_float2(ex2(e.x), ex2(e.y));
-                x[c] = pe.x;
-                x[c + 1] = pe.y;
-                ps[(c >> 1) & 3] = __fadd2_rn(ps[(c >> 1) & 3], pe);
-            }
-            const float rs = (ps[0].x + ps[0].y) + (ps[1].x + ps[1].y) + (ps[2].x + ps[2].y) + (ps[3].x + ps[3].y);
-            m_run = m_use;
-            l_run = l_run * alpha + rs;
-
-            if (j >= 1) {
-                // previous PV done: P buffer free, O stable
-                if (!wait_or_fail(&bar[P_FREE], (j - 1) & 1, a, err)) { ok = false; break; }
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, move)) {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t orow[32];
-                        tmem_ld32(tO + lane_off + c * 32, orow);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
-                        tmem_st32(tO + lane_off + c * 32, orow);
-                    }
-                    tmem_wait_st();
-                }
-            }
-            // P row -> bf16, K-major with the 128-byte swizzle: 16-byte chunk c of half hh at chunk c ^ (r & 7)
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const int e = hh * 64 + c * 8;
-                    uint4 w;
-                    w.x = pack_bf16x2(x[e + 0], x[e + 1]);
-                    w.y = pack_bf16x2(x[e + 2], x[e + 3]);
-                    w.z = pack_bf16x2(x[e + 4], x[e + 5]);
-                    w.w = pack_bf16x2(x[e + 6], x[e + 7]);
-                    *reinterpret_cast<uint4 *>(prow + hh * kHalfTile + ((c ^ (r & 7)) << 4)) = w;
-                }
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bar[P_FULL]);
-        }
-        if (ok && wait_or_fail(&bar[O_FULL], 0, a, err)) {
-            tc_fence_after();
-            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-            // log-sum-exp of the row's scaled scores, natural log: (m + log2 l) ln 2
-            if (a.lse && qrow < a.S)
-                a.lse[((size_t)b * a.Hq + h) * a.S + qrow] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
-            __nv_bfloat16 *orow_g = a.out + (((size_t)b * a.S + qrow) * a.Hq + h) * kD;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t orow[32];
-                tmem_ld32(tO + lane_off + c * 32, orow);
-                tmem_wait_ld();
-                if (qrow < a.S) {
-#pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint4 w;
-                        w.x = pack_bf16x2(__uint_as_float(orow[i + 0]) * inv, __uint_as_float(orow[i + 1]) * inv);
-                        w.y = pack_bf16x2(__uint_as_float(orow[i + 2]) * inv, __uint_as_float(orow[i + 3]) * inv);
-                        w.z = pack_bf16x2(__uint_as_float(orow[i + 4]) * inv, __uint_as_float(orow[i + 5]) * inv);
-                        w.w = pack_bf16x2(__uint_as_float(orow[i + 6]) * inv, __uint_as_float(orow[i + 7]) * inv);
-                        *reinterpret_cast<uint4 *>(orow_g + c * 32 + i) = w;
-                    }
-                }
-            }
-        }
-    }
-
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
-    }
-}
-
-
 // ----------------------------------------------------------------------------
-// Paired-head variant for even group sizes.  One CTA computes the same
-// 128-row query tile of two query heads of one group (h, h+1): they read the
-// same KV head, so every K/V tile in shared memory serves both, and they have
-// the same causal shape.  Two softmax warpgroups (one per head) alternate on
-// the tensor core: while one works through its softmax, the MMAs of the other
-// run.  Each warpgroup's P goes back into tensor memory over its own S (bf16,
-// two per 32-bit column) and the PV product reads it from there, so both Q
-// tiles and a two-stage K/V ring fit in shared memory.
+// Paired variant: one CTA computes two 128-row query tiles ("streams") that
+// read the same KV head, so every K/V tile in shared memory serves both.  For
+// even group sizes the streams are the same query tile of two heads of one
+// group (h, h+1), with the same causal shape; for odd group sizes (MHA
+// included) they are query tiles 2k and 2k+1 of one head, which share key
+// tiles 0..2k (the second stream has one more, its own diagonal).  Two softmax
+// warpgroups (one per stream) alternate on the tensor core: while one works
+// through its softmax, the MMAs of the other run.  Each warpgroup's P goes
+// back into tensor memory over its own S (bf16, two per 32-bit column) and the
+// PV product reads it from there, so both Q tiles and a two-stage K/V ring fit
+// in shared memory.
 //
-// Warps: 0..3 softmax of head h, 4..7 softmax of head h+1 (TMEM lane quarter =
+// Warps: 0..3 softmax of stream 0, 4..7 softmax of stream 1 (TMEM lane quarter =
 // warp % 4), 8 TMA producer, 9 TMEM allocator + MMA issuer.
 // TMEM columns: S_A 0..127 (P_A over 0..63), S_B 128..255, O_A 256..383, O_B 384..511.
 constexpr int kPairThreads = 320;
@@ -403,18 +116,32 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + PairSmem::tmem_slot);
     volatile int *err = reinterpret_cast<volatile int *>(smem + PairSmem::err);
 
-    // heaviest query tiles first; the pairs of one group are neighbours
+    // heaviest work first; the head pairs of one group (or the heads of one group) are neighbours
     const int nqt = (a.S + kBM - 1) / kBM;
-    const int pairs = a.Hq / 2;
-    const int per_qt = a.B * pairs;
     const int id = blockIdx.x;
-    const int qt = nqt - 1 - id / per_qt;
-    const int rem = id % per_qt;
-    const int b = rem / pairs;
-    const int hA = 2 * (rem % pairs);
-    const int kvh = hA / a.group;
-    const int q0 = qt * kBM;
-    const int ntiles = qt + 1;
+    int b, hw[2], qtw[2];
+    if (a.group % 2 == 0) {
+        const int pairs = a.Hq / 2;
+        const int per_qt = a.B * pairs;
+        const int qt = nqt - 1 - id / per_qt;
+        const int rem = id % per_qt;
+        b = rem / pairs;
+        hw[0] = 2 * (rem % pairs);
+        hw[1] = hw[0] + 1;
+        qtw[0] = qtw[1] = qt;
+    } else {
+        const int per_k = a.B * a.Hq;
+        const int k = (nqt + 1) / 2 - 1 - id / per_k;
+        const int rem = id % per_k;
+        b = rem / a.Hq;
+        hw[0] = hw[1] = rem % a.Hq;
+        qtw[0] = 2 * k;
+        qtw[1] = 2 * k + 1 < nqt ? 2 * k + 1 : -1;   // the last tile of an odd count has no partner
+    }
+    const int kvh = hw[0] / a.group;
+    const int nt0 = qtw[0] + 1, nt1 = qtw[1] + 1;     // key tiles of each stream (0: stream absent)
+    const int ntiles = nt0 > nt1 ? nt0 : nt1;
+    auto ntw = [&](int w) { return w ? nt1 : nt0; };
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -448,11 +175,13 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
-            mbar_arrive_expect_tx(&bar[PQ_FULL], 2 * kTileBytes);
+            mbar_arrive_expect_tx(&bar[PQ_FULL], (nt1 > 0 ? 2 : 1) * kTileBytes);
             for (int w = 0; w < 2; ++w) {
+                if (ntw(w) == 0) continue;
                 uint8_t *qs = smem + PairSmem::q + w * kTileBytes;
-                tma_load_4d(qs, &tmQ, &bar[PQ_FULL], 0, hA + w, q0, b);
-                tma_load_4d(qs + kHalfTile, &tmQ, &bar[PQ_FULL], 64, hA + w, q0, b);
+                const int hq = w ? hw[1] : hw[0], q0 = (w ? qtw[1] : qtw[0]) * kBM;
+                tma_load_4d(qs, &tmQ, &bar[PQ_FULL], 0, hq, q0, b);
+                tma_load_4d(qs + kHalfTile, &tmQ, &bar[PQ_FULL], 64, hq, q0, b);
             }
             int issued = 0;
             for (int j = 0; j < ntiles; ++j) {
@@ -495,16 +224,19 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             };
             if (ok) {
                 tc_fence_after();
-                issue_s(0, 0);
-                issue_s(1, 0);
+                for (int w = 0; w < 2; ++w)
+                    if (ntw(w) > 0) issue_s(w, 0);
             }
             int pv_done = 0;
             for (int j = 0; ok && j < ntiles; ++j) {
                 const int s = j & 1;
                 const uint32_t v_addr = smem_u32(smem + PairSmem::kv + s * 2 * kTileBytes + kTileBytes);
+                bool v_seen = false, k_next_seen = false;
                 for (int w = 0; w < 2; ++w) {
+                    if (j >= ntw(w)) continue;   // this stream's key tiles end before j
                     if (!wait_or_fail(&bar[PP_FULL + w], j & 1, a, err)) { ok = false; break; }
-                    if (w == 0 && !wait_or_fail(&bar[PV_FULL + s], (j >> 1) & 1, a, err)) { ok = false; break; }
+                    if (!v_seen && !wait_or_fail(&bar[PV_FULL + s], (j >> 1) & 1, a, err)) { ok = false; break; }
+                    v_seen = true;
                     tc_fence_after();
 #pragma unroll
                     for (int ks = 0; ks < kBN / 16; ++ks) {
@@ -513,39 +245,43 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                                      desc_mnmajor(v_addr + ks * 2048, kHalfTile), idesc_o,
                                      (j > 0 || ks > 0) ? 1u : 0u);
                     }
-                    if (w == 1) {
-                        umma_commit(&bar[PKV_EMPTY + s]);
-                        ++pv_done;
-                    }
-                    if (j + 1 < ntiles) {
-                        if (w == 0 && !wait_or_fail(&bar[PK_FULL + ((j + 1) & 1)], ((j + 1) >> 1) & 1, a, err)) {
+                    if (j + 1 < ntw(w)) {
+                        if (!k_next_seen && !wait_or_fail(&bar[PK_FULL + ((j + 1) & 1)], ((j + 1) >> 1) & 1, a, err)) {
                             ok = false;
                             break;
                         }
+                        k_next_seen = true;
                         tc_fence_after();
                         issue_s(w, j + 1);
                     }
                 }
+                if (!ok) break;
+                // the tile's last reader has been issued
+                umma_commit(&bar[PKV_EMPTY + s]);
+                ++pv_done;
             }
             if (ok && pv_done == ntiles) umma_commit(&bar[PO_FULL]);
             umma_commit(&bar[PDRAIN]);
             mbar_wait(&bar[PDRAIN], 0, a.wait_budget_ns);
         }
     } else {
-        // ---------------- softmax warpgroup w: head hA + w, thread owns query row r
+        // ---------------- softmax warpgroup w: stream w (head hw[w], query tile qtw[w]), thread owns query row r
         const int w = warp >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t tS = tmem + w * 128 + lane_off;
         const uint32_t tO = tmem + 256 + w * 128 + lane_off;
-        const int qrow = q0 + r;
+        const int qtile = w ? qtw[1] : qtw[0];
+        const int qrow = qtile * kBM + r;
+        const int hq = w ? hw[1] : hw[0];
+        const int nt = ntw(w);
         float m_run = -INFINITY, l_run = 0.f;
-        bool ok = true;
-        for (int j = 0; j < ntiles; ++j) {
+        bool ok = nt > 0;
+        for (int j = 0; ok && j < nt; ++j) {
             if (!wait_or_fail(&bar[PS_FULL + w], j & 1, a, err)) { ok = false; break; }
             tc_fence_after();
-            const bool diag = (j == qt);
+            const bool diag = (j == qtile);
             // pass 1: the row maximum of the raw scores (keys after the row hidden on the diagonal);
             // two 32-column loads per wait, three-input max, four independent partial maxima
             float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -627,8 +363,8 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
             // log-sum-exp of the row's scaled scores, natural log: (m + log2 l) ln 2
             if (a.lse && qrow < a.S)
-                a.lse[((size_t)b * a.Hq + hA + w) * a.S + qrow] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
-            __nv_bfloat16 *orow_g = a.out + (((size_t)b * a.S + qrow) * a.Hq + hA + w) * kD;
+                a.lse[((size_t)b * a.Hq + hq) * a.S + qrow] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
+            __nv_bfloat16 *orow_g = a.out + (((size_t)b * a.S + qrow) * a.Hq + hq) * kD;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t orow[32];
@@ -662,26 +398,20 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 cudaError_t launch_prefill(const CUtensorMap &tmQ, const CUtensorMap &tmK, const CUtensorMap &tmV,
                            const PrefillArgs &a, cudaStream_t stream)
 {
-    static bool attr_done[2][64] = {};
-    const bool paired = (a.group % 2 == 0);
-    const int smem = (paired ? PairSmem::bytes : Smem::bytes) + 1024;
+    static bool attr_done[64] = {};
+    const int smem = PairSmem::bytes + 1024;
     int dev = 0;
     cudaGetDevice(&dev);
-    if (dev < 64 && !attr_done[paired][dev]) {
-        cudaError_t e = paired ? cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                      smem)
-                               : cudaFuncSetAttribute(prefill_causal_kernel,
-                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (dev < 64 && !attr_done[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(prefill_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        attr_done[paired][dev] = true;
+        attr_done[dev] = true;
     }
+    // even groups: (query tile, sequence, head pair); odd groups: (query-tile pair, sequence, head)
     const long long nqt = (a.S + kBM - 1) / kBM;
-    const long long grid = nqt * a.B * (paired ? a.Hq / 2 : a.Hq);
+    const long long grid = a.group % 2 == 0 ? nqt * a.B * (a.Hq / 2) : ((nqt + 1) / 2) * a.B * a.Hq;
     if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
-    if (paired)
-        prefill_pair_kernel<<<(unsigned)grid, kPairThreads, smem, stream>>>(tmQ, tmK, tmV, a);
-    else
-        prefill_causal_kernel<<<(unsigned)grid, kThreads, smem, stream>>>(tmQ, tmK, tmV, a);
+    prefill_pair_kernel<<<(unsigned)grid, kPairThreads, smem, stream>>>(tmQ, tmK, tmV, a);
     return cudaGetLastError();
 }
 
