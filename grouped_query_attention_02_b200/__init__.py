@@ -92,9 +92,13 @@ def _check(status: int, where: str):
 
 
 def _stream_ptr(stream):
+    """The stream argument of an entry point: None = the current device's current stream."""
     import torch
 
     if stream is None:
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        if raw is not None:   # the handle without building a Stream object (a few microseconds a call)
+            return raw(torch._C._cuda_getDevice())
         return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     if isinstance(stream, int):
         return ctypes.c_void_p(stream)
@@ -102,8 +106,19 @@ def _stream_ptr(stream):
 
 
 def _need(t, name, dtype, ndim, device=None):
+    """Checks one tensor argument: type, dtype, rank, a CUDA device (the given one, if any), contiguous.
+    The common case costs a handful of attribute reads; the detailed checks run only to name a failure."""
+    try:
+        if t.dtype is dtype and t.dim() == ndim and t.is_contiguous():
+            d = t.get_device()
+            if d >= 0 and (device is None or d == (device if isinstance(device, int) else device.index)):
+                return
+    except AttributeError:
+        pass
     import torch
 
+    if isinstance(device, int):
+        device = torch.device("cuda", device)
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if t.dtype != dtype:
@@ -116,6 +131,7 @@ def _need(t, name, dtype, ndim, device=None):
         raise ValueError(f"{name} is on {t.device}, expected {device}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    raise ValueError(f"{name}: unsupported tensor")
 
 
 def gqa_decode(q, k_cache, v_cache, seqlens, scale=None, out=None, stream=None):
@@ -124,16 +140,17 @@ def gqa_decode(q, k_cache, v_cache, seqlens, scale=None, out=None, stream=None):
 
     _need(q, "q", torch.bfloat16, 3)
     B, Hq, d = q.shape
-    _need(k_cache, "k_cache", torch.bfloat16, 4, q.device)
-    _need(v_cache, "v_cache", torch.bfloat16, 4, q.device)
-    _need(seqlens, "seqlens", torch.int32, 1, q.device)
+    dev = q.get_device()
+    _need(k_cache, "k_cache", torch.bfloat16, 4, dev)
+    _need(v_cache, "v_cache", torch.bfloat16, 4, dev)
+    _need(seqlens, "seqlens", torch.int32, 1, dev)
     Bk, Tmax, Hkv, dk = k_cache.shape
     if (Bk, dk) != (B, d) or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
         raise ValueError("shape mismatch between q, k_cache, v_cache and seqlens")
     if out is None:
         out = torch.empty_like(q)
     else:
-        _need(out, "out", torch.bfloat16, 3, q.device)
+        _need(out, "out", torch.bfloat16, 3, dev)
         if out.shape != q.shape:
             raise ValueError("out must have q's shape")
     if scale is None:
@@ -152,20 +169,21 @@ def gqa_decode_fp8(q, k_cache, v_cache, seqlens, k_scale, v_scale, scale=None, o
 
     _need(q, "q", torch.bfloat16, 3)
     B, Hq, d = q.shape
+    dev = q.get_device()
     if k_cache.dtype == torch.float8_e4m3fn:
         k_cache = k_cache.view(torch.uint8)
     if v_cache.dtype == torch.float8_e4m3fn:
         v_cache = v_cache.view(torch.uint8)
-    _need(k_cache, "k_cache", torch.uint8, 4, q.device)
-    _need(v_cache, "v_cache", torch.uint8, 4, q.device)
-    _need(seqlens, "seqlens", torch.int32, 1, q.device)
+    _need(k_cache, "k_cache", torch.uint8, 4, dev)
+    _need(v_cache, "v_cache", torch.uint8, 4, dev)
+    _need(seqlens, "seqlens", torch.int32, 1, dev)
     Bk, Tmax, Hkv, dk = k_cache.shape
     if (Bk, dk) != (B, d) or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
         raise ValueError("shape mismatch between q, k_cache, v_cache and seqlens")
     if out is None:
         out = torch.empty_like(q)
     else:
-        _need(out, "out", torch.bfloat16, 3, q.device)
+        _need(out, "out", torch.bfloat16, 3, dev)
         if out.shape != q.shape:
             raise ValueError("out must have q's shape")
     if scale is None:

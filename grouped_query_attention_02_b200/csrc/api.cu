@@ -222,6 +222,13 @@ DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_
         if (cap > tiles) cap = tiles;
         const long long fit = per_piece ? (long long)(ws_budget / per_piece) : cap;
         if (fit < cap) cap = fit < 1 ? 1 : fit;
+        if (tiles <= kStaticPlanTiles) {
+            p.static_plan = true;
+            p.nsplit = 1;
+            p.chunk = (int)(tiles * sh.tile);
+            p.ws_bytes = 0;
+            return p;
+        }
         const long long cmin = (tiles + cap - 1) / cap;
         p.nsplit = (int)((tiles + cmin - 1) / cmin);
         p.chunk = (int)(cmin * sh.tile);
@@ -316,10 +323,6 @@ int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *s
     a.num_ctas = num_sms;
     int n = 0;
     if (p.tensor_cores) {
-        a.plan_hdr = reinterpret_cast<int *>(w + p.off_hdr);
-        a.nsplit_b = reinterpret_cast<int *>(w + p.off_nsb);
-        a.plan_scratch = reinterpret_cast<int *>(w + p.off_nsb + round256((size_t)B * 4));
-        a.items = reinterpret_cast<int4 *>(w + p.off_items);
         // the group's query rows as a 3-D map (d, heads, batch): one box = N rows of one 64-column half
         const int N = a.group <= 16 ? 16 : 32;
         cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)Hq, (cuuint64_t)B};
@@ -330,6 +333,19 @@ int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *s
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return GQA_ERR_CUDA;
+    }
+    if (p.tensor_cores && p.static_plan) {
+        // one launch: whole histories as units, nothing to plan or combine
+        a.static_plan = 1;
+        if (ev_before) cudaEventRecord(ev_before, stream);
+        if ((s = cuda_status(launch_decode_tc(tmK, tmV, tmQ, a, stream, fp8 != nullptr))) != GQA_OK) return s;
+        if (ev_after) cudaEventRecord(ev_after, stream);
+        ++n;
+    } else if (p.tensor_cores) {
+        a.plan_hdr = reinterpret_cast<int *>(w + p.off_hdr);
+        a.nsplit_b = reinterpret_cast<int *>(w + p.off_nsb);
+        a.plan_scratch = reinterpret_cast<int *>(w + p.off_nsb + round256((size_t)B * 4));
+        a.items = reinterpret_cast<int4 *>(w + p.off_items);
         if ((s = cuda_status(launch_decode_plan(a, stream))) != GQA_OK) return s;
         ++n;
         if (ev_before) cudaEventRecord(ev_before, stream);

@@ -474,10 +474,28 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 tma_prefetch_desc(&tmK);
                 tma_prefetch_desc(&tmV);
                 tma_prefetch_desc(&tmQ);
-                const int units = a.plan_hdr[1] * a.Hkv;
-                int tcount = 0, icount = 0, issued_tiles = 0;
+                // static schedule (no planner): unit u = (sequence u / Hkv, KV head u % Hkv), the whole
+                // history as one piece, units dealt round-robin over the CTAs
+                const bool stat = a.static_plan != 0;
+                const int units = stat ? a.B * a.Hkv : a.plan_hdr[1] * a.Hkv;
+                int tcount = 0, icount = 0, issued_tiles = 0, claim = 0;
                 while (true) {
-                    const int u = atomicAdd(&a.plan_hdr[0], 1);
+                    int u = stat ? blockIdx.x + (claim++) * gridDim.x : atomicAdd(&a.plan_hdr[0], 1);
+                    int4 it = make_int4(0, 0, 0, 0);
+                    if (stat) {
+                        // an empty history has no unit: its output rows are zero
+                        for (; u < units; u = blockIdx.x + (claim++) * gridDim.x) {
+                            const int bb = u / a.Hkv;
+                            int T = a.seqlens[bb];
+                            T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
+                            if (T > 0) {
+                                it = make_int4(bb, 0, 0, T);
+                                break;
+                            }
+                            uint4 *o = reinterpret_cast<uint4 *>(a.out + ((size_t)bb * a.Hq + (u % a.Hkv) * g) * kD);
+                            for (int i = 0; i < g * kD / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
+                        }
+                    }
                     const int slot = icount % kQD;
                     if (icount >= kQD && !wait_or_fail(&bar[I_EMPTY + slot], ((icount / kQD) - 1) & 1, a, err)) break;
                     volatile int *q = queue + slot * 8;
@@ -486,7 +504,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                         mbar_arrive(&bar[I_FULL + slot]);
                         break;
                     }
-                    const int4 it = a.items[u / a.Hkv];
+                    if (!stat) it = a.items[u / a.Hkv];
                     const int kvh = u % a.Hkv;
                     q[0] = it.x;
                     q[1] = kvh;
@@ -812,7 +830,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 o[h] = __float_as_uint((__uint_as_float(o[h]) + __uint_as_float(olo[h])) * ofac);
             const float *ls = lsum + pob * 4 * N;
             const int d = t;
-            const int npieces = a.nsplit_b[pb];
+            const int npieces = a.static_plan ? 1 : a.nsplit_b[pb];
             if (npieces == 1) {
                 // the whole history in one unit: normalise and write the output
 #pragma unroll
@@ -1063,10 +1081,12 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
         }
         attr_done[dev] = true;
     }
-    // programmatic dependent launch: the prologue overlaps decode_plan_kernel, which the kernel
-    // waits for (griddepcontrol.wait) before reading the plan
+    // programmatic dependent launch: the prologue overlaps decode_plan_kernel (or, with the static
+    // schedule, whatever ran before), which the kernel waits for (griddepcontrol.wait) before it
+    // touches global memory
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.num_ctas);
+    const int units = a.B * a.Hkv;
+    cfg.gridDim = dim3(a.static_plan && units < a.num_ctas ? units : a.num_ctas);
     cfg.blockDim = dim3(TcCfg<N, F8, HW, NWG>::threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;

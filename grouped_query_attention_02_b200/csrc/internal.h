@@ -14,6 +14,10 @@ constexpr int kDecodeTile = 64;     // tokens per TMA stage of the CUDA-core dec
 constexpr int kDecodeCtasPerSm = 2; // resident CUDA-core decode CTAs per SM (shared-memory bound)
 constexpr int kStatusTimeout = 6;   // device status word: a bounded wait gave up
 constexpr int kStatusMisaligned = 3; // device status word: a kernel found its shared memory misaligned
+// Caches of at most this many 128-token tiles (Tmax <= 512) take the tensor-core decode as one launch:
+// whole histories as units, no planner and no combine, whose fixed costs would exceed what splitting
+// a history this short could save.
+constexpr int kStaticPlanTiles = 4;
 
 struct DecodeArgs {
     const __nv_bfloat16 *q;   // [B,Hq,d]
@@ -36,6 +40,7 @@ struct DecodeArgs {
     // planner options for other operators that reuse decode_plan_kernel (0: the GQA decode's defaults)
     int out_row;              // output elements per (sequence, query head) row, zeroed for empty histories
     int plan_rounds;          // rounds of units per persistent CTA the pieces are sized for
+    int static_plan;          // 1: no planner; one piece per history, units dealt round-robin (short caches)
 };
 
 // Host plan of a decode call and the layout of its workspace.
@@ -43,6 +48,7 @@ struct DecodePlan {
     int tile, chunk, nsplit, hb, nhb;
     bool tensor_cores;
     size_t off_hdr, off_nsb, off_items, off_po, off_pml, ws_bytes;
+    bool static_plan;   // tensor-core path without the device planner: one launch, no workspace
 };
 // ws_budget bounds the split partials (fewer pieces per sequence when they would not fit; one piece needs none).
 // fp8: the plan of the FP8-cache decode, which always takes the tensor-core path (group sizes <= 32).

@@ -86,6 +86,18 @@ def test_fp8_tile_edges_and_empty(oracle_mod):
     assert_close(out.double().cpu().numpy(), _ref(oracle_mod, x))
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (32, 1)])
+def test_fp8_short_caches_one_launch(oracle_mod, Hq, Hkv):
+    # at most four tiles: one launch over whole histories, more units than CTAs, empty histories included
+    B = 150
+    lens = [(i * 41) % 513 for i in range(B)]
+    x = inputs.make_decode_fp8(B, Hq, Hkv, 128, 512, seqlens=lens, device=DEV, seed=31 + Hkv)
+    out = _run(x)
+    assert gqa.gqa_last_launch_count() == 1
+    assert torch.all(out[0] == 0)
+    assert_close(out.double().cpu().numpy(), _ref(oracle_mod, x))
+
+
 def test_fp8_long_history_split_and_merged(oracle_mod):
     x = inputs.make_decode_fp8(2, 8, 2, 128, 20000, seqlens=[20000, 9001], device=DEV, seed=4)
     assert_close(_run(x).double().cpu().numpy(), _ref(oracle_mod, x))

@@ -92,6 +92,21 @@ def test_tile_edges_and_empty(oracle_mod):
     _check_all(oracle_mod, x, out)
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (24, 8), (32, 1)])
+def test_short_caches_one_launch_more_units_than_ctas(oracle_mod, Hq, Hkv):
+    """Caches of at most four 128-token tiles run as one launch over whole histories, dealt round-robin:
+    here more (sequence, KV head) units than CTAs for the grouped shapes, lengths from 0 to 512."""
+    B = 150
+    lens = [(i * 37) % 513 for i in range(B)]
+    x = inputs.make_decode(B, Hq, Hkv, 128, 512, seqlens=lens, device=DEV, seed=14 + Hkv)
+    out = _run(x)
+    assert gqa.gqa_last_launch_count() == 1
+    for b, T in enumerate(lens):
+        if T == 0:
+            assert torch.all(out[b] == 0)
+    _check_all(oracle_mod, x, out)
+
+
 def test_split_boundaries(oracle_mod):
     # a long single sequence is split; lengths straddling the split chunk must merge exactly
     B, Hq, Hkv, Tmax = 2, 8, 2, 20000

@@ -18,7 +18,7 @@ class Plan(ctypes.Structure):
     _fields_ = [("tile", ctypes.c_int), ("chunk", ctypes.c_int), ("nsplit", ctypes.c_int), ("hb", ctypes.c_int),
                 ("nhb", ctypes.c_int), ("tensor_cores", ctypes.c_bool), ("off_hdr", ctypes.c_size_t),
                 ("off_nsb", ctypes.c_size_t), ("off_items", ctypes.c_size_t), ("off_po", ctypes.c_size_t),
-                ("off_pml", ctypes.c_size_t), ("ws_bytes", ctypes.c_size_t)]
+                ("off_pml", ctypes.c_size_t), ("ws_bytes", ctypes.c_size_t), ("static_plan", ctypes.c_bool)]
 
 
 @pytest.fixture(scope="module")
@@ -57,3 +57,13 @@ def test_every_split_the_budget_allows_covers_the_history(plan):
             assert p.nsplit >= 1 and p.chunk * p.nsplit >= T and p.chunk * (p.nsplit - 1) < T
             if p.nsplit > 1:
                 assert B * Hq * p.nsplit * (128 + 2) * 4 <= budget
+
+
+@pytest.mark.parametrize("T,static", [(1, True), (512, True), (513, False), (8192, False)])
+def test_short_caches_take_one_launch(plan, T, static):
+    # the tensor-core path (group 4): caches of at most four 128-token tiles run without the planner
+    # (no workspace at all), longer ones are planned on the device
+    p = plan(49, 32, 8, T, 256 << 20)
+    assert p.tensor_cores and p.static_plan == static
+    assert (p.ws_bytes == 0) == static
+    assert p.nsplit >= 1 and p.chunk * p.nsplit >= T

@@ -96,10 +96,11 @@ def test_allocates_nothing(oracle_mod):
     assert_close(out.double().cpu().numpy(), oracle_mod.decode(x.q, x.k_cache, x.v_cache, x.seqlens.cpu(), x.scale))
 
 
-def test_rejects_partials_larger_than_the_fixed_scratch():
+def test_rejects_partials_larger_than_the_fixed_scratch(oracle_mod):
     # 2048 sequences x 32 query heads: even one piece per sequence needs 2048*32*130*4 B = 34 MB of
-    # partials, more than the 32 MiB array
-    B, Hq, Hkv, Tmax = 2048, 32, 8, 256
+    # partials, more than the 32 MiB array (a cache of 1024 tokens is planned on the device; caches of
+    # at most 512 run as one launch with no partials at all, and are accepted)
+    B, Hq, Hkv, Tmax = 2048, 32, 8, 1024
     assert B * Hq * (128 + 2) * 4 > 32 << 20
     q = torch.zeros((B, Hq, 128), dtype=torch.bfloat16, device=DEV)
     k = torch.empty((B, Tmax, Hkv, 128), dtype=torch.bfloat16, device=DEV)
@@ -111,3 +112,12 @@ def test_rejects_partials_larger_than_the_fixed_scratch():
                                 ctypes.c_float(0.088), out.data_ptr(), None)
     assert st == 2, gqa.gqa_status_string(st)
     assert gqa.gqa_last_launch_count() == 0
+    # the same batch over a 512-token cache needs no scratch: one launch, right answer
+    Tmax = 512
+    x = inputs.make_decode(B, Hq, Hkv, 128, Tmax, device=DEV, seed=79)
+    assert _call_noalloc(lib, x, out) == 0
+    torch.cuda.synchronize()
+    assert gqa.gqa_last_launch_count() == 1 and gqa.gqa_get_last_device_status() == 0
+    bs = [0, 1000, 2047]
+    ref = oracle_mod.decode(x.q[bs].cpu(), x.k_cache[bs].cpu(), x.v_cache[bs].cpu(), x.seqlens[bs].cpu(), x.scale)
+    assert_close(out[bs].double().cpu().numpy(), ref)
