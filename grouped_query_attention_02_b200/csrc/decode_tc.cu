@@ -104,7 +104,8 @@ struct TcCfg {
     static constexpr int p_half = nb * 2048;                  //   each [16 token groups][8 tokens][8 heads] 16-bit
     static constexpr int red_off = p_off + pbufs * 2 * p_half; // [2][4][N] floats: tile maxima per warp
     static constexpr int lsum_off = red_off + 2 * 4 * N * 4;  // [2 O buffers][4][N] floats: l partials per warp
-    static constexpr int qfac_off = lsum_off + 2 * 4 * N * 4; // FP8: [kQD unit slots][N] score factors per head
+    static constexpr int mst_off = lsum_off + 2 * 4 * N * 4;  // [2 O buffers][N] floats: the unit's final maxima
+    static constexpr int qfac_off = mst_off + 2 * N * 4;      // FP8: [kQD unit slots][N] score factors per head
     static constexpr int vote_off = qfac_off + (F8 ? kQD * N * 4 : 0);   // [nwg][2][4] ints
     static constexpr int queue_off = vote_off + nwg * 32;     // kQD units of 8 ints
     static constexpr int bar_off = queue_off + kQD * 32;
@@ -214,7 +215,7 @@ __device__ __forceinline__ int block_sum(int part, int *red_i, int *out)
 
 // Cuts every history into pieces of C tiles and lists them longest first:
 // plan_hdr = {claim counter (reset to 0), pieces, C}; nsplit_b[b] = pieces of sequence b;
-// items[i] = {b, piece index, first token, end token}.  Full pieces come first, then the
+// items[i] = {b, piece index | pieces of b << 16, first token, end token}.  Full pieces come first, then the
 // shorter last pieces in decreasing length (a counting sort).
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeArgs a, int slots)
 {
@@ -295,6 +296,7 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
         const int tl = (T + kTok - 1) / kTok;
         const int full = tl / C, rem = tl % C;
+        const int np_b = full + (rem > 0 ? 1 : 0);
         if (tl == 0) {
             // no cached token: no unit will touch this sequence, its output rows are zero
             const int orow = a.out_row > 0 ? a.out_row : kD;
@@ -302,11 +304,11 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
             for (int i = 0; i < a.Hq * orow / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
         }
         for (int s = 0; s < full; ++s)
-            a.items[full_off[b] + s] = make_int4(b, s, s * C * kTok, min((s + 1) * C * kTok, T));
+            a.items[full_off[b] + s] = make_int4(b, s | (np_b << 16), s * C * kTok, min((s + 1) * C * kTok, T));
         if (rem > 0) {
             const int k = C - 1 - rem;
             const int pos = sort_rem ? F + hist[k] + atomicAdd(&cursor[k], 1) : F + atomicAdd(&cursor[0], 1);
-            a.items[pos] = make_int4(b, full, full * C * kTok, T);
+            a.items[pos] = make_int4(b, full | (np_b << 16), full * C * kTok, T);
         }
     }
     if (tid == 0) {
@@ -394,6 +396,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     volatile int *err = reinterpret_cast<volatile int *>(smem + C::err_off);
     float *red = reinterpret_cast<float *>(smem + C::red_off);
     float *lsum = reinterpret_cast<float *>(smem + C::lsum_off);
+    float *mst = reinterpret_cast<float *>(smem + C::mst_off);
     float *qfac = reinterpret_cast<float *>(smem + C::qfac_off);
     volatile int *vote = reinterpret_cast<volatile int *>(smem + C::vote_off);
     volatile int *queue = reinterpret_cast<volatile int *>(smem + C::queue_off);
@@ -489,7 +492,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                             int T = a.seqlens[bb];
                             T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
                             if (T > 0) {
-                                it = make_int4(bb, 0, 0, T);
+                                it = make_int4(bb, 1 << 16, 0, T);   // piece 0 of 1
                                 break;
                             }
                             uint4 *o = reinterpret_cast<uint4 *>(a.out + ((size_t)bb * a.Hq + (u % a.Hkv) * g) * kD);
@@ -813,8 +816,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         // The epilogue of a unit (its O^T from TMEM to the partials) runs after the next unit's first
         // tile, so that waiting for the unit's last PV product overlaps useful work.
         bool pend = false;
-        int pb = 0, pkvh = 0, psplit = 0, pob = 0;
-        float pm[HW];
+        int pb = 0, pkvh = 0, psplit = 0, pob = 0;   // psplit: piece index | pieces of the history << 16
         // FP8: O carries 128 p v_code; the value scale and 1/128 are applied here
         const float ofac = F8 ? a.o_factor : 1.f;
         auto epilogue = [&]() -> bool {
@@ -828,33 +830,33 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 #pragma unroll
             for (int h = 0; h < HW; ++h)
                 o[h] = __float_as_uint((__uint_as_float(o[h]) + __uint_as_float(olo[h])) * ofac);
-            const float *ls = lsum + pob * 4 * N;
+            const float *ls = lsum + pob * 4 * N;   // per-warp weight sums of the unit: [4][N]
             const int d = t;
-            const int npieces = a.static_plan ? 1 : a.nsplit_b[pb];
-            if (npieces == 1) {
+            const size_t row0 = (size_t)pb * a.Hq + pkvh * g + hs;   // the warpgroup's first (b, query head) row
+            if ((psplit >> 16) == 1) {
                 // the whole history in one unit: normalise and write the output
 #pragma unroll
                 for (int h = 0; h < HW; ++h) {
-                    const int hg = hs + h;
-                    if (hg >= g) break;
-                    const float L = ls[hg] + ls[N + hg] + ls[2 * N + hg] + ls[3 * N + hg];
+                    if (hs + h >= g) break;
+                    const float L = ls[hs + h] + ls[N + hs + h] + ls[2 * N + hs + h] + ls[3 * N + hs + h];
                     const float O = __uint_as_float(o[h]);
                     // a zero sum only for an empty history (output 0); a NaN sum (a NaN in the cache) stays NaN
-                    a.out[((size_t)pb * a.Hq + pkvh * g + hg) * kD + d] = __float2bfloat16_rn(L != 0.f ? O / L : 0.f);
+                    a.out[(row0 + h) * kD + d] = __float2bfloat16_rn(L != 0.f ? O / L : 0.f);
                 }
             } else {
                 // one piece of several: a partial (o, m, l) for decode_combine_kernel
 #pragma unroll
                 for (int h = 0; h < HW; ++h) {
-                    const int hg = hs + h;
-                    if (hg >= g) break;
-                    const float L = ls[hg] + ls[N + hg] + ls[2 * N + hg] + ls[3 * N + hg];
-                    const size_t prow = ((size_t)pb * a.Hq + pkvh * g + hg) * a.nsplit + psplit;
-                    a.part_o[prow * kD + d] = __uint_as_float(o[h]);
-                    if (d == 0) {
-                        a.part_ml[prow * 2 + 0] = pm[h];
-                        a.part_ml[prow * 2 + 1] = L;
-                    }
+                    if (hs + h >= g) break;
+                    a.part_o[((row0 + h) * a.nsplit + (psplit & 0xffff)) * kD + d] = __uint_as_float(o[h]);
+                }
+                // the (m, l) pairs: lane h of the warpgroup's first warp writes head h's, one store each
+                if (quarter == 0 && lane < HW && hs + lane < g) {
+                    const int hg = hs + lane;
+                    const float mv = mst[pob * N + hg];
+                    const float lv = ls[hg] + ls[N + hg] + ls[2 * N + hg] + ls[3 * N + hg];
+                    *reinterpret_cast<float2 *>(a.part_ml + ((row0 + lane) * a.nsplit + (psplit & 0xffff)) * 2) =
+                        make_float2(mv, lv);
                 }
             }
             tc_fence_before();
@@ -1044,8 +1046,11 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             pkvh = kvh;
             psplit = split;
             pob = ob;
+            // the maxima the unit's weights are relative to, for its (deferred) partial
+            if (t == 0) {
 #pragma unroll
-            for (int h = 0; h < HW; ++h) pm[h] = m_use[h];
+                for (int h = 0; h < HW; ++h) mst[ob * N + hs + h] = m_use[h];
+            }
             tcount += ntl;
             ++icount;
         }

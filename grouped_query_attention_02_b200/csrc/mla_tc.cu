@@ -212,7 +212,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV2, const __grid_con
                 const int hb = u % a.nhb;
                 q[0] = it.x;
                 q[1] = hb;
-                q[2] = it.y;
+                q[2] = it.y & 0xffff;   // the piece index (the planner keeps the piece count above it)
                 q[3] = it.z;
                 q[4] = it.w;
                 mbar_arrive(&bar[I_FULL + slot]);
