@@ -282,34 +282,50 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             if (!wait_or_fail(&bar[PS_FULL + w], j & 1, a, err)) { ok = false; break; }
             tc_fence_after();
             const bool diag = (j == qtile);
-            // pass 1: the row maximum of the raw scores (keys after the row hidden on the diagonal);
-            // two 32-column loads per wait, three-input max, four independent partial maxima
+            // the row's 128 raw scores, loaded once (keys after the row hidden on the diagonal)
+            uint32_t sr[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
+            tmem_wait_ld();
+            if (diag) {
+#pragma unroll
+                for (int i = 0; i < 128; ++i)
+                    if (i > r) sr[i] = __float_as_uint(-INFINITY);
+            }
+            // the row maximum: three-input max, four independent partial maxima
             float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c2 = 0; c2 < 4; c2 += 2) {
-                uint32_t sr[64];
-                tmem_ld32(tS + c2 * 32, sr);
-                tmem_ld32(tS + c2 * 32 + 32, sr + 32);
-                tmem_wait_ld();
-                if (diag) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (c2 * 32 + i > r) sr[i] = __float_as_uint(-INFINITY);
-                }
-#pragma unroll
-                for (int i = 0; i < 64; i += 8) {
-                    pm[0] = fmax3(pm[0], __uint_as_float(sr[i + 0]), __uint_as_float(sr[i + 1]));
-                    pm[1] = fmax3(pm[1], __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
-                    pm[2] = fmax3(pm[2], __uint_as_float(sr[i + 4]), __uint_as_float(sr[i + 5]));
-                    pm[3] = fmax3(pm[3], __uint_as_float(sr[i + 6]), __uint_as_float(sr[i + 7]));
-                }
+            for (int i = 0; i < 128; i += 8) {
+                pm[0] = fmax3(pm[0], __uint_as_float(sr[i + 0]), __uint_as_float(sr[i + 1]));
+                pm[1] = fmax3(pm[1], __uint_as_float(sr[i + 2]), __uint_as_float(sr[i + 3]));
+                pm[2] = fmax3(pm[2], __uint_as_float(sr[i + 4]), __uint_as_float(sr[i + 5]));
+                pm[3] = fmax3(pm[3], __uint_as_float(sr[i + 6]), __uint_as_float(sr[i + 7]));
             }
             const float mraw = fmaxf(fmax3(pm[0], pm[1], pm[2]), pm[3]);
             const float m_new = fmaxf(m_run, mraw * a.qscale);
             const bool move = (m_new > m_run + kRescaleThreshold);
             const float m_use = move ? m_new : m_run;
             const float alpha = move ? ex2(m_run - m_new) : 1.f;
-            // O holds tiles < j (the S_FULL commit covers the previous PV): rescale when the max moved
+            // p = 2^(raw*qscale - m_use), summed, packed to bf16 pairs over S columns 0..63
+            const float2 sc2 = make_float2(a.qscale, a.qscale);
+            const float2 nm2 = make_float2(-m_use, -m_use);
+            float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                            make_float2(0.f, 0.f)};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const float2 e = __ffma2_rn(
+                        make_float2(__uint_as_float(sr[h * 32 + i]), __uint_as_float(sr[h * 32 + i + 1])), sc2, nm2);
+                    const float2 pe = make_float2(ex2(e.x), ex2(e.y));
+                    ps[(i >> 1) & 3] = __fadd2_rn(ps[(i >> 1) & 3], pe);
+                    pk[i >> 1] = pack_bf16x2(pe.x, pe.y);
+                }
+                tmem_st16(tS + h * 16, pk);
+            }
+            // O holds tiles < j (the S_FULL commit covers the previous PV): rescale when the max moved;
+            // PV of this tile is issued only after P_FULL below
             if (j > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -319,36 +335,6 @@ prefill_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
 #pragma unroll
                     for (int i = 0; i < 32; ++i) orow[i] = __float_as_uint(__uint_as_float(orow[i]) * alpha);
                     tmem_st32(tO + c * 32, orow);
-                }
-            }
-            // pass 2: p = 2^(raw*qscale - m_use), summed, packed to bf16 pairs over S columns 0..63
-            const float2 sc2 = make_float2(a.qscale, a.qscale);
-            const float2 nm2 = make_float2(-m_use, -m_use);
-            float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                            make_float2(0.f, 0.f)};
-#pragma unroll
-            for (int c2 = 0; c2 < 4; c2 += 2) {
-                uint32_t sr[64];
-                tmem_ld32(tS + c2 * 32, sr);
-                tmem_ld32(tS + c2 * 32 + 32, sr + 32);
-                tmem_wait_ld();
-                if (diag) {
-#pragma unroll
-                    for (int i = 0; i < 64; ++i)
-                        if (c2 * 32 + i > r) sr[i] = __float_as_uint(-INFINITY);
-                }
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const float2 e = __ffma2_rn(
-                            make_float2(__uint_as_float(sr[h * 32 + i]), __uint_as_float(sr[h * 32 + i + 1])), sc2, nm2);
-                        const float2 pe = make_float2(ex2(e.x), ex2(e.y));
-                        ps[(i >> 1) & 3] = __fadd2_rn(ps[(i >> 1) & 3], pe);
-                        pk[i >> 1] = pack_bf16x2(pe.x, pe.y);
-                    }
-                    tmem_st16(tS + (c2 + h) * 16, pk);
                 }
             }
             tmem_wait_st();
