@@ -106,13 +106,13 @@ struct KvSmem {
     static constexpr int bytes = err + 8;
 };
 // S^T and dP^T products complete (ST_FULL, DPT_FULL); P^T written (P_READY); dS^T written (DST_READY);
-// the dV and dK products that read them complete (DV_DONE, DK_DONE)
+// (slots 13 and 14 are unused: the products that overwrite P^T and dS^T follow their readers in issue order)
 // ST_READ / DPT_READ: the first elementwise warpgroup has read the raw columns the second one's packed
 // output lands on
 // RS_FULL: the row statistics of an iteration are in shared memory (the elementwise threads load them one
 // iteration ahead, so their global-memory latency hides behind a whole iteration)
 enum KvBar { KV_FULL = 0, QD_FULL = 1, QD_EMPTY = 3, RS_FULL = 5, ST_FULL = 9, DPT_FULL = 10,
-             P_READY = 11, DST_READY = 12, DV_DONE = 13, DK_DONE = 14, ACC_FULL = 15, KDRAIN = 16, ST_READ = 17,
+             P_READY = 11, DST_READY = 12, ACC_FULL = 15, KDRAIN = 16, ST_READ = 17,
              DPT_READ = 18 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -149,8 +149,6 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_init(&bar[DPT_FULL], 1);
         mbar_init(&bar[P_READY], kEw);
         mbar_init(&bar[DST_READY], kEw);
-        mbar_init(&bar[DV_DONE], 1);
-        mbar_init(&bar[DK_DONE], 1);
         mbar_init(&bar[ACC_FULL], 1);
         mbar_init(&bar[KDRAIN], 1);
         mbar_init(&bar[ST_READ], kEw / 2);
@@ -199,30 +197,34 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
     } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer.  The elementwise pass hands over P^T before it computes dS^T, so
-        // dV += P^T dO runs while dS^T is being formed, and the next S^T once dV has read P^T.
+        // dV += P^T dO runs while dS^T is being formed, and the next S^T is issued right behind that dV
+        // product (it overwrites the P^T columns dV reads; tcgen05 products of a CTA run in issue order),
+        // so that the next iteration's scores are ready when the elementwise threads finish dS^T.  Per
+        // iteration: dP^T(n), dV(n), S^T(n+1), dK(n).
         if (lane == 0) {
             const uint32_t idesc_s = umma_idesc_bf16(kB, kB, 0, 0);   // K (K-major) x Q (K-major) -> S^T
             const uint32_t idesc_g = umma_idesc_bf16(kB, kD, 0, 1);   // P^T / dS^T (TMEM) x dO / Q (MN-major)
             const uint32_t k_addr = smem_u32(smem + KvSmem::k), v_addr = smem_u32(smem + KvSmem::v);
-            bool ok = wait_or_fail(&bar[KV_FULL], 0, a, err);
-            int done = 0;
-            for (int n = 0; ok && n < n_it; ++n) {
-                const int s = n & 1;
-                if (!wait_or_fail(&bar[QD_FULL + s], (n >> 1) & 1, a, err)) break;
-                const uint32_t q_addr = smem_u32(smem + KvSmem::q + s * kTile);
-                const uint32_t o_addr = smem_u32(smem + KvSmem::dout + s * kTile);
-                // S^T: its columns held the previous P^T, read by the previous dV product
-                if (n >= 1 && !wait_or_fail(&bar[DV_DONE], (n - 1) & 1, a, err)) break;
-                tc_fence_after();
+            auto issue_st = [&](int n) {
+                const uint32_t q_addr = smem_u32(smem + KvSmem::q + (n & 1) * kTile);
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
                     umma_ss(tS, desc_kmajor(k_addr + off), desc_kmajor(q_addr + off), idesc_s, ks > 0 ? 1u : 0u);
                 }
                 umma_commit(&bar[ST_FULL]);
-                // dP^T: its columns held the previous dS^T, read by the previous dK product
-                if (n >= 1 && !wait_or_fail(&bar[DK_DONE], (n - 1) & 1, a, err)) break;
+            };
+            bool ok = wait_or_fail(&bar[KV_FULL], 0, a, err) && wait_or_fail(&bar[QD_FULL], 0, a, err);
+            if (ok) {
                 tc_fence_after();
+                issue_st(0);
+            }
+            int done = 0;
+            for (int n = 0; ok && n < n_it; ++n) {
+                const int s = n & 1;
+                const uint32_t q_addr = smem_u32(smem + KvSmem::q + s * kTile);
+                const uint32_t o_addr = smem_u32(smem + KvSmem::dout + s * kTile);
+                // dP^T: its columns held the previous dS^T, read by the previous dK product (issued before)
 #pragma unroll
                 for (int ks = 0; ks < kD / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
@@ -235,14 +237,18 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
                 for (int ks = 0; ks < kB / 16; ++ks)
                     umma_ts(tdV, tS + ks * 8, desc_mnmajor(o_addr + ks * 2048), idesc_g, (n > 0 || ks > 0) ? 1u : 0u);
-                umma_commit(&bar[DV_DONE]);
+                // the next iteration's S^T, behind this dV product
+                if (n + 1 < n_it) {
+                    if (!wait_or_fail(&bar[QD_FULL + (s ^ 1)], ((n + 1) >> 1) & 1, a, err)) break;
+                    tc_fence_after();
+                    issue_st(n + 1);
+                }
                 // dK += dS^T Q
                 if (!wait_or_fail(&bar[DST_READY], n & 1, a, err)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < kB / 16; ++ks)
                     umma_ts(tdK, tdP + ks * 8, desc_mnmajor(q_addr + ks * 2048), idesc_g, (n > 0 || ks > 0) ? 1u : 0u);
-                umma_commit(&bar[DK_DONE]);
                 umma_commit(&bar[QD_EMPTY + s]);
                 done = n + 1;
             }
