@@ -134,7 +134,10 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int b = bk / a.Hkv, kvh = bk % a.Hkv;
     const int g = a.group;
     const int nq = nt - kt;                 // query tiles kt .. nt-1
-    const int n_it = g * nq;                // (head, query tile) iterations
+    // (head, query tile) iterations: query tiles from the last down to kt, the group's heads innermost,
+    // so that the CTAs of one KV head, which start together, read the same query and dO tiles at the
+    // same time and L2 serves all but the first of them
+    const int n_it = g * nq;
     const int k0 = kt * kB;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -180,7 +183,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             tma_load_4d(smem + KvSmem::v + kHalf, &tmV, &bar[KV_FULL], 64, kvh, k0, b);
             int issued = 0;
             for (int n = 0; n < n_it; ++n) {
-                const int h = kvh * g + n / nq, q0 = (kt + n % nq) * kB, s = n & 1;
+                const int h = kvh * g + n % g, q0 = (nt - 1 - n / g) * kB, s = n & 1;
                 if (n >= 2 && !wait_or_fail(&bar[QD_EMPTY + s], ((n >> 1) - 1) & 1, a, err)) break;
                 mbar_arrive_expect_tx(&bar[QD_FULL + s], 2 * kTile);
                 uint8_t *qs = smem + KvSmem::q + s * kTile, *ds = smem + KvSmem::dout + s * kTile;
@@ -268,7 +271,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         // row statistic t of iteration n's query tile: lse * log2(e) (warpgroup 0) or D (warpgroup 1); rows
         // past the sequence get lse = +inf (P = 0) and D = 0
         auto row_stat = [&](int n) -> float {
-            const int h = kvh * g + n / nq, r = (kt + n % nq) * kB + t;
+            const int h = kvh * g + n % g, r = (nt - 1 - n / g) * kB + t;
             const size_t i = ((size_t)b * a.Hq + h) * a.S + r;
             return w == 0 ? (r < a.S ? a.lse[i] * kLog2e : INFINITY) : (r < a.S ? a.dsum[i] : 0.f);
         };
@@ -277,7 +280,7 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         mbar_arrive(&bar[RS_FULL]);
         for (int n = 0; n < n_it; ++n) {
             const int s = n & 1;
-            const bool diag = (n % nq) == 0;      // the query tile that holds this CTA's keys
+            const bool diag = n / g == nq - 1;    // the query tile that holds this CTA's keys (the last)
             if (!wait_or_fail(&bar[RS_FULL + s], (n >> 1) & 1, a, err)) { ok = false; break; }
             // the next iteration's statistic, in flight during this iteration
             const float next_stat = n + 1 < n_it ? row_stat(n + 1) : 0.f;
@@ -532,8 +535,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 if (j < ntiles) {
                     const int s = j & 1, sk = j % QSmem::kstages, sv = j % QSmem::vstages;
                     if (!wait_or_fail(&bar[K2_FULL + sk], (j / QSmem::kstages) & 1, a, err)) break;
-                    // this S buffer's previous dS was read by the dQ product of tile j - 2
-                    if (j >= 2 && !wait_or_fail(&bar[S2_FREE + s], ((j >> 1) - 1) & 1, a, err)) break;
+                    // this S buffer's previous dS is read by the dQ product of tile j - 2, issued before
                     tc_fence_after();
                     const uint32_t k_addr = smem_u32(smem + QSmem::k + sk * kTile);
                     const uint32_t v_addr = smem_u32(smem + QSmem::v + sv * kTile);
