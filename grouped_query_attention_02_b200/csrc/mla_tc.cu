@@ -56,7 +56,10 @@ constexpr int kHW = kNh / kNWG;                   // heads per warpgroup (32)
 constexpr int kProducerWarp = 4 * kNWG;
 constexpr int kMmaWarp = kProducerWarp + 1;
 constexpr int kPrefetchWarp = kMmaWarp + 1;       // keeps the tiles kAhead ahead of the producer in L2
-constexpr int kThreads = kWG * kNWG + 96;
+// A second TMA issuer: one thread completes about one box per 300 ns whatever its size, so the odd latent
+// chunk pairs of every tile come from this warp while the producer issues the even ones and the RoPE chunk
+constexpr int kCoProducerWarp = kPrefetchWarp + 1;
+constexpr int kThreads = kWG * kNWG + 128;
 constexpr int kAhead = 2;
 constexpr int kQD = 4;                            // depth of the unit queue
 constexpr float kMoveThreshold = 8.0f;            // the running maximum moves only by more than this
@@ -165,7 +168,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV2, const __grid_con
         mbar_init(&bar[O_FREE], kWG * kNWG);
         for (int s = 0; s < kQD; ++s) {
             mbar_init(&bar[I_FULL + s], 1);
-            mbar_init(&bar[I_EMPTY + s], 2 + kWG * kNWG);   // the MMA issuer, the prefetcher, the softmax threads
+            mbar_init(&bar[I_EMPTY + s], 3 + kWG * kNWG);   // MMA issuer, prefetcher, co-producer, softmax threads
         }
         mbar_init(&bar[DRAIN], 1);
         for (int w = 0; w < kNWG; ++w) mbar_init(&bar[GRP + w], kWG);
@@ -195,8 +198,9 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV2, const __grid_con
             tma_prefetch_desc(&tmQ);
             const int units = a.plan_hdr[1] * a.nhb;
             int icount = 0, T = 0;
-            // for the drain: tiles whose loads were all issued, loads issued of the tile after them
-            int full_tiles = 0, part_groups = 0, q_loads = 0;
+            // for the drain: loads issued per group (this warp issues the even chunk pairs and the RoPE chunk)
+            int issued[kGroups] = {};
+            int q_loads = 0;
             bool ok = true;
             while (ok) {
                 const int u = atomicAdd(a.claim, 1);
@@ -225,7 +229,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV2, const __grid_con
                 const int ntl = (it.w - it.z + kTok - 1) / kTok;
                 for (int jj = 0; jj < ntl && ok; ++jj, ++T) {
                     const int t0 = it.z + jj * kTok;
-                    for (int g = 0; g < kGroups; ++g) {
+                    for (int g = 0; g < kGroups; g += 2) {
                         // the previous tile's PV product has finished with these slots (its O^T block, or
                         // for the last slot the whole product that read P^T there)
                         if (T >= 1 && !wait_or_fail(&bar[g < kGroups - 1 ? EMPTY_PAIR + g : EMPTY_P], (T - 1) & 1,
@@ -243,22 +247,48 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV2, const __grid_con
                             mbar_arrive_expect_tx(&bar[CH_FULL + g], kChunkBytes);
                             tma_load_3d(dst, &tmKV1, &bar[CH_FULL + g], kMlaLatent, t0, it.x);
                         }
-                        part_groups = g + 1;
+                        ++issued[g];
                     }
-                    if (part_groups == kGroups) {
-                        ++full_tiles;
-                        part_groups = 0;
-                        *reinterpret_cast<volatile int *>(smem + kIssuedOff) = full_tiles;
-                    }
+                    if (ok) *reinterpret_cast<volatile int *>(smem + kIssuedOff) = T + 1;
                 }
                 ++icount;
             }
             // leave no copy in flight
-            for (int g = 0; g < kGroups; ++g) {
-                const int n = full_tiles + (g < part_groups ? 1 : 0);   // loads issued for group g
-                if (n >= 1) mbar_wait(&bar[CH_FULL + g], (n - 1) & 1, a.wait_budget_ns);
-            }
+            for (int g = 0; g < kGroups; g += 2)
+                if (issued[g] >= 1) mbar_wait(&bar[CH_FULL + g], (issued[g] - 1) & 1, a.wait_budget_ns);
             if (q_loads >= 1) mbar_wait(&bar[Q_FULL], (q_loads - 1) & 1, a.wait_budget_ns);
+        }
+    } else if (warp == kCoProducerWarp) {
+        // ---------------- co-producer: the odd latent chunk pairs of every tile, in the producer's order
+        if (lane == 0) {
+            int icount = 0, T = 0;
+            int issued[kGroups] = {};
+            bool ok = true;
+            while (ok) {
+                const int slot = icount % kQD;
+                if (!wait_or_fail(&bar[I_FULL + slot], (icount / kQD) & 1, a, err)) break;
+                volatile int *q = queue + slot * 8;
+                const int b = q[0], t_begin = q[3], t_end = q[4];
+                mbar_arrive(&bar[I_EMPTY + slot]);
+                if (t_end < 0) break;
+                const int ntl = (t_end - t_begin + kTok - 1) / kTok;
+                for (int jj = 0; jj < ntl && ok; ++jj, ++T) {
+                    const int t0 = t_begin + jj * kTok;
+                    for (int g = 1; g < kGroups - 1; g += 2) {
+                        if (T >= 1 && !wait_or_fail(&bar[EMPTY_PAIR + g], (T - 1) & 1, a, err)) {
+                            ok = false;
+                            break;
+                        }
+                        uint8_t *dst = smem + kSlotOff + 2 * g * kChunkBytes;
+                        mbar_arrive_expect_tx(&bar[CH_FULL + g], 2 * kChunkBytes);
+                        tma_load_4d(dst, &tmKV2, &bar[CH_FULL + g], 0, t0, 2 * g, b);
+                        ++issued[g];
+                    }
+                }
+                ++icount;
+            }
+            for (int g = 1; g < kGroups - 1; g += 2)
+                if (issued[g] >= 1) mbar_wait(&bar[CH_FULL + g], (issued[g] - 1) & 1, a.wait_budget_ns);
         }
     } else if (warp == kPrefetchWarp) {
         // ---------------- L2 prefetcher: tile T of the CTA's stream goes to L2 once the producer has issued
