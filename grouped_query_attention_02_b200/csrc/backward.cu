@@ -8,20 +8,20 @@
 //   dP = dO V^T,  D = rowsum(dO * O),   dS = P * (dP - D)
 //   dV = sum over the group of P^T dO,  dK = scale * sum over the group of dS^T Q,  dQ = scale * dS K
 //
-// Three kernels:
-//   bwd_rowdot_kernel   D = rowsum(dO * O) in fp32, one warp per (sequence, row, head)
+// Two kernels, the dQ kernel first:
 //   bwd_dkdv_kernel     one CTA per (sequence, KV head, 128-key tile): loops over the g query heads
 //                       of the group and over the query tiles at or after the key tile; S^T = K Q^T and
 //                       dP^T = V dO^T into tensor memory, P^T and dS^T back into tensor memory as bf16,
 //                       then dV += P^T dO and dK += dS^T Q with the accumulators resident in tensor
 //                       memory for the whole loop, so the group sum costs nothing extra
-//   bwd_dq_kernel       one CTA per (sequence, query head, 128-row tile): loops over the key tiles up
-//                       to the diagonal; S = Q K^T and dP = dO V^T, dS back into tensor memory, then
-//                       dQ += dS K
+//   bwd_dq_kernel       one CTA per (sequence, query head, 128-row tile): first D = rowsum(dO * O) of
+//                       its rows (left in the workspace for the dK/dV kernel), then a loop over the key
+//                       tiles up to the diagonal: S = Q K^T and dP = dO V^T, dS back into tensor memory,
+//                       then dQ += dS K
 //
-// Roles in both tensor-core kernels (192 threads): warps 0..3 elementwise (one TMEM lane each: a key
-// row of S^T in the dK/dV kernel, a query row of S in the dQ kernel), warp 4 TMA producer, warp 5
-// TMEM allocator + MMA issuer.  The probabilities and dS are rounded to bf16 for the products, as the
+// Roles in both kernels (320 threads): warps 0..7 elementwise in two warpgroups of 64 columns each (one
+// TMEM lane per thread: a key row of S^T in the dK/dV kernel, a query row of S in the dQ kernel),
+// warp 8 TMA producer, warp 9 TMEM allocator + MMA issuer.  The probabilities and dS are rounded to bf16 for the products, as the
 // forward rounds P.  Every wait is bounded; a kernel that gives up records GQA_ERR_DEVICE_TIMEOUT.
 #include "internal.h"
 #include "ptx.cuh"
@@ -68,25 +68,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
-}
-
-// D[b][h][r] = sum_j dO[b,r,h,j] * O[b,r,h,j]: one warp per row, four elements per lane.
-__global__ void bwd_rowdot_kernel(const BackwardArgs a)
-{
-    const long long rows = (long long)a.B * a.S * a.Hq;
-    const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (wid >= rows) return;
-    const int h = (int)(wid % a.Hq);
-    const long long br = wid / a.Hq;
-    const int r = (int)(br % a.S), b = (int)(br / a.S);
-    const uint2 o = *reinterpret_cast<const uint2 *>(a.out + wid * kD + lane * 4);
-    const uint2 g = *reinterpret_cast<const uint2 *>(a.dout + wid * kD + lane * 4);
-    float s = bf16_lo(o.x) * bf16_lo(g.x) + bf16_hi(o.x) * bf16_hi(g.x) + bf16_lo(o.y) * bf16_lo(g.y) +
-              bf16_hi(o.y) * bf16_hi(g.y);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) a.dsum[((size_t)b * a.Hq + h) * a.S + r] = s;
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -587,11 +568,30 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         const int qrow = q0 + r;
         const size_t rs = ((size_t)b * a.Hq + h) * a.S + qrow;
         const float lse2 = qrow < a.S ? a.lse[rs] * kLog2e : INFINITY;
-        const float dsum = qrow < a.S ? a.dsum[rs] : 0.f;
+        // D = rowsum(dO * O) of this row in fp32, from the dO tile in shared memory and the row of O in
+        // global memory; the first warpgroup leaves it in the workspace for the dK/dV kernel, which runs next
+        bool ok = wait_or_fail(&bar[QO_FULL], 0, a, err);
+        float dsum = 0.f;
+        if (ok && qrow < a.S) {
+            const uint4 *orow = reinterpret_cast<const uint4 *>(a.out + (((size_t)b * a.S + qrow) * a.Hq + h) * kD);
+            const uint8_t *grow = smem + QSmem::dout + r * 128;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    // the 128-byte swizzle: chunk c of row r sits at chunk c ^ (r % 8)
+                    const uint4 gv = *reinterpret_cast<const uint4 *>(grow + hf * kHalf + ((c ^ (r & 7)) << 4));
+                    const uint4 ov = orow[hf * 8 + c];
+                    dsum += bf16_lo(gv.x) * bf16_lo(ov.x) + bf16_hi(gv.x) * bf16_hi(ov.x) + bf16_lo(gv.y) * bf16_lo(ov.y) +
+                            bf16_hi(gv.y) * bf16_hi(ov.y) + bf16_lo(gv.z) * bf16_lo(ov.z) + bf16_hi(gv.z) * bf16_hi(ov.z) +
+                            bf16_lo(gv.w) * bf16_lo(ov.w) + bf16_hi(gv.w) * bf16_hi(ov.w);
+                }
+            }
+            if (w == 0) a.dsum[rs] = dsum;
+        }
         const float2 qs2 = make_float2(a.qscale, a.qscale), nl2 = make_float2(-lse2, -lse2);
         const float2 nd2 = make_float2(-dsum, -dsum);
-        bool ok = true;
-        for (int j = 0; j < ntiles; ++j) {
+        for (int j = 0; ok && j < ntiles; ++j) {
             const int s = j & 1;
             // dP into registers first, then release it for the next tile's product
             if (!wait_or_fail(&bar[DP_FULL], j & 1, a, err)) { ok = false; break; }
@@ -684,19 +684,15 @@ cudaError_t launch_prefill_backward(const CUtensorMap &tmQ, const CUtensorMap &t
             return e;
         attr_done[dev] = true;
     }
-    const long long rows = (long long)a.B * a.S * a.Hq;
-    const long long blocks = (rows * 32 + 255) / 256;
     const long long nt = (a.S + kB - 1) / kB;
     const long long grid_kv = nt * a.B * a.Hkv, grid_q = nt * a.B * a.Hq;
-    if (blocks > 0x7fffffffLL || grid_q > 0x7fffffffLL) return cudaErrorInvalidValue;
-    bwd_rowdot_kernel<<<(unsigned)blocks, 256, 0, stream>>>(a);
+    if (grid_q > 0x7fffffffLL) return cudaErrorInvalidValue;
+    // the dQ kernel first: it also forms D = rowsum(dO * O), which the dK/dV kernel reads
+    bwd_dq_kernel<<<(unsigned)grid_q, kThreads, smem_q, stream>>>(tmQ, tmK, tmV, tmDO, a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     ++*launches;
     bwd_dkdv_kernel<<<(unsigned)grid_kv, kThreads, smem_kv, stream>>>(tmQ, tmK, tmV, tmDO, a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    ++*launches;
-    bwd_dq_kernel<<<(unsigned)grid_q, kThreads, smem_q, stream>>>(tmQ, tmK, tmV, tmDO, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;
     return cudaSuccess;

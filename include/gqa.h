@@ -184,8 +184,9 @@ gqa_status gqa_prefill_causal_fwd(const void *q, const void *k, const void *v, i
  * With P = exp(q.k / sqrt(d) - lse) (causal), dP = dout v^T, D = rowsum(dout * out),
  * dS = P (dP - D): dv = sum_h P^T dout, dk = sum_h dS^T q / sqrt(d), dq = dS k / sqrt(d).
  * P and dS are rounded to bf16 for the tensor-core products (fp32 accumulation); D is
- * computed from the bf16 out.  Uses B*Hq*S*4 bytes of the library workspace; three
- * kernels.  Same layouts, alignment and error rules as gqa_prefill_causal.
+ * computed from the bf16 out.  Uses B*Hq*S*4 bytes of the library workspace; two
+ * kernels (dq, which also forms D, then dk/dv).  Same layouts, alignment and error rules as
+ * gqa_prefill_causal.
  */
 gqa_status gqa_prefill_causal_bwd(const void *q, const void *k, const void *v, const void *out, const float *lse,
                                   const void *dout, int B, int S, int Hq, int Hkv, int d, void *dq, void *dk,
@@ -312,7 +313,7 @@ gqa_status gqa_selftest_wait_timeout(int timeout_us, void *stream);
  * gqa_mla_decode / gqa_prefill_causal(_fwd) / gqa_decode_expanded records `before` on its stream
  * immediately before its dominant kernel (the decode kernel; the prefill
  * kernel) and `after` immediately after it; gqa_prefill_causal_bwd records
- * them around its three kernels; gqa_decode_noalloc records nothing.  NULL,
+ * them around its two kernels; gqa_decode_noalloc records nothing.  NULL,
  * NULL turns the hook off.
  */
 gqa_status gqa_set_profile_events(void *before, void *after);
