@@ -227,6 +227,10 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     __shared__ int s_C, s_sum;
     int *full_off = a.plan_scratch;     // per-sequence offsets of the full pieces (B ints, global)
 
+    // launched as a programmatic dependent of whatever ran before on the stream (the previous call's
+    // combine, say, which still reads nsplit_b): wait for it before touching anything, so that only the
+    // launch overlaps it
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // the persistent kernel may start its prologue now; it reads this plan only after griddepcontrol.wait
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -1107,8 +1111,16 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
 
 cudaError_t launch_decode_plan(const DecodeArgs &a, cudaStream_t stream)
 {
-    decode_plan_kernel<<<1, kPlanThreads, 0, stream>>>(a, a.num_ctas);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kPlanThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_plan_kernel, a, a.num_ctas);
 }
 
 cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, const CUtensorMap &tmQ,
