@@ -257,10 +257,6 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             return w == 0 ? (r < a.S ? a.lse[i] * kLog2e : INFINITY) : (r < a.S ? a.dsum[i] : 0.f);
         };
         float *stat_smem = reinterpret_cast<float *>(smem + (w == 0 ? KvSmem::lse : KvSmem::dsum));
-        // launched as a programmatic dependent of the dQ kernel, which writes D: the elementwise threads
-        // (the only readers of D) wait for it here; the loads and products of the other roles read only
-        // the inputs and may start in the dQ kernel's tail
-        asm volatile("griddepcontrol.wait;" ::: "memory");
         stat_smem[t] = row_stat(0);
         mbar_arrive(&bar[RS_FULL]);
         for (int n = 0; n < n_it; ++n) {
@@ -464,8 +460,6 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    // the dK/dV kernel may be scheduled into this grid's tail; it waits for D before reading it
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
     // S[2] (dS is packed into the S buffer it came from), dP, the dQ accumulator
     const uint32_t tS0 = tmem, tdP = tmem + 256, tdQ = tmem + 384;
@@ -698,19 +692,8 @@ cudaError_t launch_prefill_backward(const CUtensorMap &tmQ, const CUtensorMap &t
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     ++*launches;
-    {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)grid_kv);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = smem_kv;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if ((e = cudaLaunchKernelEx(&cfg, bwd_dkdv_kernel, tmQ, tmK, tmV, tmDO, a)) != cudaSuccess) return e;
-    }
+    bwd_dkdv_kernel<<<(unsigned)grid_kv, kThreads, smem_kv, stream>>>(tmQ, tmK, tmV, tmDO, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     ++*launches;
     return cudaSuccess;
 }
