@@ -278,16 +278,31 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     __syncthreads();
     const int C = s_C;
     const bool sort_rem = C <= kPlanMaxC;
+    // A history's remainder (tl % C tiles) is cut into up to tail_split pieces of nearly equal size
+    // (never more than nsplit pieces in all): the shortest units are claimed last, so that the CTAs
+    // finish together even when some of them stream their tiles more slowly than others.
+    const int tsplit = a.tail_split > 1 ? a.tail_split : 1;
+    auto tail_pieces = [&](int full, int rem) -> int {
+        if (rem <= 0) return 0;
+        int k = tsplit < rem ? tsplit : rem;
+        if (k > a.nsplit - full) k = a.nsplit - full;
+        return k > 1 ? k : 1;
+    };
     int npieces = 0;
     for (int b = tid; b < a.B; b += blockDim.x) {
         int T = a.seqlens[b];
         T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
         const int tl = (T + kTok - 1) / kTok;
-        const int rem = tl % C;
-        full_off[b] = tl / C;
-        a.nsplit_b[b] = tl / C + (rem > 0 ? 1 : 0);
-        npieces += tl / C + (rem > 0 ? 1 : 0);
-        if (rem > 0 && sort_rem) atomicAdd(&hist[C - 1 - rem], 1);   // reversed: longest remainder first
+        const int full = tl / C, rem = tl % C;
+        const int k = tail_pieces(full, rem);
+        full_off[b] = full;
+        a.nsplit_b[b] = full + k;
+        npieces += full + k;
+        if (sort_rem)
+            for (int j = 0; j < k; ++j) {
+                const int size = rem / k + (j < rem % k ? 1 : 0);
+                atomicAdd(&hist[C - 1 - size], 1);   // reversed: longest first
+            }
     }
     __syncthreads();
     const int P = block_sum(npieces, red_i, &s_sum);
@@ -295,13 +310,14 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     for (int b = tid; b < a.B; b += blockDim.x) nfull += full_off[b];
     const int F = block_sum(nfull, red_i, &s_sum);
     block_exclusive_scan(full_off, a.B, warp_tot);
-    if (sort_rem) block_exclusive_scan(hist, C, warp_tot);   // hist[C-1-r]: remainders longer than r
+    if (sort_rem) block_exclusive_scan(hist, C, warp_tot);   // hist[C-1-r]: tail pieces longer than r
     for (int b = tid; b < a.B; b += blockDim.x) {
         int T = a.seqlens[b];
         T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
         const int tl = (T + kTok - 1) / kTok;
         const int full = tl / C, rem = tl % C;
-        const int np_b = full + (rem > 0 ? 1 : 0);
+        const int k = tail_pieces(full, rem);
+        const int np_b = full + k;
         if (tl == 0) {
             // no cached token: no unit will touch this sequence, its output rows are zero
             const int orow = a.out_row > 0 ? a.out_row : kD;
@@ -310,10 +326,13 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         }
         for (int s = 0; s < full; ++s)
             a.items[full_off[b] + s] = make_int4(b, s | (np_b << 16), s * C * kTok, min((s + 1) * C * kTok, T));
-        if (rem > 0) {
-            const int k = C - 1 - rem;
-            const int pos = sort_rem ? F + hist[k] + atomicAdd(&cursor[k], 1) : F + atomicAdd(&cursor[0], 1);
-            a.items[pos] = make_int4(b, full | (np_b << 16), full * C * kTok, T);
+        int start = full * C;   // first tile of the next tail piece
+        for (int j = 0; j < k; ++j) {
+            const int size = rem / k + (j < rem % k ? 1 : 0);
+            const int kk = C - 1 - size;
+            const int pos = sort_rem ? F + hist[kk] + atomicAdd(&cursor[kk], 1) : F + atomicAdd(&cursor[0], 1);
+            a.items[pos] = make_int4(b, (full + j) | (np_b << 16), start * kTok, min((start + size) * kTok, T));
+            start += size;
         }
     }
     if (tid == 0) {

@@ -41,6 +41,7 @@ struct DecodeArgs {
     int out_row;              // output elements per (sequence, query head) row, zeroed for empty histories
     int plan_rounds;          // rounds of units per persistent CTA the pieces are sized for
     int static_plan;          // 1: no planner; one piece per history, units dealt round-robin (short caches)
+    int tail_split;           // planner: a history's remainder is cut into up to this many pieces (0, 1: one)
 };
 
 // Host plan of a decode call and the layout of its workspace.
