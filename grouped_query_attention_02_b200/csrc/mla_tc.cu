@@ -652,7 +652,10 @@ cudaError_t launch_mla_decode_tc(const CUtensorMap &tmKV2, const CUtensorMap &tm
     pa.items = reinterpret_cast<int4 *>(w + p.off_items);
     pa.num_ctas = num_sms;
     pa.out_row = kMlaLatent;
-    pa.plan_rounds = 2;
+    // one round of long pieces per CTA, each history's remainder cut into four (a sweep over 1-6 rounds
+    // and 1-4 tail pieces at the DeepSeek-V3 shape: 190 -> 180 us against two rounds of whole pieces)
+    pa.plan_rounds = 1;
+    pa.tail_split = 4;
     cudaError_t e = launch_decode_plan(pa, stream);
     if (e != cudaSuccess) return e;
     ++*launches;
