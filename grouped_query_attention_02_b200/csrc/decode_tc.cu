@@ -264,10 +264,10 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
             T += red_ll[i];
             M = max(M, red_i[i]);
         }
-        // rounds of (piece, KV head) units per persistent CTA: eight for groups up to 8, four for groups
-        // of 9-16 and two above 16, whose units of more heads carry a larger fixed cost each (measured
-        // on the benchmark shapes); never more than nsplit pieces
-        const long long rounds = a.plan_rounds > 0 ? a.plan_rounds : (a.group > 16 ? 2 : (a.group > 8 ? 4 : 8));
+        // rounds of (piece, KV head) units per persistent CTA: eight for groups up to 8, two above, whose
+        // units of more heads carry a larger fixed cost each (measured on the benchmark shapes); never
+        // more than nsplit pieces
+        const long long rounds = a.plan_rounds > 0 ? a.plan_rounds : (a.group > 8 ? 2 : 8);
         long long C = (T * a.Hkv + rounds * slots - 1) / (rounds * slots);
         const long long cmin = (M + a.nsplit - 1) / a.nsplit;
         if (C < cmin) C = cmin;
