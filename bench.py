@@ -207,6 +207,30 @@ def time_decode(gqa, torch, x, steps: int, warmup: int, expanded=None):
     return step_ms, kern_ms, launches, out
 
 
+def time_decode_graph(gqa, torch, x, calls: int = 20, replays: int = 50):
+    """Mean step time (ms) of the decode replayed from a CUDA graph that captured `calls` calls (the
+    serving loop's form: no host work per step)."""
+    out = torch.empty_like(x.q)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            decode_call(gqa, x, out)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(calls):
+            decode_call(gqa, x, out)
+    g.replay()
+    torch.cuda.synchronize()
+    s0, s1 = _events(torch)
+    s0.record()
+    for _ in range(replays):
+        g.replay()
+    s1.record()
+    torch.cuda.synchronize()
+    return s0.elapsed_time(s1) / (replays * calls)
+
+
 def time_prefill(gqa, torch, p, steps: int, warmup: int):
     out = torch.empty_like(p.q)
     for _ in range(warmup):
@@ -716,6 +740,8 @@ def main():
                              "kernel_frac_hbm": uu / (k_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                              "frac_hbm": uu / (st_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                              "tokens_per_s": ww.B / (st_ms * 1e-3), "launches_per_step": n / (10 if ww.B * ww.Tmax > 1e5 else 50)}
+            if ww is workloads.TINY_DECODE:
+                rows[ww.name]["graph_ms_per_step"] = time_decode_graph(gqa, torch, xx)
             del xx
             torch.cuda.empty_cache()
         # expanded repeat-KV baseline on the headline workload

@@ -233,3 +233,35 @@ def test_profile_events_bracket_the_decode_kernel():
     finally:
         gqa.gqa_set_profile_events(None, None)
     assert e0.elapsed_time(e1) > 0
+
+
+# ---------------------------------------------------------------- CUDA graphs
+
+
+@pytest.mark.parametrize("shape", [(1, 8, 2, 256, None), (4, 32, 8, 4096, [4096, 3000, 129, 1]), (3, 32, 1, 3000, None)],
+                         ids=["one-launch", "planned-split", "mqa"])
+def test_decode_replays_in_a_cuda_graph(oracle_mod, shape):
+    """A decode call captured once in a CUDA graph and replayed: no allocation, host work or
+    synchronisation inside the call (after a first call has sized the workspace), and the graph reads
+    the live inputs at every replay."""
+    B, Hq, Hkv, Tmax, lens = shape
+    x = inputs.make_decode(B, Hq, Hkv, 128, Tmax, seqlens=lens, device=DEV, seed=60 + Hkv)
+    out = torch.empty_like(x.q)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out)   # sizes the workspace
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        gqa.gqa_decode(x.q, x.k_cache, x.v_cache, x.seqlens, x.scale, out=out)
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    _check_all(oracle_mod, x, out)
+    # new query rows in place: the replay must see them
+    x.q.copy_(inputs.make_decode(B, Hq, Hkv, 128, Tmax, seqlens=lens, device=DEV, seed=160 + Hkv).q)
+    g.replay()
+    torch.cuda.synchronize()
+    assert gqa.gqa_get_last_device_status() == 0
+    _check_all(oracle_mod, x, out)
+

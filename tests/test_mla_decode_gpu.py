@@ -155,3 +155,26 @@ def test_mla_deterministic_on_a_side_stream(oracle_mod):
         b = gqa.gqa_mla_decode(x.q, x.kv_cache, x.seqlens, x.scale, stream=s)
     s.synchronize()
     assert torch.equal(a, b)
+
+
+def test_mla_decode_replays_in_a_cuda_graph(oracle_mod):
+    """The planned MLA decode (planner, tensor-core kernel, combine) captured once in a CUDA graph and
+    replayed, with new query rows in place between replays."""
+    x = inputs.make_mla_decode(4, 64, 3000, device=DEV, seed=12, seqlen_range=(1, 3000))
+    out = torch.empty((4, 64, x.d_c), dtype=torch.bfloat16, device=DEV)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        gqa.gqa_mla_decode(x.q, x.kv_cache, x.seqlens, x.scale, out=out)   # sizes the workspace
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        gqa.gqa_mla_decode(x.q, x.kv_cache, x.seqlens, x.scale, out=out)
+    out.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    _check_tc(out, _ref(oracle_mod, x), x)
+    x.q.copy_(inputs.make_mla_decode(4, 64, 3000, device=DEV, seed=13, seqlen_range=(1, 3000)).q)
+    g.replay()
+    torch.cuda.synchronize()
+    assert gqa.gqa_get_last_device_status() == 0
+    _check_tc(out, _ref(oracle_mod, x), x)
