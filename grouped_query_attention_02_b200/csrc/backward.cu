@@ -278,6 +278,13 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                 tmem_ld32(tS + lane_off + w * 64 + 32, sr + 32);
                 tmem_wait_ld();
                 if (w == 0) mbar_arrive(&bar[ST_READ]);
+                if (diag) {
+                    // query c of the tile sees key t only when c >= t on the diagonal tile (weight 2^-inf = 0);
+                    // masked before the loop below, which then has no branch
+#pragma unroll
+                    for (int i = 0; i < 64; ++i)
+                        if (w * 64 + i < t) sr[i] = __float_as_uint(-INFINITY);
+                }
                 const float4 *ls4 = reinterpret_cast<const float4 *>(ls);
                 uint32_t pw[32];
 #pragma unroll
@@ -291,14 +298,6 @@ bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
                     p[i + 1] = ex2(x01.y);
                     p[i + 2] = ex2(x23.x);
                     p[i + 3] = ex2(x23.y);
-                    if (diag) {
-                        // query c of the tile sees key t only when c >= t on the diagonal tile
-                        const int c = w * 64 + i;
-                        if (c < t) p[i] = 0.f;
-                        if (c + 1 < t) p[i + 1] = 0.f;
-                        if (c + 2 < t) p[i + 2] = 0.f;
-                        if (c + 3 < t) p[i + 3] = 0.f;
-                    }
                     pw[i >> 1] = pack_bf16x2(p[i], p[i + 1]);
                     pw[(i >> 1) + 1] = pack_bf16x2(p[i + 2], p[i + 3]);
                 }
@@ -612,17 +611,20 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tmem_ld32(tS0 + s * 128 + lane_off + w * 64 + 32, sr + 32);
             tmem_wait_ld();
             if (w == 0) mbar_arrive(&bar[S2_READ]);
+            if (edge) {
+                // key c of the tile: after the row on the diagonal tile, or past the sequence (its weight
+                // is 2^-inf = 0); masked before the loop below, which then has no branch
+#pragma unroll
+                for (int i = 0; i < 64; ++i) {
+                    const int c = w * 64 + i;
+                    if ((diag && c > r) || c >= kend) sr[i] = __float_as_uint(-INFINITY);
+                }
+            }
             uint32_t dw[32];
 #pragma unroll
             for (int i = 0; i < 64; i += 2) {
-                const int c = w * 64 + i;
                 const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), qs2, nl2);
-                float2 p = make_float2(ex2(x.x), ex2(x.y));
-                if (edge) {
-                    // key c of the tile: after the row on the diagonal tile, or past the sequence
-                    if ((diag && c > r) || c >= kend) p.x = 0.f;
-                    if ((diag && c + 1 > r) || c + 1 >= kend) p.y = 0.f;
-                }
+                const float2 p = make_float2(ex2(x.x), ex2(x.y));
                 const float2 d = __fmul2_rn(p, __fadd2_rn(make_float2(__uint_as_float(pr[i]), __uint_as_float(pr[i + 1])), nd2));
                 dw[i >> 1] = pack_bf16x2(d.x, d.y);
             }
