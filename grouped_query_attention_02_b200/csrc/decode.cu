@@ -317,44 +317,68 @@ __global__ void __launch_bounds__(kD) decode_combine_kernel(const DecodeArgs a)
 {
     // launched as a programmatic dependent of the split kernel: wait for its results
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    __shared__ float wgt[kD];
-    __shared__ float red[kD / 32];
     const int h = blockIdx.x, b = blockIdx.y, j = threadIdx.x;
-    int T = a.seqlens[b];
-    T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
-    int nv = a.nsplit_b ? a.nsplit_b[b] : (T + a.chunk - 1) / a.chunk;
+    const size_t row = (size_t)b * a.Hq + h;
+    const float2 *ml = reinterpret_cast<const float2 *>(a.part_ml) + row * a.nsplit;
+    const float *po = a.part_o + row * a.nsplit * kD + j;
+    // The first kSpec slots are fetched together with the piece count, so that one round trip serves
+    // every history of up to kSpec pieces; slots past the count are never used (they may hold anything).
+    constexpr int kSpec = 8;
+    float2 mlv[kSpec];
+    float ov[kSpec];
+    int nv;
+    if (a.nsplit_b) {
+        nv = a.nsplit_b[b];
+    } else {
+        int T = a.seqlens[b];
+        T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
+        nv = (T + a.chunk - 1) / a.chunk;
+    }
+#pragma unroll
+    for (int s = 0; s < kSpec; ++s) {
+        if (s < a.nsplit) {
+            mlv[s] = ml[s];
+            ov[s] = po[(size_t)s * kD];
+        } else {
+            mlv[s] = make_float2(-INFINITY, 0.f);
+            ov[s] = 0.f;
+        }
+    }
     // with the device plan, a history of one piece (or none) was written out by the split kernel
     if (a.nsplit_b && nv <= 1) return;
     nv = nv > a.nsplit ? a.nsplit : nv;
-    const size_t row = (size_t)b * a.Hq + h;
-    const float *ml = a.part_ml + row * a.nsplit * 2;
-    const float *po = a.part_o + row * a.nsplit * kD;
-    // M = max over the splits
+    // M = max over the pieces
     float M = -INFINITY;
-    for (int s = j; s < nv; s += kD) M = fmaxf(M, ml[2 * s]);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if ((j & 31) == 0) red[j >> 5] = M;
-    __syncthreads();
-    M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    for (int s = 0; s < kSpec; ++s)
+        if (s < nv) M = fmaxf(M, mlv[s].x);
+    for (int s = kSpec; s < nv; ++s) M = fmaxf(M, ml[s].x);
     float Lsum = 0.f, O = 0.f;
-    for (int c = 0; c < nv; c += kD) {
-        const int n = min(kD, nv - c);
-        __syncthreads();
-        if (j < n) wgt[j] = ex2(ml[2 * (c + j)] - M);
-        __syncthreads();
-        int s = 0;
-        for (; s + 4 <= n; s += 4) {
-            const float o0 = po[(size_t)(c + s + 0) * kD + j], o1 = po[(size_t)(c + s + 1) * kD + j];
-            const float o2 = po[(size_t)(c + s + 2) * kD + j], o3 = po[(size_t)(c + s + 3) * kD + j];
-            const float l0 = ml[2 * (c + s + 0) + 1], l1 = ml[2 * (c + s + 1) + 1];
-            const float l2 = ml[2 * (c + s + 2) + 1], l3 = ml[2 * (c + s + 3) + 1];
-            O += o0 * wgt[s] + o1 * wgt[s + 1] + o2 * wgt[s + 2] + o3 * wgt[s + 3];
-            Lsum += l0 * wgt[s] + l1 * wgt[s + 1] + l2 * wgt[s + 2] + l3 * wgt[s + 3];
+#pragma unroll
+    for (int s = 0; s < kSpec; ++s) {
+        if (s < nv) {
+            const float wgt = ex2(mlv[s].x - M);
+            O += ov[s] * wgt;
+            Lsum += mlv[s].y * wgt;
         }
-        for (; s < n; ++s) {
-            O += po[(size_t)(c + s) * kD + j] * wgt[s];
-            Lsum += ml[2 * (c + s) + 1] * wgt[s];
+    }
+    for (int s = kSpec; s < nv; s += 4) {
+        float2 m4[4];
+        float o4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (s + e < nv) {
+                m4[e] = ml[s + e];
+                o4[e] = po[(size_t)(s + e) * kD];
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (s + e < nv) {
+                const float wgt = ex2(m4[e].x - M);
+                O += o4[e] * wgt;
+                Lsum += m4[e].y * wgt;
+            }
         }
     }
     // a zero sum only for an empty history (output 0); a NaN sum (a NaN in the cache) stays NaN

@@ -52,7 +52,8 @@ constexpr int kHalf = kTile / 2;          // one 64-column half
 constexpr int kWG = 128;                  // threads of one softmax warpgroup (one token each)
 constexpr int kQD = 4;                    // depth of the unit queue in shared memory
 constexpr float kMoveThreshold = 8.0f;
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 512;
+constexpr int kPlanSmemB = 2048;          // sequences whose planner scratch fits shared memory
 constexpr int kPlanMaxC = 4096;           // remainder sizes sorted by a shared-memory histogram up to this
 
 // barrier slots: each name owns a contiguous range (sizes checked against the configuration below)
@@ -161,71 +162,79 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
 }
 
 // ---------------------------------------------------------------------------------------------
-// Exclusive scan of n ints in shared memory by the whole block.
-__device__ void block_exclusive_scan(int *v, int n, int *warp_tot)
+// Exclusive scans of two int arrays (n1 and n2 entries) by the whole block in one pass; *tot1 and *tot2
+// receive their totals.  Each thread scans a contiguous run of each array.
+__device__ void block_exclusive_scan2(int *v1, int n1, int *v2, int n2, int (*warp_tot)[32], int *tot1, int *tot2)
 {
-    const int tid = threadIdx.x, nt = blockDim.x;
-    const int per = (n + nt - 1) / nt;
-    const int lo = min(n, tid * per), hi = min(n, lo + per);
-    int run = 0;
-    for (int i = lo; i < hi; ++i) run += v[i];
-    int x = run;   // inclusive scan of the per-thread runs
+    const int tid = threadIdx.x, nt = blockDim.x, nw = nt >> 5;
     const int lane = tid & 31, w = tid >> 5;
+    const int per1 = (n1 + nt - 1) / nt, per2 = (n2 + nt - 1) / nt;
+    const int lo1 = min(n1, tid * per1), hi1 = min(n1, lo1 + per1);
+    const int lo2 = min(n2, tid * per2), hi2 = min(n2, lo2 + per2);
+    int run1 = 0, run2 = 0;
+    for (int i = lo1; i < hi1; ++i) run1 += v1[i];
+    for (int i = lo2; i < hi2; ++i) run2 += v2[i];
+    int x1 = run1, x2 = run2;   // inclusive scans of the per-thread runs
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+        const int y1 = __shfl_up_sync(0xffffffffu, x1, o), y2 = __shfl_up_sync(0xffffffffu, x2, o);
+        if (lane >= o) {
+            x1 += y1;
+            x2 += y2;
+        }
     }
-    if (lane == 31) warp_tot[w] = x;
+    if (lane == 31) {
+        warp_tot[0][w] = x1;
+        warp_tot[1][w] = x2;
+    }
     __syncthreads();
-    if (w == 0) {
-        int t = lane < (nt >> 5) ? warp_tot[lane] : 0;
+    if (w < 2) {   // warp 0 scans the first array's warp totals, warp 1 the second's
+        int t = lane < nw ? warp_tot[w][lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, t, o);
             if (lane >= o) t += y;
         }
-        if (lane < (nt >> 5)) warp_tot[lane] = t;
+        if (lane < nw) warp_tot[w][lane] = t;
+        if (lane == nw - 1) *(w == 0 ? tot1 : tot2) = t;
     }
     __syncthreads();
-    int base = x - run + (w > 0 ? warp_tot[w - 1] : 0);
-    for (int i = lo; i < hi; ++i) {
-        const int c = v[i];
-        v[i] = base;
-        base += c;
+    int base1 = x1 - run1 + (w > 0 ? warp_tot[0][w - 1] : 0);
+    int base2 = x2 - run2 + (w > 0 ? warp_tot[1][w - 1] : 0);
+    for (int i = lo1; i < hi1; ++i) {
+        const int c = v1[i];
+        v1[i] = base1;
+        base1 += c;
+    }
+    for (int i = lo2; i < hi2; ++i) {
+        const int c = v2[i];
+        v2[i] = base2;
+        base2 += c;
     }
     __syncthreads();
 }
 
-__device__ __forceinline__ int block_sum(int part, int *red_i, int *out)
+__device__ __forceinline__ int plan_tiles(const DecodeArgs &a, int b)
 {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    if (lane == 0) red_i[w] = part;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int s = 0;
-        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += red_i[i];
-        *out = s;
-    }
-    __syncthreads();
-    return *out;
+    int T = __ldg(a.seqlens + b);
+    T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
+    return (T + kTok - 1) / kTok;
 }
 
 // Cuts every history into pieces of C tiles and lists them longest first:
 // plan_hdr = {claim counter (reset to 0), pieces, C}; nsplit_b[b] = pieces of sequence b;
 // items[i] = {b, piece index | pieces of b << 16, first token, end token}.  Full pieces come first, then the
-// shorter last pieces in decreasing length (a counting sort).
+// shorter last pieces in decreasing length (a counting sort).  One block; up to kPlanSmemB sequences keep
+// their scratch in shared memory, so that the only global reads are the lengths.
 __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeArgs a, int slots)
 {
     __shared__ long long red_ll[32];
     __shared__ int red_i[32];
-    __shared__ int warp_tot[32];
-    __shared__ int hist[kPlanMaxC];
-    __shared__ int cursor[kPlanMaxC];
-    __shared__ int s_C, s_sum;
-    int *full_off = a.plan_scratch;     // per-sequence offsets of the full pieces (B ints, global)
+    __shared__ int warp_tot[2][32];
+    __shared__ int hist[kPlanMaxC];        // tail pieces per size class, then each class's next slot
+    __shared__ int s_full[kPlanSmemB];     // full pieces per sequence, then its first slot
+    __shared__ int s_C, s_F, s_tail;
+    int *full_off = a.B <= kPlanSmemB ? s_full : a.plan_scratch;
 
     // launched as a programmatic dependent of whatever ran before on the stream (the previous call's
     // combine, say, which still reads nsplit_b): wait for it before touching anything, so that only the
@@ -233,13 +242,12 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // the persistent kernel may start its prologue now; it reads this plan only after griddepcontrol.wait
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+    for (int i = tid; i < kPlanMaxC; i += blockDim.x) hist[i] = 0;
     long long tot = 0;
     int mx = 0;
     for (int b = tid; b < a.B; b += blockDim.x) {
-        int T = a.seqlens[b];
-        T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
-        const int tl = (T + kTok - 1) / kTok;
+        const int tl = plan_tiles(a, b);
         tot += tl;
         mx = max(mx, tl);
     }
@@ -252,31 +260,32 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         red_ll[w] = tot;
         red_i[w] = mx;
     }
-    for (int i = tid; i < kPlanMaxC; i += blockDim.x) {
-        hist[i] = 0;
-        cursor[i] = 0;
-    }
     __syncthreads();
-    if (tid == 0) {
-        long long T = 0;
-        int M = 0;
-        for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
-            T += red_ll[i];
-            M = max(M, red_i[i]);
+    if (w == 0) {
+        long long T = lane < nw ? red_ll[lane] : 0;
+        int M = lane < nw ? red_i[lane] : 0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            T += __shfl_xor_sync(0xffffffffu, T, o);
+            M = max(M, __shfl_xor_sync(0xffffffffu, M, o));
         }
-        // rounds of (piece, KV head) units per persistent CTA: eight for groups up to 8, two above, whose
-        // units of more heads carry a larger fixed cost each (measured on the benchmark shapes); never
-        // more than nsplit pieces
-        const long long rounds = a.plan_rounds > 0 ? a.plan_rounds : (a.group > 8 ? 2 : 8);
-        long long C = (T * a.Hkv + rounds * slots - 1) / (rounds * slots);
-        const long long cmin = (M + a.nsplit - 1) / a.nsplit;
-        if (C < cmin) C = cmin;
-        if (C > M) C = M;
-        if (C < 1) C = 1;
-        s_C = (int)C;
+        if (lane == 0) {
+            // rounds of (piece, KV head) units per persistent CTA: eight for groups up to 8, two above,
+            // whose units of more heads carry a larger fixed cost each (measured on the benchmark shapes);
+            // never more than nsplit pieces
+            const long long rounds = a.plan_rounds > 0 ? a.plan_rounds : (a.group > 8 ? 2 : 8);
+            long long C = (T * a.Hkv + rounds * slots - 1) / (rounds * slots);
+            const long long cmin = (M + a.nsplit - 1) / a.nsplit;
+            if (C < cmin) C = cmin;
+            if (C > M) C = M;
+            if (C < 1) C = 1;
+            s_C = (int)C;
+        }
     }
     __syncthreads();
     const int C = s_C;
+    // remainder sizes sort by a shared histogram up to kPlanMaxC; past that they keep no order and
+    // hist[0] counts and then places them
     const bool sort_rem = C <= kPlanMaxC;
     // A history's remainder (tl % C tiles) is cut into up to tail_split pieces of nearly equal size
     // (never more than nsplit pieces in all): the shortest units are claimed last, so that the CTAs
@@ -288,56 +297,52 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         if (k > a.nsplit - full) k = a.nsplit - full;
         return k > 1 ? k : 1;
     };
-    int npieces = 0;
     for (int b = tid; b < a.B; b += blockDim.x) {
-        int T = a.seqlens[b];
-        T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
-        const int tl = (T + kTok - 1) / kTok;
+        const int tl = plan_tiles(a, b);
         const int full = tl / C, rem = tl % C;
         const int k = tail_pieces(full, rem);
         full_off[b] = full;
         a.nsplit_b[b] = full + k;
-        npieces += full + k;
-        if (sort_rem)
+        if (sort_rem) {
             for (int j = 0; j < k; ++j) {
                 const int size = rem / k + (j < rem % k ? 1 : 0);
                 atomicAdd(&hist[C - 1 - size], 1);   // reversed: longest first
             }
-    }
-    __syncthreads();
-    const int P = block_sum(npieces, red_i, &s_sum);
-    int nfull = 0;
-    for (int b = tid; b < a.B; b += blockDim.x) nfull += full_off[b];
-    const int F = block_sum(nfull, red_i, &s_sum);
-    block_exclusive_scan(full_off, a.B, warp_tot);
-    if (sort_rem) block_exclusive_scan(hist, C, warp_tot);   // hist[C-1-r]: tail pieces longer than r
-    for (int b = tid; b < a.B; b += blockDim.x) {
-        int T = a.seqlens[b];
-        T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
-        const int tl = (T + kTok - 1) / kTok;
-        const int full = tl / C, rem = tl % C;
-        const int k = tail_pieces(full, rem);
-        const int np_b = full + k;
+        } else if (k > 0) {
+            atomicAdd(&hist[0], k);
+        }
         if (tl == 0) {
             // no cached token: no unit will touch this sequence, its output rows are zero
             const int orow = a.out_row > 0 ? a.out_row : kD;
             uint4 *o = reinterpret_cast<uint4 *>(a.out + (size_t)b * a.Hq * orow);
             for (int i = 0; i < a.Hq * orow / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
         }
+    }
+    __syncthreads();
+    // full_off[b]: first slot of b's full pieces; hist[C-1-r]: tail pieces longer than r
+    block_exclusive_scan2(full_off, a.B, hist, sort_rem ? C : 1, warp_tot, &s_F, &s_tail);
+    const int F = s_F;
+    for (int b = tid; b < a.B; b += blockDim.x) {
+        int T = __ldg(a.seqlens + b);
+        T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
+        const int tl = (T + kTok - 1) / kTok;
+        const int full = tl / C, rem = tl % C;
+        const int k = tail_pieces(full, rem);
+        const int np_b = full + k;
+        const int f0 = full_off[b];
         for (int s = 0; s < full; ++s)
-            a.items[full_off[b] + s] = make_int4(b, s | (np_b << 16), s * C * kTok, min((s + 1) * C * kTok, T));
+            a.items[f0 + s] = make_int4(b, s | (np_b << 16), s * C * kTok, min((s + 1) * C * kTok, T));
         int start = full * C;   // first tile of the next tail piece
         for (int j = 0; j < k; ++j) {
             const int size = rem / k + (j < rem % k ? 1 : 0);
-            const int kk = C - 1 - size;
-            const int pos = sort_rem ? F + hist[kk] + atomicAdd(&cursor[kk], 1) : F + atomicAdd(&cursor[0], 1);
+            const int pos = F + atomicAdd(&hist[sort_rem ? C - 1 - size : 0], 1);
             a.items[pos] = make_int4(b, (full + j) | (np_b << 16), start * kTok, min((start + size) * kTok, T));
             start += size;
         }
     }
     if (tid == 0) {
         a.plan_hdr[0] = 0;   // claim counter
-        a.plan_hdr[1] = P;
+        a.plan_hdr[1] = F + s_tail;
         a.plan_hdr[2] = C;
     }
 }
