@@ -236,7 +236,7 @@ DecodePlan decode_plan_host(int B, int Hq, int Hkv, int Tmax, int num_sms, size_
         p.off_hdr = off;
         off += 256;
         p.off_nsb = off;
-        off += round256((size_t)B * 4) * 2;   // pieces per sequence, then the planner's scratch
+        off += round256((size_t)B * 4);   // pieces per sequence
         p.off_items = off;
         off += round256((size_t)B * p.nsplit * 16);
         p.off_po = off;
@@ -347,7 +347,6 @@ int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *s
     } else if (p.tensor_cores) {
         a.plan_hdr = reinterpret_cast<int *>(w + p.off_hdr);
         a.nsplit_b = reinterpret_cast<int *>(w + p.off_nsb);
-        a.plan_scratch = reinterpret_cast<int *>(w + p.off_nsb + round256((size_t)B * 4));
         a.items = reinterpret_cast<int4 *>(w + p.off_items);
         if ((s = cuda_status(launch_decode_plan(a, stream))) != GQA_OK) return s;
         ++n;

@@ -52,8 +52,6 @@ constexpr int kHalf = kTile / 2;          // one 64-column half
 constexpr int kWG = 128;                  // threads of one softmax warpgroup (one token each)
 constexpr int kQD = 4;                    // depth of the unit queue in shared memory
 constexpr float kMoveThreshold = 8.0f;
-constexpr int kPlanThreads = 512;
-constexpr int kPlanSmemB = 2048;          // sequences whose planner scratch fits shared memory
 constexpr int kPlanMaxC = 4096;           // remainder sizes sorted by a shared-memory histogram up to this
 
 // barrier slots: each name owns a contiguous range (sizes checked against the configuration below)
@@ -162,79 +160,36 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
 }
 
 // ---------------------------------------------------------------------------------------------
-// Exclusive scans of two int arrays (n1 and n2 entries) by the whole block in one pass; *tot1 and *tot2
-// receive their totals.  Each thread scans a contiguous run of each array.
-__device__ void block_exclusive_scan2(int *v1, int n1, int *v2, int n2, int (*warp_tot)[32], int *tot1, int *tot2)
+__device__ __forceinline__ int plan_tokens(const DecodeArgs &a, int b)
 {
-    const int tid = threadIdx.x, nt = blockDim.x, nw = nt >> 5;
-    const int lane = tid & 31, w = tid >> 5;
-    const int per1 = (n1 + nt - 1) / nt, per2 = (n2 + nt - 1) / nt;
-    const int lo1 = min(n1, tid * per1), hi1 = min(n1, lo1 + per1);
-    const int lo2 = min(n2, tid * per2), hi2 = min(n2, lo2 + per2);
-    int run1 = 0, run2 = 0;
-    for (int i = lo1; i < hi1; ++i) run1 += v1[i];
-    for (int i = lo2; i < hi2; ++i) run2 += v2[i];
-    int x1 = run1, x2 = run2;   // inclusive scans of the per-thread runs
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y1 = __shfl_up_sync(0xffffffffu, x1, o), y2 = __shfl_up_sync(0xffffffffu, x2, o);
-        if (lane >= o) {
-            x1 += y1;
-            x2 += y2;
-        }
-    }
-    if (lane == 31) {
-        warp_tot[0][w] = x1;
-        warp_tot[1][w] = x2;
-    }
-    __syncthreads();
-    if (w < 2) {   // warp 0 scans the first array's warp totals, warp 1 the second's
-        int t = lane < nw ? warp_tot[w][lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, t, o);
-            if (lane >= o) t += y;
-        }
-        if (lane < nw) warp_tot[w][lane] = t;
-        if (lane == nw - 1) *(w == 0 ? tot1 : tot2) = t;
-    }
-    __syncthreads();
-    int base1 = x1 - run1 + (w > 0 ? warp_tot[0][w - 1] : 0);
-    int base2 = x2 - run2 + (w > 0 ? warp_tot[1][w - 1] : 0);
-    for (int i = lo1; i < hi1; ++i) {
-        const int c = v1[i];
-        v1[i] = base1;
-        base1 += c;
-    }
-    for (int i = lo2; i < hi2; ++i) {
-        const int c = v2[i];
-        v2[i] = base2;
-        base2 += c;
-    }
-    __syncthreads();
+    const int T = __ldg(a.seqlens + b);
+    return T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
 }
 
-__device__ __forceinline__ int plan_tiles(const DecodeArgs &a, int b)
+// Exclusive scan over the warp; *total receives the sum of all lanes' values.
+__device__ __forceinline__ int warp_exclusive_scan(int v, int &total)
 {
-    int T = __ldg(a.seqlens + b);
-    T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
-    return (T + kTok - 1) / kTok;
+    const int lane = threadIdx.x & 31;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    total = __shfl_sync(0xffffffffu, x, 31);
+    return x - v;
 }
 
 // Cuts every history into pieces of C tiles and lists them longest first:
 // plan_hdr = {claim counter (reset to 0), pieces, C}; nsplit_b[b] = pieces of sequence b;
-// items[i] = {b, piece index | pieces of b << 16, first token, end token}.  Full pieces come first, then the
-// shorter last pieces in decreasing length (a counting sort).  One block; up to kPlanSmemB sequences keep
-// their scratch in shared memory, so that the only global reads are the lengths.
-__global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeArgs a, int slots)
+// items[i] = {b, piece index | pieces of b << 16, first token, end token}.  Full pieces come first, in
+// sequence order, then the shorter last pieces in decreasing length (a counting sort).
+// One warp: its time is latency (one read of the lengths and a few dependent steps), which a warp
+// takes with shuffles where a larger block would need barriers.  Lane l owns the contiguous sequences
+// [l * per, (l + 1) * per).
+__global__ void __launch_bounds__(32) decode_plan_kernel(const DecodeArgs a, int slots)
 {
-    __shared__ long long red_ll[32];
-    __shared__ int red_i[32];
-    __shared__ int warp_tot[2][32];
-    __shared__ int hist[kPlanMaxC];        // tail pieces per size class, then each class's next slot
-    __shared__ int s_full[kPlanSmemB];     // full pieces per sequence, then its first slot
-    __shared__ int s_C, s_F, s_tail;
-    int *full_off = a.B <= kPlanSmemB ? s_full : a.plan_scratch;
+    __shared__ int hist[kPlanMaxC];   // tail pieces per size class, then each class's next slot
 
     // launched as a programmatic dependent of whatever ran before on the stream (the previous call's
     // combine, say, which still reads nsplit_b): wait for it before touching anything, so that only the
@@ -242,12 +197,13 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
     asm volatile("griddepcontrol.wait;" ::: "memory");
     // the persistent kernel may start its prologue now; it reads this plan only after griddepcontrol.wait
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
-    for (int i = tid; i < kPlanMaxC; i += blockDim.x) hist[i] = 0;
+    const int lane = threadIdx.x;
+    const int per = (a.B + 31) / 32;
+    const int b0 = min(a.B, lane * per), b1 = min(a.B, b0 + per);
     long long tot = 0;
     int mx = 0;
-    for (int b = tid; b < a.B; b += blockDim.x) {
-        const int tl = plan_tiles(a, b);
+    for (int b = b0; b < b1; ++b) {
+        const int tl = (plan_tokens(a, b) + kTok - 1) / kTok;
         tot += tl;
         mx = max(mx, tl);
     }
@@ -256,37 +212,22 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         tot += __shfl_xor_sync(0xffffffffu, tot, o);
         mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
-    if (lane == 0) {
-        red_ll[w] = tot;
-        red_i[w] = mx;
-    }
-    __syncthreads();
-    if (w == 0) {
-        long long T = lane < nw ? red_ll[lane] : 0;
-        int M = lane < nw ? red_i[lane] : 0;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            T += __shfl_xor_sync(0xffffffffu, T, o);
-            M = max(M, __shfl_xor_sync(0xffffffffu, M, o));
-        }
-        if (lane == 0) {
-            // rounds of (piece, KV head) units per persistent CTA: eight for groups up to 8, two above,
-            // whose units of more heads carry a larger fixed cost each (measured on the benchmark shapes);
-            // never more than nsplit pieces
-            const long long rounds = a.plan_rounds > 0 ? a.plan_rounds : (a.group > 8 ? 2 : 8);
-            long long C = (T * a.Hkv + rounds * slots - 1) / (rounds * slots);
-            const long long cmin = (M + a.nsplit - 1) / a.nsplit;
-            if (C < cmin) C = cmin;
-            if (C > M) C = M;
-            if (C < 1) C = 1;
-            s_C = (int)C;
-        }
-    }
-    __syncthreads();
-    const int C = s_C;
+    // rounds of (piece, KV head) units per persistent CTA: eight for groups up to 8, two above, whose
+    // units of more heads carry a larger fixed cost each (measured on the benchmark shapes); never more
+    // than nsplit pieces
+    const long long rounds = a.plan_rounds > 0 ? a.plan_rounds : (a.group > 8 ? 2 : 8);
+    long long Cl = (tot * a.Hkv + rounds * slots - 1) / (rounds * slots);
+    const long long cmin = (mx + a.nsplit - 1) / a.nsplit;
+    if (Cl < cmin) Cl = cmin;
+    if (Cl > mx) Cl = mx;
+    if (Cl < 1) Cl = 1;
+    const int C = (int)Cl;
     // remainder sizes sort by a shared histogram up to kPlanMaxC; past that they keep no order and
     // hist[0] counts and then places them
     const bool sort_rem = C <= kPlanMaxC;
+    const int nclass = sort_rem ? C : 1;
+    for (int i = lane; i < nclass; i += 32) hist[i] = 0;
+    __syncwarp();
     // A history's remainder (tl % C tiles) is cut into up to tail_split pieces of nearly equal size
     // (never more than nsplit pieces in all): the shortest units are claimed last, so that the CTAs
     // finish together even when some of them stream their tiles more slowly than others.
@@ -297,12 +238,15 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         if (k > a.nsplit - full) k = a.nsplit - full;
         return k > 1 ? k : 1;
     };
-    for (int b = tid; b < a.B; b += blockDim.x) {
-        const int tl = plan_tiles(a, b);
+    int nfull = 0;
+    bool empty = false;
+    for (int b = b0; b < b1; ++b) {
+        const int tl = (plan_tokens(a, b) + kTok - 1) / kTok;
         const int full = tl / C, rem = tl % C;
         const int k = tail_pieces(full, rem);
-        full_off[b] = full;
         a.nsplit_b[b] = full + k;
+        nfull += full;
+        empty |= tl == 0;
         if (sort_rem) {
             for (int j = 0; j < k; ++j) {
                 const int size = rem / k + (j < rem % k ? 1 : 0);
@@ -311,39 +255,55 @@ __global__ void __launch_bounds__(kPlanThreads) decode_plan_kernel(const DecodeA
         } else if (k > 0) {
             atomicAdd(&hist[0], k);
         }
-        if (tl == 0) {
-            // no cached token: no unit will touch this sequence, its output rows are zero
-            const int orow = a.out_row > 0 ? a.out_row : kD;
+    }
+    if (__any_sync(0xffffffffu, empty)) {
+        // no cached token: no unit will touch such a sequence, its output rows are zero
+        const int orow = a.out_row > 0 ? a.out_row : kD;
+        for (int b = 0; b < a.B; ++b) {
+            if (plan_tokens(a, b) > 0) continue;
             uint4 *o = reinterpret_cast<uint4 *>(a.out + (size_t)b * a.Hq * orow);
-            for (int i = 0; i < a.Hq * orow / 8; ++i) o[i] = make_uint4(0, 0, 0, 0);
+            for (int i = lane; i < a.Hq * orow / 8; i += 32) o[i] = make_uint4(0, 0, 0, 0);
         }
     }
-    __syncthreads();
-    // full_off[b]: first slot of b's full pieces; hist[C-1-r]: tail pieces longer than r
-    block_exclusive_scan2(full_off, a.B, hist, sort_rem ? C : 1, warp_tot, &s_F, &s_tail);
-    const int F = s_F;
-    for (int b = tid; b < a.B; b += blockDim.x) {
-        int T = __ldg(a.seqlens + b);
-        T = T < 0 ? 0 : (T > a.Tmax ? a.Tmax : T);
+    __syncwarp();
+    int F;
+    int f0 = warp_exclusive_scan(nfull, F);   // first slot of this lane's full pieces
+    // hist[C-1-r] becomes the first slot (after the full pieces) of the tail pieces of r tiles
+    {
+        const int cper = (nclass + 31) / 32;
+        const int c0 = min(nclass, lane * cper), c1 = min(nclass, c0 + cper);
+        int run = 0;
+        for (int c = c0; c < c1; ++c) run += hist[c];
+        int ntail;
+        int base = F + warp_exclusive_scan(run, ntail);
+        for (int c = c0; c < c1; ++c) {
+            const int n = hist[c];
+            hist[c] = base;
+            base += n;
+        }
+        if (lane == 0) {
+            a.plan_hdr[0] = 0;   // claim counter
+            a.plan_hdr[1] = F + ntail;
+            a.plan_hdr[2] = C;
+        }
+    }
+    __syncwarp();
+    for (int b = b0; b < b1; ++b) {
+        const int T = plan_tokens(a, b);
         const int tl = (T + kTok - 1) / kTok;
         const int full = tl / C, rem = tl % C;
         const int k = tail_pieces(full, rem);
         const int np_b = full + k;
-        const int f0 = full_off[b];
         for (int s = 0; s < full; ++s)
             a.items[f0 + s] = make_int4(b, s | (np_b << 16), s * C * kTok, min((s + 1) * C * kTok, T));
+        f0 += full;
         int start = full * C;   // first tile of the next tail piece
         for (int j = 0; j < k; ++j) {
             const int size = rem / k + (j < rem % k ? 1 : 0);
-            const int pos = F + atomicAdd(&hist[sort_rem ? C - 1 - size : 0], 1);
+            const int pos = atomicAdd(&hist[sort_rem ? C - 1 - size : 0], 1);
             a.items[pos] = make_int4(b, (full + j) | (np_b << 16), start * kTok, min((start + size) * kTok, T));
             start += size;
         }
-    }
-    if (tid == 0) {
-        a.plan_hdr[0] = 0;   // claim counter
-        a.plan_hdr[1] = F + s_tail;
-        a.plan_hdr[2] = C;
     }
 }
 
@@ -1138,7 +1098,7 @@ cudaError_t launch_decode_plan(const DecodeArgs &a, cudaStream_t stream)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(1);
-    cfg.blockDim = dim3(kPlanThreads);
+    cfg.blockDim = dim3(32);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -34,7 +34,6 @@ struct DecodeArgs {
     // device-planned schedule (tensor-core path): see decode_tc.cu
     int *plan_hdr;            // {claim counter, pieces, C}
     int *nsplit_b;            // [B] pieces per sequence (the combine reads it when non-null)
-    int *plan_scratch;        // [B] planner scratch
     int4 *items;              // [B * nsplit] pieces, longest first
     int num_ctas;             // persistent CTAs (one per SM)
     // planner options for other operators that reuse decode_plan_kernel (0: the GQA decode's defaults)

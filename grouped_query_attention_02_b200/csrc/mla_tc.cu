@@ -616,7 +616,7 @@ MlaTcPlan mla_tc_plan_host(int B, int Hq, int Tmax, size_t ws_budget)
     p.off_hdr = off;
     off += 256;
     p.off_nsb = off;
-    off += round256((size_t)B * 4) * 2;   // pieces per sequence, then the planner's scratch
+    off += round256((size_t)B * 4);   // pieces per sequence
     p.off_items = off;
     off += round256((size_t)B * p.nsplit * 16);
     p.off_po = off;
@@ -648,7 +648,6 @@ cudaError_t launch_mla_decode_tc(const CUtensorMap &tmKV2, const CUtensorMap &tm
     pa.nsplit = p.nsplit;
     pa.plan_hdr = reinterpret_cast<int *>(w + p.off_hdr);
     pa.nsplit_b = reinterpret_cast<int *>(w + p.off_nsb);
-    pa.plan_scratch = reinterpret_cast<int *>(w + p.off_nsb + round256((size_t)B * 4));
     pa.items = reinterpret_cast<int4 *>(w + p.off_items);
     pa.num_ctas = num_sms;
     pa.out_row = kMlaLatent;
