@@ -74,8 +74,10 @@ constexpr bool barrier_ranges_fit()
 // warpgroup widens them exactly to f16 (every E4M3 value is an f16 value): the keys into tensor
 // memory, where they are the A operand of S^T, the values into a 128-byte-swizzled f16 tile that
 // takes the place of the stage's two code tiles (each thread rewrites only the two 128-byte rows it
-// has just read, so no thread waits for another).  Q is converted in place to f16 with a power-of-two scale per head, and P enters the second
-// product as f16 hi + lo terms (of 128 p, so that small weights stay normal), with f16 MMAs throughout.
+// has just read, so no thread waits for another).  Q is converted in place to f16 with a power-of-two
+// scale per head, and P enters the second product as one f16 term of 128 p (so that small weights stay
+// normal; relative rounding 2^-11 per weight, against the bf16 path's hi + lo pair), with f16 MMAs
+// throughout.
 // HW: heads one softmax warpgroup handles (4, 8 or 16), NWG: softmax warpgroups.  Groups of up to 4
 // or 8 heads only compute their own columns of the N = 16 wide products; more warpgroups with fewer
 // heads each shorten the softmax's per-tile chain.
@@ -93,6 +95,9 @@ struct TcCfg {
     static constexpr int threads = regsplit ? 512 : kWG * nwg + 32 * conv_warps + 96;
     static constexpr int sbufs = 4;                            // S^T buffers: QK^T runs up to four tiles ahead
     static constexpr int pbufs = (F8 || N == 16) ? 2 : 1;      // P^T buffers (2: the softmax runs a tile ahead)
+    // P as one 16-bit term (FP8: f16 of 128 p, relative rounding 2^-11 on each weight) or as bf16 hi + lo
+    // terms (bf16: 2^-8 on its own would be as coarse as the output's rounding)
+    static constexpr int p_terms = F8 ? 1 : 2;
     static constexpr int stages = F8 ? (N == 32 ? 5 : 6) : 3;
     // K then V (FP8: two 16 KB code tiles, then the f16 V tile in their place)
     static constexpr int stage_bytes = F8 ? kTile : 2 * kTile;
@@ -113,8 +118,8 @@ struct TcCfg {
     static constexpr int err_off = tmem_off + 8;
     static constexpr int bytes = err_off + 8;
     // FP8: K[2] (64 columns each: 128 f16 keys per token, packed in pairs) first, then as below.
-    // S[sbufs] (N columns each) and O[2] (2N columns each: the hi and lo products side by side; the lo
-    // columns start 8 * nb columns after the hi ones)
+    // S[sbufs] (N columns each) and O[2] (2N columns each: the hi and lo products side by side, the lo
+    // columns 8 * nb after the hi ones; FP8 reads only the hi columns)
     static constexpr uint32_t s_base = F8 ? 128 : 0;
     static constexpr uint32_t o_base = s_base + sbufs * N;
     static constexpr uint32_t tmem_used = o_base + 4 * N;
@@ -321,8 +326,6 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__device__ __forceinline__ float f16_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu))); }
-__device__ __forceinline__ float f16_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
 
 // 32 lanes x 32 bits, NC (4, 8 or 16) consecutive columns per thread.
 template <int NC>
@@ -624,7 +627,8 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         } else if (warp == pv_warp) {
             // ---------------- PV issuer: [O_hi | O_lo] += V^T (MN-major) . [P_hi | P_lo]^T (MN-major)
             if (lane == 0) {
-                constexpr int npv = 16 * C::nb;   // the hi and lo blocks that carry heads
+                // the hi (and lo) blocks that carry heads; N of an M = 128 product is at least 16
+                constexpr int npv = C::p_terms * 8 * C::nb < 16 ? 16 : C::p_terms * 8 * C::nb;
                 const uint32_t idesc_o = F8 ? umma_idesc_f16(kD, npv, 1, 1) : umma_idesc_bf16(kD, npv, 1, 1);
                 int tcount = 0, icount = 0;
                 bool ok = true;
@@ -814,11 +818,11 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             tc_fence_after();
             uint32_t o[HW], olo[HW];
             tmem_ldn<HW>(tO0 + pob * 2 * N + lane_off + hs, o);
-            tmem_ldn<HW>(tO0 + pob * 2 * N + lane_off + 8 * C::nb + hs, olo);
+            if constexpr (C::p_terms == 2) tmem_ldn<HW>(tO0 + pob * 2 * N + lane_off + 8 * C::nb + hs, olo);
             tmem_wait_ld();
 #pragma unroll
             for (int h = 0; h < HW; ++h)
-                o[h] = __float_as_uint((__uint_as_float(o[h]) + __uint_as_float(olo[h])) * ofac);
+                o[h] = __float_as_uint((__uint_as_float(o[h]) + (C::p_terms == 2 ? __uint_as_float(olo[h]) : 0.f)) * ofac);
             const float *ls = lsum + pob * 4 * N;   // per-warp weight sums of the unit: [4][N]
             const int d = t;
             const size_t row0 = (size_t)pb * a.Hq + pkvh * g + hs;   // the warpgroup's first (b, query head) row
@@ -955,7 +959,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 tc_fence_after();
                 if (rescale_o) {
 #pragma unroll
-                    for (int part = 0; part < 2; ++part) {   // the hi and the lo columns
+                    for (int part = 0; part < C::p_terms; ++part) {   // the hi (and the lo) columns
                         uint32_t o[HW];
                         tmem_ldn<HW>(tO0 + ob * 2 * N + lane_off + part * 8 * C::nb + hs, o);
                         tmem_wait_ld();
@@ -981,10 +985,10 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                         }
                     }
                 }
-                // P^T, MN-major without swizzle: core matrices of 8 tokens x 8 heads (128 B), each weight
-                // as hi plus lo = (p - hi) in the products' 16-bit type (FP8: f16 terms of 128 p).  With
-                // four heads only the first half of each 16-byte core-matrix row is written: the other
-                // four columns of the products are never read.
+                // P^T, MN-major without swizzle: core matrices of 8 tokens x 8 heads (128 B).  bf16: each
+                // weight as hi plus lo = (p - hi), the lo blocks p_half after the hi ones; FP8: f16 of
+                // 128 p alone (small weights stay normal).  With four heads only the first half of each
+                // 16-byte core-matrix row is written: the other four columns of the products are never read.
                 uint8_t *pdst = ps + pbuf * 2 * C::p_half + (t >> 3) * 128 + (t & 7) * 16;
 #pragma unroll
                 for (int hb = 0; hb < (HW + 7) / 8; ++hb) {
@@ -993,9 +997,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 #pragma unroll
                     for (int e = 0; e < E; ++e) {
                         if constexpr (F8) {
-                            const float a0 = p[hb * 8 + 2 * e] * 128.f, a1 = p[hb * 8 + 2 * e + 1] * 128.f;
-                            hi[e] = pack_f16x2(a0, a1);
-                            lo[e] = pack_f16x2(a0 - f16_lo(hi[e]), a1 - f16_hi(hi[e]));
+                            hi[e] = pack_f16x2(p[hb * 8 + 2 * e] * 128.f, p[hb * 8 + 2 * e + 1] * 128.f);
                         } else {
                             const float a0 = p[hb * 8 + 2 * e], a1 = p[hb * 8 + 2 * e + 1];
                             hi[e] = pack2(a0, a1);
@@ -1005,10 +1007,12 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     uint8_t *dst = pdst + (hs / 8 + hb) * 2048;
                     if constexpr (E == 4) {
                         *reinterpret_cast<uint4 *>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                        *reinterpret_cast<uint4 *>(dst + C::p_half) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                        if constexpr (C::p_terms == 2)
+                            *reinterpret_cast<uint4 *>(dst + C::p_half) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                     } else {
                         *reinterpret_cast<uint2 *>(dst) = make_uint2(hi[0], hi[1]);
-                        *reinterpret_cast<uint2 *>(dst + C::p_half) = make_uint2(lo[0], lo[1]);
+                        if constexpr (C::p_terms == 2)
+                            *reinterpret_cast<uint2 *>(dst + C::p_half) = make_uint2(lo[0], lo[1]);
                     }
                 }
                 fence_proxy_async_smem();
