@@ -60,13 +60,13 @@ enum : int { K_FULL = 0, V_FULL = 3, KV_EMPTY = 6, S_FULL = 9, S_FREE = 13, P_FU
              // FP8 only: code ring (R_EMPTY: the stage's PV product is done), converted K (tensor memory),
              // converted V (in the stage), converted Q, and the unit slot's score factors (the softmax
              // releases the slot after reading them)
-             R_FULL = 45, R_EMPTY = 51, KT_FULL = 57, KT_FREE = 59, VC_FULL = 61, QC_FULL = 67, QF_FULL = 69,
-             kBarSlots = 73 };
+             R_FULL = 47, R_EMPTY = 53, KT_FULL = 59, KT_FREE = 61, VC_FULL = 63, QC_FULL = 69, QF_FULL = 71,
+             kBarSlots = 75 };
 constexpr int kBarSlotsFor(bool f8) { return f8 ? kBarSlots : R_FULL; }
 template <class C, bool F8>
 constexpr bool barrier_ranges_fit()
 {
-    return (F8 ? C::stages <= 6 : C::stages <= 3) && C::sbufs <= 4 && C::pbufs <= 4 && C::nwg <= 2 && kQD <= 4;
+    return (F8 ? C::stages <= 6 : C::stages <= 3) && C::sbufs <= 4 && C::pbufs <= 4 && C::nwg <= 4 && kQD <= 4;
 }
 
 // F8 = false: bf16 cache; the K and V tiles go from TMA straight to the tensor cores.
@@ -88,11 +88,19 @@ struct TcCfg {
     static constexpr int nb = NWG * HW <= 8 ? 1 : NWG * HW / 8;   // 8-head blocks of P^T / O^T that carry heads
     static constexpr int conv_warps = F8 ? 4 : 0;             // FP8: the converter warpgroup
     // + TMA warp + S^T issuer warp + PV issuer warp.  FP8 with 32 heads: the last three warps are padded
-    // to a warpgroup and the registers are redistributed (setmaxnreg): 512 threads launch with 128
-    // registers each, the softmax warpgroups then take 176, the converter 104 and the last warpgroup 56
-    // (2 * 176 + 104 + 56 = 4 * 128, so every increase is covered by the decreases)
+    // to a warpgroup and the registers are redistributed (setmaxnreg).  Two softmax warpgroups: 512
+    // threads launch with 128 registers each, the softmax warpgroups then take 176, the converter 104
+    // and the last warpgroup 56; four: 768 threads launch with 80, then 88, 88 and 40 (the sum never
+    // exceeds the launch's share, so every increase is covered by the decreases)
     static constexpr bool regsplit = F8 && N == 32;
-    static constexpr int threads = regsplit ? 512 : kWG * nwg + 32 * conv_warps + 96;
+    static constexpr int threads = regsplit ? kWG * (nwg + 2) : kWG * nwg + 32 * conv_warps + 96;
+    static constexpr int reg_launch = nwg == 4 ? 80 : 128;
+    static constexpr int reg_soft = nwg == 4 ? 88 : 176;
+    static constexpr int reg_conv = nwg == 4 ? 88 : 104;
+    static constexpr int reg_last = nwg == 4 ? 40 : 56;
+    static_assert(!regsplit || (nwg == 2 || nwg == 4), "register split for two or four softmax warpgroups");
+    static_assert(!regsplit || kWG * (nwg * reg_soft + reg_conv + reg_last) <= threads * reg_launch,
+                  "register split within the launch's share");
     static constexpr int sbufs = 4;                            // S^T buffers: QK^T runs up to four tiles ahead
     static constexpr int pbufs = (F8 || N == 16) ? 2 : 1;      // P^T buffers (2: the softmax runs a tile ahead)
     // P as one 16-bit term (FP8: f16 of 128 p, relative rounding 2^-11 on each weight) or as bf16 hi + lo
@@ -363,6 +371,16 @@ __device__ __forceinline__ void tmem_stn(uint32_t taddr, const uint32_t (&r)[NC]
     }
 }
 
+// The warp's register share becomes R (from L at launch): setmaxnreg.inc waits for the registers that
+// other warps' setmaxnreg.dec release.
+template <int R, int L>
+__device__ __forceinline__ void set_max_regs()
+{
+    static_assert(R % 8 == 0 && R >= 24 && R <= 256, "setmaxnreg takes multiples of 8 in [24, 256]");
+    if constexpr (R > L) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R) : "memory");
+    else if constexpr (R < L) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R) : "memory");
+}
+
 // ---------------------------------------------------------------------------------------------
 template <int N, bool F8, int HW, int NWG>
 __global__ void __launch_bounds__(TcCfg<N, F8, HW, NWG>::threads, 1)
@@ -458,11 +476,10 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     const uint32_t tO0 = tmem + C::o_base;
 
     // Register split (FP8, 32 heads): each warpgroup sets its share first thing in its own branch, the
-    // same instruction for all four of its warps; 2 * 176 + 104 + 56 = 4 * 128, the launch's share.
-    static_assert(!C::regsplit || (C::threads == 512 && 2 * 176 + 104 + 56 == 4 * 128), "register split");
+    // same instruction for all four of its warps (the shares are checked against the launch's in TcCfg).
     if (warp >= producer_warp) {
         // the last warpgroup: producer, S^T issuer, PV issuer (and, with the split, one idle warp)
-        if constexpr (C::regsplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+        if constexpr (C::regsplit) set_max_regs<C::reg_last, C::reg_launch>();
         if (warp == producer_warp) {
             // ---------------- claims units, loads the group's query rows and streams the K/V tiles
             if (lane == 0) {
@@ -679,7 +696,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         }
     } else if (F8 && warp >= conv_warp0) {
         // ---------------- FP8 converter: thread ct owns token ct of each tile (TMEM lane ct of K)
-        if constexpr (C::regsplit) asm volatile("setmaxnreg.dec.sync.aligned.u32 104;" ::: "memory");
+        if constexpr (C::regsplit) set_max_regs<C::reg_conv, C::reg_launch>();
         const int ct = threadIdx.x - kWG * C::nwg;
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         int tcount = 0, icount = 0;
@@ -797,7 +814,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     } else {
         // ---------------- softmax warpgroup wg: heads HW*wg .. HW*wg+HW-1; thread t owns token t of
         // each tile (TMEM lane t of S^T) and column d = t of O^T
-        if constexpr (C::regsplit) asm volatile("setmaxnreg.inc.sync.aligned.u32 176;" ::: "memory");
+        if constexpr (C::regsplit) set_max_regs<C::reg_soft, C::reg_launch>();
         const int wg = warp >> 2;
         const int quarter = warp & 3;              // TMEM lane quarter this warp may access
         const int t = quarter * 32 + lane;
@@ -1074,7 +1091,8 @@ cudaError_t launch_persistent(const CUtensorMap &tmK, const CUtensorMap &tmV, co
             // launched with: refuse to launch unless the launch holds the whole split
             cudaFuncAttributes fa;
             if ((e = cudaFuncGetAttributes(&fa, decode_persistent_kernel<N, F8, HW, NWG>)) != cudaSuccess) return e;
-            if ((long long)fa.numRegs * TcCfg<N, F8, HW, NWG>::threads < 4LL * 128 * 128)
+            using Cf = TcCfg<N, F8, HW, NWG>;
+            if ((long long)fa.numRegs * Cf::threads < (long long)kWG * (Cf::nwg * Cf::reg_soft + Cf::reg_conv + Cf::reg_last))
                 return cudaErrorInvalidConfiguration;
         }
         attr_done[dev] = true;
@@ -1119,7 +1137,7 @@ cudaError_t launch_decode_tc(const CUtensorMap &tmK, const CUtensorMap &tmV, con
         if (a.group <= 4) return launch_persistent<16, true, 4, 1>(tmK, tmV, tmQ, a, stream);
         if (a.group <= 8) return launch_persistent<16, true, 8, 1>(tmK, tmV, tmQ, a, stream);
         if (a.group <= 16) return launch_persistent<16, true, 8, 2>(tmK, tmV, tmQ, a, stream);
-        if (a.group <= 32) return launch_persistent<32, true, 16, 2>(tmK, tmV, tmQ, a, stream);
+        if (a.group <= 32) return launch_persistent<32, true, 8, 4>(tmK, tmV, tmQ, a, stream);
         return cudaErrorInvalidValue;
     }
     if (a.group <= 4) return launch_persistent<16, false, 4, 1>(tmK, tmV, tmQ, a, stream);
