@@ -117,6 +117,29 @@ def test_split_boundaries(oracle_mod):
     _check_all(oracle_mod, x, _run(x))
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (32, 1)])
+def test_many_pieces_per_history(oracle_mod, Hq, Hkv):
+    # one sequence of 128 tiles on 148 SMs: the planner cuts it into the most pieces allowed (64, two tiles
+    # each), so the merge runs well past the pieces it fetches together with the count
+    x = inputs.make_decode(1, Hq, Hkv, 128, 16384, device=DEV, seed=70 + Hq)
+    _check_all(oracle_mod, x, _run(x))
+
+
+def test_large_batch_planned_by_one_warp(oracle_mod):
+    # 2500 histories (about 78 per planner lane), some empty, some one tile, most split into pieces
+    B, Hq, Hkv, Tmax = 2500, 8, 2, 640
+    g = torch.Generator().manual_seed(90)
+    lens = torch.randint(0, Tmax + 1, (B,), generator=g)
+    lens[::97] = 0
+    lens[5::89] = 1
+    lens[7::83] = Tmax
+    x = inputs.make_decode(B, Hq, Hkv, 128, Tmax, seqlens=lens.tolist(), device=DEV, seed=91)
+    out = _run(x)
+    sl = x.seqlens.cpu()
+    bs = sorted({0, 1, 5, 7, 97, 1249, B - 1, int(sl.argmax()), int(sl.argmin())} | set(range(1200, 1216)))
+    assert_close(out[bs].double().cpu().numpy(), _oracle_rows(oracle_mod, x, bs))
+
+
 def test_nan_poisoned_padding_is_never_read(oracle_mod):
     lens = [5, 64, 100, 777]
     x = inputs.make_decode(4, 16, 4, 128, 800, seqlens=lens, device=DEV, seed=5, poison=True)
