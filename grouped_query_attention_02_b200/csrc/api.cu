@@ -321,9 +321,10 @@ int decode_enqueue(const void *q, const void *k, const void *v, const int32_t *s
     }
     a.wait_budget_ns = kWaitBudgetNs;
     a.num_ctas = num_sms;
-    // groups above 8 are planned in two rounds of long pieces: their remainders are cut in two (sweeps
-    // over 1-8 rounds and 1-8 tail pieces: +1.5 % on the MQA shape, +2-3 % at g = 16)
-    a.tail_split = a.group > 8 ? 2 : 1;
+    // groups of 9-16 are planned in two rounds of long pieces with their remainders cut in two, larger
+    // groups in one round with remainders cut in four (sweeps over rounds and tail pieces: +2-3 % at
+    // g = 16; at g = 32, +1-1.5 % bf16 and +3 % FP8 over two rounds)
+    a.tail_split = a.group > 16 ? 4 : (a.group > 8 ? 2 : 1);
     int n = 0;
     if (p.tensor_cores) {
         // the group's query rows as a 3-D map (d, heads, batch): one box = N rows of one 64-column half

@@ -227,10 +227,10 @@ __global__ void __launch_bounds__(32) decode_plan_kernel(const DecodeArgs a, int
         tot += __shfl_xor_sync(0xffffffffu, tot, o);
         mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
-    // rounds of (piece, KV head) units per persistent CTA: eight for groups up to 8, two above, whose
-    // units of more heads carry a larger fixed cost each (measured on the benchmark shapes); never more
-    // than nsplit pieces
-    const long long rounds = a.plan_rounds > 0 ? a.plan_rounds : (a.group > 8 ? 2 : 8);
+    // rounds of (piece, KV head) units per persistent CTA: eight for groups up to 8, two up to 16 and one
+    // above, whose units of more heads carry a larger fixed cost each (measured on the benchmark shapes);
+    // never more than nsplit pieces
+    const long long rounds = a.plan_rounds > 0 ? a.plan_rounds : (a.group > 16 ? 1 : (a.group > 8 ? 2 : 8));
     long long Cl = (tot * a.Hkv + rounds * slots - 1) / (rounds * slots);
     const long long cmin = (mx + a.nsplit - 1) / a.nsplit;
     if (Cl < cmin) Cl = cmin;
