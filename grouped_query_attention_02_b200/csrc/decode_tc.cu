@@ -200,11 +200,15 @@ __device__ __forceinline__ int warp_exclusive_scan(int v, int &total)
 // items[i] = {b, piece index | pieces of b << 16, first token, end token}.  Full pieces come first, in
 // sequence order, then the shorter last pieces in decreasing length (a counting sort).
 // One warp: its time is latency (one read of the lengths and a few dependent steps), which a warp
-// takes with shuffles where a larger block would need barriers.  Lane l owns the contiguous sequences
+// takes with shuffles where a larger block would need barriers.  The lengths are read once, eight
+// coalesced loads in flight per lane, into shared memory; lane l then owns the contiguous sequences
 // [l * per, (l + 1) * per).
+constexpr int kPlanLenCache = 4096;   // lengths kept in shared memory (any further ones are re-read)
+
 __global__ void __launch_bounds__(32) decode_plan_kernel(const DecodeArgs a, int slots)
 {
-    __shared__ int hist[kPlanMaxC];   // tail pieces per size class, then each class's next slot
+    __shared__ int hist[kPlanMaxC];          // tail pieces per size class, then each class's next slot
+    __shared__ int s_len[kPlanLenCache];     // clamped lengths of the first kPlanLenCache sequences
 
     // launched as a programmatic dependent of whatever ran before on the stream (the previous call's
     // combine, say, which still reads nsplit_b): wait for it before touching anything, so that only the
@@ -213,12 +217,28 @@ __global__ void __launch_bounds__(32) decode_plan_kernel(const DecodeArgs a, int
     // the persistent kernel may start its prologue now; it reads this plan only after griddepcontrol.wait
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int lane = threadIdx.x;
+    const int ncache = min(a.B, kPlanLenCache);
+    for (int i0 = 0; i0 < ncache; i0 += 8 * 32) {
+        int v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * 32 + lane;
+            v[u] = i < ncache ? __ldg(a.seqlens + i) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int i = i0 + u * 32 + lane;
+            if (i < ncache) s_len[i] = v[u] < 0 ? 0 : (v[u] > a.Tmax ? a.Tmax : v[u]);
+        }
+    }
+    __syncwarp();
+    auto tokens = [&](int b) { return b < kPlanLenCache ? s_len[b] : plan_tokens(a, b); };
     const int per = (a.B + 31) / 32;
     const int b0 = min(a.B, lane * per), b1 = min(a.B, b0 + per);
     long long tot = 0;
     int mx = 0;
     for (int b = b0; b < b1; ++b) {
-        const int tl = (plan_tokens(a, b) + kTok - 1) / kTok;
+        const int tl = (tokens(b) + kTok - 1) / kTok;
         tot += tl;
         mx = max(mx, tl);
     }
@@ -256,7 +276,7 @@ __global__ void __launch_bounds__(32) decode_plan_kernel(const DecodeArgs a, int
     int nfull = 0;
     bool empty = false;
     for (int b = b0; b < b1; ++b) {
-        const int tl = (plan_tokens(a, b) + kTok - 1) / kTok;
+        const int tl = (tokens(b) + kTok - 1) / kTok;
         const int full = tl / C, rem = tl % C;
         const int k = tail_pieces(full, rem);
         a.nsplit_b[b] = full + k;
@@ -275,7 +295,7 @@ __global__ void __launch_bounds__(32) decode_plan_kernel(const DecodeArgs a, int
         // no cached token: no unit will touch such a sequence, its output rows are zero
         const int orow = a.out_row > 0 ? a.out_row : kD;
         for (int b = 0; b < a.B; ++b) {
-            if (plan_tokens(a, b) > 0) continue;
+            if (tokens(b) > 0) continue;
             uint4 *o = reinterpret_cast<uint4 *>(a.out + (size_t)b * a.Hq * orow);
             for (int i = lane; i < a.Hq * orow / 8; i += 32) o[i] = make_uint4(0, 0, 0, 0);
         }
@@ -304,7 +324,7 @@ __global__ void __launch_bounds__(32) decode_plan_kernel(const DecodeArgs a, int
     }
     __syncwarp();
     for (int b = b0; b < b1; ++b) {
-        const int T = plan_tokens(a, b);
+        const int T = tokens(b);
         const int tl = (T + kTok - 1) / kTok;
         const int full = tl / C, rem = tl % C;
         const int k = tail_pieces(full, rem);
