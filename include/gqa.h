@@ -103,7 +103,9 @@ gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache, c
  * are widened to f16 on the SM, exactly, after one TMA read of each tile;
  * the query is carried in f16 with a power-of-two scale per head (elements
  * below 2^-24 of the head's largest |q| flush to zero), the products run on
- * the tensor cores with fp32 accumulation.  NaN codes inside the history
+ * the tensor cores with fp32 accumulation, and the softmax weights enter the
+ * P.V product as f16 values of 128 p (relative rounding at most 2^-11 per
+ * weight; the normalising sum is taken in fp32).  NaN codes inside the history
  * propagate to the output; rows past seqlens[b] are never used.  Same
  * workspace, stream and error rules as gqa_decode.
  */
