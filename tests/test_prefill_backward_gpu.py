@@ -26,7 +26,7 @@ def _run(x, dout):
 
 def _check(got, ref, name):
     """The stated bar (normwise relative 2e-2; absolute 2e-2, scaled by max|ref| where gradients exceed 1,
-    since rounding a gradient of magnitude m to bf16 alone moves it by up to 2^-9 m) and a tight gate
+    since rounding a gradient of magnitude m to bf16 alone moves it by up to 2^-8 m) and a tight gate
     from the arithmetic: every product term carries at most about 2^-8 relative error (P or dS rounded
     to bf16, D from the bf16 output), the gradient itself is rounded to bf16, and the terms' absolute
     sum stays within a few times max|ref| here, so |g - r| <= 2^-8 |r| + 2^-7 max(max|ref|, 2^-10)."""
