@@ -125,9 +125,11 @@ def test_many_pieces_per_history(oracle_mod, Hq, Hkv):
     _check_all(oracle_mod, x, _run(x))
 
 
-def test_large_batch_planned_by_one_warp(oracle_mod):
-    # 2500 histories (about 78 per planner lane), some empty, some one tile, most split into pieces
-    B, Hq, Hkv, Tmax = 2500, 8, 2, 640
+@pytest.mark.parametrize("B", [2500, 4200])
+def test_large_batch_planned_by_one_warp(oracle_mod, B):
+    # thousands of histories (78 or 131 per planner lane; past 4096 the planner re-reads lengths it does
+    # not keep), some empty, some one tile, most split into pieces
+    Hq, Hkv, Tmax = 8, 2, 640
     g = torch.Generator().manual_seed(90)
     lens = torch.randint(0, Tmax + 1, (B,), generator=g)
     lens[::97] = 0
@@ -136,7 +138,8 @@ def test_large_batch_planned_by_one_warp(oracle_mod):
     x = inputs.make_decode(B, Hq, Hkv, 128, Tmax, seqlens=lens.tolist(), device=DEV, seed=91)
     out = _run(x)
     sl = x.seqlens.cpu()
-    bs = sorted({0, 1, 5, 7, 97, 1249, B - 1, int(sl.argmax()), int(sl.argmin())} | set(range(1200, 1216)))
+    bs = sorted({0, 1, 5, 7, 97, 1249, B - 1, int(sl.argmax()), int(sl.argmin())} | set(range(1200, 1216)) |
+                set(range(min(B, 4090), min(B, 4102))))
     assert_close(out[bs].double().cpu().numpy(), _oracle_rows(oracle_mod, x, bs))
 
 
