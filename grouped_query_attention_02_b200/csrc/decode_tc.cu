@@ -57,11 +57,11 @@ constexpr int kPlanMaxC = 4096;           // remainder sizes sorted by a shared-
 // barrier slots: each name owns a contiguous range (sizes checked against the configuration below)
 enum : int { K_FULL = 0, V_FULL = 3, KV_EMPTY = 6, S_FULL = 9, S_FREE = 13, P_FULL = 17, P_FREE = 21, O_FULL = 25,
              O_FREE = 27, Q_FULL = 29, Q_EMPTY = 31, I_FULL = 33, I_EMPTY = 37, DRAIN = 41, DRAIN_PV = 42, GRP = 43,
-             // FP8 only: code ring (R_EMPTY: the stage's PV product is done), converted K (tensor memory),
-             // converted V (in the stage), converted Q, and the unit slot's score factors (the softmax
-             // releases the slot after reading them)
-             R_FULL = 47, R_EMPTY = 53, KT_FULL = 59, KT_FREE = 61, VC_FULL = 63, QC_FULL = 69, QF_FULL = 71,
-             kBarSlots = 75 };
+             // FP8 only: code ring (R_EMPTY: the stage's PV product is done), converted V (in the stage),
+             // the query's E4M3 terms, the unit slot's score factors (the softmax releases the slot after
+             // reading them), and the stage's key codes read by the S^T products
+             R_FULL = 47, R_EMPTY = 53, VC_FULL = 59, QC_FULL = 65, QF_FULL = 67, K_READ = 71,
+             kBarSlots = 77 };
 constexpr int kBarSlotsFor(bool f8) { return f8 ? kBarSlots : R_FULL; }
 template <class C, bool F8>
 constexpr bool barrier_ranges_fit()
@@ -70,14 +70,14 @@ constexpr bool barrier_ranges_fit()
 }
 
 // F8 = false: bf16 cache; the K and V tiles go from TMA straight to the tensor cores.
-// F8 = true: FP8 (E4M3) cache.  TMA brings the raw code tiles (16 KB each) into a ring; one converter
-// warpgroup widens them exactly to f16 (every E4M3 value is an f16 value): the keys into tensor
-// memory, where they are the A operand of S^T, the values into a 128-byte-swizzled f16 tile that
-// takes the place of the stage's two code tiles (each thread rewrites only the two 128-byte rows it
-// has just read, so no thread waits for another).  Q is converted in place to f16 with a power-of-two
-// scale per head, and P enters the second product as one f16 term of 128 p (so that small weights stay
-// normal; relative rounding 2^-11 per weight, against the bf16 path's hi + lo pair), with f16 MMAs
-// throughout.
+// F8 = true: FP8 (E4M3) cache.  TMA brings the raw code tiles (16 KB each) into a ring.  S^T is an
+// E4M3 product (kind::f8f6f4) straight from the key codes: the query enters it as two E4M3 terms of
+// q 2^e per head (t0 = e4m3(v), t1 = e4m3(v - t0), which carry a bf16 element exactly down to about
+// 2^-9 of the head's largest), stacked as 2N rows of B, and the softmax adds the two products.  One
+// converter warpgroup widens the values exactly to f16 (every E4M3 value is an f16 value) into a
+// 128-byte-swizzled tile that takes the place of the stage's two code tiles, once S^T has read the
+// keys.  P enters the second product as one f16 term of 128 p (so that small weights stay normal;
+// relative rounding 2^-11 per weight, against the bf16 path's hi + lo pair), an f16 MMA.
 // HW: heads one softmax warpgroup handles (4, 8 or 16), NWG: softmax warpgroups.  Groups of up to 4
 // or 8 heads only compute their own columns of the N = 16 wide products; more warpgroups with fewer
 // heads each shorten the softmax's per-tile chain.
@@ -130,8 +130,10 @@ struct TcCfg {
     // FP8: K[2] (64 columns each: 128 f16 keys per token, packed in pairs) first, then as below.
     // S[sbufs] (N columns each) and O[2] (2N columns each: the hi and lo products side by side, the lo
     // columns 8 * nb after the hi ones; FP8 reads only the hi columns)
-    static constexpr uint32_t s_base = F8 ? 128 : 0;
-    static constexpr uint32_t o_base = s_base + sbufs * N;
+    // FP8: each S buffer holds the products with the query's two E4M3 terms side by side (2N columns)
+    static constexpr uint32_t s_cols = F8 ? 2 * N : N;
+    static constexpr uint32_t s_base = 0;
+    static constexpr uint32_t o_base = s_base + sbufs * s_cols;
     static constexpr uint32_t tmem_used = o_base + 4 * N;
     static constexpr uint32_t tmem_cols = tmem_used <= 128 ? 128 : (tmem_used <= 256 ? 256 : 512);
     static_assert(bytes <= 227 * 1024, "shared memory budget");
@@ -443,10 +445,9 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 mbar_init(&bar[R_FULL + s], 1);
                 mbar_init(&bar[R_EMPTY + s], 1);
                 mbar_init(&bar[VC_FULL + s], kWG);
+                mbar_init(&bar[K_READ + s], 1);
             }
             for (int s = 0; s < 2; ++s) {
-                mbar_init(&bar[KT_FULL + s], kWG);
-                mbar_init(&bar[KT_FREE + s], 1);
                 mbar_init(&bar[QC_FULL + s], kWG);
             }
             for (int s = 0; s < kQD; ++s) mbar_init(&bar[QF_FULL + s], kWG);
@@ -493,7 +494,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS0 = tmem + C::s_base;   // S buffer i at tS0 + i * N
+    const uint32_t tS0 = tmem + C::s_base;   // S buffer i at tS0 + i * s_cols
     // O buffer i at tO0 + 2N i: V^T P_hi^T, then (8 nb columns later) V^T P_lo^T
     const uint32_t tO0 = tmem + C::o_base;
 
@@ -603,7 +604,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             // ---------------- S^T issuer: S^T = K (K-major) . Q^T (K-major), as soon as the keys and a free
             // S buffer allow (up to four tiles ahead of the softmax)
             if (lane == 0) {
-                const uint32_t idesc_s = F8 ? umma_idesc_f16(kTok, N, 0, 0) : umma_idesc_bf16(kTok, N, 0, 0);
+                const uint32_t idesc_s = F8 ? umma_idesc_f16(kTok, 2 * N, 0, 0) : umma_idesc_bf16(kTok, N, 0, 0);
                 int tcount = 0, icount = 0;
                 bool ok = true;
                 while (ok) {
@@ -620,8 +621,7 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                     for (int jj = 0; jj < ntl; ++jj) {
                         const int T = tcount + jj;
                         const int s = T % C::stages, sb = T % C::sbufs;
-                        if (!wait_or_fail(&bar[(F8 ? KT_FULL + (T & 1) : K_FULL + s)],
-                                          F8 ? ((T >> 1) & 1) : ((T / C::stages) & 1), a, err)) {
+                        if (!wait_or_fail(&bar[(F8 ? R_FULL : K_FULL) + s], (T / C::stages) & 1, a, err)) {
                             ok = false;
                             break;
                         }
@@ -631,18 +631,18 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t d_tmem = tS0 + sb * N;
+                        const uint32_t d_tmem = tS0 + sb * C::s_cols;
                         if constexpr (F8) {
-                            // A = the converted keys in tensor memory: 16 head coordinates = 8 columns
-                            const uint32_t k_tmem = tmem + (T & 1) * 64;
+                            // A = the stage's key codes as TMA left them ([128 tokens][128 codes], 128-byte
+                            // swizzle), B = the query's two E4M3 terms as 2N rows (term 0, then term 1): the
+                            // keys cross shared memory once, 32 codes of K per product
+                            const uint32_t k_addr = smem_u32(smem + s * C::stage_bytes);
     #pragma unroll
-                            for (int ks = 0; ks < kD / 16; ++ks) {
-                                const uint32_t qa = q_addr + (ks >> 2) * C::q_half + (ks & 3) * 32;
-                                umma_ts(d_tmem, k_tmem + ks * 8, umma_smem_desc(qa, 16, 1024, 2), idesc_s,
-                                        ks > 0 ? 1u : 0u);
-                            }
+                            for (int ks = 0; ks < kD / 32; ++ks)
+                                umma_ss_e4m3(d_tmem, umma_smem_desc(k_addr + ks * 32, 16, 1024, 2),
+                                             umma_smem_desc(q_addr + ks * 32, 16, 1024, 2), idesc_s, ks > 0 ? 1u : 0u);
                             umma_commit(&bar[S_FULL + sb]);
-                            umma_commit(&bar[KT_FREE + (T & 1)]);
+                            umma_commit(&bar[K_READ + s]);   // the key codes may now be overwritten
                         } else {
                             const uint32_t k_addr = smem_u32(smem + s * C::stage_bytes);
     #pragma unroll
@@ -720,7 +720,6 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
         // ---------------- FP8 converter: thread ct owns token ct of each tile (TMEM lane ct of K)
         if constexpr (C::regsplit) set_max_regs<C::reg_conv, C::reg_launch>();
         const int ct = threadIdx.x - kWG * C::nwg;
-        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         int tcount = 0, icount = 0;
         while (true) {
             const int slot = icount % kQD;
@@ -729,12 +728,16 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             const int t_begin = qq[3], t_end = qq[4];
             mbar_arrive(&bar[I_EMPTY + slot]);
             if (t_end < 0) break;
-            // the group's query rows, in place: bf16 -> f16 times 2^e per head, e putting the head's
-            // largest |q| in [2^14, 2^15); the softmax undoes 2^e in its score factor
+            // the group's query rows as two E4M3 terms of q 2^e per head (e putting the head's largest |q| in
+            // [2^7, 2^8), below E4M3's largest 448): t0 = e4m3(v), t1 = e4m3(v - t0), the residual exact in
+            // fp32.  A bf16 element (8 significant bits) leaves a residual of at most 4, so the two terms carry
+            // it exactly unless the residual falls below E4M3's normal range (elements below about 2^-9 of
+            // the head's largest); the softmax undoes 2^e in its score factor.  The terms take the places of
+            // the row's two bf16 halves, so B of S^T is the buffer read as 2N rows of 128 codes.
             const int qb = icount & 1;
             if (!wait_or_fail(&bar[Q_FULL + qb], (icount >> 1) & 1, a, err)) break;
             {
-                constexpr int tpr = kWG / N;         // threads per query row
+                constexpr int tpr = kWG / N;         // threads per query row (all in one warp)
                 constexpr int cpt = 16 / tpr;        // 16-byte chunks per thread (16 per row: 2 halves x 8)
                 const int row = ct / tpr, j0 = ct % tpr;
                 uint8_t *qs = smem + C::q_off + qb * C::q_bytes;
@@ -752,18 +755,47 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
 #pragma unroll
                 for (int o = tpr / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                 const int ex = (int)((__float_as_uint(mx) >> 23) & 0xFF) - 127;
-                const int e = min(14 - ex, 100);      // e in [-114, 100]: both 2^e and 2^-e are normal floats
+                const int e = min(7 - ex, 100);       // e in [-120, 100]: both 2^e and 2^-e are normal floats
                 const float up = __uint_as_float((uint32_t)(127 + e) << 23);
                 const float down = __uint_as_float((uint32_t)(127 - e) << 23);
+                // every bf16 element of this row is in registers before any term overwrites the row
+                __syncwarp();
 #pragma unroll
                 for (int i = 0; i < cpt; ++i) {
+                    // physical chunk (k & 7) of half k >> 3 holds logical chunk l: elements 64 (k >> 3) + 8 l ..,
+                    // which are codes 8 (l & 1) .. of logical code chunk 4 (k >> 3) + l / 2
                     const int k = j0 + i * tpr;
-                    uint4 o;
-                    o.x = pack_f16x2(bf16_lo(v[i].x) * up, bf16_hi(v[i].x) * up);
-                    o.y = pack_f16x2(bf16_lo(v[i].y) * up, bf16_hi(v[i].y) * up);
-                    o.z = pack_f16x2(bf16_lo(v[i].z) * up, bf16_hi(v[i].z) * up);
-                    o.w = pack_f16x2(bf16_lo(v[i].w) * up, bf16_hi(v[i].w) * up);
-                    *reinterpret_cast<uint4 *>(qs + (k >> 3) * C::q_half + row * 128 + (k & 7) * 16) = o;
+                    const int l = (k & 7) ^ (row & 7);
+                    const int c = 4 * (k >> 3) + (l >> 1);
+                    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+                    float r[8];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        r[2 * q] = bf16_lo(w[q]) * up;
+                        r[2 * q + 1] = bf16_hi(w[q]) * up;
+                    }
+#pragma unroll
+                    for (int tt = 0; tt < 2; ++tt) {
+                        uint32_t packed[2];
+#pragma unroll
+                        for (int q = 0; q < 2; ++q) {
+                            uint32_t code4 = 0;
+#pragma unroll
+                            for (int pr = 0; pr < 2; ++pr) {
+                                const int e0 = 4 * q + 2 * pr;
+                                uint16_t c2;
+                                asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(c2) : "f"(r[e0 + 1]), "f"(r[e0]));
+                                uint32_t f2;   // the two codes back as f16 (exact), low element first
+                                asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f2) : "h"(c2));
+                                r[e0] -= __half2float(__ushort_as_half((unsigned short)(f2 & 0xffffu)));
+                                r[e0 + 1] -= __half2float(__ushort_as_half((unsigned short)(f2 >> 16)));
+                                code4 |= (uint32_t)c2 << (16 * pr);
+                            }
+                            packed[q] = code4;
+                        }
+                        *reinterpret_cast<uint2 *>(qs + tt * C::q_half + row * 128 + ((c ^ (row & 7)) << 4) + (l & 1) * 8) =
+                            make_uint2(packed[0], packed[1]);
+                    }
                 }
                 if (j0 == 0) qfac[slot * N + row] = a.qk_factor * down;
             }
@@ -774,42 +806,20 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             bool ok = true;
             for (int jj = 0; jj < ntl; ++jj) {
                 const int T = tcount + jj;
-                const int s = T % C::stages, cb = T & 1;
+                const int s = T % C::stages;
                 if (!wait_or_fail(&bar[R_FULL + s], (T / C::stages) & 1, a, err)) { ok = false; break; }
                 // the raw tiles were stored with the 128-byte swizzle: chunk c of row ct at c ^ (ct & 7)
                 uint8_t *krow = smem + s * C::stage_bytes + ct * 128;
-                // tokens past the piece's end may hold anything (NaN codes included): they become zeros,
-                // so that no 0 * NaN reaches an accumulator
+                // tokens past the piece's end may hold anything (NaN codes included): their values become
+                // zeros, so that no 0 * NaN reaches an accumulator (their scores are masked by position)
                 const bool valid = (t_begin + jj * kTok + ct) < t_end;
-                // keys -> tensor memory, row ct: column j holds head coordinates 2j, 2j+1
-                if (T >= 2 && !wait_or_fail(&bar[KT_FREE + cb], ((T >> 1) - 1) & 1, a, err)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t w[32];
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint4 r = *reinterpret_cast<const uint4 *>(krow + (((h * 4 + c) ^ (ct & 7)) << 4));
-                        e4m3x4_to_f16x4(r.x, w[c * 8 + 0], w[c * 8 + 1]);
-                        e4m3x4_to_f16x4(r.y, w[c * 8 + 2], w[c * 8 + 3]);
-                        e4m3x4_to_f16x4(r.z, w[c * 8 + 4], w[c * 8 + 5]);
-                        e4m3x4_to_f16x4(r.w, w[c * 8 + 6], w[c * 8 + 7]);
-                    }
-                    if (!valid) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) w[i] = 0u;
-                    }
-                    tmem_st32(tmem + cb * 64 + lane_off + h * 32, w);
-                }
-                tmem_wait_st();
-                tc_fence_before();
-                mbar_arrive(&bar[KT_FULL + cb]);
                 // values -> f16 tile [2 halves][128 rows][128 B] with the 128-byte swizzle over the stage:
-                // row ct of half 0 is where this thread's key codes were (all read above), row ct of half 1
-                // where its value codes are (read into registers first)
+                // row ct of half 0 is where the key codes are (rewritten once the S^T products have read
+                // them), row ct of half 1 where this thread's value codes are (read into registers first)
                 uint4 vr[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) vr[c] = *reinterpret_cast<const uint4 *>(krow + kHalf + ((c ^ (ct & 7)) << 4));
+                if (!wait_or_fail(&bar[K_READ + s], (T / C::stages) & 1, a, err)) { ok = false; break; }
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint4 lo4, hi4;
@@ -933,7 +943,15 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
                 if (!wait_or_fail(&bar[S_FULL + sbuf], (T / C::sbufs) & 1, a, err)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t raw[HW];
-                tmem_ldn<HW>(tS0 + sbuf * N + lane_off + hs, raw);
+                tmem_ldn<HW>(tS0 + sbuf * C::s_cols + lane_off + hs, raw);
+                if constexpr (F8) {
+                    // the score is the sum of the products with the query's two terms
+                    uint32_t raw1[HW];
+                    tmem_ldn<HW>(tS0 + sbuf * C::s_cols + N + lane_off + hs, raw1);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < HW; ++h) raw[h] = __float_as_uint(__uint_as_float(raw[h]) + __uint_as_float(raw1[h]));
+                }
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&bar[S_FREE + sbuf]);
