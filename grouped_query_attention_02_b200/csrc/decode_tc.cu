@@ -72,8 +72,9 @@ constexpr bool barrier_ranges_fit()
 // F8 = false: bf16 cache; the K and V tiles go from TMA straight to the tensor cores.
 // F8 = true: FP8 (E4M3) cache.  TMA brings the raw code tiles (16 KB each) into a ring.  S^T is an
 // E4M3 product (kind::f8f6f4) straight from the key codes: the query enters it as two E4M3 terms of
-// q 2^e per head (t0 = e4m3(v), t1 = e4m3(v - t0), which carry a bf16 element exactly down to about
-// 2^-9 of the head's largest), stacked as 2N rows of B, and the softmax adds the two products.  One
+// q 2^e per head (t0 = e4m3(v), t1 = e4m3(v - t0), which carry a bf16 element exactly down to 2^-10
+// of the head's largest |q| and within 2^-17 of it below), stacked as 2N rows of B, and the softmax adds
+// the two products.  One
 // converter warpgroup widens the values exactly to f16 (every E4M3 value is an f16 value) into a
 // 128-byte-swizzled tile that takes the place of the stage's two code tiles, once S^T has read the
 // keys.  P enters the second product as one f16 term of 128 p (so that small weights stay normal;
@@ -730,10 +731,11 @@ decode_persistent_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_c
             if (t_end < 0) break;
             // the group's query rows as two E4M3 terms of q 2^e per head (e putting the head's largest |q| in
             // [2^7, 2^8), below E4M3's largest 448): t0 = e4m3(v), t1 = e4m3(v - t0), the residual exact in
-            // fp32.  A bf16 element (8 significant bits) leaves a residual of at most 4, so the two terms carry
-            // it exactly unless the residual falls below E4M3's normal range (elements below about 2^-9 of
-            // the head's largest); the softmax undoes 2^e in its score factor.  The terms take the places of
-            // the row's two bf16 halves, so B of S^T is the buffer read as 2N rows of 128 codes.
+            // fp32.  A bf16 element v = m 2^(E-7) (m of 8 bits) leaves a residual k 2^(E-7) with |k| <= 8,
+            // which E4M3 holds exactly while 2^(E-7) >= 2^-9, its subnormal step: every element down to 2^-10
+            // of the head's largest is carried exactly, smaller ones within 2^-10 absolute (2^-17 of the
+            // largest); the softmax undoes 2^e in its score factor.  The terms take the places of the row's
+            // two bf16 halves, so B of S^T is the buffer read as 2N rows of 128 codes.
             const int qb = icount & 1;
             if (!wait_or_fail(&bar[Q_FULL + qb], (icount >> 1) & 1, a, err)) break;
             {

@@ -99,13 +99,14 @@ gqa_status gqa_decode(const void *q, const void *k_cache, const void *v_cache, c
  *   out[b,h] = sum_{t < seqlens[b]} softmax_t(scale q[b,h].K[b,t,h/g]) V[b,t,h/g]
  *   with K = e4m3(k_cache) * k_scale and V = e4m3(v_cache) * v_scale.
  *
- * Group sizes g = Hq / Hkv up to 32 (GQA_ERR_UNSUPPORTED above).  The codes
- * are widened to f16 on the SM, exactly, after one TMA read of each tile;
- * the query is carried in f16 with a power-of-two scale per head (elements
- * below 2^-24 of the head's largest |q| flush to zero), the products run on
- * the tensor cores with fp32 accumulation, and the softmax weights enter the
- * P.V product as f16 values of 128 p (relative rounding at most 2^-11 per
- * weight; the normalising sum is taken in fp32).  NaN codes inside the history
+ * Group sizes g = Hq / Hkv up to 32 (GQA_ERR_UNSUPPORTED above).  Each tile
+ * is read once by TMA.  The scores are E4M3 tensor-core products straight
+ * from the key codes, with the query as two E4M3 terms of q 2^e per head:
+ * every query element down to 2^-10 of its head's largest |q| is carried
+ * exactly, smaller ones within 2^-17 of that largest.  The value codes are
+ * widened to f16 on the SM, exactly, and the softmax weights enter the P.V
+ * product as f16 values of 128 p (relative rounding at most 2^-11 per weight;
+ * the normalising sum is taken in fp32); every product accumulates in fp32.  NaN codes inside the history
  * propagate to the output; rows past seqlens[b] are never used.  Same
  * workspace, stream and error rules as gqa_decode.
  */
