@@ -124,6 +124,21 @@ def test_fp8_query_magnitudes(oracle_mod, gain):
     assert_close(_run(x).double().cpu().numpy(), _ref(oracle_mod, x), abs_bar=gain < 100)
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (16, 1), (32, 1)])
+def test_fp8_query_with_a_wide_range(oracle_mod, Hq, Hkv):
+    # the scores are E4M3 products with the query split into two E4M3 terms per head: elements spread
+    # over 2^0 .. 2^-24 of a head's largest (every bf16 exponent step the split handles differently:
+    # exact, exact with a subnormal residual, rounded, flushed), with the largest element once per head
+    x = inputs.make_decode_fp8(2, Hq, Hkv, 128, 700, seqlens=[700, 129], device=DEV, seed=31 + Hq)
+    g = torch.Generator().manual_seed(32 + Hq)
+    mag = torch.pow(2.0, -torch.randint(0, 25, (2, Hq, 128), generator=g).double())
+    sign = torch.where(torch.rand((2, Hq, 128), generator=g) < 0.5, -1.0, 1.0).double()
+    q = (mag * sign * 3.0).to(torch.bfloat16)
+    q[:, :, 5] = 3.0   # the head's largest
+    x = inputs.DecodeFp8Inputs(q.to(DEV), x.k_cache, x.v_cache, x.k_scale, x.v_scale, x.seqlens, x.scale)
+    assert_close(_run(x).double().cpu().numpy(), _ref(oracle_mod, x))
+
+
 def test_fp8_peaky_softmax(oracle_mod):
     x = inputs.make_decode_fp8(4, 32, 8, 128, 2048, seqlens=[2048, 1500, 33, 700], device=DEV, seed=6, q_gain=8.0)
     assert_close(_run(x).double().cpu().numpy(), _ref(oracle_mod, x), abs_bar=False)
