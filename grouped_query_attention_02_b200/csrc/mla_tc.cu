@@ -33,9 +33,10 @@
 // mla_combine_planned_kernel merges the pieces of split histories.  All three are chained with
 // programmatic dependent launch.
 //
-// Warps: 0..7 softmax and epilogue (two warpgroups of 32 heads; thread = token of S^T, latent
-// row of O^T), 8 the TMA producer (it also claims units), 9 the tensor-memory allocator and MMA
-// issuer.  Every wait is bounded and reports a timeout through the device status word.
+// Warps: 0..15 softmax and epilogue (four warpgroups of 16 heads; thread = token of S^T, latent
+// row of O^T), 16 the TMA producer (it also claims units), 17 the tensor-memory allocator and MMA
+// issuer, 18 an L2 prefetcher, 19 a second TMA issuer.  Every wait is bounded and reports a timeout
+// through the device status word.
 #include "internal.h"
 #include "mla.h"
 #include "ptx.cuh"
@@ -51,8 +52,8 @@ constexpr int kRopeSlot = kLatChunks;             // the RoPE chunk's slot, then
 constexpr int kChunkBytes = kTok * 128;           // 16 KB: one chunk of a tile
 constexpr int kQChunkBytes = kNh * 128;           // 8 KB: one chunk of the block's query rows
 constexpr int kWG = 128;
-constexpr int kNWG = 2;                           // softmax / epilogue warpgroups
-constexpr int kHW = kNh / kNWG;                   // heads per warpgroup (32)
+constexpr int kNWG = 4;                           // softmax / epilogue warpgroups
+constexpr int kHW = kNh / kNWG;                   // heads per warpgroup (16)
 constexpr int kProducerWarp = 4 * kNWG;
 constexpr int kMmaWarp = kProducerWarp + 1;
 constexpr int kPrefetchWarp = kMmaWarp + 1;       // keeps the tiles kAhead ahead of the producer in L2
@@ -131,6 +132,18 @@ __device__ __forceinline__ bool group_sync(uint64_t *grp, int &uses, const MlaTc
     const bool r = wait_or_fail(grp, uses & 1, a, err);
     ++uses;
     return r;
+}
+
+// kHW consecutive tensor-memory columns per thread (16 or 32)
+__device__ __forceinline__ void tmem_ld_hw(uint32_t taddr, uint32_t (&r)[kHW])
+{
+    if constexpr (kHW == 16) tmem_ld16(taddr, r);
+    else tmem_ld32(taddr, r);
+}
+__device__ __forceinline__ void tmem_st_hw(uint32_t taddr, const uint32_t (&r)[kHW])
+{
+    if constexpr (kHW == 16) tmem_st16(taddr, r);
+    else tmem_st32(taddr, r);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
@@ -421,7 +434,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV2, const __grid_con
                 if (!wait_or_fail(&bar[S_FULL], T & 1, a, err)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t raw[kHW];
-                tmem_ld32(tS + lane_off + hs, raw);
+                tmem_ld_hw(tS + lane_off + hs, raw);
                 tmem_wait_ld();
                 const bool valid = (t_begin + jj * kTok + t) < t_end;
                 float x[kHW];
@@ -483,21 +496,22 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV2, const __grid_con
 #pragma unroll 1
                     for (int j = 0; j < kLatChunks / 2; ++j) {
                         uint32_t o[kHW];
-                        tmem_ld32(tmem + j * kNh + lane_off + hs, o);
+                        tmem_ld_hw(tmem + j * kNh + lane_off + hs, o);
                         tmem_wait_ld();
 #pragma unroll
                         for (int h = 0; h < kHW; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-                        tmem_st32(tmem + j * kNh + lane_off + hs, o);
+                        tmem_st_hw(tmem + j * kNh + lane_off + hs, o);
                     }
                     tmem_wait_st();
                 }
                 if (!valid) {
                     // Rows past the piece may hold anything (NaN included) and the tensor cores would
                     // form 0 * NaN: the token's latent row is zeroed once it has landed (each warpgroup
-                    // zeroes four of the eight chunks)
+                    // zeroes its share of the eight chunks)
+                    constexpr int kZ = kLatChunks / kNWG;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int ch = wg * 4 + c;
+                    for (int c = 0; c < kZ; ++c) {
+                        const int ch = wg * kZ + c;
                         if (!wait_or_fail(&bar[CH_FULL + ch / 2], T & 1, a, err)) { ok = false; break; }
                         uint4 *row = reinterpret_cast<uint4 *>(smem + kSlotOff + ch * kChunkBytes + t * 128);
 #pragma unroll
@@ -527,7 +541,7 @@ mla_decode_tc_kernel(const __grid_constant__ CUtensorMap tmKV2, const __grid_con
 #pragma unroll 1
             for (int j = 0; j < kLatChunks / 2; ++j) {
                 uint32_t o[kHW];
-                tmem_ld32(tmem + j * kNh + lane_off + hs, o);
+                tmem_ld_hw(tmem + j * kNh + lane_off + hs, o);
                 tmem_wait_ld();
                 const int d = j * 128 + t;
 #pragma unroll
