@@ -91,15 +91,15 @@ struct TcCfg {
     // + TMA warp + S^T issuer warp + PV issuer warp.  FP8 with 32 heads: the last three warps are padded
     // to a warpgroup and the registers are redistributed (setmaxnreg).  Two softmax warpgroups: 512
     // threads launch with 128 registers each, the softmax warpgroups then take 176, the converter 104
-    // and the last warpgroup 56; four: 768 threads launch with 80, the softmax keeps 80, the converter
-    // takes 104 and the last warpgroup 40 (the sum never exceeds the launch's share, so every increase is
-    // covered by the decreases; interleaved A/B at g = 32: 80/104 is 2 % faster than 88/88, 72/120 6 %
-    // slower)
+    // and the last warpgroup 56; four: 768 threads launch with 80, the softmax takes 88, the converter
+    // 72 and the last warpgroup 40 (the sum never exceeds the launch's share, so every increase is covered
+    // by the decreases).  Interleaved A/B at g = 32: with the keys multiplied as codes the converter only
+    // widens the values, and 88/72 (no spills) is 2.7 % faster than 80/104 and 96/56.
     static constexpr bool regsplit = F8 && N == 32;
     static constexpr int threads = regsplit ? kWG * (nwg + 2) : kWG * nwg + 32 * conv_warps + 96;
     static constexpr int reg_launch = nwg == 4 ? 80 : 128;
-    static constexpr int reg_soft = nwg == 4 ? 80 : 176;
-    static constexpr int reg_conv = 104;
+    static constexpr int reg_soft = nwg == 4 ? 88 : 176;
+    static constexpr int reg_conv = nwg == 4 ? 72 : 104;
     static constexpr int reg_last = nwg == 4 ? 40 : 56;
     static_assert(!regsplit || (nwg == 2 || nwg == 4), "register split for two or four softmax warpgroups");
     static_assert(!regsplit || kWG * (nwg * reg_soft + reg_conv + reg_last) <= threads * reg_launch,
