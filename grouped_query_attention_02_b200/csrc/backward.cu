@@ -393,7 +393,7 @@ struct QSmem {
     static constexpr int k = dout + kTile;           // K[3] tiles
     static constexpr int v = k + kstages * kTile;    // V[2] tiles
     static constexpr int bars = v + vstages * kTile;
-    static constexpr int nbars = 22;
+    static constexpr int nbars = 24;
     static constexpr int tmem_slot = bars + nbars * 8;
     static constexpr int err = tmem_slot + 8;
     static constexpr int bytes = err + 8;
@@ -401,9 +401,13 @@ struct QSmem {
 // S2_FULL / S2_FREE / DS_READY: per S buffer (the pass of tile j + 1 can finish before the issuer has
 // seen tile j's, so DS_READY alternates like the buffers); DP_FREE: the pass has dP in registers
 enum QBar { QO_FULL = 0, K2_FULL = 1, K2_EMPTY = 4, S2_FULL = 7, S2_FREE = 9, DP_FULL = 11, DP_FREE = 12,
-            DS_READY = 13, DQ_FULL = 15, QDRAIN = 16, S2_READ = 17,   // S2_READ: see the dK/dV kernel's ST_READ
-            V2_FULL = 18, V2_EMPTY = 20 };
-static_assert(V2_EMPTY + QSmem::vstages <= QSmem::nbars && K2_FULL + QSmem::kstages <= K2_EMPTY &&
+            DS_READY = 13, DQ_FULL = 15, QDRAIN = 16, V2_FULL = 18, V2_EMPTY = 20,
+            // per S buffer: the first warpgroup has read the raw columns the second one packs its dS onto (see
+            // the dK/dV kernel's ST_READ).  One barrier per buffer: S is double-buffered, so the first
+            // warpgroup can read the next tile's S before the second looks at this tile's phase; reading S of
+            // tile j + 2 needs the dS of tile j from both warpgroups, so per buffer no phase is passed unseen
+            S2_READ = 22 };
+static_assert(V2_EMPTY + QSmem::vstages <= S2_READ && S2_READ + 2 <= QSmem::nbars && K2_FULL + QSmem::kstages <= K2_EMPTY &&
                   K2_EMPTY + QSmem::kstages <= S2_FULL && DPT_READ < KvSmem::nbars, "barrier slots");
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -448,7 +452,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(&bar[DS_READY + 1], kEw);
         mbar_init(&bar[DQ_FULL], 1);
         mbar_init(&bar[QDRAIN], 1);
-        mbar_init(&bar[S2_READ], kEw / 2);
+        for (int s = 0; s < 2; ++s) mbar_init(&bar[S2_READ + s], kEw / 2);
         *err = 0;
         fence_barrier_init();
     }
@@ -610,7 +614,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tmem_ld32(tS0 + s * 128 + lane_off + w * 64, sr);
             tmem_ld32(tS0 + s * 128 + lane_off + w * 64 + 32, sr + 32);
             tmem_wait_ld();
-            if (w == 0) mbar_arrive(&bar[S2_READ]);
+            if (w == 0) mbar_arrive(&bar[S2_READ + s]);
             if (edge) {
                 // key c of the tile: after the row on the diagonal tile, or past the sequence (its weight
                 // is 2^-inf = 0); masked before the loop below, which then has no branch
@@ -630,7 +634,7 @@ bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             // packed: key columns 64w.. land on packed columns 32w.., which for w = 1 are raw columns the
             // first warpgroup reads
-            if (w == 1 && !wait_or_fail(&bar[S2_READ], j & 1, a, err)) { ok = false; break; }
+            if (w == 1 && !wait_or_fail(&bar[S2_READ + s], (j >> 1) & 1, a, err)) { ok = false; break; }
             tmem_st32(tS0 + s * 128 + lane_off + w * 32, dw);
             tmem_wait_st();
             tc_fence_before();
