@@ -107,3 +107,23 @@ def test_backward_deterministic():
     for u, v in zip(a, b):
         assert torch.equal(u, v)
     assert gqa.gqa_last_launch_count() == 2   # the dQ kernel (which also forms D), then dK/dV
+
+
+def test_backward_repeated_long_sequence():
+    """Many key tiles per CTA (S = 8192: up to 64 per dQ CTA and 64 query tiles per dK/dV CTA), run
+    repeatedly: every run ends with the device status clear (no bounded wait gave up, as a handshake whose
+    phase a fast warpgroup could complete twice before its waiter looks would make one) and every run
+    gives the same bits."""
+    x = inputs.make_prefill(1, 8192, 8, 2, 128, device=DEV, seed=97)
+    dout = inputs.make_dout(1, 8192, 8, 128, device=DEV, seed=97)
+    out, lse = gqa.gqa_prefill_causal_fwd(x.q, x.k, x.v)
+    first = None
+    for _ in range(12):
+        grads = gqa.gqa_prefill_causal_bwd(x.q, x.k, x.v, out, lse, dout)
+        torch.cuda.synchronize()
+        assert gqa.gqa_get_last_device_status() == 0
+        if first is None:
+            first = [g.clone() for g in grads]
+        else:
+            for u, v in zip(first, grads):
+                assert torch.equal(u, v)
